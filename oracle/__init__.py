@@ -1,0 +1,190 @@
+"""fp64 CPU oracle for the fused LM-head linear + softcapped cross-entropy.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import this
+package.  The product path (``lm_head_linear_gemm_b200``) never imports it and
+shares no code with it.
+
+What it computes is the plain definition, written out in float64 on bf16-rounded
+inputs (the GPU path reads the same bf16 values):
+
+* logits of the untied LM head, ``z = X W^T`` over all ``Vpad`` rows of ``W``
+  (little-lm 3.8B write-up, "Setup": LM head of 154.5M = 50304 x 3072 parameters);
+* the logit softcap ``s = cap * tanh(z / cap)`` with ``cap = 15`` (config
+  appendix: ``logit_softcap: 15.0``; loss ``LigerFusedLinearCrossEntropyLoss(softcap=15.0)``).
+  The pages name the softcap but print no formula; ``cap*tanh(z/cap)`` is the
+  reading adopted.  ``cap <= 0`` means no softcap (``s = z``);
+* the padded vocabulary (50257 real tokens padded to 50304 for the tensor cores,
+  "Increasing throughput" / vocabulary padding): padded columns ``j >= Vreal``
+  take no part in the softmax;
+* cross entropy averaged over the positions whose target is not ``ignore_index``
+  (the pages state neither an ignore index nor a reduction; mean over valid rows
+  is the reading adopted; with no valid row the loss is 0);
+* analytic gradients ``dX = dz W`` and ``dW = dz^T X`` with
+  ``dz = g/Nv * (softmax(s) - onehot(t)) * (1 - tanh^2(z/cap))``.
+
+The fused method (the lm_head matmul computed chunk by chunk inside the loss so
+the ``(B*T, vocab)`` logits are never materialised -- "Increasing throughput",
+fused linear cross-entropy) reaches this same result up to rounding order; the
+oracle materialises the logits.  Rows are independent, so large inputs are
+processed in blocks of rows; the only cross-row quantities (the loss sum, the
+valid count and ``dW``) are plain sums over those blocks.
+
+Targets outside ``[0, Vreal)`` that are not ``ignore_index`` are invalid; they
+are counted and treated as ignored (the GPU path raises a status bit for them).
+
+Parity pins (``tests/test_oracle.py``): W = 0 closed form (loss = ln Vreal),
+softmax-minus-onehot rows summing to zero, zero gradient in padded rows,
+no-softcap case against ``torch.nn.functional.cross_entropy`` in fp64, central
+finite differences, and a brute-force per-element loop on tiny shapes.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+__all__ = [
+    "logits", "softcap", "softcap_derivative", "valid_rows", "row_forward", "forward",
+    "row_dlogits", "backward", "forward_backward", "dW_rows",
+]
+
+
+def logits(X: np.ndarray, W: np.ndarray) -> np.ndarray:
+    """``z = X W^T``: hidden states [n, d] times the untied LM head [Vpad, d]."""
+    return np.asarray(X, np.float64) @ np.asarray(W, np.float64).T
+
+
+def softcap(z: np.ndarray, cap: float) -> np.ndarray:
+    """``s = cap * tanh(z / cap)``; identity when ``cap <= 0``."""
+    if cap > 0:
+        return cap * np.tanh(z / cap)
+    return z
+
+
+def softcap_derivative(z: np.ndarray, cap: float) -> np.ndarray:
+    """``ds/dz = 1 - tanh(z/cap)^2``, evaluated from z (not from s, which would
+    cancel badly near saturation); 1 when there is no softcap."""
+    if cap > 0:
+        th = np.tanh(z / cap)
+        return 1.0 - th * th
+    return np.ones_like(z)
+
+
+def valid_rows(t: np.ndarray, Vreal: int, ignore_index: int):
+    """Boolean mask of rows that enter the loss, and the number of invalid targets
+    (neither ignore_index nor inside [0, Vreal))."""
+    t = np.asarray(t, np.int64)
+    in_range = (t >= 0) & (t < Vreal)
+    ignored = t == ignore_index
+    bad = int(np.count_nonzero(~in_range & ~ignored))
+    return in_range & ~ignored, bad
+
+
+def row_forward(X, W, t, Vreal: int, cap: float, ignore_index: int):
+    """Per-row log-sum-exp over the real columns and the target's softcapped logit.
+
+    Returns ``(lse [n], s_target [n] (0 for rows not in the loss), valid [n])``."""
+    z = logits(X, W)
+    s = softcap(z, cap)[:, :Vreal]                       # padded columns excluded
+    m = s.max(axis=1)
+    lse = m + np.log(np.exp(s - m[:, None]).sum(axis=1))
+    valid, _ = valid_rows(t, Vreal, ignore_index)
+    rows = np.nonzero(valid)[0]
+    s_t = np.zeros(len(t), np.float64)
+    s_t[rows] = s[rows, np.asarray(t, np.int64)[rows]]
+    return lse, s_t, valid
+
+
+def forward(X, W, t, Vreal: int, cap: float, ignore_index: int, block_rows: int = 1024):
+    """Mean cross entropy over valid rows.  Returns dict(loss, lse [N], n_valid, n_bad)."""
+    N = X.shape[0]
+    lse = np.empty(N, np.float64)
+    total = 0.0
+    for r0 in range(0, N, block_rows):
+        r1 = min(N, r0 + block_rows)
+        l, st, v = row_forward(X[r0:r1], W, t[r0:r1], Vreal, cap, ignore_index)
+        lse[r0:r1] = l
+        total += float(np.sum((l - st)[v]))
+    valid, bad = valid_rows(t, Vreal, ignore_index)
+    nv = int(np.count_nonzero(valid))
+    loss = total / nv if nv > 0 else 0.0
+    return dict(loss=loss, lse=lse, n_valid=nv, n_bad=bad)
+
+
+def row_dlogits(X, W, t, lse, Vreal: int, cap: float, ignore_index: int, n_valid: int,
+                g: float = 1.0, with_parts: bool = False):
+    """``dz = g/Nv * (softmax(s) - onehot(t)) * (1 - tanh^2(z/cap))`` for a block of rows.
+
+    Columns ``j >= Vreal`` and rows not in the loss get 0.  With ``with_parts``
+    also returns ``g_s = dL/ds`` (softmax minus onehot, scaled) for invariant tests."""
+    z = logits(X, W)
+    Vpad = z.shape[1]
+    s = softcap(z, cap)
+    valid, _ = valid_rows(t, Vreal, ignore_index)
+    gs = np.zeros_like(z)
+    if n_valid > 0:
+        p = np.exp(s[:, :Vreal] - np.asarray(lse, np.float64)[:, None])
+        rows = np.nonzero(valid)[0]
+        p[rows, np.asarray(t, np.int64)[rows]] -= 1.0
+        p[~valid] = 0.0
+        gs[:, :Vreal] = (g / n_valid) * p
+    dz = gs * softcap_derivative(z, cap)
+    assert Vpad == W.shape[0]
+    return (dz, gs) if with_parts else dz
+
+
+def backward(X, W, t, Vreal: int, cap: float, ignore_index: int, g: float = 1.0, lse=None,
+             block_rows: int = 1024):
+    """Gradients of ``g * loss``: ``dX = dz W`` [N, d] and ``dW = dz^T X`` [Vpad, d]."""
+    X = np.asarray(X, np.float64)
+    W = np.asarray(W, np.float64)
+    N = X.shape[0]
+    valid, _ = valid_rows(t, Vreal, ignore_index)
+    nv = int(np.count_nonzero(valid))
+    if lse is None:
+        lse = forward(X, W, t, Vreal, cap, ignore_index, block_rows)["lse"]
+    dX = np.zeros_like(X)
+    dW = np.zeros_like(W)
+    for r0 in range(0, N, block_rows):
+        r1 = min(N, r0 + block_rows)
+        dz = row_dlogits(X[r0:r1], W, t[r0:r1], lse[r0:r1], Vreal, cap, ignore_index, nv, g)
+        dX[r0:r1] = dz @ W
+        dW += dz.T @ X[r0:r1]
+    return dX, dW
+
+
+def forward_backward(X, W, t, Vreal: int, cap: float, ignore_index: int, g: float = 1.0,
+                     block_rows: int = 1024):
+    """Loss, lse and both gradients in one call (what one fused training step needs)."""
+    f = forward(X, W, t, Vreal, cap, ignore_index, block_rows)
+    dX, dW = backward(X, W, t, Vreal, cap, ignore_index, g, f["lse"], block_rows)
+    f.update(dX=dX, dW=dW)
+    return f
+
+
+def dW_rows(X, W, t, lse, vocab_rows, Vreal: int, cap: float, ignore_index: int,
+            g: float = 1.0, block_rows: int = 4096):
+    """Selected rows ``j`` of ``dW = dz^T X``, given the lse of every token row.
+
+    Only the logit columns ``j`` in ``vocab_rows`` are formed, so this costs
+    ``N * d * len(vocab_rows)`` instead of a full backward."""
+    X = np.asarray(X, np.float64)
+    Wj = np.asarray(W, np.float64)[np.asarray(vocab_rows)]
+    vocab_rows = np.asarray(vocab_rows, np.int64)
+    valid, _ = valid_rows(t, Vreal, ignore_index)
+    nv = int(np.count_nonzero(valid))
+    out = np.zeros((len(vocab_rows), X.shape[1]), np.float64)
+    if nv == 0:
+        return out
+    t = np.asarray(t, np.int64)
+    real = vocab_rows < Vreal
+    for r0 in range(0, X.shape[0], block_rows):
+        r1 = min(X.shape[0], r0 + block_rows)
+        z = X[r0:r1] @ Wj.T                                   # [rows, len(vocab_rows)]
+        s = softcap(z, cap)
+        p = np.exp(s - np.asarray(lse[r0:r1], np.float64)[:, None])
+        p -= (t[r0:r1, None] == vocab_rows[None, :])
+        p[~valid[r0:r1]] = 0.0
+        p[:, ~real] = 0.0
+        dz = (g / nv) * p * softcap_derivative(z, cap)
+        out += dz.T @ X[r0:r1]
+    return out

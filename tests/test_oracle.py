@@ -1,0 +1,319 @@
+"""Pins of the fp64 oracle against facts that do not come from the oracle itself.
+
+* the pages' printed shape constants (tests/golden/pages_constants.json);
+* closed forms (W = 0: loss = ln Vreal, dX = 0, dW from the column means of X);
+* invariants (softmax-minus-onehot rows sum to zero, zero gradient for padded
+  rows and ignored tokens, lse bounds, permutation and split additivity);
+* a library special case (no softcap: torch.nn.functional.cross_entropy in fp64,
+  gradients from torch autograd, also through torch.tanh with the softcap);
+* central finite differences of the loss;
+* a brute-force per-element loop with a streaming (online) softmax.
+
+The planted-mistake tests at the end patch the oracle on the CPU and check that
+these pins catch each plausible error.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+PAGES = json.load(open(os.path.join(HERE, "golden", "pages_constants.json")))
+
+
+def _tiny(N=8, d=16, Vr=40, Vp=48, w_std=0.3, ign=2, seed=1, x_std=1.0):
+    rng = np.random.default_rng(seed)
+    X = rng.standard_normal((N, d)) * x_std
+    W = rng.standard_normal((Vp, d)) * w_std
+    t = rng.integers(0, Vr, N)
+    if ign:
+        t[rng.permutation(N)[:ign]] = -1
+    return X, W, t
+
+
+# --------------------------------------------------------------------------- pages
+def test_pages_shapes_pin_the_workloads():
+    Vr, Vp = PAGES["vocab_real"]["value"], PAGES["vocab_padded"]["value"]
+    d, mult = PAGES["d_model"]["value"], PAGES["pad_multiple"]["value"]
+    assert Vp % mult == 0 and Vp - mult < Vr <= Vp          # smallest multiple of 64 >= Vreal
+    assert Vp - Vr == PAGES["unused_rows"]["value"]
+    assert round(d * Vp / 1e6, 1) == PAGES["lm_head_params_millions"]["value"]
+    # the padded rows are real rows of W: 3072 x 50257 would print as 154.4M
+    assert round(d * Vr / 1e6, 1) != PAGES["lm_head_params_millions"]["value"]
+    b, T = PAGES["per_rank_micro_batch"]["value"]
+    assert b * T * PAGES["grad_accum_steps"]["value"] * 8 == PAGES["total_batch_tokens"]["value"]
+    for name in ("small", "3.8b", "3.8b-2k"):
+        c = synth.CONFIGS[name]
+        assert (c.Vreal, c.Vpad, c.cap) == (Vr, Vp, PAGES["logit_softcap"]["value"])
+    assert synth.CONFIGS["3.8b"].d == d
+
+
+# --------------------------------------------------------------------------- P1 closed form
+@pytest.mark.parametrize("Vr,Vp", [(1000, 1024), (50257, 50304)])
+def test_zero_weight_closed_form(Vr, Vp):
+    rng = np.random.default_rng(0)
+    N, d = 6, 8
+    X = rng.standard_normal((N, d))
+    W = np.zeros((Vp, d))
+    t = rng.integers(0, Vr, N)
+    t[2] = -1
+    f = oracle.forward(X, W, t, Vr, 15.0, -1)
+    assert abs(f["loss"] - math.log(Vr)) < 1e-12
+    # the padded columns would give ln(Vpad) if they leaked into the softmax
+    assert abs(f["loss"] - math.log(Vp)) > 1e-5 or Vr == Vp
+    np.testing.assert_allclose(f["lse"], math.log(Vr), rtol=0, atol=1e-12)
+    dX, dW = oracle.backward(X, W, t, Vr, 15.0, -1, lse=f["lse"])
+    assert np.abs(dX).max() == 0.0
+    v = t != -1
+    nv = int(v.sum())
+    expect = np.zeros((Vp, d))
+    expect[:Vr] = X[v].sum(0) / Vr / nv
+    for i in np.nonzero(v)[0]:
+        expect[t[i]] -= X[i] / nv
+    np.testing.assert_allclose(dW, expect, rtol=0, atol=1e-14)
+
+
+def test_pages_headline_closed_form_value():
+    # loss at W = 0 over the pages' real vocabulary
+    assert abs(math.log(50257) - 10.824905119702) < 1e-11
+
+
+# --------------------------------------------------------------------------- P2 invariants
+def test_invariants():
+    X, W, t = _tiny(N=12, d=16, Vr=40, Vp=48, w_std=2.0, ign=3)
+    Vr, cap = 40, 15.0
+    f = oracle.forward(X, W, t, Vr, cap, -1)
+    nv = f["n_valid"]
+    z = oracle.logits(X, W)
+    s = oracle.softcap(z, cap)[:, :Vr]
+    # lse bounds
+    assert np.all(s.max(1) <= f["lse"] + 1e-12)
+    assert np.all(f["lse"] <= s.max(1) + math.log(Vr) + 1e-12)
+    # per-row loss bounds 0 <= lse - s_t <= 2c + ln Vr
+    v = t != -1
+    li = f["lse"][v] - s[np.nonzero(v)[0], t[v]]
+    assert np.all(li >= 0) and np.all(li <= 2 * cap + math.log(Vr))
+    dz, gs = oracle.row_dlogits(X, W, t, f["lse"], Vr, cap, -1, nv, with_parts=True)
+    np.testing.assert_allclose(gs[v].sum(1), 0.0, atol=1e-15)
+    assert np.abs(dz[~v]).max() == 0 and np.abs(dz[:, Vr:]).max() == 0
+    # dz / (1 - tanh^2) recovers the zero-sum g_s (the softcap derivative is the only factor)
+    np.testing.assert_allclose((dz / oracle.softcap_derivative(z, cap))[v].sum(1), 0, atol=1e-15)
+    dX, dW = oracle.backward(X, W, t, Vr, cap, -1, lse=f["lse"])
+    assert np.abs(dW[Vr:]).max() == 0.0
+    assert np.abs(dX[~v]).max() == 0.0
+
+
+def test_permutation_and_split():
+    X, W, t = _tiny(N=16, w_std=1.5, ign=4, seed=3)
+    Vr, cap = 40, 15.0
+    full = oracle.forward_backward(X, W, t, Vr, cap, -1)
+    perm = np.random.default_rng(5).permutation(16)
+    p = oracle.forward_backward(X[perm], W, t[perm], Vr, cap, -1)
+    assert abs(p["loss"] - full["loss"]) < 1e-13
+    np.testing.assert_allclose(p["lse"], full["lse"][perm], atol=1e-13)
+    np.testing.assert_allclose(p["dX"], full["dX"][perm], atol=1e-15)
+    np.testing.assert_allclose(p["dW"], full["dW"], atol=1e-15)
+    a = oracle.forward_backward(X[:7], W, t[:7], Vr, cap, -1)
+    b = oracle.forward_backward(X[7:], W, t[7:], Vr, cap, -1)
+    na, nb = a["n_valid"], b["n_valid"]
+    assert abs((na * a["loss"] + nb * b["loss"]) / (na + nb) - full["loss"]) < 1e-13
+    np.testing.assert_allclose((na * a["dW"] + nb * b["dW"]) / (na + nb), full["dW"], atol=1e-15)
+    # blocked evaluation equals the one-block evaluation
+    blk = oracle.forward_backward(X, W, t, Vr, cap, -1, block_rows=3)
+    assert abs(blk["loss"] - full["loss"]) < 1e-13
+    np.testing.assert_allclose(blk["dW"], full["dW"], atol=1e-15)
+
+
+def test_no_valid_rows_and_bad_targets():
+    X, W, t = _tiny(N=5, ign=0)
+    t[:] = -1
+    f = oracle.forward_backward(X, W, t, 40, 15.0, -1)
+    assert f["loss"] == 0.0 and f["n_valid"] == 0
+    assert np.abs(f["dX"]).max() == 0 and np.abs(f["dW"]).max() == 0
+    t2 = np.array([3, 40, -7, 47, -1], np.int64)       # 40 and 47 are padded ids, -7 invalid
+    valid, bad = oracle.valid_rows(t2, 40, -1)
+    assert valid.tolist() == [True, False, False, False, False] and bad == 3
+
+
+# --------------------------------------------------------------------------- P3 library case
+def _torch_reference(X, W, t, Vr, cap, ii):
+    torch = pytest.importorskip("torch")
+    Xt = torch.tensor(X, dtype=torch.float64, requires_grad=True)
+    Wt = torch.tensor(W, dtype=torch.float64, requires_grad=True)
+    z = Xt @ Wt.T
+    s = cap * torch.tanh(z / cap) if cap > 0 else z
+    loss = torch.nn.functional.cross_entropy(s[:, :Vr], torch.tensor(t), ignore_index=ii)
+    loss.backward()
+    return loss.item(), Xt.grad.numpy(), Wt.grad.numpy()
+
+
+@pytest.mark.parametrize("cap", [0.0, 15.0, 2.0])
+def test_against_torch_cross_entropy(cap):
+    X, W, t = _tiny(N=10, d=12, Vr=30, Vp=32, w_std=1.0, ign=2, seed=7)
+    ref_loss, ref_dX, ref_dW = _torch_reference(X, W, t, 30, cap, -1)
+    f = oracle.forward_backward(X, W, t, 30, cap, -1)
+    assert abs(f["loss"] - ref_loss) < 1e-12
+    np.testing.assert_allclose(f["dX"], ref_dX, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(f["dW"], ref_dW, rtol=0, atol=1e-12)
+
+
+def test_softcap_against_library_tanh():
+    torch = pytest.importorskip("torch")
+    z = np.linspace(-80, 80, 2001)
+    np.testing.assert_allclose(oracle.softcap(z, 15.0),
+                               15.0 * torch.tanh(torch.tensor(z) / 15.0).numpy(), atol=1e-13)
+    assert np.all(np.abs(oracle.softcap(z, 15.0)) <= 15.0)
+    np.testing.assert_allclose(oracle.softcap_derivative(z, 15.0),
+                               1.0 / np.cosh(z / 15.0) ** 2, rtol=1e-10, atol=1e-300)
+    # (1 - tanh^2 loses ~eps/(1 - tanh^2) relative accuracy near saturation: 2e-12 at |z/c| = 5.3)
+
+
+# --------------------------------------------------------------------------- P4 finite differences
+@pytest.mark.parametrize("cap,w_std,g", [(15.0, 3.0, 1.0), (2.0, 1.0, 0.7), (0.0, 1.0, 1.0)])
+def test_finite_differences(cap, w_std, g):
+    X, W, t = _tiny(N=8, d=16, Vr=40, Vp=48, w_std=w_std, ign=2, seed=11)
+    Vr, h = 40, 1e-6
+    dX, dW = oracle.backward(X, W, t, Vr, cap, -1, g=g)
+
+    def L(X_, W_):
+        return g * oracle.forward(X_, W_, t, Vr, cap, -1)["loss"]
+
+    num_dX = np.zeros_like(X)
+    for idx in np.ndindex(*X.shape):
+        Xp, Xm = X.copy(), X.copy()
+        Xp[idx] += h
+        Xm[idx] -= h
+        num_dX[idx] = (L(Xp, W) - L(Xm, W)) / (2 * h)
+    num_dW = np.zeros_like(W)
+    for idx in np.ndindex(*W.shape):
+        Wp, Wm = W.copy(), W.copy()
+        Wp[idx] += h
+        Wm[idx] -= h
+        num_dW[idx] = (L(X, Wp) - L(X, Wm)) / (2 * h)
+    assert np.linalg.norm(num_dX - dX) <= 1e-6 * np.linalg.norm(dX)
+    assert np.linalg.norm(num_dW - dW) <= 1e-6 * np.linalg.norm(dW)
+    assert np.abs(num_dW[Vr:]).max() < 1e-9          # padded rows: the loss does not see them
+
+
+# --------------------------------------------------------------------------- P5 brute force
+def _brute(X, W, t, Vr, cap, ii, g=1.0):
+    """Per-element loops; streaming (online) max / sum-exp per row."""
+    N, d = len(X), len(X[0])
+    Vp = len(W)
+    z = [[sum(X[i][k] * W[j][k] for k in range(d)) for j in range(Vp)] for i in range(N)]
+    s = [[cap * math.tanh(z[i][j] / cap) if cap > 0 else z[i][j] for j in range(Vp)]
+         for i in range(N)]
+    lse = []
+    for i in range(N):
+        m, l = -math.inf, 0.0
+        for j in range(Vr):
+            if s[i][j] > m:
+                l = l * math.exp(m - s[i][j]) + 1.0
+                m = s[i][j]
+            else:
+                l += math.exp(s[i][j] - m)
+        lse.append(m + math.log(l))
+    valid = [t[i] != ii for i in range(N)]
+    nv = sum(valid)
+    loss = sum(lse[i] - s[i][t[i]] for i in range(N) if valid[i]) / nv
+    dX = [[0.0] * d for _ in range(N)]
+    dW = [[0.0] * d for _ in range(Vp)]
+    for i in range(N):
+        if not valid[i]:
+            continue
+        for j in range(Vr):
+            p = math.exp(s[i][j] - lse[i]) - (1.0 if j == t[i] else 0.0)
+            der = 1.0 - math.tanh(z[i][j] / cap) ** 2 if cap > 0 else 1.0
+            dz = g / nv * p * der
+            for k in range(d):
+                dX[i][k] += dz * W[j][k]
+                dW[j][k] += dz * X[i][k]
+    return loss, np.array(lse), np.array(dX), np.array(dW)
+
+
+@pytest.mark.parametrize("cap", [15.0, 0.0])
+def test_brute_force(cap):
+    X, W, t = _tiny(N=5, d=4, Vr=7, Vp=8, w_std=2.0, ign=1, seed=2)
+    loss, lse, dX, dW = _brute(X.tolist(), W.tolist(), t.tolist(), 7, cap, -1, g=1.3)
+    f = oracle.forward_backward(X, W, t, 7, cap, -1, g=1.3)
+    assert abs(f["loss"] - loss) < 1e-12
+    np.testing.assert_allclose(f["lse"], lse, atol=1e-12)
+    np.testing.assert_allclose(f["dX"], dX, atol=1e-12)
+    np.testing.assert_allclose(f["dW"], dW, atol=1e-12)
+
+
+# --------------------------------------------------------------------------- sampled helpers
+def test_dW_rows_matches_full_backward():
+    X, W, t = _tiny(N=20, d=8, Vr=30, Vp=32, w_std=1.0, ign=3, seed=4)
+    f = oracle.forward_backward(X, W, t, 30, 15.0, -1, g=0.5)
+    rows = np.array([0, 5, 29, 30, 31])
+    got = oracle.dW_rows(X, W, t, f["lse"], rows, 30, 15.0, -1, g=0.5, block_rows=7)
+    np.testing.assert_allclose(got, f["dW"][rows], atol=1e-15)
+
+
+def test_synth_is_seeded_and_shaped():
+    a = synth.make_inputs("tiny")
+    b = synth.make_inputs("tiny")
+    assert np.array_equal(a["X"], b["X"]) and np.array_equal(a["W"], b["W"])
+    assert np.array_equal(a["targets"], b["targets"])
+    c = a["cfg"]
+    assert a["X"].shape == (64, 128) and a["W"].shape == (1024, 128)
+    assert int((a["targets"] == -1).sum()) == 2
+    assert a["targets"].max() < 1000
+    s = synth.make_inputs("small", N=2048)
+    x = synth.bf16_to_f64(s["X"])
+    np.testing.assert_allclose(np.sqrt((x * x).mean(1)), 1.0, atol=5e-3)   # unit RMS rows
+    assert int((s["targets"] == -1).sum()) == round(0.02 * 2048)
+    tv = s["targets"][s["targets"] >= 0]
+    assert tv.max() < 50257 and np.mean(tv == 0) > 0.05                   # Zipf head
+    # bf16 rounding is round-to-nearest-even
+    v = np.array([1.0, 1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, -2.5], np.float32)
+    assert synth.bf16_to_f32(synth.f32_to_bf16_bits(v)).tolist() == [1.0, 1.0, 1.0 + 2 ** -6, -2.5]
+    assert c.cap == 15.0
+
+
+# --------------------------------------------------------------------------- planted mistakes
+def test_planted_mistakes_are_caught(monkeypatch):
+    """Patch a plausible bug into the oracle (on the CPU) and check a pin fails."""
+    X, W, t = _tiny(N=6, d=6, Vr=10, Vp=12, w_std=2.0, ign=1, seed=9)
+
+    def pins_hold():
+        try:
+            ref_loss, ref_dX, ref_dW = _torch_reference(X, W, t, 10, 15.0, -1)
+            f = oracle.forward_backward(X, W, t, 10, 15.0, -1)
+            ok = abs(f["loss"] - ref_loss) < 1e-12
+            ok &= np.allclose(f["dX"], ref_dX, atol=1e-12)
+            ok &= np.allclose(f["dW"], ref_dW, atol=1e-12)
+            z0 = oracle.forward(X, np.zeros_like(W), t, 10, 15.0, -1)["loss"]
+            ok &= abs(z0 - math.log(10)) < 1e-12
+            return bool(ok)
+        except Exception:
+            return False
+
+    assert pins_hold()
+    real_softcap, real_der, real_logits = oracle.softcap, oracle.softcap_derivative, oracle.logits
+    real_row_forward = oracle.row_forward
+    mutants = {
+        "dropped softcap derivative": ("softcap_derivative", lambda z, cap: np.ones_like(z)),
+        "derivative from wrong sign": ("softcap_derivative",
+                                       lambda z, cap: 1.0 + np.tanh(z / cap) ** 2),
+        "softcap without outer scale": ("softcap", lambda z, cap: np.tanh(z / cap)),
+        "transposed head": ("logits", lambda X_, W_: (np.asarray(X_) @ np.asarray(W_).T)[:, ::-1]),
+        "padded columns in softmax": ("row_forward", None),
+    }
+    for name, (attr, fn) in mutants.items():
+        if name == "padded columns in softmax":
+            def fn(X_, W_, t_, Vreal, cap, ii):
+                return real_row_forward(X_, W_, t_, W_.shape[0], cap, ii)
+        monkeypatch.setattr(oracle, attr, fn)
+        assert not pins_hold(), name
+        monkeypatch.setattr(oracle, attr, {"softcap": real_softcap,
+                                           "softcap_derivative": real_der,
+                                           "logits": real_logits,
+                                           "row_forward": real_row_forward}[attr])
+    assert pins_hold()
