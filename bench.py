@@ -1,0 +1,447 @@
+#!/usr/bin/env python
+"""Benchmark of the fused LM-head linear + softcapped cross-entropy, forward + backward.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl flce|reference]
+
+One step = one fused forward that forms loss, lse, dX and dW (flce_forward with
+want_grads=1) plus the backward call that applies the upstream gradient (a device
+scalar equal to 1, the autograd default for a scalar loss), on one batch of the
+3.8B model's head: N = 16384 tokens (batch 16 x context 1024), d = 3072,
+V = 50257 -> 50304, softcap 15.  Credited work: 6*N*d*Vpad FLOP per step.
+
+Multi-GPU (torchrun): every rank runs an independent replica on its own batch
+(weak scaling, no collective in the data path); the time is the max over ranks.
+``--impl reference`` times the fp64 CPU oracle on a bounded sample of rows of the
+same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "fused linear-CE fwd+bwd tokens/sec and TFLOP/s (% bf16 peak) at d=3072,V=50304"
+UNIT = "tokens/s"
+DATASHEET_BF16_TFLOPS = 2250.0
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["flce", "reference"], default="flce")
+    ap.add_argument("--config", default="3.8b")
+    ap.add_argument("--chunk-rows", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-unfused", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="target CPU time of the oracle baseline sample")
+    ap.add_argument("--ref-rows", type=int, default=128,
+                    help="rows per step of the --impl reference arm")
+    return ap.parse_args()
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def workload_desc(c, chunk):
+    return {
+        "workload": f"{c.name}: fused linear-CE fwd+bwd, N={c.N} tokens, d={c.d}, "
+                    f"Vreal={c.Vreal} padded to Vpad={c.Vpad}, softcap={c.cap:g}",
+        "N": c.N, "d": c.d, "Vreal": c.Vreal, "Vpad": c.Vpad, "cap": c.cap,
+        "ignore_index": c.ignore_index, "ignored_rows": c.ignore_count,
+        "targets": "Zipf(1.1)" if c.target_dist == "zipf" else c.target_dist,
+        "x": c.x_dist, "w_std": c.w_std, "chunk_rows": chunk,
+        "l2": f"inputs larger than L2: X {c.N * c.d * 2 / 1e6:.1f} MB + W "
+              f"{c.Vpad * c.d * 2 / 1e6:.1f} MB > 126 MB L2 (no flush)",
+    }
+
+
+# ----------------------------------------------------------------------------------- CPU oracle
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def oracle_step(inp, r0: int, rows: int):
+    """Oracle forward + backward on rows [r0, r0+rows) of the workload (all Vpad, all d)."""
+    import oracle
+    import synth
+    c = inp["cfg"]
+    X = synth.bf16_to_f64(inp["X"][r0:r0 + rows])
+    W = inp.get("_W64")
+    if W is None:
+        W = inp["_W64"] = synth.bf16_to_f64(inp["W"])
+    t = inp["targets"][r0:r0 + rows]
+    return oracle.forward_backward(X, W, t, c.Vreal, c.cap, c.ignore_index)
+
+
+def cpu_baseline(inp, target_s: float):
+    """Time the oracle as it stands on a contiguous row slice sized for ~target_s seconds."""
+    c = inp["cfg"]
+    probe = min(32, c.N)
+    t0 = time.perf_counter()
+    oracle_step(inp, 0, probe)
+    dt = time.perf_counter() - t0
+    rows = int(max(probe, min(c.N, probe * target_s / max(dt, 1e-3))))
+    rows = max(probe, (rows // 32) * 32)
+    t0 = time.perf_counter()
+    oracle_step(inp, 0, rows)
+    dt = time.perf_counter() - t0
+    return {"value": rows / dt, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": f"rows [0, {rows}) of the {c.name} workload: fp64 forward + backward over "
+                      f"all Vpad={c.Vpad} columns and d={c.d} (that slice's dW contribution "
+                      f"included); {dt:.1f} s"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import synth
+    inp = synth.make_inputs(args.config)
+    c = inp["cfg"]
+    rows = max(1, min(args.ref_rows, c.N))
+    times = []
+    for s in range(args.warmup + args.steps):
+        r0 = (s * rows) % max(1, c.N - rows + 1)
+        t0 = time.perf_counter()
+        oracle_step(inp, r0, rows)
+        if s >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    step_s = sum(times) / len(times)
+    value = rows / step_s
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": workload_desc(c, 0),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                         "sample": f"{rows} contiguous rows per step (fp64 forward + backward "
+                                   f"over all Vpad and d, dW contribution included)"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str | None):
+        self.proc = None
+        self.path = None
+        self.gpu_id = gpu_id
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                   "-lms", "100"]
+            if self.gpu_id:
+                cmd += ["-i", self.gpu_id]
+            self.proc = subprocess.Popen(cmd, stdout=open(self.path, "w"),
+                                         stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append(dict(sm=float(parts[1]), max=float(parts[2]),
+                                 power=float(parts[3]) if parts[3] not in ("[N/A]", "") else 0.0,
+                                 hw=parts[5], hwt=parts[6], swt=parts[7], pcap=parts[8]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        reasons = set()
+        for r in rows:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
+                              ("swt", "sw_thermal_slowdown"), ("pcap", "sw_power_cap")):
+                if r[key].lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in rows),
+                "sm_max_mhz": max(r["max"] for r in rows),
+                "power_w_max": max(r["power"] for r in rows),
+                "samples": len(rows), "reasons": sorted(reasons)}
+
+
+# ----------------------------------------------------------------------------------- GPU arm
+def main_gpu(args):
+    import torch
+    import torch.distributed as dist
+    import lm_head_linear_gemm_b200 as flce
+    import synth
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (B200); the CPU oracle arm is --impl reference")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    cfg = synth.CONFIGS[args.config]
+    inp = synth.make_inputs(cfg, seed=cfg.seed + rank)
+    c = inp["cfg"]
+    N, d, Vp, Vr = c.N, c.d, c.Vpad, c.Vreal
+
+    def host_bf16(a):
+        import numpy as np
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16)
+
+    X_h = host_bf16(inp["X"]).pin_memory()
+    t_h = torch.from_numpy(inp["targets"]).pin_memory()
+    W = host_bf16(inp["W"]).to(dev)
+    X = X_h.to(dev)
+    t = t_h.to(dev)
+    torch.cuda.synchronize()
+    mem_inputs = torch.cuda.memory_allocated(dev)
+    g_one = torch.ones((), dtype=torch.float32, device=dev)
+    dX = torch.empty_like(X)
+    dW = torch.empty((Vp, d), dtype=torch.float32, device=dev)
+    shape = flce.make_shape(N, d, Vp, Vr, c.cap, c.ignore_index, args.chunk_rows)
+    ws = flce.alloc_workspace(shape, True, dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        loss, lse, _, _, _ = flce.forward(X, W, t, Vr, c.cap, c.ignore_index, True, dX=dX, dW=dW,
+                                          workspace=ws, chunk_rows=args.chunk_rows)
+        flce.backward(X, W, t, lse, Vr, c.cap, c.ignore_index, grad_out=g_one, dX=dX, dW=dW,
+                      grads_precomputed=True)
+        return loss
+
+    # ---- device-resident timing
+    torch.cuda.reset_peak_memory_stats(dev)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    status, nv = flce.read_status(ws)
+    # everything the fused step holds beyond its inputs: dX, dW, workspace, lse, loss
+    peak_fused = torch.cuda.max_memory_allocated(dev) - mem_inputs
+    barrier()
+    gpu_id = None
+    try:
+        gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        pass
+    clocks = ClockSampler(gpu_id)
+    clocks.start()
+    flce.instrument(True)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(args.steps):
+        loss = step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    elapsed_ms = e0.elapsed_time(e1)
+    kstats = flce.instrument_read()
+    flce.instrument(False)
+    clk = clocks.stop()
+    if world > 1:
+        tt = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(tt.item())
+    ms_per_step = elapsed_ms / args.steps
+    value = world * N / (ms_per_step / 1e3)
+    credited = 6.0 * N * d * Vp
+    tflops = credited / (ms_per_step / 1e3) / 1e12 * world
+
+    # ---- end-to-end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        loss_h = torch.empty((), dtype=torch.float32).pin_memory()
+
+        def e2e_step():
+            X.copy_(X_h, non_blocking=True)
+            t.copy_(t_h, non_blocking=True)
+            loss = step()
+            loss_h.copy_(loss, non_blocking=True)
+
+        for _ in range(max(1, args.warmup)):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        f1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        e2e_ms = f0.elapsed_time(f1)
+        if world > 1:
+            tt = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            e2e_ms = float(tt.item())
+        e2e = {"value": world * N / (e2e_ms / args.steps / 1e3), "unit": UNIT,
+               "h2d_bytes_per_step": X.numel() * 2 + t.numel() * 8, "d2h_bytes_per_step": 4,
+               "ms_per_step": e2e_ms / args.steps,
+               "what": "pinned-host X and targets copied in, loss copied out, every step; "
+                       "W and dW stay resident (the head's parameter and its gradient)"}
+
+    peaks, peaks_src = load_peaks()
+    sustained = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    kinds = {}
+    for name, k in kstats["gemm"].items():
+        if k["launches"]:
+            kinds[name] = {"launches": k["launches"], "ms_per_launch": k["ms"] / k["launches"],
+                           "tflops": k["flop"] / (k["ms"] / 1e3) / 1e12,
+                           "share_of_step": k["ms"] / elapsed_ms if elapsed_ms else None}
+    dom = max(kinds, key=lambda n: kstats["gemm"][n]["ms"]) if kinds else None
+    traffic = None
+    tpath = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    if dom and os.path.exists(tpath):
+        tj = json.load(open(tpath))
+        ent = tj.get(dom)
+        if ent and ent.get("kernel_rev") == KERNEL_REV and ent.get("config") == c.name:
+            traffic = ent.get("bytes_per_launch")
+    roofline = None
+    if dom:
+        ach = kinds[dom]["tflops"]
+        roofline = {"bound": "tensor", "kernel": dom, "achieved": ach, "peak": sustained,
+                    "unit": "TFLOP/s", "frac": ach / sustained, "traffic": traffic,
+                    "peak_source": f"bf16_tflops_sustained ({peaks_src} MEASURED_PEAKS.json; "
+                                   "the kernel runs inside a long step)",
+                    "algorithmic": "2*rows*Vpad*d FLOP per launch (each of the three "
+                                   "contractions of a chunk carries one third of 6*N*d*Vpad)"}
+
+    unfused = None
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_unfused:
+        unfused = unfused_torch_baseline(X, W, t, c, args)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(inp, args.cpu_seconds)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": dict(workload_desc(c, shape.chunk_rows or min(N, 4096)),
+                           parallelism=f"replicas x{world}" if world > 1 else "single GPU"),
+            "tflops": tflops,
+            "pct_of_bf16_datasheet_2250": tflops / world / DATASHEET_BF16_TFLOPS,
+            "pct_of_measured_bf16_burst": tflops / world / burst,
+            "pct_of_measured_bf16_sustained": tflops / world / sustained,
+            "credited_flop_per_step": credited, "executed_flop_per_step": credited,
+            "roofline": roofline, "kernels": kinds, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": kstats["launches_total"],
+            "gpu_launches_per_step": kstats["launches_total"] / args.steps,
+            "clocks": clk,
+            "peak_mem_MiB": {"fused_step": peak_fused / 2**20,
+                             "workspace": ws.numel() / 2**20,
+                             "unfused_torch": unfused["peak_MiB"] if unfused else None},
+            "unfused_torch": unfused, "device_status": status, "n_valid": nv,
+            "loss": float(loss.item()),
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+KERNEL_REV = "v1"
+
+
+def unfused_torch_baseline(X, W, t, c, args):
+    """Comparator only (not the product path): materialised bf16 logits, fp32 softcap,
+    torch cross_entropy and autograd, as a plain PyTorch training loss would do."""
+    import torch
+    dev = X.device
+    Xg = X.detach().clone().requires_grad_(True)
+    Wg = W.detach().clone().requires_grad_(True)
+
+    def step():
+        z = Xg @ Wg.T
+        s = c.cap * torch.tanh(z.float() / c.cap)
+        loss = torch.nn.functional.cross_entropy(s[:, :c.Vreal], t, ignore_index=c.ignore_index)
+        loss.backward()
+        Xg.grad = None
+        Wg.grad = None
+        return loss
+
+    try:
+        torch.cuda.synchronize()
+        torch.cuda.reset_peak_memory_stats(dev)
+        base = torch.cuda.memory_allocated(dev)   # beyond its (cloned) inputs: logits, grads
+        for _ in range(2):
+            step()
+        torch.cuda.synchronize()
+        peak = torch.cuda.max_memory_allocated(dev) - base
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n = max(3, min(args.steps, 10))
+        e0.record()
+        for _ in range(n):
+            step()
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / n
+        return {"tokens_per_s": c.N / (ms / 1e3), "ms_per_step": ms, "peak_MiB": peak / 2**20,
+                "what": "torch: bf16 X@W.T, fp32 cap*tanh, F.cross_entropy, autograd"}
+    except torch.cuda.OutOfMemoryError:
+        return {"error": "out of memory"}
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return main_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,144 @@
+/*
+ * flce.h -- C ABI of the fused LM-head linear + softcapped cross-entropy for B200 (sm_100a).
+ *
+ * The operation (little-lm 3.8B write-ups):
+ *   - the untied LM head W [Vpad, d] (154.5M = 50304 x 3072 parameters; "Setup" table);
+ *   - logits z = X W^T with a logit softcap s = cap * tanh(z / cap), cap = 15 (config appendix:
+ *     logit_softcap: 15.0, LigerFusedLinearCrossEntropyLoss(softcap=15.0); the pages print no
+ *     formula, cap*tanh(z/cap) is the reading used);
+ *   - a vocabulary of Vreal = 50257 tokens padded to Vpad = 50304, a multiple of 64, for the
+ *     tensor cores ("Increasing throughput", vocabulary padding; config appendix).  Padded
+ *     columns j >= Vreal take no part in the softmax and get zero gradient;
+ *   - cross entropy averaged over the rows whose target is not ignore_index;
+ *   - fused: the lm_head matmul is computed in chunks inside the loss, so the full
+ *     (B*T, vocab) logits are never materialised ("Increasing throughput", fused linear
+ *     cross-entropy).
+ *
+ *   loss   = (1/Nv) * sum_{i in V} (lse_i - s_{i, t_i}),   lse_i = log sum_{j < Vreal} exp(s_ij)
+ *   dz_ij  = g/Nv * (softmax(s_i)_j - [j = t_i]) * (1 - tanh^2(z_ij / cap))    (0 for j >= Vreal)
+ *   dX     = dz W,   dW = dz^T X
+ * with V = {i : t_i != ignore_index and 0 <= t_i < Vreal}, Nv = |V|.  Nv = 0 gives loss 0 and
+ * zero gradients.
+ *
+ * Conventions for every entry point:
+ *   - Data pointers are DEVICE pointers owned by the caller; the library never allocates or
+ *     frees memory.  Scratch space is the caller's `workspace` (see flce_workspace_bytes).
+ *   - Layouts are row-major and dense: X [N, d] bf16, W [Vpad, d] bf16, targets [N] int64,
+ *     lse [N] fp32, loss [1] fp32, dX [N, d] bf16, dW [Vpad, d] fp32.
+ *   - Every data pointer must be 16-byte aligned; d and Vpad must be multiples of 8 (the
+ *     tensor-memory-accelerator row stride must be a multiple of 16 bytes).
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).  Calls are
+ *     stream-ordered and asynchronous; calls on different streams are independent when their
+ *     workspaces and outputs differ.
+ *   - Argument errors are detected on the host before anything is launched and returned as a
+ *     negative flce_status.  Targets outside [0, Vreal) that are not ignore_index are not an
+ *     argument error: the row is treated as ignored and the device status word gets
+ *     FLCE_DEV_BAD_TARGET (read it with flce_read_status).  No kernel ever traps.
+ *   - Every wait inside a kernel is bounded; a wait that runs out sets FLCE_DEV_TIMEOUT.
+ *   - Results are bitwise reproducible from call to call (fixed reduction orders).
+ *   - The device must be compute capability 10.0 (B200, sm_100a).
+ */
+#ifndef FLCE_H_
+#define FLCE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FLCE_OK = 0,
+  FLCE_ERR_ARG = -1,       /* null pointer, bad size, inconsistent shape */
+  FLCE_ERR_ALIGN = -2,     /* pointer not 16-byte aligned, or d / Vpad not a multiple of 8 */
+  FLCE_ERR_WORKSPACE = -3, /* workspace smaller than flce_workspace_bytes() */
+  FLCE_ERR_DEVICE = -4,    /* current device is not compute capability 10.0 */
+  FLCE_ERR_CUDA = -5,      /* a CUDA runtime call or kernel launch failed */
+  FLCE_ERR_TIMEOUT = -6    /* reserved: a device wait ran out (reported via the status word) */
+} flce_status;
+
+/* Bits of the device status word (flce_read_status). */
+enum { FLCE_DEV_BAD_TARGET = 1u, FLCE_DEV_TIMEOUT = 2u };
+
+typedef struct {
+  int64_t N;            /* tokens (rows of X, targets); N = 0 is allowed and gives loss 0 */
+  int64_t d;            /* hidden size; multiple of 8 */
+  int64_t Vpad;         /* rows of W; multiple of 8 */
+  int64_t Vreal;        /* real vocabulary, 1 <= Vreal <= Vpad */
+  float cap;            /* logit softcap; <= 0 disables it */
+  int64_t ignore_index; /* target value that leaves a row out of the loss (e.g. -1) */
+  int64_t chunk_rows;   /* rows per fused chunk (bounds the scratch); 0 = automatic */
+} flce_shape;
+
+/*
+ * Bytes of device scratch the calls below need for this shape.  want_grads = 0: the
+ * statistics-only forward; want_grads = 1: the forward that also forms the gradients, and the
+ * recomputing backward.  The scratch grows with chunk_rows * Vpad (the per-chunk gradient
+ * operand) and linearly with N; it never holds an N x Vpad buffer.  Returns 0 when the shape is
+ * invalid.
+ */
+size_t flce_workspace_bytes(const flce_shape* shape, int want_grads);
+
+/*
+ * Forward.  Writes loss[0] (mean over rows in the loss) and lse[i] for every row (ignored rows
+ * included).  With want_grads = 1 it also forms the gradients of the mean loss (upstream
+ * gradient g = 1) in the same pass over the logits: dX [N, d] bf16 is written, and dW [Vpad, d]
+ * fp32 is written (accumulate_dW = 0) or added to (accumulate_dW = 1, gradient accumulation over
+ * micro-batches as in the pages' 7-step accumulation).  With want_grads = 0, dX and dW may be
+ * NULL and are not touched.
+ * workspace: device scratch of at least flce_workspace_bytes(shape, want_grads) bytes,
+ * 256-byte aligned; its contents on entry are ignored.
+ */
+int flce_forward(const flce_shape* shape, const void* X, const void* W, const int64_t* targets,
+                 float* loss, float* lse, int want_grads, void* dX, float* dW, int accumulate_dW,
+                 void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Backward.
+ *   grads_precomputed = 1: dX and dW were formed by flce_forward(want_grads = 1); they are
+ *     multiplied in place by the device scalar *grad_out (nothing runs when grad_out is NULL;
+ *     the kernel returns at once when *grad_out == 1).  When the forward accumulated into dW,
+ *     the whole dW buffer is scaled.
+ *   grads_precomputed = 0: recomputes the logits chunk by chunk from X and W, using lse from
+ *     flce_forward, and forms dX (written) and dW (written, or added to when
+ *     accumulate_dW = 1) for upstream gradient *grad_out (1 when grad_out is NULL).
+ * workspace: at least flce_workspace_bytes(shape, 1) bytes.
+ */
+int flce_backward(const flce_shape* shape, const void* X, const void* W, const int64_t* targets,
+                  const float* lse, const float* grad_out, void* dX, float* dW, int accumulate_dW,
+                  int grads_precomputed, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Reads the device status word (FLCE_DEV_* bits) and the number of rows in the loss from the
+ * workspace of the last call on `stream`.  Synchronises that stream.  Either output may be
+ * NULL.
+ */
+int flce_read_status(const void* workspace, uint32_t* dev_status_out, int64_t* n_valid_out,
+                     void* stream);
+
+/*
+ * Instrumentation (not part of the computation).  flce_instrument(1) resets the counters and
+ * starts recording: every kernel the library launches is counted, and each tensor-core
+ * contraction launch (kind 0: logits, 1: dX, 2: dW) is bracketed by CUDA events on its own
+ * stream.  flce_instrument(0) stops recording.  flce_instrument_read waits for the recorded
+ * events and fills `out` with the totals since the last reset.  Process-wide; host-thread safe.
+ */
+typedef struct {
+  int64_t launches_total;      /* all kernels launched while recording */
+  int64_t gemm_launches[3];    /* contraction launches by kind */
+  double gemm_ms[3];           /* summed event-timed durations by kind, milliseconds */
+  double gemm_flop[3];         /* 2*M*N*K summed over those launches */
+} flce_kernel_stats;
+
+int flce_instrument(int enable);
+int flce_instrument_read(flce_kernel_stats* out);
+
+/* Human-readable name of an flce_status value. */
+const char* flce_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FLCE_H_ */

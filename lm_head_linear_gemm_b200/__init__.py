@@ -1,0 +1,18 @@
+"""Fused LM-head linear + softcapped cross-entropy for B200 (sm_100a).
+
+The compute path is the C-ABI library ``libflce.so`` (include/flce.h), built in-tree
+by ``python -m lm_head_linear_gemm_b200.build``; this package only marshals
+arguments to it.  Entry points raise if the library is missing: there is no
+fallback implementation.
+"""
+from ._abi import (DEV_BAD_TARGET, DEV_TIMEOUT, FlceError, alloc_workspace, backward,
+                   declared_functions, forward, instrument, instrument_read, lib, make_shape, raw_backward, raw_forward,
+                   read_status, status_string, workspace_bytes)
+from .autograd import FusedLinearCrossEntropy, fused_linear_cross_entropy
+
+__all__ = [
+    "DEV_BAD_TARGET", "DEV_TIMEOUT", "FlceError", "alloc_workspace", "backward",
+    "declared_functions", "forward", "instrument", "instrument_read", "lib", "make_shape", "raw_backward", "raw_forward",
+    "read_status", "status_string", "workspace_bytes", "FusedLinearCrossEntropy",
+    "fused_linear_cross_entropy",
+]

@@ -1,0 +1,241 @@
+"""ctypes binding of ``libflce.so`` (include/flce.h).  Argument marshalling only.
+
+PyTorch provides device memory and the current CUDA stream; every step of the
+fused linear cross-entropy runs in the library's kernels.  There is no fallback:
+if the library is missing, importing the binding's entry points raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libflce.so")
+HEADER_PATH = os.path.join(os.path.dirname(HERE), "include", "flce.h")
+
+FLCE_OK = 0
+DEV_BAD_TARGET = 1
+DEV_TIMEOUT = 2
+
+
+class FlceError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what}: {status_string(code)} ({code})")
+        self.code = code
+
+
+class flce_shape(ctypes.Structure):
+    _fields_ = [
+        ("N", ctypes.c_int64),
+        ("d", ctypes.c_int64),
+        ("Vpad", ctypes.c_int64),
+        ("Vreal", ctypes.c_int64),
+        ("cap", ctypes.c_float),
+        ("ignore_index", ctypes.c_int64),
+        ("chunk_rows", ctypes.c_int64),
+    ]
+
+
+class flce_kernel_stats(ctypes.Structure):
+    _fields_ = [
+        ("launches_total", ctypes.c_int64),
+        ("gemm_launches", ctypes.c_int64 * 3),
+        ("gemm_ms", ctypes.c_double * 3),
+        ("gemm_flop", ctypes.c_double * 3),
+    ]
+
+
+GEMM_KINDS = ("logits", "dX", "dW")
+
+_lib = None
+
+
+def declared_functions(header: str = HEADER_PATH) -> list[str]:
+    """Names of the functions include/flce.h declares."""
+    text = open(header).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(flce_[a-z_]+)\s*\(", text)))
+
+
+def lib() -> ctypes.CDLL:
+    """Load libflce.so (built in-tree by ``python -m lm_head_linear_gemm_b200.build``)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing; build it with "
+                          "`python -m lm_head_linear_gemm_b200.build` (nvcc, sm_100a)")
+    L = ctypes.CDLL(LIB_PATH)
+    P = ctypes.c_void_p
+    shp = ctypes.POINTER(flce_shape)
+    L.flce_workspace_bytes.argtypes = [shp, ctypes.c_int]
+    L.flce_workspace_bytes.restype = ctypes.c_size_t
+    L.flce_forward.argtypes = [shp, P, P, P, P, P, ctypes.c_int, P, P, ctypes.c_int, P,
+                               ctypes.c_size_t, P]
+    L.flce_forward.restype = ctypes.c_int
+    L.flce_backward.argtypes = [shp, P, P, P, P, P, P, P, ctypes.c_int, ctypes.c_int, P,
+                                ctypes.c_size_t, P]
+    L.flce_backward.restype = ctypes.c_int
+    L.flce_read_status.argtypes = [P, ctypes.POINTER(ctypes.c_uint32),
+                                   ctypes.POINTER(ctypes.c_int64), P]
+    L.flce_read_status.restype = ctypes.c_int
+    L.flce_instrument.argtypes = [ctypes.c_int]
+    L.flce_instrument.restype = ctypes.c_int
+    L.flce_instrument_read.argtypes = [ctypes.POINTER(flce_kernel_stats)]
+    L.flce_instrument_read.restype = ctypes.c_int
+    L.flce_status_string.argtypes = [ctypes.c_int]
+    L.flce_status_string.restype = ctypes.c_char_p
+    _lib = L
+    return L
+
+
+def status_string(code: int) -> str:
+    try:
+        return lib().flce_status_string(int(code)).decode()
+    except ImportError:
+        return f"status {code}"
+
+
+def make_shape(N: int, d: int, Vpad: int, Vreal: int, cap: float = 15.0,
+               ignore_index: int = -1, chunk_rows: int = 0) -> flce_shape:
+    return flce_shape(int(N), int(d), int(Vpad), int(Vreal), float(cap), int(ignore_index),
+                      int(chunk_rows))
+
+
+def workspace_bytes(shape: flce_shape, want_grads: bool) -> int:
+    return int(lib().flce_workspace_bytes(ctypes.byref(shape), 1 if want_grads else 0))
+
+
+def _ptr(t) -> int | None:
+    return None if t is None else int(t.data_ptr())
+
+
+def _stream(stream) -> int | None:
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def raw_forward(shape, X_ptr, W_ptr, t_ptr, loss_ptr, lse_ptr, want_grads, dX_ptr, dW_ptr,
+                accumulate_dW, ws_ptr, ws_bytes, stream_handle) -> int:
+    """Direct C-ABI call with integer pointers; returns the flce_status code."""
+    return lib().flce_forward(ctypes.byref(shape), X_ptr, W_ptr, t_ptr, loss_ptr, lse_ptr,
+                              int(want_grads), dX_ptr, dW_ptr, int(accumulate_dW), ws_ptr,
+                              int(ws_bytes), stream_handle)
+
+
+def raw_backward(shape, X_ptr, W_ptr, t_ptr, lse_ptr, g_ptr, dX_ptr, dW_ptr, accumulate_dW,
+                 grads_precomputed, ws_ptr, ws_bytes, stream_handle) -> int:
+    return lib().flce_backward(ctypes.byref(shape), X_ptr, W_ptr, t_ptr, lse_ptr, g_ptr, dX_ptr,
+                               dW_ptr, int(accumulate_dW), int(grads_precomputed), ws_ptr,
+                               int(ws_bytes), stream_handle)
+
+
+def read_status(workspace, stream=None) -> tuple[int, int]:
+    """(device status bits, rows in the loss) of the last call that used ``workspace``."""
+    st = ctypes.c_uint32(0)
+    nv = ctypes.c_int64(0)
+    rc = lib().flce_read_status(_ptr(workspace), ctypes.byref(st), ctypes.byref(nv),
+                                _stream(stream))
+    if rc != FLCE_OK:
+        raise FlceError(rc, "flce_read_status")
+    return int(st.value), int(nv.value)
+
+
+def instrument(enable: bool) -> None:
+    """Start (reset) or stop per-launch event timing of the contraction kernels."""
+    lib().flce_instrument(1 if enable else 0)
+
+
+def instrument_read() -> dict:
+    """Totals since the last ``instrument(True)``: launches and per-kind time / FLOPs."""
+    st = flce_kernel_stats()
+    rc = lib().flce_instrument_read(ctypes.byref(st))
+    if rc != FLCE_OK:
+        raise FlceError(rc, "flce_instrument_read")
+    kinds = {}
+    for k, name in enumerate(GEMM_KINDS):
+        kinds[name] = dict(launches=int(st.gemm_launches[k]), ms=float(st.gemm_ms[k]),
+                           flop=float(st.gemm_flop[k]))
+    return dict(launches_total=int(st.launches_total), gemm=kinds)
+
+
+def _check(X, W, targets):
+    import torch
+    if not (X.is_cuda and W.is_cuda and targets.is_cuda):
+        raise ValueError("X, W and targets must be CUDA tensors")
+    if X.dtype != torch.bfloat16 or W.dtype != torch.bfloat16:
+        raise TypeError("X and W must be bfloat16")
+    if targets.dtype != torch.int64:
+        raise TypeError("targets must be int64")
+    if X.dim() != 2 or W.dim() != 2 or targets.dim() != 1:
+        raise ValueError("expected X [N, d], W [Vpad, d], targets [N]")
+    if X.shape[1] != W.shape[1] or X.shape[0] != targets.shape[0]:
+        raise ValueError(f"shape mismatch: X {tuple(X.shape)}, W {tuple(W.shape)}, "
+                         f"targets {tuple(targets.shape)}")
+    for name, t in (("X", X), ("W", W), ("targets", targets)):
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+
+
+def alloc_workspace(shape: flce_shape, want_grads: bool, device):
+    import torch
+    nbytes = workspace_bytes(shape, want_grads)
+    if nbytes == 0:
+        raise FlceError(-1, "flce_workspace_bytes")
+    return torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+
+def forward(X, W, targets, Vreal: int, cap: float = 15.0, ignore_index: int = -1,
+            want_grads: bool = False, dX=None, dW=None, accumulate_dW: bool = False,
+            workspace=None, chunk_rows: int = 0, stream=None):
+    """Fused forward.  Returns ``(loss [] fp32, lse [N] fp32, dX, dW, workspace)``;
+    dX/dW are None unless ``want_grads``."""
+    import torch
+    _check(X, W, targets)
+    N, d = X.shape
+    shape = make_shape(N, d, W.shape[0], Vreal, cap, ignore_index, chunk_rows)
+    dev = X.device
+    loss = torch.empty((), dtype=torch.float32, device=dev)
+    lse = torch.empty(max(N, 1), dtype=torch.float32, device=dev)[:N]
+    if want_grads:
+        if dX is None:
+            dX = torch.empty_like(X)
+        if dW is None:
+            dW = torch.empty(W.shape, dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = alloc_workspace(shape, want_grads, dev)
+    rc = raw_forward(shape, _ptr(X), _ptr(W), _ptr(targets), _ptr(loss), _ptr(lse),
+                     want_grads, _ptr(dX) if want_grads else None,
+                     _ptr(dW) if want_grads else None, accumulate_dW, _ptr(workspace),
+                     workspace.numel(), _stream(stream))
+    if rc != FLCE_OK:
+        raise FlceError(rc, "flce_forward")
+    return loss, lse, (dX if want_grads else None), (dW if want_grads else None), workspace
+
+
+def backward(X, W, targets, lse, Vreal: int, cap: float = 15.0, ignore_index: int = -1,
+             grad_out=None, dX=None, dW=None, accumulate_dW: bool = False,
+             grads_precomputed: bool = False, workspace=None, chunk_rows: int = 0, stream=None):
+    """Backward.  Returns ``(dX bf16 [N, d], dW fp32 [Vpad, d])``."""
+    import torch
+    _check(X, W, targets)
+    N, d = X.shape
+    shape = make_shape(N, d, W.shape[0], Vreal, cap, ignore_index, chunk_rows)
+    dev = X.device
+    if dX is None:
+        dX = torch.empty_like(X)
+    if dW is None:
+        dW = torch.empty(W.shape, dtype=torch.float32, device=dev)
+    if grad_out is not None and (grad_out.dtype != torch.float32 or not grad_out.is_cuda):
+        raise TypeError("grad_out must be a float32 CUDA scalar")
+    if workspace is None and not grads_precomputed:
+        workspace = alloc_workspace(shape, True, dev)
+    rc = raw_backward(shape, _ptr(X), _ptr(W), _ptr(targets), _ptr(lse), _ptr(grad_out),
+                      _ptr(dX), _ptr(dW), accumulate_dW, grads_precomputed, _ptr(workspace),
+                      0 if workspace is None else workspace.numel(), _stream(stream))
+    if rc != FLCE_OK:
+        raise FlceError(rc, "flce_backward")
+    return dX, dW

@@ -1,0 +1,572 @@
+// C ABI of the fused LM-head linear + softcapped cross-entropy (include/flce.h):
+// argument validation, workspace layout, tensor maps and the launch sequence.
+//
+// Launch sequence of one fused forward + backward (flce_forward with want_grads = 1):
+//   prep_targets                                  targets -> effective ids, Nv, status
+//   for each chunk of Nc rows:
+//     logits GEMM   z = X_c W^T  (tcgen05, fused softcap / sum-exp / target / A' epilogue)
+//     row_finish    lse, per-row loss, r = 1/(Nv S), target patch of A', Xs = r . X_c
+//     dX GEMM       dX_c = r . (A' W)              (A' K-major, W MN-major)
+//     dW GEMM       dW (+)= A'^T Xs                (both MN-major)
+//   loss          deterministic mean over rows in the loss
+// The logits of a chunk exist only as the bf16 operand A' [Nc, Vpad]; nothing of size N x Vpad
+// is ever allocated.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "../../include/flce.h"
+#include "gemm.cuh"
+#include "rowwise.cuh"
+
+using namespace flce;
+
+namespace {
+
+using CfgLogits = GemmCfg<192, 5, Major::K, Major::K, 8>;
+using CfgDx = GemmCfg<256, 4, Major::K, Major::MN, 8>;
+using CfgDw = GemmCfg<256, 4, Major::MN, Major::MN, 8>;
+
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s bound on every in-kernel wait
+constexpr float kFixedRefMaxCap = 32.f;           // exp(s - cap) >= e^{-64}: no underflow in fp32
+constexpr int64_t kAutoChunkRows = 4096;
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+struct Layout {
+  int64_t chunk;      // rows per pass
+  int n_slabs;        // per-row partial slots of the logits pass
+  bool fixed_ref;
+  size_t hdr, tgt, s_t, der_t, e_t, row_loss, partial, r, A, Xs, total;
+};
+
+bool shape_ok(const flce_shape* s) {
+  if (s == nullptr) return false;
+  if (s->N < 0 || s->d <= 0 || s->Vpad <= 0 || s->Vreal <= 0 || s->Vreal > s->Vpad) return false;
+  if (s->chunk_rows < 0) return false;
+  if (!std::isfinite(s->cap)) return false;
+  // 32-bit tile and row indices inside the kernels
+  if (s->N > (int64_t(1) << 31) - 1 || s->d > (int64_t(1) << 24) || s->Vpad > (int64_t(1) << 28))
+    return false;
+  return true;
+}
+
+Layout make_layout(const flce_shape* s, int want_grads) {
+  Layout L{};
+  const int64_t N = s->N;
+  int64_t nc = s->chunk_rows > 0 ? s->chunk_rows : kAutoChunkRows;
+  if (nc > N) nc = N;
+  if (nc < 1) nc = 1;
+  L.chunk = nc;
+  L.fixed_ref = s->cap > 0.f && s->cap <= kFixedRefMaxCap;
+  const int64_t vtiles = (s->Vpad + CfgLogits::BN - 1) / CfgLogits::BN;
+  L.n_slabs = static_cast<int>(vtiles * CfgLogits::COL_SPLIT);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align_up(off + bytes);
+    return at;
+  };
+  const size_t n = static_cast<size_t>(N > 0 ? N : 1);
+  L.hdr = take(sizeof(DevHeader));
+  L.tgt = take(n * sizeof(int));
+  L.s_t = take(n * sizeof(float));
+  L.der_t = take(n * sizeof(float));
+  L.e_t = take(n * sizeof(float));
+  L.row_loss = take(n * sizeof(float));
+  L.partial = take(static_cast<size_t>(nc) * L.n_slabs * 2 * sizeof(float));
+  if (want_grads) {
+    L.r = take(static_cast<size_t>(nc) * sizeof(float));
+    L.A = take(static_cast<size_t>(nc) * s->Vpad * sizeof(__nv_bfloat16));
+    L.Xs = take(static_cast<size_t>(nc) * s->d * sizeof(__nv_bfloat16));
+  }
+  L.total = off;
+  return L;
+}
+
+// ------------------------------------------------------------------------------ device facts
+struct DeviceInfo {
+  bool checked = false;
+  bool ok = false;
+  int sms = 0;
+  bool attrs_set = false;
+};
+std::mutex g_mu;
+DeviceInfo g_dev[64];
+
+int device_info(DeviceInfo** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FLCE_ERR_CUDA;
+  if (dev < 0 || dev >= 64) return FLCE_ERR_DEVICE;
+  std::lock_guard<std::mutex> lock(g_mu);
+  DeviceInfo& di = g_dev[dev];
+  if (!di.checked) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return FLCE_ERR_CUDA;
+    di.ok = (major == 10 && minor == 0);
+    di.sms = sms;
+    di.checked = true;
+  }
+  if (!di.ok) return FLCE_ERR_DEVICE;
+  if (!di.attrs_set) {
+    if (cudaFuncSetAttribute(gemm_kernel<CfgLogits, LogitsEpi>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             CfgLogits::SMEM_BYTES) != cudaSuccess ||
+        cudaFuncSetAttribute(gemm_kernel<CfgDx, DxEpi>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             CfgDx::SMEM_BYTES) != cudaSuccess ||
+        cudaFuncSetAttribute(gemm_kernel<CfgDw, DwEpi>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             CfgDw::SMEM_BYTES) != cudaSuccess)
+      return FLCE_ERR_CUDA;
+    di.attrs_set = true;
+  }
+  *out = &di;
+  return FLCE_OK;
+}
+
+// ------------------------------------------------------------------------------ tensor maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// bf16 matrix [outer][inner] (row-major, row stride `ld` elements), 128-byte swizzled boxes of
+// {64 inner elements, box_outer rows}.  Out-of-range box elements read as zero.
+int make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t ld,
+             uint32_t box_outer) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return FLCE_ERR_CUDA;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {ld * 2};
+  const cuuint32_t box[2] = {64, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FLCE_OK : FLCE_ERR_CUDA;
+}
+
+// ------------------------------------------------------------------------------ instrumentation
+struct TimedLaunch {
+  int kind;
+  double flop;
+  cudaEvent_t start, stop;
+};
+std::atomic<int> g_instr{0};
+std::atomic<long long> g_launches{0};
+std::mutex g_instr_mu;
+std::vector<TimedLaunch> g_timed;      // recorded since the last reset
+std::vector<cudaEvent_t> g_event_pool; // reusable events
+double g_done_ms[3] = {0, 0, 0};
+double g_done_flop[3] = {0, 0, 0};
+long long g_done_n[3] = {0, 0, 0};
+
+void count_launch() {
+  if (g_instr.load(std::memory_order_relaxed)) g_launches.fetch_add(1, std::memory_order_relaxed);
+}
+
+cudaEvent_t pooled_event() {
+  if (!g_event_pool.empty()) {
+    cudaEvent_t e = g_event_pool.back();
+    g_event_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+  return e;
+}
+
+template <class C, class Epi>
+int launch_gemm(const DeviceInfo* di, const CUtensorMap& a, const CUtensorMap& b, int M, int N,
+                int K, int m_fastest, uint32_t* status, const typename Epi::Params& ep,
+                cudaStream_t st, int kind) {
+  const long long tiles = static_cast<long long>((M + C::BM - 1) / C::BM) * ((N + C::BN - 1) / C::BN);
+  if (tiles <= 0) return FLCE_OK;
+  const int grid = static_cast<int>(tiles < di->sms ? tiles : di->sms);
+  GemmArgs args{M, N, K, m_fastest, status, kWaitLimitNs};
+  cudaEvent_t e0 = nullptr, e1 = nullptr;
+  const bool timed = g_instr.load(std::memory_order_relaxed) != 0;
+  if (timed) {
+    std::lock_guard<std::mutex> lock(g_instr_mu);
+    e0 = pooled_event();
+    e1 = pooled_event();
+    if (e0 != nullptr) cudaEventRecord(e0, st);
+  }
+  gemm_kernel<C, Epi><<<grid, C::THREADS, C::SMEM_BYTES, st>>>(a, b, args, ep);
+  const bool ok = cudaGetLastError() == cudaSuccess;
+  count_launch();
+  if (timed && e0 != nullptr && e1 != nullptr) {
+    cudaEventRecord(e1, st);
+    std::lock_guard<std::mutex> lock(g_instr_mu);
+    g_timed.push_back(TimedLaunch{kind, 2.0 * M * N * static_cast<double>(K), e0, e1});
+  }
+  return ok ? FLCE_OK : FLCE_ERR_CUDA;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+#define FLCE_TRY(expr)             \
+  do {                             \
+    const int _rc = (expr);        \
+    if (_rc != FLCE_OK) return _rc; \
+  } while (0)
+
+int launch_ok() {
+  count_launch();
+  return cudaGetLastError() == cudaSuccess ? FLCE_OK : FLCE_ERR_CUDA;
+}
+
+struct Ctx {
+  const flce_shape* s;
+  Layout L;
+  uint8_t* ws;
+  DevHeader* hdr;
+  const DeviceInfo* di;
+  cudaStream_t st;
+  template <class T>
+  T* at(size_t off) const {
+    return reinterpret_cast<T*>(ws + off);
+  }
+};
+
+// One chunk of the gradient path: logits GEMM (mode FUSED or RECOMPUTE), row finish, dX, dW.
+int grad_chunk(const Ctx& c, int64_t row0, int rows, const __nv_bfloat16* X,
+               const __nv_bfloat16* W, const float* lse_in, float* lse_out, const float* grad_out,
+               __nv_bfloat16* dX, float* dW, int accumulate, int mode) {
+  const flce_shape* s = c.s;
+  const int d = static_cast<int>(s->d), Vpad = static_cast<int>(s->Vpad);
+  const __nv_bfloat16* Xc = X + row0 * s->d;
+  __nv_bfloat16* Abuf = c.at<__nv_bfloat16>(c.L.A);
+  __nv_bfloat16* Xs = c.at<__nv_bfloat16>(c.L.Xs);
+  float* r = c.at<float>(c.L.r);
+
+  CUtensorMap mX, mW, mA_k, mW_mn, mA_mn, mXs_mn;
+  FLCE_TRY(make_map(&mX, Xc, d, rows, d, CfgLogits::BM));
+  FLCE_TRY(make_map(&mW, W, d, Vpad, d, CfgLogits::BN));
+  FLCE_TRY(make_map(&mA_k, Abuf, Vpad, rows, Vpad, CfgDx::BM));
+  FLCE_TRY(make_map(&mW_mn, W, d, Vpad, d, 64));
+  FLCE_TRY(make_map(&mA_mn, Abuf, Vpad, rows, Vpad, 64));
+  FLCE_TRY(make_map(&mXs_mn, Xs, d, rows, d, 64));
+
+  LogitsParams lp{};
+  lp.rows = rows;
+  lp.Vreal = static_cast<int>(s->Vreal);
+  lp.Vpad = Vpad;
+  lp.mode = mode;
+  lp.fixed_ref = c.L.fixed_ref ? 1 : 0;
+  lp.cap = s->cap;
+  lp.k_u = s->cap > 0.f ? 2.0f / s->cap * 1.4426950408889634f : 0.f;
+  lp.tgt = c.at<int>(c.L.tgt) + row0;
+  lp.ref = lse_in ? lse_in + row0 : nullptr;
+  lp.partial = c.at<float>(c.L.partial);
+  lp.n_slabs = c.L.n_slabs;
+  lp.s_t = c.at<float>(c.L.s_t) + row0;
+  lp.der_t = c.at<float>(c.L.der_t) + row0;
+  lp.e_t = c.at<float>(c.L.e_t) + row0;
+  lp.A = Abuf;
+  FLCE_TRY((launch_gemm<CfgLogits, LogitsEpi>(c.di, mX, mW, rows, Vpad, d, 1, &c.hdr->status, lp,
+                                               c.st, 0)));
+
+  RowFinishParams rp{};
+  rp.rows = rows;
+  rp.d = d;
+  rp.Vpad = Vpad;
+  rp.n_slabs = c.L.n_slabs;
+  rp.cap = s->cap;
+  rp.fixed_ref = lp.fixed_ref;
+  rp.from_partials = mode == LOGITS_FUSED ? 1 : 0;
+  rp.want_grads = 1;
+  rp.partial = lp.partial;
+  rp.tgt = lp.tgt;
+  rp.s_t = lp.s_t;
+  rp.der_t = lp.der_t;
+  rp.e_t = lp.e_t;
+  rp.lse_in = lse_in ? lse_in + row0 : nullptr;
+  rp.lse_out = lse_out ? lse_out + row0 : nullptr;
+  rp.row_loss = c.at<float>(c.L.row_loss) + row0;
+  rp.hdr = c.hdr;
+  rp.grad_out = grad_out;
+  rp.r = r;
+  rp.A = Abuf;
+  rp.X = Xc;
+  rp.Xs = Xs;
+  row_finish_kernel<<<(rows + 7) / 8, 256, 0, c.st>>>(rp);
+  FLCE_TRY(launch_ok());
+
+  DxParams xp{rows, d, r, dX + row0 * s->d};
+  FLCE_TRY((launch_gemm<CfgDx, DxEpi>(c.di, mA_k, mW_mn, rows, d, Vpad, 0, &c.hdr->status, xp,
+                                       c.st, 1)));
+  DwParams wp{Vpad, d, accumulate, dW};
+  FLCE_TRY((launch_gemm<CfgDw, DwEpi>(c.di, mA_mn, mXs_mn, Vpad, d, rows, 0, &c.hdr->status, wp,
+                                       c.st, 2)));
+  return FLCE_OK;
+}
+
+// Statistics-only pass over all rows: lse and per-row loss terms.
+int stats_pass(const Ctx& c, const __nv_bfloat16* X, const __nv_bfloat16* W, float* lse) {
+  const flce_shape* s = c.s;
+  const int d = static_cast<int>(s->d), Vpad = static_cast<int>(s->Vpad);
+  CUtensorMap mW;
+  FLCE_TRY(make_map(&mW, W, d, Vpad, d, CfgLogits::BN));
+  for (int64_t row0 = 0; row0 < s->N; row0 += c.L.chunk) {
+    const int rows = static_cast<int>(s->N - row0 < c.L.chunk ? s->N - row0 : c.L.chunk);
+    CUtensorMap mX;
+    FLCE_TRY(make_map(&mX, X + row0 * s->d, d, rows, d, CfgLogits::BM));
+    LogitsParams lp{};
+    lp.rows = rows;
+    lp.Vreal = static_cast<int>(s->Vreal);
+    lp.Vpad = Vpad;
+    lp.mode = LOGITS_STATS;
+    lp.fixed_ref = c.L.fixed_ref ? 1 : 0;
+    lp.cap = s->cap;
+    lp.k_u = s->cap > 0.f ? 2.0f / s->cap * 1.4426950408889634f : 0.f;
+    lp.tgt = c.at<int>(c.L.tgt) + row0;
+    lp.partial = c.at<float>(c.L.partial);
+    lp.n_slabs = c.L.n_slabs;
+    lp.s_t = c.at<float>(c.L.s_t) + row0;
+    lp.der_t = c.at<float>(c.L.der_t) + row0;
+    lp.e_t = c.at<float>(c.L.e_t) + row0;
+    FLCE_TRY((launch_gemm<CfgLogits, LogitsEpi>(c.di, mX, mW, rows, Vpad, d, 1, &c.hdr->status,
+                                                 lp, c.st, 0)));
+    RowFinishParams rp{};
+    rp.rows = rows;
+    rp.d = d;
+    rp.Vpad = Vpad;
+    rp.n_slabs = c.L.n_slabs;
+    rp.cap = s->cap;
+    rp.fixed_ref = lp.fixed_ref;
+    rp.from_partials = 1;
+    rp.want_grads = 0;
+    rp.partial = lp.partial;
+    rp.tgt = lp.tgt;
+    rp.s_t = lp.s_t;
+    rp.der_t = lp.der_t;
+    rp.e_t = lp.e_t;
+    rp.lse_out = lse + row0;
+    rp.row_loss = c.at<float>(c.L.row_loss) + row0;
+    rp.hdr = c.hdr;
+    row_finish_kernel<<<(rows + 7) / 8, 256, 0, c.st>>>(rp);
+    FLCE_TRY(launch_ok());
+  }
+  return FLCE_OK;
+}
+
+__global__ void fill_zero_f32_kernel(float* p, long long n) {
+  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
+       i += stride)
+    p[i] = 0.f;
+}
+
+int zero_dW(const Ctx& c, float* dW) {
+  const long long n = c.s->Vpad * c.s->d;
+  fill_zero_f32_kernel<<<4 * c.di->sms, 256, 0, c.st>>>(dW, n);
+  return launch_ok();
+}
+
+int common_checks(const flce_shape* s, const void* X, const void* W, const int64_t* targets,
+                  void* workspace, size_t ws_bytes, int want_grads) {
+  if (!shape_ok(s)) return FLCE_ERR_ARG;
+  if ((s->d % 8) != 0 || (s->Vpad % 8) != 0) return FLCE_ERR_ALIGN;
+  // X and targets may be NULL only when there are no rows.
+  if ((s->N > 0 && (X == nullptr || targets == nullptr)) || W == nullptr || workspace == nullptr)
+    return FLCE_ERR_ARG;
+  if (!aligned16(X) || !aligned16(W) || !aligned16(targets) ||
+      (reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0)
+    return FLCE_ERR_ALIGN;
+  if (ws_bytes < make_layout(s, want_grads).total) return FLCE_ERR_WORKSPACE;
+  return FLCE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t flce_workspace_bytes(const flce_shape* shape, int want_grads) {
+  if (!shape_ok(shape)) return 0;
+  return make_layout(shape, want_grads ? 1 : 0).total;
+}
+
+int flce_forward(const flce_shape* s, const void* X, const void* W, const int64_t* targets,
+                 float* loss, float* lse, int want_grads, void* dX, float* dW, int accumulate_dW,
+                 void* workspace, size_t workspace_bytes, void* stream) {
+  want_grads = want_grads ? 1 : 0;
+  FLCE_TRY(common_checks(s, X, W, targets, workspace, workspace_bytes, want_grads));
+  if (loss == nullptr || lse == nullptr) return FLCE_ERR_ARG;
+  if (!aligned16(loss) || !aligned16(lse)) return FLCE_ERR_ALIGN;
+  if (want_grads) {
+    if ((s->N > 0 && dX == nullptr) || dW == nullptr) return FLCE_ERR_ARG;
+    if (!aligned16(dX) || !aligned16(dW)) return FLCE_ERR_ALIGN;
+  }
+  DeviceInfo* di = nullptr;
+  FLCE_TRY(device_info(&di));
+  Ctx c{s, make_layout(s, want_grads), static_cast<uint8_t*>(workspace), nullptr, di,
+        static_cast<cudaStream_t>(stream)};
+  c.hdr = c.at<DevHeader>(c.L.hdr);
+  const auto* Xb = static_cast<const __nv_bfloat16*>(X);
+  const auto* Wb = static_cast<const __nv_bfloat16*>(W);
+
+  prep_targets_kernel<<<1, 1024, 0, c.st>>>(reinterpret_cast<const long long*>(targets), s->N,
+                                            s->Vreal, s->ignore_index, c.at<int>(c.L.tgt), c.hdr);
+  FLCE_TRY(launch_ok());
+  if (s->N == 0) {
+    zero_loss_kernel<<<1, 1, 0, c.st>>>(loss);
+    FLCE_TRY(launch_ok());
+    if (want_grads && !accumulate_dW) FLCE_TRY(zero_dW(c, dW));
+    return FLCE_OK;
+  }
+  if (want_grads && c.L.fixed_ref) {
+    for (int64_t row0 = 0; row0 < s->N; row0 += c.L.chunk) {
+      const int rows = static_cast<int>(s->N - row0 < c.L.chunk ? s->N - row0 : c.L.chunk);
+      FLCE_TRY(grad_chunk(c, row0, rows, Xb, Wb, nullptr, lse, nullptr,
+                          static_cast<__nv_bfloat16*>(dX), dW,
+                          (row0 > 0 || accumulate_dW) ? 1 : 0, LOGITS_FUSED));
+    }
+  } else {
+    FLCE_TRY(stats_pass(c, Xb, Wb, lse));
+  }
+  loss_kernel<<<1, 1024, 0, c.st>>>(c.at<float>(c.L.row_loss), s->N, c.hdr, loss);
+  FLCE_TRY(launch_ok());
+  if (want_grads && !c.L.fixed_ref) {
+    // Without a fixed exp reference the gradient needs lse first: recompute with it.
+    for (int64_t row0 = 0; row0 < s->N; row0 += c.L.chunk) {
+      const int rows = static_cast<int>(s->N - row0 < c.L.chunk ? s->N - row0 : c.L.chunk);
+      FLCE_TRY(grad_chunk(c, row0, rows, Xb, Wb, lse, nullptr, nullptr,
+                          static_cast<__nv_bfloat16*>(dX), dW,
+                          (row0 > 0 || accumulate_dW) ? 1 : 0, LOGITS_RECOMPUTE));
+    }
+  }
+  return FLCE_OK;
+}
+
+int flce_backward(const flce_shape* s, const void* X, const void* W, const int64_t* targets,
+                  const float* lse, const float* grad_out, void* dX, float* dW, int accumulate_dW,
+                  int grads_precomputed, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!shape_ok(s)) return FLCE_ERR_ARG;
+  if ((s->N > 0 && dX == nullptr) || dW == nullptr) return FLCE_ERR_ARG;
+  if (!aligned16(dX) || !aligned16(dW)) return FLCE_ERR_ALIGN;
+  if (grad_out != nullptr && (reinterpret_cast<uintptr_t>(grad_out) & 3u) != 0)
+    return FLCE_ERR_ALIGN;
+  if (grads_precomputed) {
+    if ((s->d % 8) != 0) return FLCE_ERR_ALIGN;
+    DeviceInfo* di = nullptr;
+    FLCE_TRY(device_info(&di));
+    if (grad_out == nullptr) return FLCE_OK;
+    const long long nX8 = s->N * s->d / 8, nW4 = s->Vpad * s->d / 4;
+    scale_grads_kernel<<<4 * di->sms, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        static_cast<__nv_bfloat16*>(dX), nX8, dW, nW4, grad_out);
+    return launch_ok();
+  }
+  FLCE_TRY(common_checks(s, X, W, targets, workspace, workspace_bytes, 1));
+  if (lse == nullptr) return FLCE_ERR_ARG;
+  if (!aligned16(lse)) return FLCE_ERR_ALIGN;
+  DeviceInfo* di = nullptr;
+  FLCE_TRY(device_info(&di));
+  Ctx c{s, make_layout(s, 1), static_cast<uint8_t*>(workspace), nullptr, di,
+        static_cast<cudaStream_t>(stream)};
+  c.hdr = c.at<DevHeader>(c.L.hdr);
+  prep_targets_kernel<<<1, 1024, 0, c.st>>>(reinterpret_cast<const long long*>(targets), s->N,
+                                            s->Vreal, s->ignore_index, c.at<int>(c.L.tgt), c.hdr);
+  FLCE_TRY(launch_ok());
+  if (s->N == 0) {
+    if (!accumulate_dW) FLCE_TRY(zero_dW(c, dW));
+    return FLCE_OK;
+  }
+  for (int64_t row0 = 0; row0 < s->N; row0 += c.L.chunk) {
+    const int rows = static_cast<int>(s->N - row0 < c.L.chunk ? s->N - row0 : c.L.chunk);
+    FLCE_TRY(grad_chunk(c, row0, rows, static_cast<const __nv_bfloat16*>(X),
+                        static_cast<const __nv_bfloat16*>(W), lse, nullptr, grad_out,
+                        static_cast<__nv_bfloat16*>(dX), dW, (row0 > 0 || accumulate_dW) ? 1 : 0,
+                        LOGITS_RECOMPUTE));
+  }
+  return FLCE_OK;
+}
+
+int flce_read_status(const void* workspace, uint32_t* dev_status_out, int64_t* n_valid_out,
+                     void* stream) {
+  if (workspace == nullptr) return FLCE_ERR_ARG;
+  DevHeader h;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(&h, workspace, sizeof(h), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return FLCE_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return FLCE_ERR_CUDA;
+  if (dev_status_out) *dev_status_out = h.status;
+  if (n_valid_out) *n_valid_out = h.n_valid;
+  return FLCE_OK;
+}
+
+int flce_instrument(int enable) {
+  std::lock_guard<std::mutex> lock(g_instr_mu);
+  if (enable) {
+    for (auto& t : g_timed) {
+      g_event_pool.push_back(t.start);
+      g_event_pool.push_back(t.stop);
+    }
+    g_timed.clear();
+    for (int k = 0; k < 3; ++k) g_done_ms[k] = g_done_flop[k] = 0, g_done_n[k] = 0;
+    g_launches.store(0);
+  }
+  g_instr.store(enable ? 1 : 0);
+  return FLCE_OK;
+}
+
+int flce_instrument_read(flce_kernel_stats* out) {
+  if (out == nullptr) return FLCE_ERR_ARG;
+  std::lock_guard<std::mutex> lock(g_instr_mu);
+  for (auto& t : g_timed) {
+    if (cudaEventSynchronize(t.stop) != cudaSuccess) return FLCE_ERR_CUDA;
+    float ms = 0.f;
+    if (cudaEventElapsedTime(&ms, t.start, t.stop) != cudaSuccess) return FLCE_ERR_CUDA;
+    g_done_ms[t.kind] += ms;
+    g_done_flop[t.kind] += t.flop;
+    g_done_n[t.kind] += 1;
+    g_event_pool.push_back(t.start);
+    g_event_pool.push_back(t.stop);
+  }
+  g_timed.clear();
+  out->launches_total = g_launches.load();
+  for (int k = 0; k < 3; ++k) {
+    out->gemm_launches[k] = g_done_n[k];
+    out->gemm_ms[k] = g_done_ms[k];
+    out->gemm_flop[k] = g_done_flop[k];
+  }
+  return FLCE_OK;
+}
+
+const char* flce_status_string(int status) {
+  switch (status) {
+    case FLCE_OK: return "FLCE_OK";
+    case FLCE_ERR_ARG: return "FLCE_ERR_ARG: invalid argument";
+    case FLCE_ERR_ALIGN: return "FLCE_ERR_ALIGN: pointer or row stride not 16-byte aligned";
+    case FLCE_ERR_WORKSPACE: return "FLCE_ERR_WORKSPACE: workspace too small";
+    case FLCE_ERR_DEVICE: return "FLCE_ERR_DEVICE: device is not compute capability 10.0";
+    case FLCE_ERR_CUDA: return "FLCE_ERR_CUDA: CUDA runtime error";
+    case FLCE_ERR_TIMEOUT: return "FLCE_ERR_TIMEOUT: a device wait ran out";
+    default: return "unknown flce status";
+  }
+}
+
+}  // extern "C"

@@ -1,0 +1,201 @@
+// Row-wise kernels around the tensor-core contractions: target preparation, the
+// cross-slab log-sum-exp merge with the gradient-operand patch, the loss reduction
+// and the upstream-gradient scaling.  All reductions run in a fixed order, so
+// results are bitwise reproducible.
+#pragma once
+#include "sm100.cuh"
+
+namespace flce {
+
+struct DevHeader {
+  uint32_t status;           // DEV_* bits
+  uint32_t pad0;
+  long long n_valid;         // rows whose target enters the loss
+  uint32_t reserved[60];
+};
+static_assert(sizeof(DevHeader) == 256, "header is one 256-byte block");
+
+// One block: effective targets (t, or -1 when ignored or invalid), count of rows in
+// the loss, and the bad-target bit.  Resets the status word for this call.
+__global__ void __launch_bounds__(1024) prep_targets_kernel(const long long* __restrict__ targets,
+                                                            long long N, long long Vreal,
+                                                            long long ignore_index,
+                                                            int* __restrict__ tgt,
+                                                            DevHeader* __restrict__ hdr) {
+  __shared__ int s_count[32];
+  __shared__ int s_bad;
+  if (threadIdx.x == 0) s_bad = 0;
+  __syncthreads();
+  int count = 0, bad = 0;
+  for (long long i = threadIdx.x; i < N; i += blockDim.x) {
+    const long long t = targets[i];
+    const bool ignored = t == ignore_index;
+    const bool in_range = t >= 0 && t < Vreal;
+    const bool ok = in_range && !ignored;
+    count += ok ? 1 : 0;
+    bad |= (!ok && !ignored) ? 1 : 0;
+    tgt[i] = ok ? static_cast<int>(t) : -1;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) count += __shfl_xor_sync(0xffffffffu, count, o);
+  if ((threadIdx.x & 31) == 0) s_count[threadIdx.x >> 5] = count;
+  if (bad) atomicOr(&s_bad, 1);
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    long long total = 0;
+    for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) total += s_count[w];
+    hdr->n_valid = total;
+    hdr->status = s_bad ? DEV_BAD_TARGET : 0u;
+  }
+}
+
+struct RowFinishParams {
+  int rows;                     // rows of this pass
+  int d, Vpad;
+  int n_slabs;
+  float cap;                    // softcap value (the exp reference when fixed_ref)
+  int fixed_ref;                // 1: partials are sum-exp against cap; 0: (max, sum-exp) pairs
+  int from_partials;            // 1: lse from the per-slab partials; 0: lse given (lse_in)
+  int want_grads;               // 1: also r, the target patch of A and Xs = r . X
+  const float* partial;         // [rows][n_slabs] (x2 when cap <= 0)
+  const int* tgt;               // [rows]
+  const float* s_t;             // [rows]
+  const float* der_t;           // [rows]
+  const float* e_t;             // [rows]
+  const float* lse_in;          // [rows] (from_partials == 0)
+  float* lse_out;               // [rows] (from_partials == 1)
+  float* row_loss;              // [rows] lse - s_t for rows in the loss, else 0 (from_partials)
+  const DevHeader* hdr;         // n_valid
+  const float* grad_out;        // device scalar g, or null for g = 1
+  float* r;                     // [rows]
+  __nv_bfloat16* A;             // [rows][Vpad]
+  const __nv_bfloat16* X;       // [rows][d]
+  __nv_bfloat16* Xs;            // [rows][d]
+};
+
+// One warp per row.
+__global__ void __launch_bounds__(256) row_finish_kernel(const RowFinishParams p) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp >= p.rows) return;
+  const int row = warp;
+  float lse, S = 1.f, ref;
+  if (p.from_partials) {
+    if (p.fixed_ref) {
+      const float* pp = p.partial + static_cast<size_t>(row) * p.n_slabs;
+      float acc = 0.f;
+      for (int k = lane; k < p.n_slabs; k += 32) acc += pp[k];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+      S = acc;
+      ref = p.cap;
+      lse = ref + logf(S);
+    } else {
+      const float* pp = p.partial + static_cast<size_t>(row) * p.n_slabs * 2;
+      float m = -INFINITY;
+      for (int k = lane; k < p.n_slabs; k += 32) m = fmaxf(m, pp[2 * k]);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      float l = 0.f;
+      for (int k = lane; k < p.n_slabs; k += 32) {
+        const float mk = pp[2 * k];
+        if (mk != -INFINITY) l += pp[2 * k + 1] * expf(mk - m);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+      lse = m + logf(l);
+      ref = lse;
+      S = 1.f;
+    }
+  } else {
+    lse = p.lse_in[row];
+    ref = p.fixed_ref ? p.cap : lse;
+    S = p.fixed_ref ? expf(lse - ref) : 1.f;
+  }
+  const int t = p.tgt[row];
+  const bool valid = t >= 0;
+  if (lane == 0 && p.from_partials) {
+    p.lse_out[row] = lse;
+    p.row_loss[row] = valid ? lse - p.s_t[row] : 0.f;
+  }
+  if (!p.want_grads) return;
+  const long long nv = p.hdr->n_valid;
+  const float g = p.grad_out ? *p.grad_out : 1.f;
+  const float r = (valid && nv > 0) ? g / (static_cast<float>(nv) * S) : 0.f;
+  if (lane == 0) {
+    p.r[row] = r;
+    if (valid) {
+      const float patched = p.der_t[row] * (p.e_t[row] - S);
+      p.A[static_cast<size_t>(row) * p.Vpad + t] = __float2bfloat16_rn(patched);
+    }
+  }
+  const __nv_bfloat16* xr = p.X + static_cast<size_t>(row) * p.d;
+  __nv_bfloat16* xs = p.Xs + static_cast<size_t>(row) * p.d;
+  for (int k = lane * 8; k < p.d; k += 256) {
+    const uint4 raw = *reinterpret_cast<const uint4*>(xr + k);
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
+    uint4 w;
+    uint32_t* wo = reinterpret_cast<uint32_t*>(&w);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float2 f = __bfloat1622float2(h[q]);
+      wo[q] = pack_bf16x2(f.x * r, f.y * r);
+    }
+    *reinterpret_cast<uint4*>(xs + k) = w;
+  }
+}
+
+// One block: loss = sum(row_loss) / n_valid, 0 when no row is in the loss.
+__global__ void __launch_bounds__(1024) loss_kernel(const float* __restrict__ row_loss, long long N,
+                                                    const DevHeader* __restrict__ hdr,
+                                                    float* __restrict__ loss) {
+  __shared__ double s_part[1024];
+  double acc = 0.0;
+  for (long long i = threadIdx.x; i < N; i += blockDim.x) acc += static_cast<double>(row_loss[i]);
+  s_part[threadIdx.x] = acc;
+  __syncthreads();
+  for (int w = blockDim.x >> 1; w > 0; w >>= 1) {
+    if (static_cast<int>(threadIdx.x) < w) s_part[threadIdx.x] += s_part[threadIdx.x + w];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    const long long nv = hdr->n_valid;
+    loss[0] = nv > 0 ? static_cast<float>(s_part[0] / static_cast<double>(nv)) : 0.f;
+  }
+}
+
+// dX *= g, dW *= g for gradients formed with g = 1; returns at once when g == 1.
+__global__ void scale_grads_kernel(__nv_bfloat16* __restrict__ dX, long long nX8,
+                                   float* __restrict__ dW, long long nW4,
+                                   const float* __restrict__ grad_out) {
+  const float g = *grad_out;
+  if (g == 1.f) return;
+  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < nX8;
+       i += stride) {
+    uint4 raw = reinterpret_cast<uint4*>(dX)[i];
+    __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&raw);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float2 f = __bfloat1622float2(h[q]);
+      h[q] = __floats2bfloat162_rn(f.x * g, f.y * g);
+    }
+    reinterpret_cast<uint4*>(dX)[i] = raw;
+  }
+  if (dW != nullptr) {
+    for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < nW4;
+         i += stride) {
+      float4 v = reinterpret_cast<float4*>(dW)[i];
+      v.x *= g;
+      v.y *= g;
+      v.z *= g;
+      v.w *= g;
+      reinterpret_cast<float4*>(dW)[i] = v;
+    }
+  }
+}
+
+// Writes loss = 0 (used for N = 0, where nothing else runs).
+__global__ void zero_loss_kernel(float* loss) { loss[0] = 0.f; }
+
+}  // namespace flce

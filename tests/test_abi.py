@@ -1,0 +1,111 @@
+"""Host-side checks of the C-ABI library: it loads without a GPU, exports every
+function include/flce.h declares, sizes its scratch without any N x Vpad term, and
+rejects bad arguments on the host before anything is launched."""
+import ctypes
+import os
+import subprocess
+
+import pytest
+
+import lm_head_linear_gemm_b200 as flce
+from lm_head_linear_gemm_b200 import _abi
+from lm_head_linear_gemm_b200 import build as flce_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    flce_build.build(quiet=True)
+    return flce.lib()
+
+
+def test_exports_every_declared_symbol(L):
+    names = flce.declared_functions()
+    assert set(names) == {"flce_workspace_bytes", "flce_forward", "flce_backward",
+                          "flce_read_status", "flce_status_string", "flce_instrument",
+                          "flce_instrument_read"}
+    for n in names:
+        assert hasattr(L, n), n
+    out = subprocess.run(["nm", "-D", "--defined-only", _abi.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    assert set(names) <= exported
+
+
+def test_library_is_built_for_sm100a():
+    flags = flce_build.nvcc_flags()
+    assert "arch=compute_100a,code=sm_100a" in flags
+
+
+def test_status_strings(L):
+    assert flce.status_string(0) == "FLCE_OK"
+    for code in (-1, -2, -3, -4, -5, -6):
+        assert flce.status_string(code).startswith("FLCE_ERR")
+
+
+def test_workspace_has_no_tokens_by_vocab_term(L):
+    s = flce.make_shape(16384, 3072, 50304, 50257, 15.0, -1, 0)
+    fwd = flce.workspace_bytes(s, False)
+    grads = flce.workspace_bytes(s, True)
+    logits_bytes = 16384 * 50304 * 2                     # one bf16 N x Vpad buffer
+    W_bytes = 50304 * 3072 * 2
+    assert 0 < fwd < grads < logits_bytes / 3
+    assert grads < 2 * W_bytes                            # O(Vpad * chunk) with chunk <= 4096
+    # doubling N grows the scratch only by O(N) per-row words, not by Vpad per row
+    s2 = flce.make_shape(32768, 3072, 50304, 50257, 15.0, -1, 0)
+    assert flce.workspace_bytes(s2, True) - grads < 32 * 16384
+    # the chunk bounds the gradient operand
+    s3 = flce.make_shape(16384, 3072, 50304, 50257, 15.0, -1, 1024)
+    assert flce.workspace_bytes(s3, True) < grads / 3
+
+
+def test_invalid_shapes_give_zero_workspace(L):
+    for bad in [dict(N=-1), dict(d=0), dict(Vreal=60000), dict(Vreal=0), dict(chunk_rows=-4)]:
+        kw = dict(N=8, d=64, Vpad=128, Vreal=100, cap=15.0, ignore_index=-1, chunk_rows=0)
+        kw.update(bad)
+        s = flce.make_shape(**kw)
+        assert flce.workspace_bytes(s, True) == 0, bad
+
+
+def test_host_rejects_bad_arguments_before_launch(L):
+    """These return before any CUDA call, so they run without a GPU."""
+    s = flce.make_shape(8, 64, 128, 100)
+    ws = flce.workspace_bytes(s, True)
+    good = 0x10000000  # never dereferenced: every call below fails validation first
+    args = dict(X=good, W=good, t=good, loss=good, lse=good, dX=good, dW=good, ws=good)
+
+    def fwd(**over):
+        a = dict(args)
+        a.update(over)
+        return flce.raw_forward(s, a["X"], a["W"], a["t"], a["loss"], a["lse"], 1, a["dX"],
+                                a["dW"], 0, a["ws"], over.get("ws_bytes", ws), None)
+
+    assert fwd(X=None) == -1
+    assert fwd(t=None) == -1
+    assert fwd(loss=None) == -1
+    assert fwd(dW=None) == -1
+    assert fwd(X=good + 2) == -2
+    assert fwd(ws=good + 16) == -2                 # workspace must be 256-byte aligned
+    assert fwd(ws_bytes=ws - 1) == -3
+    bad_d = flce.make_shape(8, 60, 128, 100)
+    assert flce.raw_forward(bad_d, good, good, good, good, good, 0, None, None, 0, good, 1 << 30,
+                            None) == -2
+    assert flce.raw_backward(s, good, good, good, None, None, good, good, 0, 0, good, ws,
+                             None) == -1       # lse missing on the recompute path
+    assert flce.raw_backward(s, good, good, good, good, None, None, good, 0, 0, good, ws,
+                             None) == -1
+
+
+def test_instrumentation_counters_without_gpu(L):
+    flce.instrument(True)
+    st = flce.instrument_read()
+    flce.instrument(False)
+    assert st["launches_total"] == 0
+    assert all(v["launches"] == 0 and v["ms"] == 0 for v in st["gemm"].values())
+
+
+def test_shape_struct_matches_header():
+    # int64 N, d, Vpad, Vreal; float cap (+4 padding); int64 ignore_index, chunk_rows
+    assert ctypes.sizeof(_abi.flce_shape) == 56
+    assert _abi.flce_shape.cap.offset == 32 and _abi.flce_shape.ignore_index.offset == 40

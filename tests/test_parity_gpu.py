@@ -1,0 +1,274 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on the same
+seeded inputs.
+
+Tolerances (fp32 accumulation of bf16 products, bf16 dX and gradient operand):
+  |loss_gpu - loss_ref| <= 2e-3, max |lse_gpu - lse_ref| <= 2e-3,
+  relL2(dX) <= 1e-2, relL2(dW) <= 1e-2,
+plus a per-element guard (max error <= 5% of the tensor's max magnitude) so that a
+single wrong tile cannot hide inside the L2 norm.  Small cases compare every element;
+the full-size workloads, run in the launch configuration bench.py times, compare
+sampled rows that the oracle computes one by one.
+"""
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+
+pytestmark = pytest.mark.gpu
+
+LOSS_TOL = 2e-3
+LSE_TOL = 2e-3
+REL_L2 = 1e-2
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def to_dev(a_u16_or_i64):
+    torch = _torch()
+    a = np.ascontiguousarray(a_u16_or_i64)
+    if a.dtype == np.uint16:
+        return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).cuda()
+    return torch.from_numpy(a).cuda()
+
+
+def rel_l2(got, ref):
+    den = np.linalg.norm(ref)
+    return np.linalg.norm(got - ref) / (den if den > 0 else 1.0)
+
+
+def check_tensor(name, got, ref, tol=REL_L2):
+    got = np.asarray(got, np.float64)
+    ref = np.asarray(ref, np.float64)
+    assert got.shape == ref.shape, name
+    assert np.all(np.isfinite(got)), f"{name}: non-finite values"
+    r = rel_l2(got, ref)
+    assert r <= tol, f"{name}: relL2 {r:.3e} > {tol}"
+    scale = np.abs(ref).max()
+    if scale > 0:
+        worst = np.abs(got - ref).max()
+        assert worst <= 0.05 * scale, f"{name}: max err {worst:.3e} vs max |ref| {scale:.3e}"
+    return r
+
+
+def run_gpu(inp, *, want_grads=True, chunk_rows=0, cap=None, recompute=False, g=None):
+    import lm_head_linear_gemm_b200 as flce
+    torch = _torch()
+    c = inp["cfg"]
+    cap = c.cap if cap is None else cap
+    X, W, t = to_dev(inp["X"]), to_dev(inp["W"]), to_dev(inp["targets"])
+    if recompute:
+        loss, lse, _, _, ws = flce.forward(X, W, t, c.Vreal, cap, c.ignore_index, False,
+                                           chunk_rows=chunk_rows)
+        gt = None if g is None else torch.tensor(g, dtype=torch.float32, device="cuda")
+        dX, dW = flce.backward(X, W, t, lse, c.Vreal, cap, c.ignore_index, grad_out=gt,
+                               chunk_rows=chunk_rows)
+    else:
+        loss, lse, dX, dW, ws = flce.forward(X, W, t, c.Vreal, cap, c.ignore_index, want_grads,
+                                             chunk_rows=chunk_rows)
+    torch.cuda.synchronize()
+    status, nv = flce.read_status(ws)
+    out = dict(loss=float(loss.item()), lse=lse.double().cpu().numpy(), status=status, n_valid=nv)
+    if dX is not None:
+        out["dX"] = dX.double().cpu().numpy()
+        out["dW"] = dW.double().cpu().numpy()
+    return out
+
+
+def oracle_full(inp, cap=None, g=1.0):
+    c = inp["cfg"]
+    cap = c.cap if cap is None else cap
+    X = synth.bf16_to_f64(inp["X"])
+    W = synth.bf16_to_f64(inp["W"])
+    return oracle.forward_backward(X, W, inp["targets"], c.Vreal, cap, c.ignore_index, g)
+
+
+def compare_full(got, ref, grads=True):
+    assert abs(got["loss"] - ref["loss"]) <= LOSS_TOL, (got["loss"], ref["loss"])
+    err = np.abs(got["lse"] - ref["lse"]).max() if len(ref["lse"]) else 0.0
+    assert err <= LSE_TOL, f"lse max err {err:.3e}"
+    assert got["n_valid"] == ref["n_valid"]
+    if grads:
+        check_tensor("dX", got["dX"], ref["dX"])
+        check_tensor("dW", got["dW"], ref["dW"])
+
+
+# ----------------------------------------------------------------------------- small, every element
+def test_tiny_fused_and_recompute(cuda_device):
+    inp = synth.make_inputs("tiny")
+    ref = oracle_full(inp)
+    got = run_gpu(inp)
+    compare_full(got, ref)
+    assert got["status"] == 0
+    rec = run_gpu(inp, recompute=True)
+    compare_full(rec, ref)
+    c = inp["cfg"]
+    assert np.abs(got["dW"][c.Vreal:]).max() == 0.0          # padded vocabulary rows
+
+
+RAGGED = synth.custom_config("ragged", N=300, d=200, Vreal=1500, Vpad=1544, x_dist="normal",
+                             w_std=0.05, target_dist="uniform", ignore_count=7)
+
+
+@pytest.mark.parametrize("chunk_rows", [0, 128, 100])
+def test_ragged_multi_tile(cuda_device, chunk_rows):
+    """300 rows (3 row tiles, ragged), d = 200 (K tail), Vpad = 1544 (ragged vocabulary
+    tile), chunks of 128 / 100 rows (ragged last chunk)."""
+    inp = synth.make_inputs(RAGGED)
+    ref = oracle_full(inp)
+    compare_full(run_gpu(inp, chunk_rows=chunk_rows), ref)
+    compare_full(run_gpu(inp, chunk_rows=chunk_rows, recompute=True), ref)
+
+
+@pytest.mark.parametrize("cap,w_std", [(0.0, 0.05), (2.0, 0.3), (50.0, 0.3), (15.0, 1.0)])
+def test_softcap_variants(cuda_device, cap, w_std):
+    """No softcap (online max path), a small cap (deep saturation), a large cap (softcap
+    with the lse reference) and cap 15 with wide logits (|z| well beyond cap)."""
+    c = synth.custom_config("cap", N=256, d=128, Vreal=900, Vpad=1024, x_dist="normal",
+                            w_std=w_std, target_dist="uniform", ignore_count=3, cap=cap)
+    inp = synth.make_inputs(c)
+    ref = oracle_full(inp, cap=cap)
+    compare_full(run_gpu(inp, cap=cap, chunk_rows=128), ref)
+    compare_full(run_gpu(inp, cap=cap, recompute=True), ref)
+
+
+def test_pages_vocabulary_every_element(cuda_device):
+    """The pages' vocabulary (50257 -> 50304) and the small model's d = 1536, 512 rows."""
+    inp = synth.make_inputs("small", N=512)
+    ref = oracle_full(inp)
+    got = run_gpu(inp)
+    compare_full(got, ref)
+    assert np.abs(got["dW"][50257:]).max() == 0.0
+    compare_full(run_gpu(inp, recompute=True, chunk_rows=256), ref)
+
+
+def test_bad_targets_are_ignored_and_flagged(cuda_device):
+    inp = synth.make_inputs(RAGGED)
+    t = inp["targets"].copy()
+    t[5] = 1500          # a padded id: not a real token
+    t[17] = 1_000_000
+    t[40] = -3
+    inp = dict(inp, targets=t)
+    ref = oracle_full(inp)
+    got = run_gpu(inp)
+    assert got["status"] & 1
+    compare_full(got, ref)
+    assert np.abs(got["dX"][[5, 17, 40]]).max() == 0.0
+
+
+def test_edge_cases(cuda_device):
+    import lm_head_linear_gemm_b200 as flce
+    torch = _torch()
+    # one row
+    inp = synth.make_inputs(synth.custom_config("one", 1, 64, 100, 128, w_std=0.1))
+    compare_full(run_gpu(inp), oracle_full(inp))
+    # no row in the loss: loss 0, zero gradients
+    inp = synth.make_inputs(RAGGED)
+    inp = dict(inp, targets=np.full(300, -1, np.int64))
+    got = run_gpu(inp)
+    assert got["loss"] == 0.0 and got["n_valid"] == 0
+    assert np.abs(got["dX"]).max() == 0.0 and np.abs(got["dW"]).max() == 0.0
+    # N = 0: loss 0, dW written as zeros (not accumulated)
+    X = torch.zeros((0, 64), dtype=torch.bfloat16, device="cuda")
+    W = torch.randn((128, 64), device="cuda").to(torch.bfloat16)
+    t = torch.zeros((0,), dtype=torch.int64, device="cuda")
+    dW = torch.full((128, 64), 7.0, device="cuda")
+    loss, lse, dX, dW, _ = flce.forward(X, W, t, 100, 15.0, -1, True, dW=dW)
+    torch.cuda.synchronize()
+    assert loss.item() == 0.0 and lse.numel() == 0 and float(dW.abs().max()) == 0.0
+
+
+def test_accumulate_and_upstream_gradient(cuda_device):
+    import lm_head_linear_gemm_b200 as flce
+    torch = _torch()
+    inp = synth.make_inputs(RAGGED)
+    c = inp["cfg"]
+    ref = oracle_full(inp)
+    X, W, t = to_dev(inp["X"]), to_dev(inp["W"]), to_dev(inp["targets"])
+    R = torch.randn(W.shape, device="cuda", generator=torch.Generator("cuda").manual_seed(3))
+    # fused forward accumulating onto R (gradient accumulation over micro-batches)
+    _, _, _, dW, _ = flce.forward(X, W, t, c.Vreal, c.cap, -1, True, dW=R.clone(),
+                                  accumulate_dW=True, chunk_rows=128)
+    check_tensor("dW accumulated", (dW - R).double().cpu().numpy(), ref["dW"])
+    # precomputed gradients scaled in place by g = 0.5
+    _, _, dX, dW, _ = flce.forward(X, W, t, c.Vreal, c.cap, -1, True)
+    flce.backward(X, W, t, None, c.Vreal, c.cap, -1, grad_out=torch.tensor(0.5, device="cuda"),
+                  dX=dX, dW=dW, grads_precomputed=True)
+    check_tensor("dX*g", dX.double().cpu().numpy(), 0.5 * ref["dX"])
+    check_tensor("dW*g", dW.double().cpu().numpy(), 0.5 * ref["dW"])
+    # recomputing backward with g = 2 accumulated onto R
+    loss, lse, _, _, _ = flce.forward(X, W, t, c.Vreal, c.cap, -1, False)
+    dX3, dW3 = flce.backward(X, W, t, lse, c.Vreal, c.cap, -1,
+                             grad_out=torch.tensor(2.0, device="cuda"), dW=R.clone(),
+                             accumulate_dW=True, chunk_rows=128)
+    check_tensor("dX g=2", dX3.double().cpu().numpy(), 2 * ref["dX"])
+    check_tensor("dW g=2 acc", (dW3 - R).double().cpu().numpy(), 2 * ref["dW"])
+
+
+def test_deterministic(cuda_device):
+    inp = synth.make_inputs("small", N=640)
+    a = run_gpu(inp, chunk_rows=256)
+    b = run_gpu(inp, chunk_rows=256)
+    assert a["loss"] == b["loss"]
+    for k in ("lse", "dX", "dW"):
+        assert np.array_equal(a[k], b[k]), k
+
+
+def test_autograd_drop_in(cuda_device):
+    import lm_head_linear_gemm_b200 as flce
+    torch = _torch()
+    inp = synth.make_inputs(RAGGED)
+    c = inp["cfg"]
+    ref = oracle_full(inp, g=3.0)
+    X = to_dev(inp["X"]).requires_grad_(True)
+    W = to_dev(inp["W"]).requires_grad_(True)
+    t = to_dev(inp["targets"])
+    loss = flce.fused_linear_cross_entropy(X, W, t, c.Vreal, c.cap, -1)
+    (3.0 * loss).backward()
+    assert abs(loss.item() - ref["loss"]) <= LOSS_TOL
+    check_tensor("X.grad", X.grad.double().cpu().numpy(), ref["dX"])
+    check_tensor("W.grad", W.grad.double().cpu().numpy(), ref["dW"])
+
+
+# ----------------------------------------------------------------------------- full size, sampled
+def _sampled_full_size(name, samples=48, seed=0):
+    """The named workload at full size, default chunking (the bench's launch configuration).
+    lse and dX are compared on sampled rows; dW on sampled vocabulary rows (random ones, all
+    47 padded rows and the most frequent targets) using the oracle's lse of every row."""
+    inp = synth.make_inputs(name)
+    c = inp["cfg"]
+    got = run_gpu(inp)
+    assert got["status"] == 0
+    X = synth.bf16_to_f64(inp["X"])
+    W = synth.bf16_to_f64(inp["W"])
+    t = inp["targets"]
+    f = oracle.forward(X, W, t, c.Vreal, c.cap, c.ignore_index, block_rows=2048)
+    assert abs(got["loss"] - f["loss"]) <= LOSS_TOL, (got["loss"], f["loss"])
+    assert np.abs(got["lse"] - f["lse"]).max() <= LSE_TOL
+    rng = np.random.default_rng(seed)
+    rows = np.sort(rng.choice(c.N, samples, replace=False))
+    dz = oracle.row_dlogits(X[rows], W, t[rows], f["lse"][rows], c.Vreal, c.cap, c.ignore_index,
+                            f["n_valid"])
+    check_tensor("dX rows", got["dX"][rows], dz @ W)
+    counts = np.bincount(t[t >= 0], minlength=c.Vreal)
+    frequent = np.argsort(-counts)[:16]
+    vrows = np.unique(np.concatenate([rng.choice(c.Vreal, samples, replace=False), frequent,
+                                      np.arange(c.Vreal, c.Vpad)]))
+    ref_dW = oracle.dW_rows(X, W, t, f["lse"], vrows, c.Vreal, c.cap, c.ignore_index)
+    check_tensor("dW rows", got["dW"][vrows], ref_dW)
+    assert np.abs(got["dW"][c.Vreal:]).max() == 0.0
+    return got, f
+
+
+def test_full_size_small_model(cuda_device):
+    _sampled_full_size("small")
+
+
+def test_full_size_headline(cuda_device):
+    got, f = _sampled_full_size("3.8b")
+    assert math.isfinite(got["loss"])
