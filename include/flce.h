@@ -86,7 +86,7 @@ size_t flce_workspace_bytes(const flce_shape* shape, int want_grads);
  * gradient g = 1) in the same pass over the logits: dX [N, d] bf16 is written, and dW [Vpad, d]
  * fp32 is written (accumulate_dW = 0) or added to (accumulate_dW = 1, gradient accumulation over
  * micro-batches as in the pages' 7-step accumulation).  With want_grads = 0, dX and dW may be
- * NULL and are not touched.
+ * NULL and are not touched.  When N = 0, X, targets, lse and dX may be NULL.
  * workspace: device scratch of at least flce_workspace_bytes(shape, want_grads) bytes,
  * 256-byte aligned; its contents on entry are ignored.
  */

@@ -415,7 +415,7 @@ int flce_forward(const flce_shape* s, const void* X, const void* W, const int64_
                  void* workspace, size_t workspace_bytes, void* stream) {
   want_grads = want_grads ? 1 : 0;
   FLCE_TRY(common_checks(s, X, W, targets, workspace, workspace_bytes, want_grads));
-  if (loss == nullptr || lse == nullptr) return FLCE_ERR_ARG;
+  if (loss == nullptr || (s->N > 0 && lse == nullptr)) return FLCE_ERR_ARG;
   if (!aligned16(loss) || !aligned16(lse)) return FLCE_ERR_ALIGN;
   if (want_grads) {
     if ((s->N > 0 && dX == nullptr) || dW == nullptr) return FLCE_ERR_ARG;
@@ -481,7 +481,7 @@ int flce_backward(const flce_shape* s, const void* X, const void* W, const int64
     return launch_ok();
   }
   FLCE_TRY(common_checks(s, X, W, targets, workspace, workspace_bytes, 1));
-  if (lse == nullptr) return FLCE_ERR_ARG;
+  if (s->N > 0 && lse == nullptr) return FLCE_ERR_ARG;
   if (!aligned16(lse)) return FLCE_ERR_ALIGN;
   DeviceInfo* di = nullptr;
   FLCE_TRY(device_info(&di));
