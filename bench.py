@@ -42,6 +42,8 @@ def parse_args():
     ap.add_argument("--impl", choices=["flce", "reference"], default="flce")
     ap.add_argument("--config", default="3.8b")
     ap.add_argument("--chunk-rows", type=int, default=0)
+    ap.add_argument("--rows", type=int, default=0,
+                    help="override the token count N (small profiling cases)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-unfused", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -231,7 +233,7 @@ def main_gpu(args):
             dist.barrier()
 
     cfg = synth.CONFIGS[args.config]
-    inp = synth.make_inputs(cfg, seed=cfg.seed + rank)
+    inp = synth.make_inputs(cfg, seed=cfg.seed + rank, N=args.rows or None)
     c = inp["cfg"]
     N, d, Vp, Vr = c.N, c.d, c.Vpad, c.Vreal
 
