@@ -110,6 +110,30 @@ int flce_backward(const flce_shape* shape, const void* X, const void* W, const i
                   int grads_precomputed, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Forward without any caller-provided scratch: loss[0] and lse[N] exactly as flce_forward with
+ * want_grads = 0, but the scratch lives in a device array of FLCE_NOALLOC_SCRATCH_BYTES inside the
+ * library, so the call allocates nothing and needs no workspace.  It is meant for callers that
+ * cannot obtain device memory at call time: a plugin whose host framework owns every device
+ * allocation and hands it no allocator, or a latency-critical caller that must not risk the
+ * implicit device synchronisation of cudaMalloc.  The write-ups describe no such entry point.
+ *   - The array is a file-scope __device__ object: every GPU that loads the library holds it
+ *     until the process exits.
+ *   - The first call on each device looks up the array's device address with that device
+ *     current (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   - Shapes whose scratch exceeds the array are rejected with FLCE_ERR_WORKSPACE before
+ *     anything runs (chunk_rows = 0 picks the largest chunk of 4096, 2048, ..., 128 rows that
+ *     fits; at d = 3072, Vpad = 50304 that admits N up to several hundred thousand rows).
+ *   - All calls share the array and it keeps the last call's contents (nothing in it needs to
+ *     start at zero).  Calls that overlap on the GPU (different streams, or different host
+ *     threads without ordering) race on it and must not be issued.
+ *   - The status word of the call stays inside the array and is not reported.
+ * Same argument rules as flce_forward otherwise.
+ */
+#define FLCE_NOALLOC_SCRATCH_BYTES (16u << 20)
+int flce_forward_noalloc(const flce_shape* shape, const void* X, const void* W,
+                         const int64_t* targets, float* loss, float* lse, void* stream);
+
+/*
  * Reads the device status word (FLCE_DEV_* bits) and the number of rows in the loss from the
  * workspace of the last call on `stream`.  Synchronises that stream.  Either output may be
  * NULL.

@@ -7,12 +7,12 @@ fallback implementation.
 """
 from ._abi import (DEV_BAD_TARGET, DEV_TIMEOUT, FlceError, alloc_workspace, backward,
                    declared_functions, forward, instrument, instrument_read, lib, make_shape, raw_backward, raw_forward,
-                   read_status, status_string, workspace_bytes)
+                   raw_forward_noalloc, read_status, status_string, workspace_bytes)
 from .autograd import FusedLinearCrossEntropy, fused_linear_cross_entropy
 
 __all__ = [
     "DEV_BAD_TARGET", "DEV_TIMEOUT", "FlceError", "alloc_workspace", "backward",
     "declared_functions", "forward", "instrument", "instrument_read", "lib", "make_shape", "raw_backward", "raw_forward",
-    "read_status", "status_string", "workspace_bytes", "FusedLinearCrossEntropy",
+    "raw_forward_noalloc", "read_status", "status_string", "workspace_bytes", "FusedLinearCrossEntropy",
     "fused_linear_cross_entropy",
 ]

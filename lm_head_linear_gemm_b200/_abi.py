@@ -15,6 +15,7 @@ LIB_PATH = os.path.join(HERE, "libflce.so")
 HEADER_PATH = os.path.join(os.path.dirname(HERE), "include", "flce.h")
 
 FLCE_OK = 0
+NOALLOC_SCRATCH_BYTES = 16 << 20      # FLCE_NOALLOC_SCRATCH_BYTES in include/flce.h
 DEV_BAD_TARGET = 1
 DEV_TIMEOUT = 2
 
@@ -80,6 +81,8 @@ def lib() -> ctypes.CDLL:
     L.flce_read_status.argtypes = [P, ctypes.POINTER(ctypes.c_uint32),
                                    ctypes.POINTER(ctypes.c_int64), P]
     L.flce_read_status.restype = ctypes.c_int
+    L.flce_forward_noalloc.argtypes = [shp, P, P, P, P, P, P]
+    L.flce_forward_noalloc.restype = ctypes.c_int
     L.flce_instrument.argtypes = [ctypes.c_int]
     L.flce_instrument.restype = ctypes.c_int
     L.flce_instrument_read.argtypes = [ctypes.POINTER(flce_kernel_stats)]
@@ -124,6 +127,13 @@ def raw_forward(shape, X_ptr, W_ptr, t_ptr, loss_ptr, lse_ptr, want_grads, dX_pt
     return lib().flce_forward(ctypes.byref(shape), X_ptr, W_ptr, t_ptr, loss_ptr, lse_ptr,
                               int(want_grads), dX_ptr, dW_ptr, int(accumulate_dW), ws_ptr,
                               int(ws_bytes), stream_handle)
+
+
+def raw_forward_noalloc(shape, X_ptr, W_ptr, t_ptr, loss_ptr, lse_ptr, stream_handle) -> int:
+    """flce_forward_noalloc: loss and lse with the library's own fixed device scratch (no
+    workspace, nothing allocated); returns the flce_status code."""
+    return lib().flce_forward_noalloc(ctypes.byref(shape), X_ptr, W_ptr, t_ptr, loss_ptr,
+                                      lse_ptr, stream_handle)
 
 
 def raw_backward(shape, X_ptr, W_ptr, t_ptr, lse_ptr, g_ptr, dX_ptr, dW_ptr, accumulate_dW,

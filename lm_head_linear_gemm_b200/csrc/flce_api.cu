@@ -401,6 +401,28 @@ int common_checks(const flce_shape* s, const void* X, const void* W, const int64
   return FLCE_OK;
 }
 
+// ------------------------------------------------------------------------------ no-alloc scratch
+// Scratch of flce_forward_noalloc.  In host code this name is only a stand-in for the device
+// object: its device address comes from cudaGetSymbolAddress, once per device.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[FLCE_NOALLOC_SCRATCH_BYTES];
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[64] = {};
+
+int noalloc_scratch_address(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FLCE_ERR_CUDA;
+  if (dev < 0 || dev >= 64) return FLCE_ERR_DEVICE;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_addr[dev] == nullptr) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || p == nullptr) return FLCE_ERR_CUDA;
+    g_noalloc_addr[dev] = p;
+  }
+  *out = g_noalloc_addr[dev];
+  return FLCE_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -503,6 +525,30 @@ int flce_backward(const flce_shape* s, const void* X, const void* W, const int64
                         LOGITS_RECOMPUTE));
   }
   return FLCE_OK;
+}
+
+int flce_forward_noalloc(const flce_shape* shape, const void* X, const void* W,
+                         const int64_t* targets, float* loss, float* lse, void* stream) {
+  if (!shape_ok(shape)) return FLCE_ERR_ARG;
+  flce_shape s = *shape;
+  if (s.chunk_rows == 0) {
+    s.chunk_rows = 128;
+    for (int64_t c = 4096; c >= 128; c /= 2) {
+      flce_shape t = s;
+      t.chunk_rows = c;
+      if (make_layout(&t, 0).total <= FLCE_NOALLOC_SCRATCH_BYTES) {
+        s.chunk_rows = c;
+        break;
+      }
+    }
+  }
+  if (make_layout(&s, 0).total > FLCE_NOALLOC_SCRATCH_BYTES) return FLCE_ERR_WORKSPACE;
+  DeviceInfo* di = nullptr;
+  FLCE_TRY(device_info(&di));
+  void* scratch = nullptr;
+  FLCE_TRY(noalloc_scratch_address(&scratch));
+  return flce_forward(&s, X, W, targets, loss, lse, 0, nullptr, nullptr, 0, scratch,
+                      FLCE_NOALLOC_SCRATCH_BYTES, stream);
 }
 
 int flce_read_status(const void* workspace, uint32_t* dev_status_out, int64_t* n_valid_out,
