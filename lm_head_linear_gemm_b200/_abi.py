@@ -11,7 +11,7 @@ import os
 import re
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "libflce.so")
+LIB_PATH = os.environ.get("FLCE_LIBRARY") or os.path.join(HERE, "libflce.so")
 HEADER_PATH = os.path.join(os.path.dirname(HERE), "include", "flce.h")
 
 FLCE_OK = 0

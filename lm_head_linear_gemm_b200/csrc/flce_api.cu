@@ -28,9 +28,24 @@ using namespace flce;
 
 namespace {
 
+// Contraction tiles.  Pairs of SMs (cta_group::2, 256 x 256 tiles) by default; the single-SM
+// kernels (128 x 192 / 128 x 256 tiles) remain available with -DFLCE_PAIR=0.
+#ifndef FLCE_PAIR
+#define FLCE_PAIR 1
+#endif
+#if FLCE_PAIR
+using CfgLogits = GemmPairCfg<256, 6, Major::K, Major::K, 8>;
+using CfgDx = GemmPairCfg<256, 6, Major::K, Major::MN, 8>;
+using CfgDw = GemmPairCfg<256, 6, Major::MN, Major::MN, 8>;
+template <class C, class E>
+constexpr auto gemm_entry = gemm_pair_kernel<C, E>;
+#else
 using CfgLogits = GemmCfg<192, 5, Major::K, Major::K, 8>;
 using CfgDx = GemmCfg<256, 4, Major::K, Major::MN, 8>;
 using CfgDw = GemmCfg<256, 4, Major::MN, Major::MN, 8>;
+template <class C, class E>
+constexpr auto gemm_entry = gemm_kernel<C, E>;
+#endif
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s bound on every in-kernel wait
 constexpr float kFixedRefMaxCap = 32.f;           // exp(s - cap) >= e^{-64}: no underflow in fp32
@@ -118,12 +133,12 @@ int device_info(DeviceInfo** out) {
   }
   if (!di.ok) return FLCE_ERR_DEVICE;
   if (!di.attrs_set) {
-    if (cudaFuncSetAttribute(gemm_kernel<CfgLogits, LogitsEpi>,
+    if (cudaFuncSetAttribute(gemm_entry<CfgLogits, LogitsEpi>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                              CfgLogits::SMEM_BYTES) != cudaSuccess ||
-        cudaFuncSetAttribute(gemm_kernel<CfgDx, DxEpi>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaFuncSetAttribute(gemm_entry<CfgDx, DxEpi>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              CfgDx::SMEM_BYTES) != cudaSuccess ||
-        cudaFuncSetAttribute(gemm_kernel<CfgDw, DwEpi>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaFuncSetAttribute(gemm_entry<CfgDw, DwEpi>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              CfgDw::SMEM_BYTES) != cudaSuccess)
       return FLCE_ERR_CUDA;
     di.attrs_set = true;
@@ -205,7 +220,9 @@ int launch_gemm(const DeviceInfo* di, const CUtensorMap& a, const CUtensorMap& b
                 cudaStream_t st, int kind) {
   const long long tiles = static_cast<long long>((M + C::BM - 1) / C::BM) * ((N + C::BN - 1) / C::BN);
   if (tiles <= 0) return FLCE_OK;
-  const int grid = static_cast<int>(tiles < di->sms ? tiles : di->sms);
+  // persistent: one CTA (or CTA pair) per SM (pair of SMs), never more than there are tiles
+  const long long units = C::PAIR ? di->sms / 2 : di->sms;
+  const int grid = static_cast<int>((tiles < units ? tiles : units) * (C::PAIR ? 2 : 1));
   GemmArgs args{M, N, K, m_fastest, status, kWaitLimitNs};
   cudaEvent_t e0 = nullptr, e1 = nullptr;
   const bool timed = g_instr.load(std::memory_order_relaxed) != 0;
@@ -215,7 +232,7 @@ int launch_gemm(const DeviceInfo* di, const CUtensorMap& a, const CUtensorMap& b
     e1 = pooled_event();
     if (e0 != nullptr) cudaEventRecord(e0, st);
   }
-  gemm_kernel<C, Epi><<<grid, C::THREADS, C::SMEM_BYTES, st>>>(a, b, args, ep);
+  gemm_entry<C, Epi><<<grid, C::THREADS, C::SMEM_BYTES, st>>>(a, b, args, ep);
   const bool ok = cudaGetLastError() == cudaSuccess;
   count_launch();
   if (timed && e0 != nullptr && e1 != nullptr) {
@@ -264,9 +281,9 @@ int grad_chunk(const Ctx& c, int64_t row0, int rows, const __nv_bfloat16* X,
   float* r = c.at<float>(c.L.r);
 
   CUtensorMap mX, mW, mA_k, mW_mn, mA_mn, mXs_mn;
-  FLCE_TRY(make_map(&mX, Xc, d, rows, d, CfgLogits::BM));
-  FLCE_TRY(make_map(&mW, W, d, Vpad, d, CfgLogits::BN));
-  FLCE_TRY(make_map(&mA_k, Abuf, Vpad, rows, Vpad, CfgDx::BM));
+  FLCE_TRY(make_map(&mX, Xc, d, rows, d, CfgLogits::BM_CTA));
+  FLCE_TRY(make_map(&mW, W, d, Vpad, d, CfgLogits::BN_CTA));
+  FLCE_TRY(make_map(&mA_k, Abuf, Vpad, rows, Vpad, CfgDx::BM_CTA));
   FLCE_TRY(make_map(&mW_mn, W, d, Vpad, d, 64));
   FLCE_TRY(make_map(&mA_mn, Abuf, Vpad, rows, Vpad, 64));
   FLCE_TRY(make_map(&mXs_mn, Xs, d, rows, d, 64));
@@ -279,6 +296,7 @@ int grad_chunk(const Ctx& c, int64_t row0, int rows, const __nv_bfloat16* X,
   lp.fixed_ref = c.L.fixed_ref ? 1 : 0;
   lp.cap = s->cap;
   lp.k_u = s->cap > 0.f ? 2.0f / s->cap * 1.4426950408889634f : 0.f;
+  lp.m2c_log2e = -2.0f * s->cap * 1.4426950408889634f;
   lp.tgt = c.at<int>(c.L.tgt) + row0;
   lp.ref = lse_in ? lse_in + row0 : nullptr;
   lp.partial = c.at<float>(c.L.partial);
@@ -330,11 +348,11 @@ int stats_pass(const Ctx& c, const __nv_bfloat16* X, const __nv_bfloat16* W, flo
   const flce_shape* s = c.s;
   const int d = static_cast<int>(s->d), Vpad = static_cast<int>(s->Vpad);
   CUtensorMap mW;
-  FLCE_TRY(make_map(&mW, W, d, Vpad, d, CfgLogits::BN));
+  FLCE_TRY(make_map(&mW, W, d, Vpad, d, CfgLogits::BN_CTA));
   for (int64_t row0 = 0; row0 < s->N; row0 += c.L.chunk) {
     const int rows = static_cast<int>(s->N - row0 < c.L.chunk ? s->N - row0 : c.L.chunk);
     CUtensorMap mX;
-    FLCE_TRY(make_map(&mX, X + row0 * s->d, d, rows, d, CfgLogits::BM));
+    FLCE_TRY(make_map(&mX, X + row0 * s->d, d, rows, d, CfgLogits::BM_CTA));
     LogitsParams lp{};
     lp.rows = rows;
     lp.Vreal = static_cast<int>(s->Vreal);
@@ -343,6 +361,7 @@ int stats_pass(const Ctx& c, const __nv_bfloat16* X, const __nv_bfloat16* W, flo
     lp.fixed_ref = c.L.fixed_ref ? 1 : 0;
     lp.cap = s->cap;
     lp.k_u = s->cap > 0.f ? 2.0f / s->cap * 1.4426950408889634f : 0.f;
+    lp.m2c_log2e = -2.0f * s->cap * 1.4426950408889634f;
     lp.tgt = c.at<int>(c.L.tgt) + row0;
     lp.partial = c.at<float>(c.L.partial);
     lp.n_slabs = c.L.n_slabs;

@@ -17,14 +17,21 @@
 #pragma once
 #include "sm100.cuh"
 
+#ifndef FLCE_SOFTCAP_SFU
+#define FLCE_SOFTCAP_SFU 0
+#endif
+
 namespace flce {
 
 enum class Major : int { K = 0, MN = 1 };
 
 template <int BN_, int STAGES_, Major AMAJ_, Major BMAJ_, int EPI_WARPS_>
 struct GemmCfg {
+  static constexpr bool PAIR = false;
   static constexpr int BM = 128;
+  static constexpr int BM_CTA = 128;
   static constexpr int BN = BN_;
+  static constexpr int BN_CTA = BN_;
   static constexpr int BK = 64;  // 64 bf16 = 128 bytes = one swizzle row
   static constexpr int STAGES = STAGES_;
   static constexpr Major AMAJ = AMAJ_;
@@ -258,6 +265,254 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 }
 
 // ==============================================================================================
+// The same GEMM on SM pairs (cta_group::2): a 256 x BN tile per pair of CTAs in a 2-CTA cluster.
+// Each CTA stages its own 128 rows of A and its own BN/2 rows of B (no multicast); both CTAs'
+// copies complete on the leader's (rank 0) stage barrier; the leader issues
+// tcgen05.mma.cta_group::2 (M = 256), which reads each half from its own CTA's shared memory and
+// leaves rows 0-127 of the accumulator in the leader's TMEM and rows 128-255 in the peer's.
+// Commits arrive on both CTAs' barriers; each CTA's epilogue drains its own TMEM half and
+// releases the accumulator on the leader.  Per SM and k-block this stages 16 KB of A and
+// BN/2 x 128 B of B, against 16 KB + BN x 128 B on a single SM.
+template <int BN_, int STAGES_, Major AMAJ_, Major BMAJ_, int EPI_WARPS_>
+struct GemmPairCfg {
+  static constexpr bool PAIR = true;
+  static constexpr int BM = 256;         // rows per pair tile
+  static constexpr int BM_CTA = 128;     // rows per CTA (one TMEM lane each)
+  static constexpr int BN = BN_;         // columns per pair tile
+  static constexpr int BN_CTA = BN_ / 2; // B rows staged by each CTA
+  static constexpr int BK = 64;
+  static constexpr int STAGES = STAGES_;
+  static constexpr Major AMAJ = AMAJ_;
+  static constexpr Major BMAJ = BMAJ_;
+  static constexpr int EPI_WARPS = EPI_WARPS_;
+  static constexpr int THREADS = 64 + 32 * EPI_WARPS;
+  static constexpr int A_BYTES = BM_CTA * BK * 2;
+  static constexpr int B_BYTES = BN_CTA * BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int TMEM_COLS = (2 * BN <= 256) ? 256 : 512;
+  static constexpr int COL_SPLIT = EPI_WARPS / 4;
+  static constexpr int COLS_PER_WARP = BN / COL_SPLIT;
+  static constexpr int BAR_BYTES = 256;
+  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
+  static_assert(EPI_WARPS % 4 == 0, "epilogue warps must cover the four TMEM lane quarters");
+  static_assert(COLS_PER_WARP % 32 == 0, "epilogue works in 32-column TMEM loads");
+  static_assert(BN_CTA % 64 == 0 || BMAJ_ == Major::K, "MN-major tiles are whole 64-wide blocks");
+  static_assert(BN % 32 == 0 && BN >= 64 && BN <= 256, "cta_group::2 M=256 needs N % 16 == 0");
+  static_assert(A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "swizzle atoms need 1 KB alignment");
+  static_assert((2 * STAGES + 5) * 8 + 8 <= BAR_BYTES, "barrier area too small");
+  static_assert(SMEM_BYTES <= 232448, "more than 227 KB of shared memory");
+};
+
+template <class C, class Epi>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
+    gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                     const GemmArgs args, const __grid_constant__ typename Epi::Params ep) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+  uint64_t* full = bars;                 // used on the leader only
+  uint64_t* empty = bars + C::STAGES;    // both CTAs
+  uint64_t* tfull = bars + 2 * C::STAGES;
+  uint64_t* tempty = tfull + 2;          // used on the leader only
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = static_cast<int>(cluster_id_x());
+  const int npairs = static_cast<int>(num_clusters_x());
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 2 * C::EPI_WARPS);   // one arrival per epilogue warp of each CTA
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
+  __syncwarp();
+  tc_fence_before();
+  cluster_sync_all();   // both CTAs' barriers initialised and TMEM allocated
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const uint32_t leader_full = mapa_shared(smem_u32(full), 0);
+  const uint32_t leader_tempty = mapa_shared(smem_u32(tempty), 0);
+
+  const int m_tiles = (args.M + C::BM - 1) / C::BM;
+  const int n_tiles = (args.N + C::BN - 1) / C::BN;
+  const int num_tiles = m_tiles * n_tiles;
+  const int num_kb = (args.K + C::BK - 1) / C::BK;
+  auto tile_coords = [&](int t, int& mb, int& nb) {
+    if (args.m_fastest) {
+      mb = t % m_tiles;
+      nb = t / m_tiles;
+    } else {
+      nb = t % n_tiles;
+      mb = t / n_tiles;
+    }
+  };
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ TMA producer (both CTAs)
+      int stage = 0;
+      uint32_t phase = 0;
+      long long arms = 0;
+      for (int t = pair; t < num_tiles && !*abort_flag; t += npairs) {
+        int mb, nb;
+        tile_coords(t, mb, nb);
+        const int a_row = mb * C::BM + static_cast<int>(rank) * C::BM_CTA;
+        const int b_row = nb * C::BN + static_cast<int>(rank) * C::BN_CTA;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, args.status, args.limit_ns)) {
+            *abort_flag = 1;
+            break;
+          }
+          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * C::STAGE_BYTES);
+          uint8_t* sA = smem + stage * C::STAGE_BYTES;
+          uint8_t* sB = sA + C::A_BYTES;
+          const uint32_t bar = leader_full + 8u * stage;
+          if constexpr (C::AMAJ == Major::K) {
+            tma_load_2d_pair(sA, &tmA, bar, kb * C::BK, a_row);
+          } else {
+#pragma unroll
+            for (int q = 0; q < C::BM_CTA / 64; ++q)
+              tma_load_2d_pair(sA + q * 8192, &tmA, bar, a_row + 64 * q, kb * C::BK);
+          }
+          if constexpr (C::BMAJ == Major::K) {
+            tma_load_2d_pair(sB, &tmB, bar, kb * C::BK, b_row);
+          } else {
+#pragma unroll
+            for (int q = 0; q < C::BN_CTA / 64; ++q)
+              tma_load_2d_pair(sB + q * 8192, &tmB, bar, b_row + 64 * q, kb * C::BK);
+          }
+          ++arms;
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (leader) {
+        // Drain: the last phases of every stage include both CTAs' copies.
+        const long long first = arms > C::STAGES ? arms - C::STAGES : 0;
+        for (long long a = first; a < arms; ++a)
+          mbar_wait_bounded(&full[a % C::STAGES], static_cast<uint32_t>((a / C::STAGES) & 1),
+                            args.status, args.limit_ns);
+      } else if (*abort_flag) {
+        // After an abort the leader may not wait for this CTA's last copies: give them time
+        // to land before the CTA can exit (copies take microseconds).
+        const uint64_t t0 = global_timer_ns();
+        while (global_timer_ns() - t0 < 200000ull) {
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      // ------------------------------------------------------------ MMA issuer (leader only)
+      constexpr uint32_t idesc =
+          instr_desc_bf16_f32(C::BM, C::BN, C::AMAJ == Major::MN, C::BMAJ == Major::MN);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool issued = false;
+      for (int t = pair; t < num_tiles && !*abort_flag; t += npairs) {
+        if (!mbar_wait_bounded_cluster(&tempty[acc], acc_phase ^ 1u, args.status, args.limit_ns)) {
+          *abort_flag = 1;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * C::BN);
+        bool ok = true;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait_bounded(&full[stage], phase, args.status, args.limit_ns)) {
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_base = smem_u32(smem + stage * C::STAGE_BYTES);
+          const uint32_t b_base = a_base + C::A_BYTES;
+#pragma unroll
+          for (int k = 0; k < C::BK / 16; ++k) {
+            mma_bf16_ss_pair(d_tmem, operand_desc<C::AMAJ>(a_base, k),
+                             operand_desc<C::BMAJ>(b_base, k), idesc, (kb | k) != 0 ? 1u : 0u);
+          }
+          issued = true;
+          mma_commit_pair_both(&empty[stage]);
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        mma_commit_pair_both(&tfull[acc]);
+        if (++acc == 2) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
+      }
+      if (issued) {
+        mma_commit_pair_both(drain);
+        mbar_wait_bounded(drain, 0, args.status, args.limit_ns);
+      }
+    }
+  } else {
+    // -------------------------------------------------------------- epilogue (both CTAs)
+    const int ew = warp - 2;
+    const int quarter = warp & 3;
+    const int slab = ew >> 2;
+    const int row_in_cta = quarter * 32 + lane;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int t = pair; t < num_tiles && !*abort_flag; t += npairs) {
+      int mb, nb;
+      tile_coords(t, mb, nb);
+      if (!mbar_wait_bounded(&tfull[acc], acc_phase, args.status, args.limit_ns)) {
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
+                             static_cast<uint32_t>(acc * C::BN + slab * C::COLS_PER_WARP);
+      Epi::template apply<C::COLS_PER_WARP>(
+          ep, mb * C::BM + static_cast<int>(rank) * C::BM_CTA + row_in_cta,
+          nb * C::BN + slab * C::COLS_PER_WARP, taddr, nb * C::COL_SPLIT + slab);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(leader_tempty + 8u * acc);
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+    }
+  }
+
+  __syncwarp();
+  tc_fence_before();
+  cluster_sync_all();   // both CTAs done with TMEM, shared memory and barriers
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+  }
+}
+
+// ==============================================================================================
 // Epilogue 1: softcapped logits -> softmax statistics, target capture, and (optionally) the
 // unnormalised gradient operand A.
 //
@@ -279,6 +534,34 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 //     tanh(|z|/cap) = (1-u)/(1+u),   1 - tanh^2 = 4u/(1+u)^2,
 //     s - cap = -2 cap u/(1+u) (z >= 0)  or  -2 cap/(1+u) (z < 0),
 // which keeps 1 - tanh^2 and s - cap free of cancellation at saturation.
+struct Softcapped {
+  float s, der, e;
+};
+
+// s = cap tanh(z/cap), der = 1 - tanh^2(z/cap) and e = exp(s - cap), from u = exp(-2|z|/cap).
+// Special-function unit: one exp2 (u).  FMA pipe: the reciprocal 1/(1+u) (Newton-Raphson) and
+// exp(s - cap) (polynomial exp2); this keeps the epilogue off the special-function unit's limit.
+__device__ __forceinline__ Softcapped softcap_fixed_ref(float z, float k_u, float m2c_log2e,
+                                                        float cap) {
+  const float u = ex2_approx(-fabsf(z) * k_u);        // exp(-2|z|/cap) in (0, 1]
+#if FLCE_SOFTCAP_SFU
+  const float q = rcp_approx(1.0f + u);
+#else
+  const float q = rcp_newton_1_2(1.0f + u);           // 1/(1+u)
+#endif
+  const float uq = u * q;
+  Softcapped r;
+  r.der = 4.0f * uq * q;                               // 4u/(1+u)^2
+  // s - cap = -2 cap u/(1+u) for z >= 0, -2 cap/(1+u) for z < 0
+#if FLCE_SOFTCAP_SFU
+  r.e = ex2_approx((z >= 0.f ? uq : q) * m2c_log2e);
+#else
+  r.e = exp2_poly((z >= 0.f ? uq : q) * m2c_log2e);
+#endif
+  r.s = copysignf(cap * (q - uq), z);                  // cap (1-u)/(1+u)
+  return r;
+}
+
 enum LogitsMode : int { LOGITS_STATS = 0, LOGITS_FUSED = 1, LOGITS_RECOMPUTE = 2 };
 
 struct LogitsParams {
@@ -288,6 +571,7 @@ struct LogitsParams {
   int fixed_ref;             // 1: exp reference is cap (requires cap > 0); 0: online / lse
   float cap;                 // > 0: softcap value; <= 0: no softcap
   float k_u;                 // 2/cap * log2(e)
+  float m2c_log2e;           // -2 cap log2(e)
   const int* tgt;            // [rows] target id, -1 when the row is not in the loss
   const float* ref;          // [rows] exp reference (lse) when !fixed_ref and mode == RECOMPUTE
   float* partial;            // [rows][n_slabs] sum-exp (pairs (max, sum-exp) when !fixed_ref)
@@ -323,25 +607,33 @@ struct LogitsEpi {
       tmem_ld32(taddr + c * 32, v);
       const int cbase = col0 + c * 32;
       if (p.fixed_ref) {
-        // softcap with the fixed reference: e = exp(s - cap)
+        // softcap with the fixed reference: e = exp(s - cap), A = e (1 - tanh^2)
+        if (static_cast<unsigned>(t - cbase) < 32u) {   // this row's target is in this chunk
+          float zt = 0.f;
 #pragma unroll
-        for (int k = 0; k < 32; ++k) {
-          const float z = v[k];
-          const float u = ex2_approx(-fabsf(z) * p.k_u);      // exp(-2|z|/cap)
-          const float q = rcp_approx(1.0f + u);
-          const float der = 4.0f * u * q * q;                // 1 - tanh^2(z/cap)
-          const float s_minus_cap = z >= 0.f ? -2.0f * p.cap * u * q : -2.0f * p.cap * q;
-          float e = ex2_approx(s_minus_cap * LOG2E);
-          const int col = cbase + k;
-          if (col >= p.Vreal) e = 0.f;
-          sum += e;
-          if (col == t) {
-            tv_s = copysignf(p.cap * (1.0f - u) * q, z);
-            tv_der = der;
-            tv_e = e;
-            has_t = true;
+          for (int k = 0; k < 32; ++k)
+            if (k == t - cbase) zt = v[k];
+          const Softcapped sc = softcap_fixed_ref(zt, p.k_u, p.m2c_log2e, p.cap);
+          tv_s = sc.s;
+          tv_der = sc.der;
+          tv_e = sc.e;
+          has_t = true;
+        }
+        if (cbase + 32 <= p.Vreal) {
+#pragma unroll
+          for (int k = 0; k < 32; ++k) {
+            const Softcapped sc = softcap_fixed_ref(v[k], p.k_u, p.m2c_log2e, p.cap);
+            sum += sc.e;
+            v[k] = sc.e * sc.der;
           }
-          v[k] = e * der;
+        } else {                                            // last vocabulary tile: padded columns
+#pragma unroll
+          for (int k = 0; k < 32; ++k) {
+            const Softcapped sc = softcap_fixed_ref(v[k], p.k_u, p.m2c_log2e, p.cap);
+            const float e = cbase + k < p.Vreal ? sc.e : 0.f;
+            sum += e;
+            v[k] = e * sc.der;
+          }
         }
       } else {
         float der[32];

@@ -58,15 +58,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // Wait until the phase with the given parity has completed.  Gives up after
 // `limit_ns` of wall time, raises DEV_TIMEOUT in *status and returns false, so
 // a lost arrival ends the kernel with an error instead of hanging the GPU.
+// try_wait itself suspends the thread for a while, so the clock is read only
+// once every 1024 unsuccessful polls.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
                                                   uint32_t* status, uint64_t limit_ns) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = global_timer_ns();
-  while (true) {
+  uint64_t t0 = 0;
+  for (uint32_t it = 0;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (global_timer_ns() - t0 > limit_ns) {
-      if (status) atomicOr(status, DEV_TIMEOUT);
-      return false;
+    if ((it & 1023u) == 1023u) {
+      const uint64_t now = global_timer_ns();
+      if (t0 == 0) {
+        t0 = now;
+      } else if (now - t0 > limit_ns) {
+        if (status) atomicOr(status, DEV_TIMEOUT);
+        return false;
+      }
     }
   }
 }
@@ -177,6 +183,104 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// ---------------------------------------------------------------- CTA pairs (cta_group::2)
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cluster_id_x() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %clusterid.x;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t num_clusters_x() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %nclusterid.x;" : "=r"(r));
+  return r;
+}
+// Address in the shared::cluster window of the same variable in CTA `rank` of this cluster.
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t local_addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local_addr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" :::
+                   "memory");
+}
+// Arrive on an mbarrier that may live in the peer CTA (shared::cluster address).
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait_cluster_acq(uint64_t* bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+// Bounded wait with cluster-scope acquire (for barriers the peer CTA arrives on).
+__device__ __forceinline__ bool mbar_wait_bounded_cluster(uint64_t* bar, uint32_t parity,
+                                                          uint32_t* status, uint64_t limit_ns) {
+  uint64_t t0 = 0;
+  for (uint32_t it = 0;; ++it) {
+    if (mbar_try_wait_cluster_acq(bar, parity)) return true;
+    if ((it & 1023u) == 1023u) {
+      const uint64_t now = global_timer_ns();
+      if (t0 == 0) {
+        t0 = now;
+      } else if (now - t0 > limit_ns) {
+        if (status) atomicOr(status, DEV_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+// Tile load whose completion is counted on the pair leader's mbarrier (cluster address).
+// Each CTA loads into its own shared memory; no multicast.
+__device__ __forceinline__ void tma_load_2d_pair(void* smem_dst, const CUtensorMap* map,
+                                                 uint32_t leader_bar, int32_t x, int32_t y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(leader_bar), "r"(x), "r"(y)
+      : "memory");
+}
+__device__ __forceinline__ void mma_bf16_ss_pair(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                                 uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Arrive on the barrier at this offset in both CTAs of the pair once the pair's MMAs complete.
+__device__ __forceinline__ void mma_commit_pair_both(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;" ::"r"(smem_u32(bar)),
+      "h"(static_cast<uint16_t>(3))
+      : "memory");
+}
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                   smem_u32(dst_smem)),
+               "r"(ncols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+
 // ---------------------------------------------------------------- fast math
 // exp2 and reciprocal on the special-function unit (documented relative errors
 // of about 2^-22 and 2^-23; ftz).
@@ -189,6 +293,39 @@ __device__ __forceinline__ float rcp_approx(float x) {
   float y;
   asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// 1/v for v in [1, 2] on the FMA pipe (Newton-Raphson division): linear seed 24/17 - 8/17 v
+// (relative error <= 1/17), then three steps x <- x + x(1 - v x); the error squares each step
+// (1/17 -> 3.5e-3 -> 1.2e-5 -> 1.4e-10), i.e. fp32 rounding level after three.
+__device__ __forceinline__ float rcp_newton_1_2(float v) {
+  float x = fmaf(-0.47058823529411764f, v, 1.4117647058823530f);
+  float r = fmaf(-v, x, 1.0f);
+  x = fmaf(x, r, x);
+  r = fmaf(-v, x, 1.0f);
+  x = fmaf(x, r, x);
+  r = fmaf(-v, x, 1.0f);
+  return fmaf(x, r, x);
+}
+
+// 2^w for w in [-126, 0] on the FMA/ALU pipes.  w = n + f with n = rint(w) obtained by adding
+// and subtracting 1.5*2^23 (the rounded integer sits in the low mantissa bits of the sum), |f| <=
+// 1/2; 2^f from the degree-6 Taylor polynomial of e^{f ln 2} (relative truncation error 1.6e-7
+// on |f| <= 1/2); 2^n applied by adding n to the exponent field.  No denormal results for w
+// above -126.
+__device__ __forceinline__ float exp2_poly(float w) {
+  const float kRound = 12582912.0f;  // 1.5 * 2^23
+  const float t = w + kRound;
+  const float n = t - kRound;
+  const float f = w - n;
+  float p = 1.5403530393381606e-4f;
+  p = fmaf(p, f, 1.3333558146428441e-3f);
+  p = fmaf(p, f, 9.6181291076284770e-3f);
+  p = fmaf(p, f, 5.5504108664821576e-2f);
+  p = fmaf(p, f, 2.4022650695910071e-1f);
+  p = fmaf(p, f, 6.9314718055994531e-1f);
+  p = fmaf(p, f, 1.0f);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
