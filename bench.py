@@ -51,6 +51,9 @@ def parse_args():
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--ref-rows", type=int, default=128,
                     help="rows per step of the --impl reference arm")
+    ap.add_argument("--compare-cublas", action="store_true",
+                    help="per-contraction efficiency at the operating clock next to cuBLAS "
+                         "(torch.matmul) on the same shapes, with NVML clock/power sampling")
     return ap.parse_args()
 
 
@@ -255,10 +258,12 @@ def main_gpu(args):
     ws = flce.alloc_workspace(shape, True, dev)
     stream = torch.cuda.current_stream()
 
-    def step():
-        loss, lse, _, _, _ = flce.forward(X, W, t, Vr, c.cap, c.ignore_index, True, dX=dX, dW=dW,
-                                          workspace=ws, chunk_rows=args.chunk_rows)
-        flce.backward(X, W, t, lse, Vr, c.cap, c.ignore_index, grad_out=g_one, dX=dX, dW=dW,
+    def step(Xd=None, td=None):
+        Xd = X if Xd is None else Xd
+        td = t if td is None else td
+        loss, lse, _, _, _ = flce.forward(Xd, W, td, Vr, c.cap, c.ignore_index, True, dX=dX,
+                                          dW=dW, workspace=ws, chunk_rows=args.chunk_rows)
+        flce.backward(Xd, W, td, lse, Vr, c.cap, c.ignore_index, grad_out=g_one, dX=dX, dW=dW,
                       grads_precomputed=True)
         return loss
 
@@ -301,25 +306,46 @@ def main_gpu(args):
     credited = 6.0 * N * d * Vp
     tflops = credited / (ms_per_step / 1e3) / 1e12 * world
 
-    # ---- end-to-end through the public API with host buffers
+    # ---- end-to-end through the public API with host buffers: every step copies its X and
+    # targets from pinned host memory and reads its loss back.  The copy for step i+2 runs on a
+    # side stream into the buffer step i has finished with, so copies overlap compute.
     e2e = None
     if not args.no_e2e:
         loss_h = torch.empty((), dtype=torch.float32).pin_memory()
+        Xb = [X, torch.empty_like(X)]
+        tb = [t, torch.empty_like(t)]
+        copy_stream = torch.cuda.Stream(device=dev)
+        copied = [torch.cuda.Event(), torch.cuda.Event()]
+        used = [torch.cuda.Event(), torch.cuda.Event()]
 
-        def e2e_step():
-            X.copy_(X_h, non_blocking=True)
-            t.copy_(t_h, non_blocking=True)
-            loss = step()
-            loss_h.copy_(loss, non_blocking=True)
+        def issue_copy(b, first=False):
+            with torch.cuda.stream(copy_stream):
+                if not first:
+                    copy_stream.wait_event(used[b])
+                Xb[b].copy_(X_h, non_blocking=True)
+                tb[b].copy_(t_h, non_blocking=True)
+                copied[b].record(copy_stream)
 
-        for _ in range(max(1, args.warmup)):
-            e2e_step()
+        def e2e_run(nsteps):
+            issue_copy(0, True)
+            if nsteps > 1:
+                issue_copy(1, True)
+            for i in range(nsteps):
+                b = i % 2
+                stream.wait_event(copied[b])
+                loss = step(Xb[b], tb[b])
+                used[b].record(stream)
+                loss_h.copy_(loss, non_blocking=True)
+                if i + 2 < nsteps:
+                    issue_copy(b)
+
+        e2e_run(max(2, args.warmup))
         torch.cuda.synchronize()
         barrier()
         f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         f0.record(stream)
-        for _ in range(args.steps):
-            e2e_step()
+        copy_stream.wait_event(f0)
+        e2e_run(args.steps)
         f1.record(stream)
         torch.cuda.synchronize()
         barrier()
@@ -331,8 +357,9 @@ def main_gpu(args):
         e2e = {"value": world * N / (e2e_ms / args.steps / 1e3), "unit": UNIT,
                "h2d_bytes_per_step": X.numel() * 2 + t.numel() * 8, "d2h_bytes_per_step": 4,
                "ms_per_step": e2e_ms / args.steps,
-               "what": "pinned-host X and targets copied in, loss copied out, every step; "
-                       "W and dW stay resident (the head's parameter and its gradient)"}
+               "what": "pinned-host X and targets copied in and the loss copied out every step "
+                       "(copies on a side stream, double-buffered, overlapping the previous "
+                       "step); W and dW stay resident (the head's parameter and its gradient)"}
 
     peaks, peaks_src = load_peaks()
     sustained = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
@@ -438,10 +465,120 @@ def unfused_torch_baseline(X, W, t, c, args):
         return {"error": "out of memory"}
 
 
+class NvmlSampler:
+    """SM clock, power and clock-event reasons every 10 ms while a loop runs (NVML)."""
+
+    def __init__(self, torch_device):
+        import threading
+        import pynvml
+        self.nv = pynvml
+        pynvml.nvmlInit()
+        self.h = pynvml.nvmlDeviceGetHandleByIndex(0)
+        uuid = str(getattr(__import__("torch").cuda.get_device_properties(torch_device), "uuid", ""))
+        for i in range(pynvml.nvmlDeviceGetCount()):
+            hh = pynvml.nvmlDeviceGetHandleByIndex(i)
+            u = pynvml.nvmlDeviceGetUUID(hh)
+            u = u.decode() if isinstance(u, bytes) else u
+            if uuid and uuid in u:
+                self.h = hh
+        self.threading = threading
+
+    def __enter__(self):
+        self.samples, self.stop = [], False
+
+        def run():
+            nv = self.nv
+            while not self.stop:
+                self.samples.append((nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM),
+                                     nv.nvmlDeviceGetPowerUsage(self.h) / 1000.0,
+                                     nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)))
+                time.sleep(0.01)
+        self.t = self.threading.Thread(target=run)
+        self.t.start()
+        return self
+
+    def __exit__(self, *exc):
+        self.stop = True
+        self.t.join()
+
+    def summary(self):
+        c = [x[0] for x in self.samples] or [0]
+        p = [x[1] for x in self.samples] or [0]
+        return {"sm_mhz": statistics.median(c), "power_w": statistics.median(p),
+                "samples": len(self.samples),
+                "power_capped": any(x[2] & 0x4 for x in self.samples)}
+
+
+def compare_cublas(args):
+    """Each contraction of one chunk (Nc rows) next to torch.matmul (cuBLAS) on the same shape,
+    each looped for ~2 s; efficiency = achieved FLOP/s / (8192 FLOP/clk/SM x SMs x median clock)."""
+    import numpy as np
+    import torch
+    import lm_head_linear_gemm_b200 as flce
+    import synth
+    dev = torch.device("cuda", 0)
+    cfg = synth.CONFIGS[args.config]
+    Nc = args.rows or 4096
+    inp = synth.make_inputs(cfg, N=Nc)
+    c = inp["cfg"]
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    flop = 2.0 * Nc * c.d * c.Vpad
+
+    def bf(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    X, W = bf(inp["X"]), bf(inp["W"])
+    t = torch.from_numpy(inp["targets"]).to(dev)
+    Ap = (torch.randn(Nc, c.Vpad, device=dev) * 1e-3).to(torch.bfloat16)
+
+    def loop(fn, seconds=2.0):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n, t0 = 0, time.time()
+        with NvmlSampler(dev) as smp:
+            e0.record()
+            while time.time() - t0 < seconds:
+                fn()
+                n += 1
+                if n % 4 == 0:
+                    torch.cuda.synchronize()
+            e1.record()
+            torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / n, smp.summary()
+
+    def row(ms, smp):
+        tf = flop / (ms * 1e-3) / 1e12
+        peak = 8192 * sms * smp["sm_mhz"] * 1e6 / 1e12
+        return {"ms": ms, "tflops": tf, "pct_of_clock_peak": 100 * tf / peak, **smp}
+
+    out = {}
+    for name, fn in (("cublas_logits_shape", lambda: torch.matmul(X, W.T)),
+                     ("cublas_dX_shape", lambda: torch.matmul(Ap, W)),
+                     ("cublas_dW_shape", lambda: torch.matmul(Ap.T, X))):
+        out[name] = row(*loop(fn))
+    dX = torch.empty_like(X)
+    dW = torch.empty((c.Vpad, c.d), dtype=torch.float32, device=dev)
+    ws = flce.alloc_workspace(flce.make_shape(Nc, c.d, c.Vpad, c.Vreal, c.cap), True, dev)
+    flce.instrument(True)
+    ms, smp = loop(lambda: flce.forward(X, W, t, c.Vreal, c.cap, c.ignore_index, True, dX=dX,
+                                        dW=dW, workspace=ws), 3.0)
+    st = flce.instrument_read()
+    flce.instrument(False)
+    for k, v in st["gemm"].items():
+        out["flce_" + k] = row(v["ms"] / v["launches"], smp)
+    out["flce_chunk_step_ms"] = ms
+    print(json.dumps({"compare_cublas": out, "rows": Nc, "config": c.name}), flush=True)
+    return 0
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
         return run_reference(args)
+    if args.compare_cublas:
+        return compare_cublas(args)
     return main_gpu(args)
 
 

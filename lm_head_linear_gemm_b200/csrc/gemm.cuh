@@ -17,9 +17,7 @@
 #pragma once
 #include "sm100.cuh"
 
-#ifndef FLCE_SOFTCAP_SFU
-#define FLCE_SOFTCAP_SFU 0
-#endif
+
 
 namespace flce {
 
@@ -538,26 +536,19 @@ struct Softcapped {
   float s, der, e;
 };
 
-// s = cap tanh(z/cap), der = 1 - tanh^2(z/cap) and e = exp(s - cap), from u = exp(-2|z|/cap).
-// Special-function unit: one exp2 (u).  FMA pipe: the reciprocal 1/(1+u) (Newton-Raphson) and
-// exp(s - cap) (polynomial exp2); this keeps the epilogue off the special-function unit's limit.
+// s = cap tanh(z/cap), der = 1 - tanh^2(z/cap) and e = exp(s - cap), from u = exp(-2|z|/cap):
+// three special-function operations (exp2, reciprocal, exp2) and a handful of FMAs per logit.
+// (Moving the reciprocal or the second exp2 to FMA-pipe Newton / polynomial forms measured
+// slower on B200: the extra instructions cost more than the special-function unit saves.)
 __device__ __forceinline__ Softcapped softcap_fixed_ref(float z, float k_u, float m2c_log2e,
                                                         float cap) {
   const float u = ex2_approx(-fabsf(z) * k_u);        // exp(-2|z|/cap) in (0, 1]
-#if FLCE_SOFTCAP_SFU
-  const float q = rcp_approx(1.0f + u);
-#else
-  const float q = rcp_newton_1_2(1.0f + u);           // 1/(1+u)
-#endif
+  const float q = rcp_approx(1.0f + u);               // 1/(1+u)
   const float uq = u * q;
   Softcapped r;
   r.der = 4.0f * uq * q;                               // 4u/(1+u)^2
   // s - cap = -2 cap u/(1+u) for z >= 0, -2 cap/(1+u) for z < 0
-#if FLCE_SOFTCAP_SFU
   r.e = ex2_approx((z >= 0.f ? uq : q) * m2c_log2e);
-#else
-  r.e = exp2_poly((z >= 0.f ? uq : q) * m2c_log2e);
-#endif
   r.s = copysignf(cap * (q - uq), z);                  // cap (1-u)/(1+u)
   return r;
 }

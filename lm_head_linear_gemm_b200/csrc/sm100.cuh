@@ -295,39 +295,6 @@ __device__ __forceinline__ float rcp_approx(float x) {
   return y;
 }
 
-// 1/v for v in [1, 2] on the FMA pipe (Newton-Raphson division): linear seed 24/17 - 8/17 v
-// (relative error <= 1/17), then three steps x <- x + x(1 - v x); the error squares each step
-// (1/17 -> 3.5e-3 -> 1.2e-5 -> 1.4e-10), i.e. fp32 rounding level after three.
-__device__ __forceinline__ float rcp_newton_1_2(float v) {
-  float x = fmaf(-0.47058823529411764f, v, 1.4117647058823530f);
-  float r = fmaf(-v, x, 1.0f);
-  x = fmaf(x, r, x);
-  r = fmaf(-v, x, 1.0f);
-  x = fmaf(x, r, x);
-  r = fmaf(-v, x, 1.0f);
-  return fmaf(x, r, x);
-}
-
-// 2^w for w in [-126, 0] on the FMA/ALU pipes.  w = n + f with n = rint(w) obtained by adding
-// and subtracting 1.5*2^23 (the rounded integer sits in the low mantissa bits of the sum), |f| <=
-// 1/2; 2^f from the degree-6 Taylor polynomial of e^{f ln 2} (relative truncation error 1.6e-7
-// on |f| <= 1/2); 2^n applied by adding n to the exponent field.  No denormal results for w
-// above -126.
-__device__ __forceinline__ float exp2_poly(float w) {
-  const float kRound = 12582912.0f;  // 1.5 * 2^23
-  const float t = w + kRound;
-  const float n = t - kRound;
-  const float f = w - n;
-  float p = 1.5403530393381606e-4f;
-  p = fmaf(p, f, 1.3333558146428441e-3f);
-  p = fmaf(p, f, 9.6181291076284770e-3f);
-  p = fmaf(p, f, 5.5504108664821576e-2f);
-  p = fmaf(p, f, 2.4022650695910071e-1f);
-  p = fmaf(p, f, 6.9314718055994531e-1f);
-  p = fmaf(p, f, 1.0f);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-}
-
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h);
