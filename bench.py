@@ -567,7 +567,11 @@ def compare_cublas(args):
     st = flce.instrument_read()
     flce.instrument(False)
     for k, v in st["gemm"].items():
-        out["flce_" + k] = row(v["ms"] / v["launches"], smp)
+        if v["launches"]:
+            r = row(v["ms"] / v["launches"], smp)
+            r["tflops"] = v["flop"] / (v["ms"] * 1e-3) / 1e12       # the dX+dW launch does 2 shapes
+            r["pct_of_clock_peak"] = 100 * r["tflops"] / (8192 * sms * smp["sm_mhz"] * 1e6 / 1e12)
+            out["flce_" + k] = r
     out["flce_chunk_step_ms"] = ms
     print(json.dumps({"compare_cublas": out, "rows": Nc, "config": c.name}), flush=True)
     return 0

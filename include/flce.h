@@ -144,8 +144,8 @@ int flce_read_status(const void* workspace, uint32_t* dev_status_out, int64_t* n
 /*
  * Instrumentation (not part of the computation).  flce_instrument(1) resets the counters and
  * starts recording: every kernel the library launches is counted, and each tensor-core
- * contraction launch (kind 0: logits, 1: dX, 2: dW) is bracketed by CUDA events on its own
- * stream.  flce_instrument(0) stops recording.  flce_instrument_read waits for the recorded
+ * contraction launch (kind 0: logits; kind 1: dX and dW, which share one launch; kind 2 is not
+ * used) is bracketed by CUDA events on its own stream.  flce_instrument(0) stops recording.  flce_instrument_read waits for the recorded
  * events and fills `out` with the totals since the last reset.  Process-wide; host-thread safe.
  */
 typedef struct {

@@ -47,7 +47,7 @@ class flce_kernel_stats(ctypes.Structure):
     ]
 
 
-GEMM_KINDS = ("logits", "dX", "dW")
+GEMM_KINDS = ("logits", "dX+dW", "unused")
 
 _lib = None
 

@@ -28,24 +28,14 @@ using namespace flce;
 
 namespace {
 
-// Contraction tiles.  Pairs of SMs (cta_group::2, 256 x 256 tiles) by default; the single-SM
-// kernels (128 x 192 / 128 x 256 tiles) remain available with -DFLCE_PAIR=0.
-#ifndef FLCE_PAIR
-#define FLCE_PAIR 1
-#endif
-#if FLCE_PAIR
-using CfgLogits = GemmPairCfg<256, 6, Major::K, Major::K, 8>;
-using CfgDx = GemmPairCfg<256, 6, Major::K, Major::MN, 8>;
-using CfgDw = GemmPairCfg<256, 6, Major::MN, Major::MN, 8>;
-template <class C, class E>
-constexpr auto gemm_entry = gemm_pair_kernel<C, E>;
-#else
-using CfgLogits = GemmCfg<192, 5, Major::K, Major::K, 8>;
-using CfgDx = GemmCfg<256, 4, Major::K, Major::MN, 8>;
-using CfgDw = GemmCfg<256, 4, Major::MN, Major::MN, 8>;
-template <class C, class E>
-constexpr auto gemm_entry = gemm_kernel<C, E>;
-#endif
+// Contraction tiles: pairs of SMs (cta_group::2), 256 x 256 tiles, 6-stage shared-memory ring.
+using Cfg = PairCfg<256, 6, 8>;
+// logits: A = X (K-major), B = W (K-major)
+constexpr auto kLogitsKernel =
+    gemm_pair_kernel<Cfg, LogitsEpi, LogitsEpi, Major::K, Major::K, Major::K, Major::K>;
+// gradients in one launch: dX = A' W (A' K-major, W MN-major), dW = A'^T Xs (both MN-major)
+constexpr auto kGradKernel =
+    gemm_pair_kernel<Cfg, DxEpi, DwEpi, Major::K, Major::MN, Major::MN, Major::MN>;
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s bound on every in-kernel wait
 constexpr float kFixedRefMaxCap = 32.f;           // exp(s - cap) >= e^{-64}: no underflow in fp32
@@ -80,8 +70,8 @@ Layout make_layout(const flce_shape* s, int want_grads) {
   if (nc < 1) nc = 1;
   L.chunk = nc;
   L.fixed_ref = s->cap > 0.f && s->cap <= kFixedRefMaxCap;
-  const int64_t vtiles = (s->Vpad + CfgLogits::BN - 1) / CfgLogits::BN;
-  L.n_slabs = static_cast<int>(vtiles * CfgLogits::COL_SPLIT);
+  const int64_t vtiles = (s->Vpad + Cfg::BN - 1) / Cfg::BN;
+  L.n_slabs = static_cast<int>(vtiles * Cfg::COL_SPLIT);
   size_t off = 0;
   auto take = [&](size_t bytes) {
     const size_t at = off;
@@ -133,13 +123,10 @@ int device_info(DeviceInfo** out) {
   }
   if (!di.ok) return FLCE_ERR_DEVICE;
   if (!di.attrs_set) {
-    if (cudaFuncSetAttribute(gemm_entry<CfgLogits, LogitsEpi>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             CfgLogits::SMEM_BYTES) != cudaSuccess ||
-        cudaFuncSetAttribute(gemm_entry<CfgDx, DxEpi>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             CfgDx::SMEM_BYTES) != cudaSuccess ||
-        cudaFuncSetAttribute(gemm_entry<CfgDw, DwEpi>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             CfgDw::SMEM_BYTES) != cudaSuccess)
+    if (cudaFuncSetAttribute(kLogitsKernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Cfg::SMEM_BYTES) != cudaSuccess ||
+        cudaFuncSetAttribute(kGradKernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Cfg::SMEM_BYTES) != cudaSuccess)
       return FLCE_ERR_CUDA;
     di.attrs_set = true;
   }
@@ -214,31 +201,40 @@ cudaEvent_t pooled_event() {
   return e;
 }
 
-template <class C, class Epi>
-int launch_gemm(const DeviceInfo* di, const CUtensorMap& a, const CUtensorMap& b, int M, int N,
-                int K, int m_fastest, uint32_t* status, const typename Epi::Params& ep,
-                cudaStream_t st, int kind) {
-  const long long tiles = static_cast<long long>((M + C::BM - 1) / C::BM) * ((N + C::BN - 1) / C::BN);
+long long pair_tiles(const PairProblem& p) {
+  if (p.M <= 0 || p.N <= 0) return 0;
+  return static_cast<long long>((p.M + Cfg::BM - 1) / Cfg::BM) * ((p.N + Cfg::BN - 1) / Cfg::BN);
+}
+
+// Launch one persistent pair kernel over one or two problems; `kind` labels the launch for the
+// instrumentation counters (0: logits, 1: dX + dW).
+template <class E0, class E1, class K>
+int launch_pair(K kernel, const DeviceInfo* di, const CUtensorMap& a0, const CUtensorMap& b0,
+                const CUtensorMap& a1, const CUtensorMap& b1, const PairProblem& p0,
+                const PairProblem& p1, uint32_t* status, const typename E0::Params& e0,
+                const typename E1::Params& e1, cudaStream_t st, int kind) {
+  const long long tiles = pair_tiles(p0) + pair_tiles(p1);
   if (tiles <= 0) return FLCE_OK;
-  // persistent: one CTA (or CTA pair) per SM (pair of SMs), never more than there are tiles
-  const long long units = C::PAIR ? di->sms / 2 : di->sms;
-  const int grid = static_cast<int>((tiles < units ? tiles : units) * (C::PAIR ? 2 : 1));
-  GemmArgs args{M, N, K, m_fastest, status, kWaitLimitNs};
-  cudaEvent_t e0 = nullptr, e1 = nullptr;
+  const long long units = di->sms / 2;   // one CTA pair per SM pair, persistent
+  const int grid = static_cast<int>(2 * (tiles < units ? tiles : units));
+  PairArgs args{{p0, p1}, status, kWaitLimitNs};
+  cudaEvent_t ev0 = nullptr, ev1 = nullptr;
   const bool timed = g_instr.load(std::memory_order_relaxed) != 0;
   if (timed) {
     std::lock_guard<std::mutex> lock(g_instr_mu);
-    e0 = pooled_event();
-    e1 = pooled_event();
-    if (e0 != nullptr) cudaEventRecord(e0, st);
+    ev0 = pooled_event();
+    ev1 = pooled_event();
+    if (ev0 != nullptr) cudaEventRecord(ev0, st);
   }
-  gemm_entry<C, Epi><<<grid, C::THREADS, C::SMEM_BYTES, st>>>(a, b, args, ep);
+  kernel<<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, st>>>(a0, b0, a1, b1, args, e0, e1);
   const bool ok = cudaGetLastError() == cudaSuccess;
   count_launch();
-  if (timed && e0 != nullptr && e1 != nullptr) {
-    cudaEventRecord(e1, st);
+  if (timed && ev0 != nullptr && ev1 != nullptr) {
+    cudaEventRecord(ev1, st);
+    const double flop = 2.0 * p0.M * p0.N * static_cast<double>(p0.K) +
+                        (p1.M > 0 ? 2.0 * p1.M * p1.N * static_cast<double>(p1.K) : 0.0);
     std::lock_guard<std::mutex> lock(g_instr_mu);
-    g_timed.push_back(TimedLaunch{kind, 2.0 * M * N * static_cast<double>(K), e0, e1});
+    g_timed.push_back(TimedLaunch{kind, flop, ev0, ev1});
   }
   return ok ? FLCE_OK : FLCE_ERR_CUDA;
 }
@@ -281,9 +277,9 @@ int grad_chunk(const Ctx& c, int64_t row0, int rows, const __nv_bfloat16* X,
   float* r = c.at<float>(c.L.r);
 
   CUtensorMap mX, mW, mA_k, mW_mn, mA_mn, mXs_mn;
-  FLCE_TRY(make_map(&mX, Xc, d, rows, d, CfgLogits::BM_CTA));
-  FLCE_TRY(make_map(&mW, W, d, Vpad, d, CfgLogits::BN_CTA));
-  FLCE_TRY(make_map(&mA_k, Abuf, Vpad, rows, Vpad, CfgDx::BM_CTA));
+  FLCE_TRY(make_map(&mX, Xc, d, rows, d, Cfg::BM_CTA));
+  FLCE_TRY(make_map(&mW, W, d, Vpad, d, Cfg::BN_CTA));
+  FLCE_TRY(make_map(&mA_k, Abuf, Vpad, rows, Vpad, Cfg::BM_CTA));
   FLCE_TRY(make_map(&mW_mn, W, d, Vpad, d, 64));
   FLCE_TRY(make_map(&mA_mn, Abuf, Vpad, rows, Vpad, 64));
   FLCE_TRY(make_map(&mXs_mn, Xs, d, rows, d, 64));
@@ -305,8 +301,9 @@ int grad_chunk(const Ctx& c, int64_t row0, int rows, const __nv_bfloat16* X,
   lp.der_t = c.at<float>(c.L.der_t) + row0;
   lp.e_t = c.at<float>(c.L.e_t) + row0;
   lp.A = Abuf;
-  FLCE_TRY((launch_gemm<CfgLogits, LogitsEpi>(c.di, mX, mW, rows, Vpad, d, 1, &c.hdr->status, lp,
-                                               c.st, 0)));
+  const PairProblem logits{rows, Vpad, d, 1}, none{0, 0, 0, 0};
+  FLCE_TRY((launch_pair<LogitsEpi, LogitsEpi>(kLogitsKernel, c.di, mX, mW, mX, mW, logits, none,
+                                               &c.hdr->status, lp, lp, c.st, 0)));
 
   RowFinishParams rp{};
   rp.rows = rows;
@@ -334,12 +331,12 @@ int grad_chunk(const Ctx& c, int64_t row0, int rows, const __nv_bfloat16* X,
   row_finish_kernel<<<(rows + 7) / 8, 256, 0, c.st>>>(rp);
   FLCE_TRY(launch_ok());
 
+  // dX (long tiles: K = Vpad) and dW (short tiles: K = rows) share one balanced launch
   DxParams xp{rows, d, r, dX + row0 * s->d};
-  FLCE_TRY((launch_gemm<CfgDx, DxEpi>(c.di, mA_k, mW_mn, rows, d, Vpad, 0, &c.hdr->status, xp,
-                                       c.st, 1)));
   DwParams wp{Vpad, d, accumulate, dW};
-  FLCE_TRY((launch_gemm<CfgDw, DwEpi>(c.di, mA_mn, mXs_mn, Vpad, d, rows, 0, &c.hdr->status, wp,
-                                       c.st, 2)));
+  const PairProblem pdx{rows, d, Vpad, 0}, pdw{Vpad, d, rows, 0};
+  FLCE_TRY((launch_pair<DxEpi, DwEpi>(kGradKernel, c.di, mA_k, mW_mn, mA_mn, mXs_mn, pdx, pdw,
+                                       &c.hdr->status, xp, wp, c.st, 1)));
   return FLCE_OK;
 }
 
@@ -348,11 +345,11 @@ int stats_pass(const Ctx& c, const __nv_bfloat16* X, const __nv_bfloat16* W, flo
   const flce_shape* s = c.s;
   const int d = static_cast<int>(s->d), Vpad = static_cast<int>(s->Vpad);
   CUtensorMap mW;
-  FLCE_TRY(make_map(&mW, W, d, Vpad, d, CfgLogits::BN_CTA));
+  FLCE_TRY(make_map(&mW, W, d, Vpad, d, Cfg::BN_CTA));
   for (int64_t row0 = 0; row0 < s->N; row0 += c.L.chunk) {
     const int rows = static_cast<int>(s->N - row0 < c.L.chunk ? s->N - row0 : c.L.chunk);
     CUtensorMap mX;
-    FLCE_TRY(make_map(&mX, X + row0 * s->d, d, rows, d, CfgLogits::BM_CTA));
+    FLCE_TRY(make_map(&mX, X + row0 * s->d, d, rows, d, Cfg::BM_CTA));
     LogitsParams lp{};
     lp.rows = rows;
     lp.Vreal = static_cast<int>(s->Vreal);
@@ -368,8 +365,9 @@ int stats_pass(const Ctx& c, const __nv_bfloat16* X, const __nv_bfloat16* W, flo
     lp.s_t = c.at<float>(c.L.s_t) + row0;
     lp.der_t = c.at<float>(c.L.der_t) + row0;
     lp.e_t = c.at<float>(c.L.e_t) + row0;
-    FLCE_TRY((launch_gemm<CfgLogits, LogitsEpi>(c.di, mX, mW, rows, Vpad, d, 1, &c.hdr->status,
-                                                 lp, c.st, 0)));
+    const PairProblem logits{rows, Vpad, d, 1}, none{0, 0, 0, 0};
+    FLCE_TRY((launch_pair<LogitsEpi, LogitsEpi>(kLogitsKernel, c.di, mX, mW, mX, mW, logits, none,
+                                                 &c.hdr->status, lp, lp, c.st, 0)));
     RowFinishParams rp{};
     rp.rows = rows;
     rp.d = d;

@@ -2,9 +2,11 @@
 //
 //   D[M, N] = A[M, K] * B[N, K]^T, bf16 operands, fp32 accumulation in TMEM.
 //
-// Roles (one CTA per SM, 64 + 32*EPI_WARPS threads):
+// Runs on pairs of SMs (2-CTA clusters, tcgen05 cta_group::2).  Roles in each CTA
+// (64 + 32*EPI_WARPS threads, one CTA per SM):
 //   warp 0 lane 0 : TMA producer, STAGES-deep shared-memory ring of (A, B) k-blocks;
-//   warp 1        : TMEM allocator; lane 0 issues tcgen05.mma (M=128, N=BN, K=16);
+//   warp 1        : TMEM allocator; lane 0 of the leader CTA issues tcgen05.mma
+//                   (M=256 across the pair, N=BN, K=16);
 //   warps 2..     : epilogue; two TMEM accumulators so the epilogue of one tile
 //                   overlaps the main loop of the next.
 // Operands may be K-major (rows of K contiguous) or MN-major (rows of M/N
@@ -17,60 +19,22 @@
 #pragma once
 #include "sm100.cuh"
 
-
-
 namespace flce {
 
 enum class Major : int { K = 0, MN = 1 };
 
-template <int BN_, int STAGES_, Major AMAJ_, Major BMAJ_, int EPI_WARPS_>
-struct GemmCfg {
-  static constexpr bool PAIR = false;
-  static constexpr int BM = 128;
-  static constexpr int BM_CTA = 128;
-  static constexpr int BN = BN_;
-  static constexpr int BN_CTA = BN_;
-  static constexpr int BK = 64;  // 64 bf16 = 128 bytes = one swizzle row
-  static constexpr int STAGES = STAGES_;
-  static constexpr Major AMAJ = AMAJ_;
-  static constexpr Major BMAJ = BMAJ_;
-  static constexpr int EPI_WARPS = EPI_WARPS_;
-  static constexpr int THREADS = 64 + 32 * EPI_WARPS;
-  static constexpr int A_BYTES = BM * BK * 2;
-  static constexpr int B_BYTES = BN * BK * 2;
-  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int TMEM_COLS = (2 * BN <= 32) ? 32 : (2 * BN <= 64) ? 64 : (2 * BN <= 128) ? 128
-                                   : (2 * BN <= 256) ? 256 : 512;
-  static constexpr int COL_SPLIT = EPI_WARPS / 4;       // warps sharing one TMEM lane quarter
-  static constexpr int COLS_PER_WARP = BN / COL_SPLIT;  // columns each epilogue thread owns
-  static constexpr int BAR_BYTES = 256;
-  static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
-  static_assert(EPI_WARPS % 4 == 0, "epilogue warps must cover the four TMEM lane quarters");
-  static_assert(COLS_PER_WARP % 32 == 0, "epilogue works in 32-column TMEM loads");
-  static_assert(BN % 64 == 0 || BMAJ_ == Major::K, "MN-major tiles are whole 64-wide blocks");
-  static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "tcgen05 M=128 needs N % 16 == 0, N <= 256");
-  static_assert(A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "swizzle atoms need 1 KB alignment");
-  static_assert((2 * STAGES + 5) * 8 + 4 <= BAR_BYTES, "barrier area too small");
-  static_assert(SMEM_BYTES <= 232448, "more than 227 KB of shared memory");
-};
-
-struct GemmArgs {
-  int M, N, K;          // problem extents (M rows of A, N rows of B, K shared)
-  int m_fastest;        // tile order: 1 = consecutive tiles walk M first
-  uint32_t* status;     // device status word (DEV_TIMEOUT is or-ed in)
-  uint64_t limit_ns;    // bound on every wait
-};
-
 // ----------------------------------------------------------------------------------------------
-// Tile loaders: K-major -> one TMA box {64 (K), rows}; MN-major -> rows/64 boxes {64 (MN), 64 (K)}
+// Tile loaders: K-major -> one TMA box {64 (K), rows}; MN-major -> rows/64 boxes {64 (MN), 64 (K)}.
+// The copy completes on the pair leader's barrier (shared::cluster address).
 template <Major MAJ, int ROWS>
-__device__ __forceinline__ void load_operand(uint8_t* dst, const CUtensorMap* map, uint64_t* bar,
-                                             int row0, int k0) {
+__device__ __forceinline__ void load_operand_pair(uint8_t* dst, const CUtensorMap* map,
+                                                  uint32_t leader_bar, int row0, int k0) {
   if constexpr (MAJ == Major::K) {
-    tma_load_2d(dst, map, bar, k0, row0);
+    tma_load_2d_pair(dst, map, leader_bar, k0, row0);
   } else {
 #pragma unroll
-    for (int q = 0; q < ROWS / 64; ++q) tma_load_2d(dst + q * 8192, map, bar, row0 + 64 * q, k0);
+    for (int q = 0; q < ROWS / 64; ++q)
+      tma_load_2d_pair(dst + q * 8192, map, leader_bar, row0 + 64 * q, k0);
   }
 }
 
@@ -84,186 +48,8 @@ __device__ __forceinline__ uint64_t operand_desc(uint32_t base, int k) {
   }
 }
 
-template <class C, class Epi>
-__global__ void __launch_bounds__(C::THREADS, 1)
-    gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                const GemmArgs args, const __grid_constant__ typename Epi::Params ep) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~static_cast<uintptr_t>(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
-  uint64_t* full = bars;
-  uint64_t* empty = bars + C::STAGES;
-  uint64_t* tfull = bars + 2 * C::STAGES;
-  uint64_t* tempty = tfull + 2;
-  uint64_t* drain = tempty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < C::STAGES; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
-    }
-    for (int a = 0; a < 2; ++a) {
-      mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], C::EPI_WARPS * 32);
-    }
-    mbar_init(drain, 1);
-    *abort_flag = 0;
-    fence_barrier_init();
-  }
-  if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&tmA);
-    tma_prefetch_desc(&tmB);
-  }
-  if (warp == 1) tmem_alloc(tmem_slot, C::TMEM_COLS);
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem_base = *tmem_slot;
-
-  const int m_tiles = (args.M + C::BM - 1) / C::BM;
-  const int n_tiles = (args.N + C::BN - 1) / C::BN;
-  const int num_tiles = m_tiles * n_tiles;
-  const int num_kb = (args.K + C::BK - 1) / C::BK;
-  auto tile_coords = [&](int t, int& mb, int& nb) {
-    if (args.m_fastest) {
-      mb = t % m_tiles;
-      nb = t / m_tiles;
-    } else {
-      nb = t % n_tiles;
-      mb = t / n_tiles;
-    }
-  };
-
-  if (warp == 0) {
-    if (lane == 0) {
-      // ------------------------------------------------------------ TMA producer
-      int stage = 0;
-      uint32_t phase = 0;
-      long long arms = 0;
-      for (int t = blockIdx.x; t < num_tiles && !*abort_flag; t += gridDim.x) {
-        int mb, nb;
-        tile_coords(t, mb, nb);
-        for (int kb = 0; kb < num_kb; ++kb) {
-          if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, args.status, args.limit_ns)) {
-            *abort_flag = 1;
-            break;
-          }
-          uint8_t* sA = smem + stage * C::STAGE_BYTES;
-          uint8_t* sB = sA + C::A_BYTES;
-          mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
-          load_operand<C::AMAJ, C::BM>(sA, &tmA, &full[stage], mb * C::BM, kb * C::BK);
-          load_operand<C::BMAJ, C::BN>(sB, &tmB, &full[stage], nb * C::BN, kb * C::BK);
-          ++arms;
-          if (++stage == C::STAGES) {
-            stage = 0;
-            phase ^= 1u;
-          }
-        }
-      }
-      // Drain: every copy issued must have landed before the CTA may exit.
-      const long long first = arms > C::STAGES ? arms - C::STAGES : 0;
-      for (long long a = first; a < arms; ++a) {
-        mbar_wait_bounded(&full[a % C::STAGES], static_cast<uint32_t>((a / C::STAGES) & 1),
-                          args.status, args.limit_ns);
-      }
-    }
-  } else if (warp == 1) {
-    if (lane == 0) {
-      // ------------------------------------------------------------ MMA issuer
-      constexpr uint32_t idesc =
-          instr_desc_bf16_f32(C::BM, C::BN, C::AMAJ == Major::MN, C::BMAJ == Major::MN);
-      int stage = 0;
-      uint32_t phase = 0;
-      int acc = 0;
-      uint32_t acc_phase = 0;
-      bool issued = false;
-      for (int t = blockIdx.x; t < num_tiles && !*abort_flag; t += gridDim.x) {
-        if (!mbar_wait_bounded(&tempty[acc], acc_phase ^ 1u, args.status, args.limit_ns)) {
-          *abort_flag = 1;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * C::BN);
-        bool ok = true;
-        for (int kb = 0; kb < num_kb; ++kb) {
-          if (!mbar_wait_bounded(&full[stage], phase, args.status, args.limit_ns)) {
-            *abort_flag = 1;
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t a_base = smem_u32(smem + stage * C::STAGE_BYTES);
-          const uint32_t b_base = a_base + C::A_BYTES;
-#pragma unroll
-          for (int k = 0; k < C::BK / 16; ++k) {
-            mma_bf16_ss(d_tmem, operand_desc<C::AMAJ>(a_base, k), operand_desc<C::BMAJ>(b_base, k),
-                        idesc, (kb | k) != 0 ? 1u : 0u);
-          }
-          issued = true;
-          mma_commit(&empty[stage]);
-          if (++stage == C::STAGES) {
-            stage = 0;
-            phase ^= 1u;
-          }
-        }
-        if (!ok) break;
-        mma_commit(&tfull[acc]);
-        if (++acc == 2) {
-          acc = 0;
-          acc_phase ^= 1u;
-        }
-      }
-      if (issued) {  // drain: all MMAs complete before TMEM is released
-        mma_commit(drain);
-        mbar_wait_bounded(drain, 0, args.status, args.limit_ns);
-      }
-    }
-  } else {
-    // -------------------------------------------------------------- epilogue
-    const int ew = warp - 2;
-    const int quarter = warp & 3;              // TMEM lanes this warp may access
-    const int slab = ew >> 2;                  // which column slab of the tile
-    const int row_in_tile = quarter * 32 + lane;
-    int acc = 0;
-    uint32_t acc_phase = 0;
-    for (int t = blockIdx.x; t < num_tiles && !*abort_flag; t += gridDim.x) {
-      int mb, nb;
-      tile_coords(t, mb, nb);
-      if (!mbar_wait_bounded(&tfull[acc], acc_phase, args.status, args.limit_ns)) {
-        *abort_flag = 1;
-        break;
-      }
-      tc_fence_after();
-      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
-                             static_cast<uint32_t>(acc * C::BN + slab * C::COLS_PER_WARP);
-      Epi::template apply<C::COLS_PER_WARP>(ep, mb * C::BM + row_in_tile,
-                                            nb * C::BN + slab * C::COLS_PER_WARP, taddr,
-                                            nb * C::COL_SPLIT + slab);
-      tc_fence_before();
-      mbar_arrive(&tempty[acc]);
-      if (++acc == 2) {
-        acc = 0;
-        acc_phase ^= 1u;
-      }
-    }
-  }
-
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc(tmem_base, C::TMEM_COLS);
-  }
-}
-
 // ==============================================================================================
-// The same GEMM on SM pairs (cta_group::2): a 256 x BN tile per pair of CTAs in a 2-CTA cluster.
+// The GEMM on SM pairs (cta_group::2): a 256 x BN tile per pair of CTAs in a 2-CTA cluster.
 // Each CTA stages its own 128 rows of A and its own BN/2 rows of B (no multicast); both CTAs'
 // copies complete on the leader's (rank 0) stage barrier; the leader issues
 // tcgen05.mma.cta_group::2 (M = 256), which reads each half from its own CTA's shared memory and
@@ -271,8 +57,13 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 // Commits arrive on both CTAs' barriers; each CTA's epilogue drains its own TMEM half and
 // releases the accumulator on the leader.  Per SM and k-block this stages 16 KB of A and
 // BN/2 x 128 B of B, against 16 KB + BN x 128 B on a single SM.
-template <int BN_, int STAGES_, Major AMAJ_, Major BMAJ_, int EPI_WARPS_>
-struct GemmPairCfg {
+//
+// One launch may carry two problems (e.g. dX = A'W and dW = A'^T Xs, whose tiles differ in
+// length by 12x): each pair first takes its round-robin share of problem 0's tiles, then a
+// contiguous run of problem 1's tiles sized so that every pair ends with about the same number
+// of k-blocks.  A launch with one problem is the plain round-robin persistent schedule.
+template <int BN_, int STAGES_, int EPI_WARPS_>
+struct PairCfg {
   static constexpr bool PAIR = true;
   static constexpr int BM = 256;         // rows per pair tile
   static constexpr int BM_CTA = 128;     // rows per CTA (one TMEM lane each)
@@ -280,8 +71,6 @@ struct GemmPairCfg {
   static constexpr int BN_CTA = BN_ / 2; // B rows staged by each CTA
   static constexpr int BK = 64;
   static constexpr int STAGES = STAGES_;
-  static constexpr Major AMAJ = AMAJ_;
-  static constexpr Major BMAJ = BMAJ_;
   static constexpr int EPI_WARPS = EPI_WARPS_;
   static constexpr int THREADS = 64 + 32 * EPI_WARPS;
   static constexpr int A_BYTES = BM_CTA * BK * 2;
@@ -294,17 +83,62 @@ struct GemmPairCfg {
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
   static_assert(EPI_WARPS % 4 == 0, "epilogue warps must cover the four TMEM lane quarters");
   static_assert(COLS_PER_WARP % 32 == 0, "epilogue works in 32-column TMEM loads");
-  static_assert(BN_CTA % 64 == 0 || BMAJ_ == Major::K, "MN-major tiles are whole 64-wide blocks");
+  static_assert(BN_CTA % 64 == 0, "MN-major tiles are whole 64-wide blocks");
   static_assert(BN % 32 == 0 && BN >= 64 && BN <= 256, "cta_group::2 M=256 needs N % 16 == 0");
   static_assert(A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "swizzle atoms need 1 KB alignment");
-  static_assert((2 * STAGES + 5) * 8 + 8 <= BAR_BYTES, "barrier area too small");
+  static_assert((2 * STAGES + 5) * 8 + 32 <= BAR_BYTES, "barrier area too small");
   static_assert(SMEM_BYTES <= 232448, "more than 227 KB of shared memory");
 };
 
-template <class C, class Epi>
+struct PairProblem {
+  int M, N, K;          // extents; M == 0 marks an absent second problem
+  int m_fastest;        // tile order: 1 = consecutive tiles walk M first
+};
+
+struct PairArgs {
+  PairProblem prob[2];
+  uint32_t* status;     // device status word (DEV_TIMEOUT is or-ed in)
+  uint64_t limit_ns;    // bound on every wait
+};
+
+// Pair `pair` of `P` takes n0 tiles of problem 0 (pair, pair + P, ...).  Problem 0 has
+// a = T0 / P tiles per pair plus one more on the first T0 % P pairs ("heavy" pairs).  Problem 1
+// then runs in two interleaved phases so that concurrently running tiles stay neighbours (and
+// share their operand slabs in L2):
+//   phase A: the light pairs alone take k = round(c0 / c1) tiles each, round-robin among
+//            themselves (tiles [0, TA)), making up for the problem-0 tile they lack;
+//   phase B: the remaining tiles [TA, T1) round-robin over all pairs.
+struct PairSchedule {
+  int n0;        // problem-0 tiles
+  int qa;        // phase-A tiles (light pairs only)
+  int qb;        // phase-B tiles
+  int la;        // index of this pair among the light pairs
+  int p_light;   // number of light pairs
+  int ta;        // problem-1 tiles handed out in phase A
+};
+
+__device__ inline PairSchedule pair_schedule(int pair, int P, int T0, int c0, int T1, int c1) {
+  PairSchedule s{0, 0, 0, 0, 1, 0};
+  const int a = T0 / P, n_hi = T0 % P;
+  s.n0 = a + (pair < n_hi ? 1 : 0);
+  if (T1 <= 0) return s;
+  s.p_light = P - n_hi;
+  int k = n_hi > 0 ? (c0 + c1 / 2) / c1 : 0;
+  if (static_cast<long long>(s.p_light) * k > T1) k = T1 / s.p_light;
+  s.ta = s.p_light * k;
+  s.qa = pair >= n_hi ? k : 0;
+  s.la = pair - n_hi;
+  const int rest = T1 - s.ta;
+  s.qb = pair < rest ? (rest - pair + P - 1) / P : 0;
+  return s;
+}
+
+template <class C, class E0, class E1, Major A0, Major B0, Major A1, Major B1>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
-    gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                     const GemmArgs args, const __grid_constant__ typename Epi::Params ep) {
+    gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
+                     const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
+                     const PairArgs args, const __grid_constant__ typename E0::Params ep0,
+                     const __grid_constant__ typename E1::Params ep1) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -316,6 +150,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
   uint64_t* drain = tempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* sched = reinterpret_cast<int*>(tmem_slot + 2);   // PairSchedule fields
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -323,6 +158,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
   const bool leader = rank == 0;
   const int pair = static_cast<int>(cluster_id_x());
   const int npairs = static_cast<int>(num_clusters_x());
+
+  const int m_tiles0 = (args.prob[0].M + C::BM - 1) / C::BM;
+  const int n_tiles0 = (args.prob[0].N + C::BN - 1) / C::BN;
+  const int nkb0 = (args.prob[0].K + C::BK - 1) / C::BK;
+  const int m_tiles1 = (args.prob[1].M + C::BM - 1) / C::BM;
+  const int n_tiles1 = (args.prob[1].N + C::BN - 1) / C::BN;
+  const int nkb1 = (args.prob[1].K + C::BK - 1) / C::BK;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
@@ -335,32 +177,61 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
+    const PairSchedule ps = pair_schedule(pair, npairs, m_tiles0 * n_tiles0, nkb0,
+                                          args.prob[1].M > 0 ? m_tiles1 * n_tiles1 : 0,
+                                          nkb1 > 0 ? nkb1 : 1);
+    sched[0] = ps.n0;
+    sched[1] = ps.qa;
+    sched[2] = ps.qb;
+    sched[3] = ps.la;
+    sched[4] = ps.p_light;
+    sched[5] = ps.ta;
     fence_barrier_init();
   }
   if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&tmA);
-    tma_prefetch_desc(&tmB);
+    tma_prefetch_desc(&tmA0);
+    tma_prefetch_desc(&tmB0);
+    if (args.prob[1].M > 0) {
+      tma_prefetch_desc(&tmA1);
+      tma_prefetch_desc(&tmB1);
+    }
   }
   if (warp == 1) tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
   __syncwarp();
   tc_fence_before();
-  cluster_sync_all();   // both CTAs' barriers initialised and TMEM allocated
+  cluster_sync_all();   // both CTAs' barriers initialised, schedule written, TMEM allocated
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  const int n0 = sched[0], qa = sched[1], total = sched[0] + sched[1] + sched[2];
+  const int la = sched[3], p_light = sched[4], ta = sched[5];
   const uint32_t leader_full = mapa_shared(smem_u32(full), 0);
   const uint32_t leader_tempty = mapa_shared(smem_u32(tempty), 0);
 
-  const int m_tiles = (args.M + C::BM - 1) / C::BM;
-  const int n_tiles = (args.N + C::BN - 1) / C::BN;
-  const int num_tiles = m_tiles * n_tiles;
-  const int num_kb = (args.K + C::BK - 1) / C::BK;
-  auto tile_coords = [&](int t, int& mb, int& nb) {
-    if (args.m_fastest) {
-      mb = t % m_tiles;
-      nb = t / m_tiles;
+  // i-th tile of this pair -> (problem, m block, n block, k-blocks)
+  auto tile_of = [&](int i, int& prob, int& mb, int& nb, int& kbs) {
+    int t, mt, nt, mf;
+    if (i < n0) {
+      prob = 0;
+      t = pair + i * npairs;
+      mt = m_tiles0;
+      nt = n_tiles0;
+      mf = args.prob[0].m_fastest;
+      kbs = nkb0;
     } else {
-      nb = t % n_tiles;
-      mb = t / n_tiles;
+      prob = 1;
+      const int j = i - n0;
+      t = j < qa ? la + j * p_light : ta + pair + (j - qa) * npairs;
+      mt = m_tiles1;
+      nt = n_tiles1;
+      mf = args.prob[1].m_fastest;
+      kbs = nkb1;
+    }
+    if (mf) {
+      mb = t % mt;
+      nb = t / mt;
+    } else {
+      nb = t % nt;
+      mb = t / nt;
     }
   };
 
@@ -370,12 +241,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
       int stage = 0;
       uint32_t phase = 0;
       long long arms = 0;
-      for (int t = pair; t < num_tiles && !*abort_flag; t += npairs) {
-        int mb, nb;
-        tile_coords(t, mb, nb);
+      for (int i = 0; i < total && !*abort_flag; ++i) {
+        int prob, mb, nb, kbs;
+        tile_of(i, prob, mb, nb, kbs);
         const int a_row = mb * C::BM + static_cast<int>(rank) * C::BM_CTA;
         const int b_row = nb * C::BN + static_cast<int>(rank) * C::BN_CTA;
-        for (int kb = 0; kb < num_kb; ++kb) {
+        for (int kb = 0; kb < kbs; ++kb) {
           if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, args.status, args.limit_ns)) {
             *abort_flag = 1;
             break;
@@ -384,19 +255,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
           uint8_t* sA = smem + stage * C::STAGE_BYTES;
           uint8_t* sB = sA + C::A_BYTES;
           const uint32_t bar = leader_full + 8u * stage;
-          if constexpr (C::AMAJ == Major::K) {
-            tma_load_2d_pair(sA, &tmA, bar, kb * C::BK, a_row);
+          if (prob == 0) {
+            load_operand_pair<A0, C::BM_CTA>(sA, &tmA0, bar, a_row, kb * C::BK);
+            load_operand_pair<B0, C::BN_CTA>(sB, &tmB0, bar, b_row, kb * C::BK);
           } else {
-#pragma unroll
-            for (int q = 0; q < C::BM_CTA / 64; ++q)
-              tma_load_2d_pair(sA + q * 8192, &tmA, bar, a_row + 64 * q, kb * C::BK);
-          }
-          if constexpr (C::BMAJ == Major::K) {
-            tma_load_2d_pair(sB, &tmB, bar, kb * C::BK, b_row);
-          } else {
-#pragma unroll
-            for (int q = 0; q < C::BN_CTA / 64; ++q)
-              tma_load_2d_pair(sB + q * 8192, &tmB, bar, b_row + 64 * q, kb * C::BK);
+            load_operand_pair<A1, C::BM_CTA>(sA, &tmA1, bar, a_row, kb * C::BK);
+            load_operand_pair<B1, C::BN_CTA>(sB, &tmB1, bar, b_row, kb * C::BK);
           }
           ++arms;
           if (++stage == C::STAGES) {
@@ -422,14 +286,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
   } else if (warp == 1) {
     if (lane == 0 && leader) {
       // ------------------------------------------------------------ MMA issuer (leader only)
-      constexpr uint32_t idesc =
-          instr_desc_bf16_f32(C::BM, C::BN, C::AMAJ == Major::MN, C::BMAJ == Major::MN);
+      constexpr uint32_t idesc0 = instr_desc_bf16_f32(C::BM, C::BN, A0 == Major::MN, B0 == Major::MN);
+      constexpr uint32_t idesc1 = instr_desc_bf16_f32(C::BM, C::BN, A1 == Major::MN, B1 == Major::MN);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
       bool issued = false;
-      for (int t = pair; t < num_tiles && !*abort_flag; t += npairs) {
+      for (int i = 0; i < total && !*abort_flag; ++i) {
+        int prob, mb, nb, kbs;
+        tile_of(i, prob, mb, nb, kbs);
         if (!mbar_wait_bounded_cluster(&tempty[acc], acc_phase ^ 1u, args.status, args.limit_ns)) {
           *abort_flag = 1;
           break;
@@ -437,7 +303,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * C::BN);
         bool ok = true;
-        for (int kb = 0; kb < num_kb; ++kb) {
+        for (int kb = 0; kb < kbs; ++kb) {
           if (!mbar_wait_bounded(&full[stage], phase, args.status, args.limit_ns)) {
             *abort_flag = 1;
             ok = false;
@@ -446,10 +312,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
           tc_fence_after();
           const uint32_t a_base = smem_u32(smem + stage * C::STAGE_BYTES);
           const uint32_t b_base = a_base + C::A_BYTES;
+          if (prob == 0) {
 #pragma unroll
-          for (int k = 0; k < C::BK / 16; ++k) {
-            mma_bf16_ss_pair(d_tmem, operand_desc<C::AMAJ>(a_base, k),
-                             operand_desc<C::BMAJ>(b_base, k), idesc, (kb | k) != 0 ? 1u : 0u);
+            for (int k = 0; k < C::BK / 16; ++k)
+              mma_bf16_ss_pair(d_tmem, operand_desc<A0>(a_base, k), operand_desc<B0>(b_base, k),
+                               idesc0, (kb | k) != 0 ? 1u : 0u);
+          } else {
+#pragma unroll
+            for (int k = 0; k < C::BK / 16; ++k)
+              mma_bf16_ss_pair(d_tmem, operand_desc<A1>(a_base, k), operand_desc<B1>(b_base, k),
+                               idesc1, (kb | k) != 0 ? 1u : 0u);
           }
           issued = true;
           mma_commit_pair_both(&empty[stage]);
@@ -478,9 +350,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
     const int row_in_cta = quarter * 32 + lane;
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int t = pair; t < num_tiles && !*abort_flag; t += npairs) {
-      int mb, nb;
-      tile_coords(t, mb, nb);
+    for (int i = 0; i < total && !*abort_flag; ++i) {
+      int prob, mb, nb, kbs;
+      tile_of(i, prob, mb, nb, kbs);
       if (!mbar_wait_bounded(&tfull[acc], acc_phase, args.status, args.limit_ns)) {
         *abort_flag = 1;
         break;
@@ -488,9 +360,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
       tc_fence_after();
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
                              static_cast<uint32_t>(acc * C::BN + slab * C::COLS_PER_WARP);
-      Epi::template apply<C::COLS_PER_WARP>(
-          ep, mb * C::BM + static_cast<int>(rank) * C::BM_CTA + row_in_cta,
-          nb * C::BN + slab * C::COLS_PER_WARP, taddr, nb * C::COL_SPLIT + slab);
+      const int row = mb * C::BM + static_cast<int>(rank) * C::BM_CTA + row_in_cta;
+      const int col0 = nb * C::BN + slab * C::COLS_PER_WARP;
+      if (prob == 0)
+        E0::template apply<C::COLS_PER_WARP>(ep0, row, col0, taddr, nb * C::COL_SPLIT + slab);
+      else
+        E1::template apply<C::COLS_PER_WARP>(ep1, row, col0, taddr, nb * C::COL_SPLIT + slab);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(leader_tempty + 8u * acc);
