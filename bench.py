@@ -168,7 +168,7 @@ class ClockSampler:
             fd, self.path = tempfile.mkstemp(suffix=".csv")
             os.close(fd)
             cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                   "-lms", "100"]
+                   "-lms", "50"]
             if self.gpu_id:
                 cmd += ["-i", self.gpu_id]
             self.proc = subprocess.Popen(cmd, stdout=open(self.path, "w"),
@@ -283,6 +283,11 @@ def main_gpu(args):
         pass
     clocks = ClockSampler(gpu_id)
     clocks.start()
+    nvml = None
+    try:
+        nvml = NvmlSampler(dev).__enter__()
+    except Exception:
+        nvml = None
     flce.instrument(True)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
@@ -297,6 +302,10 @@ def main_gpu(args):
     kstats = flce.instrument_read()
     flce.instrument(False)
     clk = clocks.stop()
+    nvml_clk = None
+    if nvml is not None:
+        nvml.__exit__(None, None, None)
+        nvml_clk = nvml.summary()
     if world > 1:
         tt = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
         dist.all_reduce(tt, op=dist.ReduceOp.MAX)
@@ -376,7 +385,7 @@ def main_gpu(args):
     if dom and os.path.exists(tpath):
         tj = json.load(open(tpath))
         ent = tj.get(dom)
-        if ent and ent.get("kernel_rev") == KERNEL_REV and ent.get("config") == c.name:
+        if ent and ent.get("kernel_rev") == kernel_rev() and ent.get("config") == c.name:
             traffic = ent.get("bytes_per_launch")
     roofline = None
     if dom:
@@ -396,6 +405,8 @@ def main_gpu(args):
         cpu = cpu_baseline(inp, args.cpu_seconds)
 
     if rank == 0:
+        if roofline is not None:
+            roofline["kernel_rev"] = kernel_rev()
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
@@ -411,6 +422,8 @@ def main_gpu(args):
             "gpu_launches": kstats["launches_total"],
             "gpu_launches_per_step": kstats["launches_total"] / args.steps,
             "clocks": clk,
+            "clocks_nvml_10ms": nvml_clk,
+            "mcycles_per_step": (ms_per_step * nvml_clk["sm_mhz"] / 1e3) if nvml_clk else None,
             "peak_mem_MiB": {"fused_step": peak_fused / 2**20,
                              "workspace": ws.numel() / 2**20,
                              "unfused_torch": unfused["peak_MiB"] if unfused else None},
@@ -423,7 +436,15 @@ def main_gpu(args):
     return 0
 
 
-KERNEL_REV = "v1"
+def kernel_rev() -> str:
+    """Hash of the kernel sources; DRAM traffic recorded for another hash is stale."""
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "lm_head_linear_gemm_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".cuh")):
+            h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()[:16]
 
 
 def unfused_torch_baseline(X, W, t, c, args):
