@@ -236,7 +236,11 @@ def main_gpu(args):
             dist.barrier()
 
     cfg = synth.CONFIGS[args.config]
-    inp = synth.make_inputs(cfg, seed=cfg.seed + rank, N=args.rows or None)
+    fp8 = args.config == "fp8"
+    if fp8:
+        inp = synth.make_fp8_inputs(cfg, seed=cfg.seed + rank, N=args.rows or None)
+    else:
+        inp = synth.make_inputs(cfg, seed=cfg.seed + rank, N=args.rows or None)
     c = inp["cfg"]
     N, d, Vp, Vr = c.N, c.d, c.Vpad, c.Vreal
 
@@ -258,11 +262,22 @@ def main_gpu(args):
     ws = flce.alloc_workspace(shape, True, dev)
     stream = torch.cuda.current_stream()
 
+    if fp8:
+        X8 = torch.from_numpy(inp["X8"]).to(dev)
+        W8 = torch.from_numpy(inp["W8"]).to(dev)
+        sX = torch.tensor(float(inp["sX"]), dtype=torch.float32, device=dev)
+        sW = torch.tensor(float(inp["sW"]), dtype=torch.float32, device=dev)
+
     def step(Xd=None, td=None):
         Xd = X if Xd is None else Xd
         td = t if td is None else td
-        loss, lse, _, _, _ = flce.forward(Xd, W, td, Vr, c.cap, c.ignore_index, True, dX=dX,
-                                          dW=dW, workspace=ws, chunk_rows=args.chunk_rows)
+        if fp8:
+            loss, lse, _, _, _ = flce.forward_fp8(X8, W8, sX, sW, Xd, W, td, Vr, c.cap,
+                                                  c.ignore_index, True, dX=dX, dW=dW,
+                                                  workspace=ws, chunk_rows=args.chunk_rows)
+        else:
+            loss, lse, _, _, _ = flce.forward(Xd, W, td, Vr, c.cap, c.ignore_index, True, dX=dX,
+                                              dW=dW, workspace=ws, chunk_rows=args.chunk_rows)
         flce.backward(Xd, W, td, lse, Vr, c.cap, c.ignore_index, grad_out=g_one, dX=dX, dW=dW,
                       grads_precomputed=True)
         return loss
@@ -410,7 +425,8 @@ def main_gpu(args):
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "scaling": "weak", "vs_baseline": None,
+            "dtype": "e4m3 logits + bf16 gradients" if fp8 else "bf16", "data": "synthetic",
             "config": dict(workload_desc(c, shape.chunk_rows or min(N, 4096)),
                            parallelism=f"replicas x{world}" if world > 1 else "single GPU"),
             "tflops": tflops,

@@ -134,6 +134,32 @@ int flce_forward_noalloc(const flce_shape* shape, const void* X, const void* W,
                          const int64_t* targets, float* loss, float* lse, void* stream);
 
 /*
+ * Forward with FP8 logits: the logits contraction z = X W^T reads e4m3 operands with dynamic
+ * tensorwise scales (x ~ X8 * *scale_x, w ~ W8 * *scale_w; the scales are device scalars) on the
+ * tensor cores' fp8 path, with both scales applied to z before the softcap.  This follows the
+ * write-ups' FP8 training ("Increasing throughput": GEMMs in FP8 with dynamic tensorwise scaling
+ * through torch._scaled_mm, +25%); here only the logits contraction reads fp8.  With
+ * want_grads = 1 the softmax gradient is formed from those logits and the two gradient
+ * contractions use the bf16 copies X [N, d] and W [Vpad, d] (dX = dz W, dW = dz^T X), which may
+ * be NULL when want_grads = 0.
+ *   X8 [N, d], W8 [Vpad, d]: e4m3 bytes, row-major; d must be a multiple of 16.
+ * Outputs, workspace (flce_workspace_bytes of the same shape) and errors as flce_forward.
+ */
+int flce_forward_fp8(const flce_shape* shape, const void* X8, const void* W8,
+                     const float* scale_x, const float* scale_w, const void* X, const void* W,
+                     const int64_t* targets, float* loss, float* lse, int want_grads, void* dX,
+                     float* dW, int accumulate_dW, void* workspace, size_t workspace_bytes,
+                     void* stream);
+
+/*
+ * Dynamic tensorwise e4m3 quantisation of n bf16 values: *scale_out = amax(|src|) / 448
+ * (1 when all values are 0) and dst[i] = e4m3(src[i] / *scale_out), rounded to nearest even and
+ * saturated to the finite e4m3 range.  scale_out is a device float; it also serves as the
+ * amax accumulator while the call runs.  Four small kernels on `stream`.
+ */
+int flce_quantize_e4m3(const void* src, int64_t n, void* dst, float* scale_out, void* stream);
+
+/*
  * Reads the device status word (FLCE_DEV_* bits) and the number of rows in the loss from the
  * workspace of the last call on `stream`.  Synchronises that stream.  Either output may be
  * NULL.

@@ -6,13 +6,13 @@ arguments to it.  Entry points raise if the library is missing: there is no
 fallback implementation.
 """
 from ._abi import (DEV_BAD_TARGET, DEV_TIMEOUT, FlceError, alloc_workspace, backward,
-                   declared_functions, forward, instrument, instrument_read, lib, make_shape, raw_backward, raw_forward,
-                   raw_forward_noalloc, read_status, status_string, workspace_bytes)
+                   declared_functions, forward, forward_fp8, instrument, instrument_read, lib, make_shape, raw_backward, raw_forward,
+                   quantize_e4m3, raw_forward_noalloc, read_status, status_string, workspace_bytes)
 from .autograd import FusedLinearCrossEntropy, fused_linear_cross_entropy
 
 __all__ = [
     "DEV_BAD_TARGET", "DEV_TIMEOUT", "FlceError", "alloc_workspace", "backward",
-    "declared_functions", "forward", "instrument", "instrument_read", "lib", "make_shape", "raw_backward", "raw_forward",
-    "raw_forward_noalloc", "read_status", "status_string", "workspace_bytes", "FusedLinearCrossEntropy",
+    "declared_functions", "forward", "forward_fp8", "instrument", "instrument_read", "lib", "make_shape", "raw_backward", "raw_forward",
+    "quantize_e4m3", "raw_forward_noalloc", "read_status", "status_string", "workspace_bytes", "FusedLinearCrossEntropy",
     "fused_linear_cross_entropy",
 ]

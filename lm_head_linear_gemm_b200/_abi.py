@@ -56,7 +56,7 @@ def declared_functions(header: str = HEADER_PATH) -> list[str]:
     """Names of the functions include/flce.h declares."""
     text = open(header).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(flce_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(flce_[a-z0-9_]+)\s*\(", text)))
 
 
 def lib() -> ctypes.CDLL:
@@ -81,6 +81,11 @@ def lib() -> ctypes.CDLL:
     L.flce_read_status.argtypes = [P, ctypes.POINTER(ctypes.c_uint32),
                                    ctypes.POINTER(ctypes.c_int64), P]
     L.flce_read_status.restype = ctypes.c_int
+    L.flce_forward_fp8.argtypes = [shp, P, P, P, P, P, P, P, P, P, ctypes.c_int, P, P,
+                                   ctypes.c_int, P, ctypes.c_size_t, P]
+    L.flce_forward_fp8.restype = ctypes.c_int
+    L.flce_quantize_e4m3.argtypes = [P, ctypes.c_int64, P, P, P]
+    L.flce_quantize_e4m3.restype = ctypes.c_int
     L.flce_forward_noalloc.argtypes = [shp, P, P, P, P, P, P]
     L.flce_forward_noalloc.restype = ctypes.c_int
     L.flce_instrument.argtypes = [ctypes.c_int]
@@ -223,6 +228,57 @@ def forward(X, W, targets, Vreal: int, cap: float = 15.0, ignore_index: int = -1
                      workspace.numel(), _stream(stream))
     if rc != FLCE_OK:
         raise FlceError(rc, "flce_forward")
+    return loss, lse, (dX if want_grads else None), (dW if want_grads else None), workspace
+
+
+def quantize_e4m3(x, out=None, scale=None, stream=None):
+    """Tensorwise e4m3 quantisation of a bf16 CUDA tensor: returns (uint8 codes, fp32 scale)
+    with x ~ codes.view(float8_e4m3fn) * scale."""
+    import torch
+    if not x.is_cuda or x.dtype != torch.bfloat16 or not x.is_contiguous():
+        raise TypeError("x must be a contiguous bf16 CUDA tensor")
+    if out is None:
+        out = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    if scale is None:
+        scale = torch.empty((), dtype=torch.float32, device=x.device)
+    rc = lib().flce_quantize_e4m3(_ptr(x), x.numel(), _ptr(out), _ptr(scale), _stream(stream))
+    if rc != FLCE_OK:
+        raise FlceError(rc, "flce_quantize_e4m3")
+    return out, scale
+
+
+def forward_fp8(X8, W8, scale_x, scale_w, X, W, targets, Vreal: int, cap: float = 15.0,
+                ignore_index: int = -1, want_grads: bool = False, dX=None, dW=None,
+                accumulate_dW: bool = False, workspace=None, chunk_rows: int = 0, stream=None):
+    """Fused forward with e4m3 logits operands (uint8 codes + fp32 device scales) and bf16
+    copies X/W for the gradient contractions.  Returns (loss, lse, dX, dW, workspace)."""
+    import torch
+    for name, t in (("X8", X8), ("W8", W8)):
+        if not t.is_cuda or t.dtype not in (torch.uint8, getattr(torch, "float8_e4m3fn", None)):
+            raise TypeError(f"{name} must be a CUDA uint8 / float8_e4m3fn tensor")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    N, d = X8.shape
+    shape = make_shape(N, d, W8.shape[0], Vreal, cap, ignore_index, chunk_rows)
+    dev = X8.device
+    loss = torch.empty((), dtype=torch.float32, device=dev)
+    lse = torch.empty(max(N, 1), dtype=torch.float32, device=dev)[:N]
+    if want_grads:
+        _check(X, W, targets)
+        if dX is None:
+            dX = torch.empty_like(X)
+        if dW is None:
+            dW = torch.empty(W.shape, dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = alloc_workspace(shape, want_grads, dev)
+    rc = lib().flce_forward_fp8(ctypes.byref(shape), _ptr(X8), _ptr(W8), _ptr(scale_x),
+                                _ptr(scale_w), _ptr(X), _ptr(W), _ptr(targets), _ptr(loss),
+                                _ptr(lse), 1 if want_grads else 0,
+                                _ptr(dX) if want_grads else None,
+                                _ptr(dW) if want_grads else None, int(accumulate_dW),
+                                _ptr(workspace), workspace.numel(), _stream(stream))
+    if rc != FLCE_OK:
+        raise FlceError(rc, "flce_forward_fp8")
     return loss, lse, (dX if want_grads else None), (dW if want_grads else None), workspace
 
 

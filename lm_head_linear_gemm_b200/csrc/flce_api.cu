@@ -33,6 +33,10 @@ using Cfg = PairCfg<256, 6, 8>;
 // logits: A = X (K-major), B = W (K-major)
 constexpr auto kLogitsKernel =
     gemm_pair_kernel<Cfg, LogitsEpi, LogitsEpi, Major::K, Major::K, Major::K, Major::K>;
+// logits from e4m3 operands (kind::f8f6f4, tensorwise scales applied in the epilogue)
+using Cfg8 = PairCfg<256, 6, 8, 1>;
+constexpr auto kLogitsKernel8 =
+    gemm_pair_kernel<Cfg8, LogitsEpi, LogitsEpi, Major::K, Major::K, Major::K, Major::K>;
 // gradients in one launch: dX = A' W (A' K-major, W MN-major), dW = A'^T Xs (both MN-major)
 constexpr auto kGradKernel =
     gemm_pair_kernel<Cfg, DxEpi, DwEpi, Major::K, Major::MN, Major::MN, Major::MN>;
@@ -126,7 +130,9 @@ int device_info(DeviceInfo** out) {
     if (cudaFuncSetAttribute(kLogitsKernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              Cfg::SMEM_BYTES) != cudaSuccess ||
         cudaFuncSetAttribute(kGradKernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             Cfg::SMEM_BYTES) != cudaSuccess)
+                             Cfg::SMEM_BYTES) != cudaSuccess ||
+        cudaFuncSetAttribute(kLogitsKernel8, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Cfg8::SMEM_BYTES) != cudaSuccess)
       return FLCE_ERR_CUDA;
     di.attrs_set = true;
   }
@@ -154,17 +160,20 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// bf16 matrix [outer][inner] (row-major, row stride `ld` elements), 128-byte swizzled boxes of
-// {64 inner elements, box_outer rows}.  Out-of-range box elements read as zero.
+// Matrix [outer][inner] of bf16 (elem_bytes 2) or e4m3 (elem_bytes 1, described as bytes),
+// row-major with row stride `ld` elements, in 128-byte swizzled boxes of {128 bytes of inner
+// elements, box_outer rows}.  Out-of-range box elements read as zero.
 int make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t ld,
-             uint32_t box_outer) {
+             uint32_t box_outer, int elem_bytes = 2) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return FLCE_ERR_CUDA;
   const cuuint64_t dims[2] = {inner, outer};
-  const cuuint64_t strides[1] = {ld * 2};
-  const cuuint32_t box[2] = {64, box_outer};
+  const cuuint64_t strides[1] = {ld * static_cast<uint64_t>(elem_bytes)};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / elem_bytes), box_outer};
   const cuuint32_t estr[2] = {1, 1};
-  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+  const CUtensorMapDataType dt =
+      elem_bytes == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const CUresult r = fn(m, dt, 2, const_cast<void*>(base), dims,
                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -208,7 +217,7 @@ long long pair_tiles(const PairProblem& p) {
 
 // Launch one persistent pair kernel over one or two problems; `kind` labels the launch for the
 // instrumentation counters (0: logits, 1: dX + dW).
-template <class E0, class E1, class K>
+template <class E0, class E1, class CF = Cfg, class K>
 int launch_pair(K kernel, const DeviceInfo* di, const CUtensorMap& a0, const CUtensorMap& b0,
                 const CUtensorMap& a1, const CUtensorMap& b1, const PairProblem& p0,
                 const PairProblem& p1, uint32_t* status, const typename E0::Params& e0,
@@ -226,7 +235,7 @@ int launch_pair(K kernel, const DeviceInfo* di, const CUtensorMap& a0, const CUt
     ev1 = pooled_event();
     if (ev0 != nullptr) cudaEventRecord(ev0, st);
   }
-  kernel<<<grid, Cfg::THREADS, Cfg::SMEM_BYTES, st>>>(a0, b0, a1, b1, args, e0, e1);
+  kernel<<<grid, CF::THREADS, CF::SMEM_BYTES, st>>>(a0, b0, a1, b1, args, e0, e1);
   const bool ok = cudaGetLastError() == cudaSuccess;
   count_launch();
   if (timed && ev0 != nullptr && ev1 != nullptr) {
@@ -252,8 +261,18 @@ int launch_ok() {
   return cudaGetLastError() == cudaSuccess ? FLCE_OK : FLCE_ERR_CUDA;
 }
 
+// Operands of the logits contraction when they are e4m3 (otherwise the bf16 X and W are used):
+// x ~ X8 * (*scale_x), w ~ W8 * (*scale_w).
+struct Fp8Logits {
+  const uint8_t* X8 = nullptr;
+  const uint8_t* W8 = nullptr;
+  const float* scale_x = nullptr;
+  const float* scale_w = nullptr;
+};
+
 struct Ctx {
   const flce_shape* s;
+  Fp8Logits fp8;
   Layout L;
   uint8_t* ws;
   DevHeader* hdr;
@@ -264,6 +283,29 @@ struct Ctx {
     return reinterpret_cast<T*>(ws + off);
   }
 };
+
+// Logits contraction of rows [row0, row0 + rows) with the given epilogue parameters, from the
+// bf16 X/W or, when the context carries them, from the e4m3 operands.
+int launch_logits(const Ctx& c, int64_t row0, int rows, const __nv_bfloat16* X,
+                  const __nv_bfloat16* W, LogitsParams lp) {
+  const flce_shape* s = c.s;
+  const int d = static_cast<int>(s->d), Vpad = static_cast<int>(s->Vpad);
+  const PairProblem logits{rows, Vpad, d, 1}, none{0, 0, 0, 0};
+  CUtensorMap mX, mW;
+  if (c.fp8.X8 != nullptr) {
+    FLCE_TRY(make_map(&mX, c.fp8.X8 + row0 * s->d, d, rows, d, Cfg8::BM_CTA, 1));
+    FLCE_TRY(make_map(&mW, c.fp8.W8, d, Vpad, d, Cfg8::BN_CTA, 1));
+    lp.scale_a = c.fp8.scale_x;
+    lp.scale_b = c.fp8.scale_w;
+    return launch_pair<LogitsEpi, LogitsEpi, Cfg8>(kLogitsKernel8, c.di, mX, mW, mX, mW, logits,
+                                                    none, &c.hdr->status, lp, lp, c.st, 0);
+  }
+  FLCE_TRY(make_map(&mX, X + row0 * s->d, d, rows, d, Cfg::BM_CTA));
+  FLCE_TRY(make_map(&mW, W, d, Vpad, d, Cfg::BN_CTA));
+  lp.scale_a = lp.scale_b = nullptr;
+  return launch_pair<LogitsEpi, LogitsEpi>(kLogitsKernel, c.di, mX, mW, mX, mW, logits, none,
+                                           &c.hdr->status, lp, lp, c.st, 0);
+}
 
 // One chunk of the gradient path: logits GEMM (mode FUSED or RECOMPUTE), row finish, dX, dW.
 int grad_chunk(const Ctx& c, int64_t row0, int rows, const __nv_bfloat16* X,
@@ -276,9 +318,7 @@ int grad_chunk(const Ctx& c, int64_t row0, int rows, const __nv_bfloat16* X,
   __nv_bfloat16* Xs = c.at<__nv_bfloat16>(c.L.Xs);
   float* r = c.at<float>(c.L.r);
 
-  CUtensorMap mX, mW, mA_k, mW_mn, mA_mn, mXs_mn;
-  FLCE_TRY(make_map(&mX, Xc, d, rows, d, Cfg::BM_CTA));
-  FLCE_TRY(make_map(&mW, W, d, Vpad, d, Cfg::BN_CTA));
+  CUtensorMap mA_k, mW_mn, mA_mn, mXs_mn;
   FLCE_TRY(make_map(&mA_k, Abuf, Vpad, rows, Vpad, Cfg::BM_CTA));
   FLCE_TRY(make_map(&mW_mn, W, d, Vpad, d, 64));
   FLCE_TRY(make_map(&mA_mn, Abuf, Vpad, rows, Vpad, 64));
@@ -301,9 +341,7 @@ int grad_chunk(const Ctx& c, int64_t row0, int rows, const __nv_bfloat16* X,
   lp.der_t = c.at<float>(c.L.der_t) + row0;
   lp.e_t = c.at<float>(c.L.e_t) + row0;
   lp.A = Abuf;
-  const PairProblem logits{rows, Vpad, d, 1}, none{0, 0, 0, 0};
-  FLCE_TRY((launch_pair<LogitsEpi, LogitsEpi>(kLogitsKernel, c.di, mX, mW, mX, mW, logits, none,
-                                               &c.hdr->status, lp, lp, c.st, 0)));
+  FLCE_TRY(launch_logits(c, row0, rows, X, W, lp));
 
   RowFinishParams rp{};
   rp.rows = rows;
@@ -344,12 +382,8 @@ int grad_chunk(const Ctx& c, int64_t row0, int rows, const __nv_bfloat16* X,
 int stats_pass(const Ctx& c, const __nv_bfloat16* X, const __nv_bfloat16* W, float* lse) {
   const flce_shape* s = c.s;
   const int d = static_cast<int>(s->d), Vpad = static_cast<int>(s->Vpad);
-  CUtensorMap mW;
-  FLCE_TRY(make_map(&mW, W, d, Vpad, d, Cfg::BN_CTA));
   for (int64_t row0 = 0; row0 < s->N; row0 += c.L.chunk) {
     const int rows = static_cast<int>(s->N - row0 < c.L.chunk ? s->N - row0 : c.L.chunk);
-    CUtensorMap mX;
-    FLCE_TRY(make_map(&mX, X + row0 * s->d, d, rows, d, Cfg::BM_CTA));
     LogitsParams lp{};
     lp.rows = rows;
     lp.Vreal = static_cast<int>(s->Vreal);
@@ -365,9 +399,7 @@ int stats_pass(const Ctx& c, const __nv_bfloat16* X, const __nv_bfloat16* W, flo
     lp.s_t = c.at<float>(c.L.s_t) + row0;
     lp.der_t = c.at<float>(c.L.der_t) + row0;
     lp.e_t = c.at<float>(c.L.e_t) + row0;
-    const PairProblem logits{rows, Vpad, d, 1}, none{0, 0, 0, 0};
-    FLCE_TRY((launch_pair<LogitsEpi, LogitsEpi>(kLogitsKernel, c.di, mX, mW, mX, mW, logits, none,
-                                                 &c.hdr->status, lp, lp, c.st, 0)));
+    FLCE_TRY(launch_logits(c, row0, rows, X, W, lp));
     RowFinishParams rp{};
     rp.rows = rows;
     rp.d = d;
@@ -440,20 +472,13 @@ int noalloc_scratch_address(void** out) {
   return FLCE_OK;
 }
 
-}  // namespace
-
-extern "C" {
-
-size_t flce_workspace_bytes(const flce_shape* shape, int want_grads) {
-  if (!shape_ok(shape)) return 0;
-  return make_layout(shape, want_grads ? 1 : 0).total;
-}
-
-int flce_forward(const flce_shape* s, const void* X, const void* W, const int64_t* targets,
-                 float* loss, float* lse, int want_grads, void* dX, float* dW, int accumulate_dW,
-                 void* workspace, size_t workspace_bytes, void* stream) {
+// Forward (and, with want_grads, the gradients of the mean loss) from bf16 X/W, or from e4m3
+// operands for the logits when fp8.X8 is set (X/W then only feed the gradient contractions).
+int forward_impl(const flce_shape* s, const void* X, const void* W, const Fp8Logits& fp8,
+                 const int64_t* targets, float* loss, float* lse, int want_grads, void* dX,
+                 float* dW, int accumulate_dW, void* workspace, size_t workspace_bytes,
+                 void* stream) {
   want_grads = want_grads ? 1 : 0;
-  FLCE_TRY(common_checks(s, X, W, targets, workspace, workspace_bytes, want_grads));
   if (loss == nullptr || (s->N > 0 && lse == nullptr)) return FLCE_ERR_ARG;
   if (!aligned16(loss) || !aligned16(lse)) return FLCE_ERR_ALIGN;
   if (want_grads) {
@@ -462,8 +487,13 @@ int flce_forward(const flce_shape* s, const void* X, const void* W, const int64_
   }
   DeviceInfo* di = nullptr;
   FLCE_TRY(device_info(&di));
-  Ctx c{s, make_layout(s, want_grads), static_cast<uint8_t*>(workspace), nullptr, di,
-        static_cast<cudaStream_t>(stream)};
+  Ctx c{};
+  c.s = s;
+  c.fp8 = fp8;
+  c.L = make_layout(s, want_grads);
+  c.ws = static_cast<uint8_t*>(workspace);
+  c.di = di;
+  c.st = static_cast<cudaStream_t>(stream);
   c.hdr = c.at<DevHeader>(c.L.hdr);
   const auto* Xb = static_cast<const __nv_bfloat16*>(X);
   const auto* Wb = static_cast<const __nv_bfloat16*>(W);
@@ -501,6 +531,70 @@ int flce_forward(const flce_shape* s, const void* X, const void* W, const int64_
   return FLCE_OK;
 }
 
+}  // namespace
+
+extern "C" {
+
+size_t flce_workspace_bytes(const flce_shape* shape, int want_grads) {
+  if (!shape_ok(shape)) return 0;
+  return make_layout(shape, want_grads ? 1 : 0).total;
+}
+
+int flce_forward(const flce_shape* s, const void* X, const void* W, const int64_t* targets,
+                 float* loss, float* lse, int want_grads, void* dX, float* dW, int accumulate_dW,
+                 void* workspace, size_t workspace_bytes, void* stream) {
+  FLCE_TRY(common_checks(s, X, W, targets, workspace, workspace_bytes, want_grads ? 1 : 0));
+  return forward_impl(s, X, W, Fp8Logits{}, targets, loss, lse, want_grads, dX, dW,
+                      accumulate_dW, workspace, workspace_bytes, stream);
+}
+
+int flce_forward_fp8(const flce_shape* s, const void* X8, const void* W8, const float* scale_x,
+                     const float* scale_w, const void* X, const void* W, const int64_t* targets,
+                     float* loss, float* lse, int want_grads, void* dX, float* dW,
+                     int accumulate_dW, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!shape_ok(s)) return FLCE_ERR_ARG;
+  if ((s->d % 16) != 0 || (s->Vpad % 8) != 0) return FLCE_ERR_ALIGN;  // 16-byte e4m3 rows
+  if ((s->N > 0 && (X8 == nullptr || targets == nullptr)) || W8 == nullptr ||
+      scale_x == nullptr || scale_w == nullptr || workspace == nullptr)
+    return FLCE_ERR_ARG;
+  if (want_grads && ((s->N > 0 && X == nullptr) || W == nullptr)) return FLCE_ERR_ARG;
+  if (!aligned16(X8) || !aligned16(W8) || !aligned16(X) || !aligned16(W) || !aligned16(targets) ||
+      (reinterpret_cast<uintptr_t>(scale_x) & 3u) != 0 ||
+      (reinterpret_cast<uintptr_t>(scale_w) & 3u) != 0 ||
+      (reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0)
+    return FLCE_ERR_ALIGN;
+  if (workspace_bytes < make_layout(s, want_grads ? 1 : 0).total) return FLCE_ERR_WORKSPACE;
+  Fp8Logits fp8;
+  fp8.X8 = static_cast<const uint8_t*>(X8);
+  fp8.W8 = static_cast<const uint8_t*>(W8);
+  fp8.scale_x = scale_x;
+  fp8.scale_w = scale_w;
+  return forward_impl(s, X, W, fp8, targets, loss, lse, want_grads, dX, dW, accumulate_dW,
+                      workspace, workspace_bytes, stream);
+}
+
+int flce_quantize_e4m3(const void* src, int64_t n, void* dst, float* scale_out, void* stream) {
+  if (n < 0 || (n > 0 && (src == nullptr || dst == nullptr)) || scale_out == nullptr)
+    return FLCE_ERR_ARG;
+  if ((reinterpret_cast<uintptr_t>(scale_out) & 3u) != 0) return FLCE_ERR_ALIGN;
+  DeviceInfo* di = nullptr;
+  FLCE_TRY(device_info(&di));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t* amax_bits = reinterpret_cast<uint32_t*>(scale_out);
+  const int grid = 4 * di->sms;
+  zero_u32_kernel<<<1, 1, 0, st>>>(amax_bits);
+  FLCE_TRY(launch_ok());
+  if (n > 0) {
+    amax_bf16_kernel<<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(src), n, amax_bits);
+    FLCE_TRY(launch_ok());
+    quantize_e4m3_kernel<<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(src), n,
+                                                 static_cast<uint8_t*>(dst), amax_bits);
+    FLCE_TRY(launch_ok());
+  }
+  finish_scale_kernel<<<1, 1, 0, st>>>(amax_bits);
+  return launch_ok();
+}
+
 int flce_backward(const flce_shape* s, const void* X, const void* W, const int64_t* targets,
                   const float* lse, const float* grad_out, void* dX, float* dW, int accumulate_dW,
                   int grads_precomputed, void* workspace, size_t workspace_bytes, void* stream) {
@@ -524,8 +618,12 @@ int flce_backward(const flce_shape* s, const void* X, const void* W, const int64
   if (!aligned16(lse)) return FLCE_ERR_ALIGN;
   DeviceInfo* di = nullptr;
   FLCE_TRY(device_info(&di));
-  Ctx c{s, make_layout(s, 1), static_cast<uint8_t*>(workspace), nullptr, di,
-        static_cast<cudaStream_t>(stream)};
+  Ctx c{};
+  c.s = s;
+  c.L = make_layout(s, 1);
+  c.ws = static_cast<uint8_t*>(workspace);
+  c.di = di;
+  c.st = static_cast<cudaStream_t>(stream);
   c.hdr = c.at<DevHeader>(c.L.hdr);
   prep_targets_kernel<<<1, 1024, 0, c.st>>>(reinterpret_cast<const long long*>(targets), s->N,
                                             s->Vreal, s->ignore_index, c.at<int>(c.L.tgt), c.hdr);

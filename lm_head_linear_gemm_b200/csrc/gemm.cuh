@@ -38,7 +38,8 @@ __device__ __forceinline__ void load_operand_pair(uint8_t* dst, const CUtensorMa
   }
 }
 
-// Descriptor of the k-th 16-deep slice of a staged operand tile.
+// Descriptor of the k-th MMA slice of a staged operand tile (32 bytes of K: 16 bf16 or 32 e4m3
+// elements; MN-major slices are bf16 only: 16 K rows = two 1 KB swizzle atoms).
 template <Major MAJ>
 __device__ __forceinline__ uint64_t operand_desc(uint32_t base, int k) {
   if constexpr (MAJ == Major::K) {
@@ -62,19 +63,21 @@ __device__ __forceinline__ uint64_t operand_desc(uint32_t base, int k) {
 // length by 12x): each pair first takes its round-robin share of problem 0's tiles, then a
 // contiguous run of problem 1's tiles sized so that every pair ends with about the same number
 // of k-blocks.  A launch with one problem is the plain round-robin persistent schedule.
-template <int BN_, int STAGES_, int EPI_WARPS_>
+template <int BN_, int STAGES_, int EPI_WARPS_, int ELEM_BYTES_ = 2>
 struct PairCfg {
   static constexpr bool PAIR = true;
+  static constexpr int ELEM_BYTES = ELEM_BYTES_;  // 2: bf16 (kind::f16), 1: e4m3 (kind::f8f6f4)
   static constexpr int BM = 256;         // rows per pair tile
   static constexpr int BM_CTA = 128;     // rows per CTA (one TMEM lane each)
   static constexpr int BN = BN_;         // columns per pair tile
   static constexpr int BN_CTA = BN_ / 2; // B rows staged by each CTA
-  static constexpr int BK = 64;
+  static constexpr int BK = 128 / ELEM_BYTES;  // one 128-byte swizzle row of K per k-block
+  static constexpr int MMA_K = 32 / ELEM_BYTES; // K per tcgen05.mma: 32 bytes of each row
   static constexpr int STAGES = STAGES_;
   static constexpr int EPI_WARPS = EPI_WARPS_;
   static constexpr int THREADS = 64 + 32 * EPI_WARPS;
-  static constexpr int A_BYTES = BM_CTA * BK * 2;
-  static constexpr int B_BYTES = BN_CTA * BK * 2;
+  static constexpr int A_BYTES = BM_CTA * 128;
+  static constexpr int B_BYTES = BN_CTA * 128;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int TMEM_COLS = (2 * BN <= 256) ? 256 : 512;
   static constexpr int COL_SPLIT = EPI_WARPS / 4;
@@ -286,8 +289,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
   } else if (warp == 1) {
     if (lane == 0 && leader) {
       // ------------------------------------------------------------ MMA issuer (leader only)
-      constexpr uint32_t idesc0 = instr_desc_bf16_f32(C::BM, C::BN, A0 == Major::MN, B0 == Major::MN);
-      constexpr uint32_t idesc1 = instr_desc_bf16_f32(C::BM, C::BN, A1 == Major::MN, B1 == Major::MN);
+      static_assert(C::ELEM_BYTES == 2 || (A0 == Major::K && B0 == Major::K && A1 == Major::K &&
+                                           B1 == Major::K),
+                    "e4m3 operands are staged K-major");
+      constexpr uint32_t idesc0 =
+          C::ELEM_BYTES == 1 ? instr_desc_e4m3_f32(C::BM, C::BN)
+                             : instr_desc_bf16_f32(C::BM, C::BN, A0 == Major::MN, B0 == Major::MN);
+      constexpr uint32_t idesc1 =
+          C::ELEM_BYTES == 1 ? instr_desc_e4m3_f32(C::BM, C::BN)
+                             : instr_desc_bf16_f32(C::BM, C::BN, A1 == Major::MN, B1 == Major::MN);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
@@ -312,14 +322,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
           tc_fence_after();
           const uint32_t a_base = smem_u32(smem + stage * C::STAGE_BYTES);
           const uint32_t b_base = a_base + C::A_BYTES;
-          if (prob == 0) {
+          if constexpr (C::ELEM_BYTES == 1) {
 #pragma unroll
-            for (int k = 0; k < C::BK / 16; ++k)
+            for (int k = 0; k < C::BK / C::MMA_K; ++k)
+              mma_e4m3_ss_pair(d_tmem, operand_desc<Major::K>(a_base, k),
+                               operand_desc<Major::K>(b_base, k), prob == 0 ? idesc0 : idesc1,
+                               (kb | k) != 0 ? 1u : 0u);
+          } else if (prob == 0) {
+#pragma unroll
+            for (int k = 0; k < C::BK / C::MMA_K; ++k)
               mma_bf16_ss_pair(d_tmem, operand_desc<A0>(a_base, k), operand_desc<B0>(b_base, k),
                                idesc0, (kb | k) != 0 ? 1u : 0u);
           } else {
 #pragma unroll
-            for (int k = 0; k < C::BK / 16; ++k)
+            for (int k = 0; k < C::BK / C::MMA_K; ++k)
               mma_bf16_ss_pair(d_tmem, operand_desc<A1>(a_base, k), operand_desc<B1>(b_base, k),
                                idesc1, (kb | k) != 0 ? 1u : 0u);
           }
@@ -438,6 +454,8 @@ struct LogitsParams {
   float cap;                 // > 0: softcap value; <= 0: no softcap
   float k_u;                 // 2/cap * log2(e)
   float m2c_log2e;           // -2 cap log2(e)
+  const float* scale_a;      // e4m3 operands: z = acc * (*scale_a) * (*scale_b); null for bf16
+  const float* scale_b;
   const int* tgt;            // [rows] target id, -1 when the row is not in the loss
   const float* ref;          // [rows] exp reference (lse) when !fixed_ref and mode == RECOMPUTE
   float* partial;            // [rows][n_slabs] sum-exp (pairs (max, sum-exp) when !fixed_ref)
@@ -459,6 +477,10 @@ struct LogitsEpi {
     const int t = row_ok ? __ldg(p.tgt + row) : -1;
     const bool capped = p.cap > 0.f;
     const bool write_a = p.mode != LOGITS_STATS;
+    // Tensorwise scales of e4m3 operands: folded into the exp2 argument on the fixed-reference
+    // path (only |z| and the sign of z are used there), applied to z elsewhere.
+    const float zs = p.scale_a != nullptr ? __ldg(p.scale_a) * __ldg(p.scale_b) : 1.0f;
+    const float k_u = p.k_u * zs;
     const bool online = !p.fixed_ref && p.mode == LOGITS_STATS;
     const float ref = p.fixed_ref ? p.cap
                                   : ((p.mode == LOGITS_RECOMPUTE && row_ok) ? __ldg(p.ref + row) : 0.f);
@@ -479,7 +501,7 @@ struct LogitsEpi {
 #pragma unroll
           for (int k = 0; k < 32; ++k)
             if (k == t - cbase) zt = v[k];
-          const Softcapped sc = softcap_fixed_ref(zt, p.k_u, p.m2c_log2e, p.cap);
+          const Softcapped sc = softcap_fixed_ref(zt, k_u, p.m2c_log2e, p.cap);
           tv_s = sc.s;
           tv_der = sc.der;
           tv_e = sc.e;
@@ -488,14 +510,14 @@ struct LogitsEpi {
         if (cbase + 32 <= p.Vreal) {
 #pragma unroll
           for (int k = 0; k < 32; ++k) {
-            const Softcapped sc = softcap_fixed_ref(v[k], p.k_u, p.m2c_log2e, p.cap);
+            const Softcapped sc = softcap_fixed_ref(v[k], k_u, p.m2c_log2e, p.cap);
             sum += sc.e;
             v[k] = sc.e * sc.der;
           }
         } else {                                            // last vocabulary tile: padded columns
 #pragma unroll
           for (int k = 0; k < 32; ++k) {
-            const Softcapped sc = softcap_fixed_ref(v[k], p.k_u, p.m2c_log2e, p.cap);
+            const Softcapped sc = softcap_fixed_ref(v[k], k_u, p.m2c_log2e, p.cap);
             const float e = cbase + k < p.Vreal ? sc.e : 0.f;
             sum += e;
             v[k] = e * sc.der;
@@ -505,6 +527,7 @@ struct LogitsEpi {
         float der[32];
 #pragma unroll
         for (int k = 0; k < 32; ++k) {
+          v[k] *= zs;
           if (capped) {
             const float z = v[k];
             const float u = ex2_approx(-fabsf(z) * p.k_u);

@@ -3,6 +3,8 @@
 // and the upstream-gradient scaling.  All reductions run in a fixed order, so
 // results are bitwise reproducible.
 #pragma once
+#include <cuda_fp8.h>
+
 #include "sm100.cuh"
 
 namespace flce {
@@ -193,6 +195,40 @@ __global__ void scale_grads_kernel(__nv_bfloat16* __restrict__ dX, long long nX8
       reinterpret_cast<float4*>(dW)[i] = v;
     }
   }
+}
+
+// ---------------------------------------------------------------- tensorwise e4m3 quantisation
+// scale = amax(|x|) / 448 (448 = largest finite e4m3), q = e4m3(x / scale) rounded to nearest
+// even and saturated to the finite range.  The amax is kept as the bit pattern of a
+// non-negative float in the scale slot (bit order = value order), then turned into the scale.
+__global__ void zero_u32_kernel(uint32_t* p) { *p = 0u; }
+
+__global__ void amax_bf16_kernel(const __nv_bfloat16* __restrict__ x, long long n,
+                                 uint32_t* __restrict__ amax_bits) {
+  float m = 0.f;
+  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
+       i += stride)
+    m = fmaxf(m, fabsf(__bfloat162float(x[i])));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((threadIdx.x & 31) == 0) atomicMax(amax_bits, __float_as_uint(m));
+}
+
+__global__ void quantize_e4m3_kernel(const __nv_bfloat16* __restrict__ x, long long n,
+                                     uint8_t* __restrict__ q, const uint32_t* __restrict__ amax_bits) {
+  const float amax = __uint_as_float(*amax_bits);
+  const float scale = amax > 0.f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n;
+       i += stride)
+    q[i] = static_cast<uint8_t>(
+        __nv_cvt_float_to_fp8(__fdiv_rn(__bfloat162float(x[i]), scale), __NV_SATFINITE, __NV_E4M3));
+}
+
+__global__ void finish_scale_kernel(uint32_t* amax_bits) {
+  const float amax = __uint_as_float(*amax_bits);
+  *reinterpret_cast<float*>(amax_bits) = amax > 0.f ? __fdiv_rn(amax, 448.0f) : 1.0f;
 }
 
 // Writes loss = 0 (used for N = 0, where nothing else runs).

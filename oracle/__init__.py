@@ -22,6 +22,9 @@ inputs (the GPU path reads the same bf16 values):
   is the reading adopted; with no valid row the loss is 0);
 * analytic gradients ``dX = dz W`` and ``dW = dz^T X`` with
   ``dz = g/Nv * (softmax(s) - onehot(t)) * (1 - tanh^2(z/cap))``.
+* FP8 variant (the write-ups train with FP8 GEMMs under dynamic tensorwise scaling,
+  "Increasing throughput"): the logits come from the e4m3 operands times their scales while
+  the two gradient products use the bf16 copies -- ``backward(..., Xg=, Wg=)``.
 
 The fused method (the lm_head matmul computed chunk by chunk inside the loss so
 the ``(B*T, vocab)`` logits are never materialised -- "Increasing throughput",
@@ -133,10 +136,15 @@ def row_dlogits(X, W, t, lse, Vreal: int, cap: float, ignore_index: int, n_valid
 
 
 def backward(X, W, t, Vreal: int, cap: float, ignore_index: int, g: float = 1.0, lse=None,
-             block_rows: int = 1024):
-    """Gradients of ``g * loss``: ``dX = dz W`` [N, d] and ``dW = dz^T X`` [Vpad, d]."""
+             block_rows: int = 1024, Xg=None, Wg=None):
+    """Gradients of ``g * loss``: ``dX = dz W`` [N, d] and ``dW = dz^T X`` [Vpad, d].
+
+    ``Xg`` / ``Wg`` (default X / W) are the operands of the two gradient products; the logits
+    and hence ``dz`` always come from X and W."""
     X = np.asarray(X, np.float64)
     W = np.asarray(W, np.float64)
+    Xg = X if Xg is None else np.asarray(Xg, np.float64)
+    Wg = W if Wg is None else np.asarray(Wg, np.float64)
     N = X.shape[0]
     valid, _ = valid_rows(t, Vreal, ignore_index)
     nv = int(np.count_nonzero(valid))
@@ -147,27 +155,29 @@ def backward(X, W, t, Vreal: int, cap: float, ignore_index: int, g: float = 1.0,
     for r0 in range(0, N, block_rows):
         r1 = min(N, r0 + block_rows)
         dz = row_dlogits(X[r0:r1], W, t[r0:r1], lse[r0:r1], Vreal, cap, ignore_index, nv, g)
-        dX[r0:r1] = dz @ W
-        dW += dz.T @ X[r0:r1]
+        dX[r0:r1] = dz @ Wg
+        dW += dz.T @ Xg[r0:r1]
     return dX, dW
 
 
 def forward_backward(X, W, t, Vreal: int, cap: float, ignore_index: int, g: float = 1.0,
-                     block_rows: int = 1024):
+                     block_rows: int = 1024, Xg=None, Wg=None):
     """Loss, lse and both gradients in one call (what one fused training step needs)."""
     f = forward(X, W, t, Vreal, cap, ignore_index, block_rows)
-    dX, dW = backward(X, W, t, Vreal, cap, ignore_index, g, f["lse"], block_rows)
+    dX, dW = backward(X, W, t, Vreal, cap, ignore_index, g, f["lse"], block_rows, Xg, Wg)
     f.update(dX=dX, dW=dW)
     return f
 
 
 def dW_rows(X, W, t, lse, vocab_rows, Vreal: int, cap: float, ignore_index: int,
-            g: float = 1.0, block_rows: int = 4096):
-    """Selected rows ``j`` of ``dW = dz^T X``, given the lse of every token row.
+            g: float = 1.0, block_rows: int = 4096, Xg=None):
+    """Selected rows ``j`` of ``dW = dz^T Xg`` (Xg defaults to X), given the lse of every
+    token row.
 
     Only the logit columns ``j`` in ``vocab_rows`` are formed, so this costs
     ``N * d * len(vocab_rows)`` instead of a full backward."""
     X = np.asarray(X, np.float64)
+    Xg = X if Xg is None else np.asarray(Xg, np.float64)
     Wj = np.asarray(W, np.float64)[np.asarray(vocab_rows)]
     vocab_rows = np.asarray(vocab_rows, np.int64)
     valid, _ = valid_rows(t, Vreal, ignore_index)
@@ -186,5 +196,5 @@ def dW_rows(X, W, t, lse, vocab_rows, Vreal: int, cap: float, ignore_index: int,
         p[~valid[r0:r1]] = 0.0
         p[:, ~real] = 0.0
         dz = (g / nv) * p * softcap_derivative(z, cap)
-        out += dz.T @ X[r0:r1]
+        out += dz.T @ Xg[r0:r1]
     return out

@@ -25,8 +25,9 @@ import zlib
 import numpy as np
 
 __all__ = [
-    "FlceConfig", "CONFIGS", "make_inputs", "f32_to_bf16_bits", "bf16_to_f32",
-    "bf16_to_f64", "zipf_targets", "uniform_targets", "place_ignored",
+    "FlceConfig", "CONFIGS", "make_inputs", "make_fp8_inputs", "quantize_e4m3", "e4m3_to_f64",
+    "f32_to_bf16_bits", "bf16_to_f32", "bf16_to_f64", "zipf_targets", "uniform_targets",
+    "place_ignored",
 ]
 
 
@@ -64,7 +65,41 @@ CONFIGS = {
     # 3.8B head at 2048 context; wider W so more logits reach the softcap's curved range.
     "3.8b-2k": FlceConfig("3.8b-2k", 32768, 3072, 50257, 50304, "unit_rms", 0.05, "zipf",
                           _ignored(0.02, 32768)),
+    # large micro-batch, X and W also given as e4m3 with tensorwise scales (make_fp8_inputs)
+    "fp8": FlceConfig("fp8", 65536, 3072, 50257, 50304, "unit_rms", 0.02, "zipf",
+                      _ignored(0.05, 65536)),
 }
+
+E4M3_MAX = 448.0   # largest finite e4m3 value
+
+
+def quantize_e4m3(bits_bf16: np.ndarray):
+    """Tensorwise e4m3 encoding of bf16 values: scale = amax/448 (fp32), codes =
+    e4m3(x / scale) with the fp32 quotient rounded to nearest even by torch's float8_e4m3fn
+    cast.  Returns (uint8 codes, float32 scale)."""
+    import torch
+    x = bf16_to_f32(bits_bf16)
+    amax = np.float32(np.max(np.abs(x))) if x.size else np.float32(0)
+    scale = np.float32(amax / np.float32(E4M3_MAX)) if amax > 0 else np.float32(1.0)
+    q = torch.from_numpy(np.ascontiguousarray(x / scale, dtype=np.float32))
+    codes = q.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    return codes, scale
+
+
+def e4m3_to_f64(codes: np.ndarray) -> np.ndarray:
+    """Exact value of e4m3 codes (finite codes only)."""
+    import torch
+    t = torch.from_numpy(np.ascontiguousarray(codes, dtype=np.uint8)).view(torch.float8_e4m3fn)
+    return t.to(torch.float64).numpy()
+
+
+def make_fp8_inputs(cfg: FlceConfig | str = "fp8", seed: int | None = None, N: int | None = None):
+    """make_inputs plus e4m3 codes and tensorwise scales of X and W (the bf16 arrays stay as
+    the reference copies)."""
+    inp = make_inputs(cfg, seed=seed, N=N)
+    inp["X8"], inp["sX"] = quantize_e4m3(inp["X"])
+    inp["W8"], inp["sW"] = quantize_e4m3(inp["W"])
+    return inp
 
 
 def _rng(seed: int, tag: str) -> np.random.Generator:

@@ -24,7 +24,8 @@ def test_exports_every_declared_symbol(L):
     names = flce.declared_functions()
     assert set(names) == {"flce_workspace_bytes", "flce_forward", "flce_backward",
                           "flce_read_status", "flce_status_string", "flce_instrument",
-                          "flce_instrument_read", "flce_forward_noalloc"}
+                          "flce_instrument_read", "flce_forward_noalloc", "flce_forward_fp8",
+                          "flce_quantize_e4m3"}
     for n in names:
         assert hasattr(L, n), n
     out = subprocess.run(["nm", "-D", "--defined-only", _abi.LIB_PATH], capture_output=True,

@@ -1,0 +1,129 @@
+"""GPU parity of the FP8 path: logits from e4m3 operands with tensorwise scales
+(tcgen05 kind::f8f6f4), gradient contractions with the bf16 copies.
+
+* The device quantiser matches the reference encoder bit for bit (codes and scale).
+* Kernel error: against the fp64 oracle evaluated on the dequantised e4m3 values for the
+  logits and on the bf16 copies for the gradient products, with the ordinary parity bar.
+* Quantisation error: against the all-bf16 oracle, reported and bounded loosely (three
+  mantissa bits per operand).
+"""
+import numpy as np
+import pytest
+
+import oracle
+import synth
+
+pytestmark = pytest.mark.gpu
+
+LOSS_TOL = 2e-3
+LSE_TOL = 2e-3
+REL_L2 = 1e-2
+
+
+def _dev(a):
+    import torch
+    a = np.ascontiguousarray(a)
+    if a.dtype == np.uint16:
+        return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).cuda()
+    return torch.from_numpy(a).cuda()
+
+
+def _rel(got, ref):
+    return float(np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-300))
+
+
+def _run_fp8(inp, chunk_rows=0, want_grads=True):
+    import torch
+    import lm_head_linear_gemm_b200 as flce
+    c = inp["cfg"]
+    sx = torch.tensor(float(inp["sX"]), dtype=torch.float32, device="cuda")
+    sw = torch.tensor(float(inp["sW"]), dtype=torch.float32, device="cuda")
+    loss, lse, dX, dW, ws = flce.forward_fp8(_dev(inp["X8"]), _dev(inp["W8"]), sx, sw,
+                                             _dev(inp["X"]), _dev(inp["W"]), _dev(inp["targets"]),
+                                             c.Vreal, c.cap, c.ignore_index, want_grads,
+                                             chunk_rows=chunk_rows)
+    torch.cuda.synchronize()
+    status, nv = flce.read_status(ws)
+    out = dict(loss=float(loss.item()), lse=lse.double().cpu().numpy(), status=status, n_valid=nv)
+    if want_grads:
+        out["dX"] = dX.double().cpu().numpy()
+        out["dW"] = dW.double().cpu().numpy()
+    return out
+
+
+def _dequantised(inp):
+    Xq = synth.e4m3_to_f64(inp["X8"]) * float(inp["sX"])
+    Wq = synth.e4m3_to_f64(inp["W8"]) * float(inp["sW"])
+    return Xq, Wq
+
+
+def test_quantiser_matches_reference_encoder(cuda_device):
+    import torch
+    import lm_head_linear_gemm_b200 as flce
+    inp = synth.make_fp8_inputs("small", N=1024)
+    for key, skey in (("X", "sX"), ("W", "sW")):
+        codes, scale = flce.quantize_e4m3(_dev(inp[key]))
+        torch.cuda.synchronize()
+        assert float(scale.item()) == float(inp[skey])
+        assert np.array_equal(codes.cpu().numpy(), inp[key + "8"])
+
+
+def test_fp8_against_dequantised_oracle(cuda_device):
+    inp = synth.make_fp8_inputs("small", N=640)        # pages' vocabulary, d = 1536
+    c = inp["cfg"]
+    Xq, Wq = _dequantised(inp)
+    ref = oracle.forward_backward(Xq, Wq, inp["targets"], c.Vreal, c.cap, c.ignore_index,
+                                  Xg=synth.bf16_to_f64(inp["X"]), Wg=synth.bf16_to_f64(inp["W"]))
+    for chunk in (0, 256):
+        got = _run_fp8(inp, chunk_rows=chunk)
+        assert got["status"] == 0 and got["n_valid"] == ref["n_valid"]
+        assert abs(got["loss"] - ref["loss"]) <= LOSS_TOL
+        assert np.abs(got["lse"] - ref["lse"]).max() <= LSE_TOL
+        assert _rel(got["dX"], ref["dX"]) <= REL_L2
+        assert _rel(got["dW"], ref["dW"]) <= REL_L2
+        assert np.abs(got["dW"][c.Vreal:]).max() == 0.0
+    stats = _run_fp8(inp, want_grads=False)
+    assert abs(stats["loss"] - ref["loss"]) <= LOSS_TOL
+
+
+def test_fp8_quantisation_error_against_bf16_oracle(cuda_device):
+    """Reported figure: how far e4m3 logits move the loss and gradients from the bf16 result."""
+    inp = synth.make_fp8_inputs("small", N=640)
+    c = inp["cfg"]
+    ref = oracle.forward_backward(synth.bf16_to_f64(inp["X"]), synth.bf16_to_f64(inp["W"]),
+                                  inp["targets"], c.Vreal, c.cap, c.ignore_index)
+    got = _run_fp8(inp)
+    dloss = abs(got["loss"] - ref["loss"])
+    rx, rw = _rel(got["dX"], ref["dX"]), _rel(got["dW"], ref["dW"])
+    print(f"fp8 vs bf16 oracle: |dloss| {dloss:.2e}, max|dlse| "
+          f"{np.abs(got['lse'] - ref['lse']).max():.2e}, relL2 dX {rx:.2e}, dW {rw:.2e}")
+    assert dloss <= 5e-2 and rx <= 0.2 and rw <= 0.2
+
+
+def test_fp8_full_size_sampled(cuda_device):
+    """The large micro-batch workload (N = 65536, 5% ignored) in the bench's launch
+    configuration: loss and lse on all rows, dX on sampled rows, dW on sampled vocabulary
+    rows (random, the most frequent targets and all padded rows), against the oracle on the
+    dequantised logits operands and the bf16 gradient operands."""
+    inp = synth.make_fp8_inputs("fp8")
+    c = inp["cfg"]
+    got = _run_fp8(inp)
+    assert got["status"] == 0
+    Xq, Wq = _dequantised(inp)
+    Xb = synth.bf16_to_f64(inp["X"])
+    Wb = synth.bf16_to_f64(inp["W"])
+    t = inp["targets"]
+    f = oracle.forward(Xq, Wq, t, c.Vreal, c.cap, c.ignore_index, block_rows=2048)
+    assert abs(got["loss"] - f["loss"]) <= LOSS_TOL
+    assert np.abs(got["lse"] - f["lse"]).max() <= LSE_TOL
+    rng = np.random.default_rng(1)
+    rows = np.sort(rng.choice(c.N, 32, replace=False))
+    dz = oracle.row_dlogits(Xq[rows], Wq, t[rows], f["lse"][rows], c.Vreal, c.cap,
+                            c.ignore_index, f["n_valid"])
+    assert _rel(got["dX"][rows], dz @ Wb) <= REL_L2
+    counts = np.bincount(t[t >= 0], minlength=c.Vreal)
+    vrows = np.unique(np.concatenate([rng.choice(c.Vreal, 24, replace=False),
+                                      np.argsort(-counts)[:8], np.arange(c.Vreal, c.Vpad)]))
+    ref_dW = oracle.dW_rows(Xq, Wq, t, f["lse"], vrows, c.Vreal, c.cap, c.ignore_index, Xg=Xb)
+    assert _rel(got["dW"][vrows], ref_dW) <= REL_L2
+    assert np.abs(got["dW"][c.Vreal:]).max() == 0.0

@@ -317,3 +317,59 @@ def test_planted_mistakes_are_caught(monkeypatch):
                                            "logits": real_logits,
                                            "row_forward": real_row_forward}[attr])
     assert pins_hold()
+
+
+# --------------------------------------------------------------------------- FP8 variant
+def test_mixed_operand_gradients_reduce_and_brute_force():
+    """Logits from one pair of operands (the dequantised e4m3 values), gradient products with
+    another (the bf16 copies): equal operands give the ordinary backward, and a per-element
+    loop with separate operands agrees."""
+    X, W, t = _tiny(N=5, d=4, Vr=7, Vp=8, w_std=2.0, ign=1, seed=12)
+    rng = np.random.default_rng(3)
+    Xg = X + 0.01 * rng.standard_normal(X.shape)
+    Wg = W + 0.01 * rng.standard_normal(W.shape)
+    base = oracle.forward_backward(X, W, t, 7, 15.0, -1)
+    same = oracle.forward_backward(X, W, t, 7, 15.0, -1, Xg=X, Wg=W)
+    np.testing.assert_array_equal(base["dX"], same["dX"])
+    np.testing.assert_array_equal(base["dW"], same["dW"])
+    mixed = oracle.forward_backward(X, W, t, 7, 15.0, -1, Xg=Xg, Wg=Wg)
+    assert mixed["loss"] == base["loss"]
+    # brute force: dz from (X, W), products with (Xg, Wg)
+    N, d, Vp, Vr = 5, 4, 8, 7
+    nv = int((t != -1).sum())
+    dXb = np.zeros((N, d))
+    dWb = np.zeros((Vp, d))
+    for i in range(N):
+        if t[i] == -1:
+            continue
+        for j in range(Vr):
+            z = sum(X[i, k] * W[j, k] for k in range(d))
+            s = 15.0 * math.tanh(z / 15.0)
+            p = math.exp(s - base["lse"][i]) - (1.0 if j == t[i] else 0.0)
+            dz = p * (1.0 - math.tanh(z / 15.0) ** 2) / nv
+            dXb[i] += dz * Wg[j]
+            dWb[j] += dz * Xg[i]
+    np.testing.assert_allclose(mixed["dX"], dXb, atol=1e-12)
+    np.testing.assert_allclose(mixed["dW"], dWb, atol=1e-12)
+    rows = np.array([0, 3, 7])
+    got = oracle.dW_rows(X, W, t, base["lse"], rows, 7, 15.0, -1, Xg=Xg)
+    np.testing.assert_allclose(got, dWb[rows], atol=1e-13)
+
+
+def test_e4m3_encoder():
+    """Tensorwise e4m3 codes: scale = amax/448, the amax element maps to +-448, and every code
+    is the nearest e4m3 value of x/scale (3 mantissa bits: half-ulp bound 2^-4 relative for
+    normal codes, 2^-10 absolute below the smallest normal 2^-6)."""
+    inp = synth.make_fp8_inputs(synth.custom_config("q", 64, 96, 40, 48, w_std=0.3))
+    for key, skey in (("X", "sX"), ("W", "sW")):
+        x = synth.bf16_to_f64(inp[key])
+        s = float(inp[skey])
+        q = synth.e4m3_to_f64(inp[key + "8"])
+        assert abs(s - np.float32(np.abs(x).max()) / np.float32(448.0)) <= 1e-7 * s
+        assert np.abs(q).max() == 448.0
+        r = x / s
+        err = np.abs(q - r)
+        normal = np.abs(r) >= 2.0 ** -6
+        assert np.all(err[normal] <= np.abs(r[normal]) * 2.0 ** -4 * 1.0001)
+        assert np.all(err[~normal] <= 2.0 ** -10 * 1.0001)
+        assert np.all(np.sign(q[np.abs(r) > 2.0 ** -10]) == np.sign(r[np.abs(r) > 2.0 ** -10]))
