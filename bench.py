@@ -47,6 +47,11 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-unfused", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--accum-steps", type=int, default=7,
+                    help="N>1: micro-batches per optimizer step; dW is accumulated over them and "
+                         "all-reduced after the last (the write-ups: 7)")
+    ap.add_argument("--no-allreduce", action="store_true",
+                    help="N>1: independent replicas with no collective (weak-scaling floor)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--ref-rows", type=int, default=128,
@@ -268,9 +273,22 @@ def main_gpu(args):
         sX = torch.tensor(float(inp["sX"]), dtype=torch.float32, device=dev)
         sW = torch.tensor(float(inp["sW"]), dtype=torch.float32, device=dev)
 
+    dp = world > 1 and not args.no_allreduce and not fp8
+    micro = [0]
+
     def step(Xd=None, td=None):
         Xd = X if Xd is None else Xd
         td = t if td is None else td
+        if dp:
+            # data-parallel micro-batch: global-count normalisation; dW accumulated over
+            # --accum-steps micro-batches and all-reduced after the last one
+            k = micro[0] % max(1, args.accum_steps)
+            micro[0] += 1
+            loss, _, _, _, _ = flce.dp_step(
+                Xd, W, td, Vr, c.cap, c.ignore_index, dW=dW, accumulate_dW=k > 0,
+                allreduce_dW=k == max(1, args.accum_steps) - 1, workspace=ws,
+                chunk_rows=args.chunk_rows)
+            return loss
         if fp8:
             loss, lse, _, _, _ = flce.forward_fp8(X8, W8, sX, sW, Xd, W, td, Vr, c.cap,
                                                   c.ignore_index, True, dX=dX, dW=dW,
@@ -428,7 +446,10 @@ def main_gpu(args):
             "scaling": "weak", "vs_baseline": None,
             "dtype": "e4m3 logits + bf16 gradients" if fp8 else "bf16", "data": "synthetic",
             "config": dict(workload_desc(c, shape.chunk_rows or min(N, 4096)),
-                           parallelism=f"replicas x{world}" if world > 1 else "single GPU"),
+                           parallelism=(f"data parallel x{world}: global-count loss, dW "
+                                        f"all-reduce every {args.accum_steps} micro-batches"
+                                        if dp else
+                                        f"replicas x{world}" if world > 1 else "single GPU")),
             "tflops": tflops,
             "pct_of_bf16_datasheet_2250": tflops / world / DATASHEET_BF16_TFLOPS,
             "pct_of_measured_bf16_burst": tflops / world / burst,

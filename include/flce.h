@@ -134,6 +134,26 @@ int flce_forward_noalloc(const flce_shape* shape, const void* X, const void* W,
                          const int64_t* targets, float* loss, float* lse, void* stream);
 
 /*
+ * Data-parallel training (the write-ups train with plain DDP on 8 GPUs, gradient all-reduce; the
+ * "distributed strategy" paragraph).  Every rank holds W and its own rows.  To make the result
+ * equal to one call on the union of all ranks' rows:
+ *   1. flce_count_valid writes this rank's number of rows in the loss to *n_valid_out (device
+ *      int64, 8-byte aligned);
+ *   2. the caller sums it over ranks (an all-reduce) into a device int64 n_valid_total;
+ *   3. flce_forward_dp runs flce_forward but normalises by *n_valid_total: loss[0] is this rank's
+ *      share of the global mean and dX / dW are the gradients of the global mean (dW: this
+ *      rank's contribution, written or accumulated as in flce_forward);
+ *   4. the caller sums loss and dW over ranks (all-reduces); dX stays with its rows.
+ * flce_forward_dp takes the same arguments as flce_forward plus n_valid_total.
+ */
+int flce_count_valid(const flce_shape* shape, const int64_t* targets, int64_t* n_valid_out,
+                     void* stream);
+int flce_forward_dp(const flce_shape* shape, const void* X, const void* W, const int64_t* targets,
+                    const int64_t* n_valid_total, float* loss, float* lse, int want_grads,
+                    void* dX, float* dW, int accumulate_dW, void* workspace,
+                    size_t workspace_bytes, void* stream);
+
+/*
  * Forward with FP8 logits: the logits contraction z = X W^T reads e4m3 operands with dynamic
  * tensorwise scales (x ~ X8 * *scale_x, w ~ W8 * *scale_w; the scales are device scalars) on the
  * tensor cores' fp8 path, with both scales applied to z before the softcap.  This follows the
@@ -158,6 +178,15 @@ int flce_forward_fp8(const flce_shape* shape, const void* X8, const void* W8,
  * amax accumulator while the call runs.  Four small kernels on `stream`.
  */
 int flce_quantize_e4m3(const void* src, int64_t n, void* dst, float* scale_out, void* stream);
+
+/*
+ * Self-test of failure detection (no counterpart on the pages): runs the library's bounded
+ * pipeline wait on a barrier that nothing arrives at, with a limit of limit_ns (1 ns .. 10 s).
+ * The wait runs out, FLCE_DEV_TIMEOUT is or-ed into the status word of `workspace` (read it with
+ * flce_read_status), and the kernel returns normally, leaving the context usable.  workspace
+ * needs 256 bytes and is otherwise untouched.
+ */
+int flce_selftest_wait_timeout(void* workspace, uint64_t limit_ns, void* stream);
 
 /*
  * Reads the device status word (FLCE_DEV_* bits) and the number of rows in the loss from the

@@ -6,13 +6,14 @@ arguments to it.  Entry points raise if the library is missing: there is no
 fallback implementation.
 """
 from ._abi import (DEV_BAD_TARGET, DEV_TIMEOUT, FlceError, alloc_workspace, backward,
-                   declared_functions, forward, forward_fp8, instrument, instrument_read, lib, make_shape, raw_backward, raw_forward,
-                   quantize_e4m3, raw_forward_noalloc, read_status, status_string, workspace_bytes)
+                   declared_functions, forward, forward_dp, forward_fp8, instrument, instrument_read, lib, make_shape, raw_backward, raw_forward,
+                   quantize_e4m3, raw_forward_noalloc, read_status, selftest_wait_timeout, status_string, workspace_bytes)
 from .autograd import FusedLinearCrossEntropy, fused_linear_cross_entropy
+from .data_parallel import dp_step
 
 __all__ = [
     "DEV_BAD_TARGET", "DEV_TIMEOUT", "FlceError", "alloc_workspace", "backward",
-    "declared_functions", "forward", "forward_fp8", "instrument", "instrument_read", "lib", "make_shape", "raw_backward", "raw_forward",
-    "quantize_e4m3", "raw_forward_noalloc", "read_status", "status_string", "workspace_bytes", "FusedLinearCrossEntropy",
-    "fused_linear_cross_entropy",
+    "declared_functions", "forward", "forward_dp", "forward_fp8", "instrument", "instrument_read", "lib", "make_shape", "raw_backward", "raw_forward",
+    "quantize_e4m3", "raw_forward_noalloc", "read_status", "selftest_wait_timeout", "status_string", "workspace_bytes", "FusedLinearCrossEntropy",
+    "fused_linear_cross_entropy", "dp_step",
 ]

@@ -86,8 +86,15 @@ def lib() -> ctypes.CDLL:
     L.flce_forward_fp8.restype = ctypes.c_int
     L.flce_quantize_e4m3.argtypes = [P, ctypes.c_int64, P, P, P]
     L.flce_quantize_e4m3.restype = ctypes.c_int
+    L.flce_count_valid.argtypes = [shp, P, P, P]
+    L.flce_count_valid.restype = ctypes.c_int
+    L.flce_forward_dp.argtypes = [shp, P, P, P, P, P, P, ctypes.c_int, P, P, ctypes.c_int, P,
+                                  ctypes.c_size_t, P]
+    L.flce_forward_dp.restype = ctypes.c_int
     L.flce_forward_noalloc.argtypes = [shp, P, P, P, P, P, P]
     L.flce_forward_noalloc.restype = ctypes.c_int
+    L.flce_selftest_wait_timeout.argtypes = [P, ctypes.c_uint64, P]
+    L.flce_selftest_wait_timeout.restype = ctypes.c_int
     L.flce_instrument.argtypes = [ctypes.c_int]
     L.flce_instrument.restype = ctypes.c_int
     L.flce_instrument_read.argtypes = [ctypes.POINTER(flce_kernel_stats)]
@@ -159,6 +166,13 @@ def read_status(workspace, stream=None) -> tuple[int, int]:
     return int(st.value), int(nv.value)
 
 
+def selftest_wait_timeout(workspace, limit_ns: int, stream=None) -> None:
+    """Run the bounded-wait self-test into ``workspace``'s status word (see read_status)."""
+    rc = lib().flce_selftest_wait_timeout(_ptr(workspace), int(limit_ns), _stream(stream))
+    if rc != FLCE_OK:
+        raise FlceError(rc, "flce_selftest_wait_timeout")
+
+
 def instrument(enable: bool) -> None:
     """Start (reset) or stop per-launch event timing of the contraction kernels."""
     lib().flce_instrument(1 if enable else 0)
@@ -228,6 +242,37 @@ def forward(X, W, targets, Vreal: int, cap: float = 15.0, ignore_index: int = -1
                      workspace.numel(), _stream(stream))
     if rc != FLCE_OK:
         raise FlceError(rc, "flce_forward")
+    return loss, lse, (dX if want_grads else None), (dW if want_grads else None), workspace
+
+
+def forward_dp(X, W, targets, n_valid_total, Vreal: int, cap: float = 15.0,
+               ignore_index: int = -1, want_grads: bool = True, dX=None, dW=None,
+               accumulate_dW: bool = False, workspace=None, chunk_rows: int = 0, stream=None):
+    """flce_forward normalised by a device int64 count of rows in the loss over all
+    data-parallel ranks.  Returns (loss share, lse, dX, dW, workspace)."""
+    import torch
+    _check(X, W, targets)
+    if not n_valid_total.is_cuda or n_valid_total.dtype != torch.int64:
+        raise TypeError("n_valid_total must be a CUDA int64 tensor")
+    N, d = X.shape
+    shape = make_shape(N, d, W.shape[0], Vreal, cap, ignore_index, chunk_rows)
+    dev = X.device
+    loss = torch.empty((), dtype=torch.float32, device=dev)
+    lse = torch.empty(max(N, 1), dtype=torch.float32, device=dev)[:N]
+    if want_grads:
+        if dX is None:
+            dX = torch.empty_like(X)
+        if dW is None:
+            dW = torch.empty(W.shape, dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = alloc_workspace(shape, want_grads, dev)
+    rc = lib().flce_forward_dp(ctypes.byref(shape), _ptr(X), _ptr(W), _ptr(targets),
+                               _ptr(n_valid_total), _ptr(loss), _ptr(lse),
+                               1 if want_grads else 0, _ptr(dX) if want_grads else None,
+                               _ptr(dW) if want_grads else None, int(accumulate_dW),
+                               _ptr(workspace), workspace.numel(), _stream(stream))
+    if rc != FLCE_OK:
+        raise FlceError(rc, "flce_forward_dp")
     return loss, lse, (dX if want_grads else None), (dW if want_grads else None), workspace
 
 

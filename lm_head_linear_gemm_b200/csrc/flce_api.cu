@@ -273,6 +273,7 @@ struct Fp8Logits {
 struct Ctx {
   const flce_shape* s;
   Fp8Logits fp8;
+  const long long* nv_total = nullptr;   // data-parallel normaliser (null: this call's rows)
   Layout L;
   uint8_t* ws;
   DevHeader* hdr;
@@ -361,6 +362,7 @@ int grad_chunk(const Ctx& c, int64_t row0, int rows, const __nv_bfloat16* X,
   rp.lse_out = lse_out ? lse_out + row0 : nullptr;
   rp.row_loss = c.at<float>(c.L.row_loss) + row0;
   rp.hdr = c.hdr;
+  rp.nv_total = c.nv_total;
   rp.grad_out = grad_out;
   rp.r = r;
   rp.A = Abuf;
@@ -477,7 +479,7 @@ int noalloc_scratch_address(void** out) {
 int forward_impl(const flce_shape* s, const void* X, const void* W, const Fp8Logits& fp8,
                  const int64_t* targets, float* loss, float* lse, int want_grads, void* dX,
                  float* dW, int accumulate_dW, void* workspace, size_t workspace_bytes,
-                 void* stream) {
+                 void* stream, const int64_t* nv_total = nullptr) {
   want_grads = want_grads ? 1 : 0;
   if (loss == nullptr || (s->N > 0 && lse == nullptr)) return FLCE_ERR_ARG;
   if (!aligned16(loss) || !aligned16(lse)) return FLCE_ERR_ALIGN;
@@ -490,6 +492,7 @@ int forward_impl(const flce_shape* s, const void* X, const void* W, const Fp8Log
   Ctx c{};
   c.s = s;
   c.fp8 = fp8;
+  c.nv_total = reinterpret_cast<const long long*>(nv_total);
   c.L = make_layout(s, want_grads);
   c.ws = static_cast<uint8_t*>(workspace);
   c.di = di;
@@ -517,7 +520,7 @@ int forward_impl(const flce_shape* s, const void* X, const void* W, const Fp8Log
   } else {
     FLCE_TRY(stats_pass(c, Xb, Wb, lse));
   }
-  loss_kernel<<<1, 1024, 0, c.st>>>(c.at<float>(c.L.row_loss), s->N, c.hdr, loss);
+  loss_kernel<<<1, 1024, 0, c.st>>>(c.at<float>(c.L.row_loss), s->N, c.hdr, c.nv_total, loss);
   FLCE_TRY(launch_ok());
   if (want_grads && !c.L.fixed_ref) {
     // Without a fixed exp reference the gradient needs lse first: recompute with it.
@@ -546,6 +549,31 @@ int flce_forward(const flce_shape* s, const void* X, const void* W, const int64_
   FLCE_TRY(common_checks(s, X, W, targets, workspace, workspace_bytes, want_grads ? 1 : 0));
   return forward_impl(s, X, W, Fp8Logits{}, targets, loss, lse, want_grads, dX, dW,
                       accumulate_dW, workspace, workspace_bytes, stream);
+}
+
+int flce_count_valid(const flce_shape* s, const int64_t* targets, int64_t* n_valid_out,
+                     void* stream) {
+  if (!shape_ok(s) || n_valid_out == nullptr || (s->N > 0 && targets == nullptr))
+    return FLCE_ERR_ARG;
+  if ((reinterpret_cast<uintptr_t>(n_valid_out) & 7u) != 0 || !aligned16(targets))
+    return FLCE_ERR_ALIGN;
+  DeviceInfo* di = nullptr;
+  FLCE_TRY(device_info(&di));
+  count_valid_kernel<<<1, 1024, 0, static_cast<cudaStream_t>(stream)>>>(
+      reinterpret_cast<const long long*>(targets), s->N, s->Vreal, s->ignore_index,
+      reinterpret_cast<long long*>(n_valid_out));
+  return launch_ok();
+}
+
+int flce_forward_dp(const flce_shape* s, const void* X, const void* W, const int64_t* targets,
+                    const int64_t* n_valid_total, float* loss, float* lse, int want_grads,
+                    void* dX, float* dW, int accumulate_dW, void* workspace,
+                    size_t workspace_bytes, void* stream) {
+  FLCE_TRY(common_checks(s, X, W, targets, workspace, workspace_bytes, want_grads ? 1 : 0));
+  if (n_valid_total == nullptr) return FLCE_ERR_ARG;
+  if ((reinterpret_cast<uintptr_t>(n_valid_total) & 7u) != 0) return FLCE_ERR_ALIGN;
+  return forward_impl(s, X, W, Fp8Logits{}, targets, loss, lse, want_grads, dX, dW,
+                      accumulate_dW, workspace, workspace_bytes, stream, n_valid_total);
 }
 
 int flce_forward_fp8(const flce_shape* s, const void* X8, const void* W8, const float* scale_x,
@@ -664,6 +692,17 @@ int flce_forward_noalloc(const flce_shape* shape, const void* X, const void* W,
   FLCE_TRY(noalloc_scratch_address(&scratch));
   return flce_forward(&s, X, W, targets, loss, lse, 0, nullptr, nullptr, 0, scratch,
                       FLCE_NOALLOC_SCRATCH_BYTES, stream);
+}
+
+int flce_selftest_wait_timeout(void* workspace, uint64_t limit_ns, void* stream) {
+  if (workspace == nullptr) return FLCE_ERR_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0) return FLCE_ERR_ALIGN;
+  if (limit_ns == 0 || limit_ns > 10000000000ull) return FLCE_ERR_ARG;   // at most 10 s
+  DeviceInfo* di = nullptr;
+  FLCE_TRY(device_info(&di));
+  wait_timeout_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+      &static_cast<DevHeader*>(workspace)->status, limit_ns);
+  return launch_ok();
 }
 
 int flce_read_status(const void* workspace, uint32_t* dev_status_out, int64_t* n_valid_out,

@@ -68,6 +68,7 @@ struct RowFinishParams {
   float* lse_out;               // [rows] (from_partials == 1)
   float* row_loss;              // [rows] lse - s_t for rows in the loss, else 0 (from_partials)
   const DevHeader* hdr;         // n_valid
+  const long long* nv_total;    // rows in the loss over all data-parallel ranks, or null (= local)
   const float* grad_out;        // device scalar g, or null for g = 1
   float* r;                     // [rows]
   __nv_bfloat16* A;             // [rows][Vpad]
@@ -121,7 +122,7 @@ __global__ void __launch_bounds__(256) row_finish_kernel(const RowFinishParams p
     p.row_loss[row] = valid ? lse - p.s_t[row] : 0.f;
   }
   if (!p.want_grads) return;
-  const long long nv = p.hdr->n_valid;
+  const long long nv = p.nv_total != nullptr ? *p.nv_total : p.hdr->n_valid;
   const float g = p.grad_out ? *p.grad_out : 1.f;
   const float r = (valid && nv > 0) ? g / (static_cast<float>(nv) * S) : 0.f;
   if (lane == 0) {
@@ -147,9 +148,11 @@ __global__ void __launch_bounds__(256) row_finish_kernel(const RowFinishParams p
   }
 }
 
-// One block: loss = sum(row_loss) / n_valid, 0 when no row is in the loss.
+// One block: loss = sum(row_loss) / n_valid, 0 when no row is in the loss.  With nv_total (the
+// count over all data-parallel ranks) the result is this rank's share of the global mean.
 __global__ void __launch_bounds__(1024) loss_kernel(const float* __restrict__ row_loss, long long N,
                                                     const DevHeader* __restrict__ hdr,
+                                                    const long long* __restrict__ nv_total,
                                                     float* __restrict__ loss) {
   __shared__ double s_part[1024];
   double acc = 0.0;
@@ -161,7 +164,7 @@ __global__ void __launch_bounds__(1024) loss_kernel(const float* __restrict__ ro
     __syncthreads();
   }
   if (threadIdx.x == 0) {
-    const long long nv = hdr->n_valid;
+    const long long nv = nv_total != nullptr ? *nv_total : hdr->n_valid;
     loss[0] = nv > 0 ? static_cast<float>(s_part[0] / static_cast<double>(nv)) : 0.f;
   }
 }
@@ -229,6 +232,39 @@ __global__ void quantize_e4m3_kernel(const __nv_bfloat16* __restrict__ x, long l
 __global__ void finish_scale_kernel(uint32_t* amax_bits) {
   const float amax = __uint_as_float(*amax_bits);
   *reinterpret_cast<float*>(amax_bits) = amax > 0.f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+}
+
+// One block: number of rows whose target enters the loss (t != ignore_index, 0 <= t < Vreal).
+__global__ void __launch_bounds__(1024) count_valid_kernel(const long long* __restrict__ targets,
+                                                           long long N, long long Vreal,
+                                                           long long ignore_index,
+                                                           long long* __restrict__ out) {
+  __shared__ long long s_count[32];
+  long long count = 0;
+  for (long long i = threadIdx.x; i < N; i += blockDim.x) {
+    const long long t = targets[i];
+    count += (t != ignore_index && t >= 0 && t < Vreal) ? 1 : 0;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) count += __shfl_xor_sync(0xffffffffu, count, o);
+  if ((threadIdx.x & 31) == 0) s_count[threadIdx.x >> 5] = count;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    long long total = 0;
+    for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) total += s_count[w];
+    *out = total;
+  }
+}
+
+// Self-test of the bounded wait used by every pipeline barrier: one thread initialises an
+// mbarrier that expects one arrival, never arrives, and waits on it with the given limit.  The
+// wait gives up, raises DEV_TIMEOUT in *status and the kernel returns normally.
+__global__ void wait_timeout_selftest_kernel(uint32_t* status, unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x != 0) return;
+  mbar_init(&bar, 1);
+  fence_barrier_init();
+  mbar_wait_bounded(&bar, 0, status, limit_ns);
 }
 
 // Writes loss = 0 (used for N = 0, where nothing else runs).

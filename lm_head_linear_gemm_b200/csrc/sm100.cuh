@@ -59,13 +59,13 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // `limit_ns` of wall time, raises DEV_TIMEOUT in *status and returns false, so
 // a lost arrival ends the kernel with an error instead of hanging the GPU.
 // try_wait itself suspends the thread for a while, so the clock is read only
-// once every 1024 unsuccessful polls.
+// once every 128 unsuccessful polls.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
                                                   uint32_t* status, uint64_t limit_ns) {
   uint64_t t0 = 0;
   for (uint32_t it = 0;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 1023u) == 1023u) {
+    if ((it & 127u) == 127u) {
       const uint64_t now = global_timer_ns();
       if (t0 == 0) {
         t0 = now;
@@ -231,7 +231,7 @@ __device__ __forceinline__ bool mbar_wait_bounded_cluster(uint64_t* bar, uint32_
   uint64_t t0 = 0;
   for (uint32_t it = 0;; ++it) {
     if (mbar_try_wait_cluster_acq(bar, parity)) return true;
-    if ((it & 1023u) == 1023u) {
+    if ((it & 127u) == 127u) {
       const uint64_t now = global_timer_ns();
       if (t0 == 0) {
         t0 = now;

@@ -25,7 +25,8 @@ def test_exports_every_declared_symbol(L):
     assert set(names) == {"flce_workspace_bytes", "flce_forward", "flce_backward",
                           "flce_read_status", "flce_status_string", "flce_instrument",
                           "flce_instrument_read", "flce_forward_noalloc", "flce_forward_fp8",
-                          "flce_quantize_e4m3"}
+                          "flce_quantize_e4m3", "flce_selftest_wait_timeout",
+                          "flce_count_valid", "flce_forward_dp"}
     for n in names:
         assert hasattr(L, n), n
     out = subprocess.run(["nm", "-D", "--defined-only", _abi.LIB_PATH], capture_output=True,
@@ -104,6 +105,14 @@ def test_instrumentation_counters_without_gpu(L):
     flce.instrument(False)
     assert st["launches_total"] == 0
     assert all(v["launches"] == 0 and v["ms"] == 0 for v in st["gemm"].values())
+
+
+def test_selftest_rejects_bad_limits(L):
+    p = 0x10000000      # never dereferenced: argument checks come first
+    assert L.flce_selftest_wait_timeout(None, 1000, None) == -1
+    assert L.flce_selftest_wait_timeout(p, 0, None) == -1
+    assert L.flce_selftest_wait_timeout(p, 11_000_000_000, None) == -1
+    assert L.flce_selftest_wait_timeout(p + 16, 1000, None) == -2
 
 
 def test_shape_struct_matches_header():
