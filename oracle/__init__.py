@@ -47,7 +47,8 @@ import numpy as np
 
 __all__ = [
     "logits", "softcap", "softcap_derivative", "valid_rows", "row_forward", "forward",
-    "row_dlogits", "backward", "forward_backward", "dW_rows",
+    "row_dlogits", "backward", "forward_backward", "dW_rows", "rmsnorm_forward",
+    "rmsnorm_backward",
 ]
 
 
@@ -198,3 +199,30 @@ def dW_rows(X, W, t, lse, vocab_rows, Vreal: int, cap: float, ignore_index: int,
         dz = (g / nv) * p * softcap_derivative(z, cap)
         out += dz.T @ Xg[r0:r1]
     return out
+
+
+# ------------------------------------------------------------------------ final RMSNorm
+# The model's last RMSNorm feeds the head (the write-ups' model is Llama-style with RMSNorm;
+# config appendix: rms_norm_eps = 1.0e-6):  x_i = h_i * rstd_i * gamma,
+# rstd_i = 1 / sqrt(mean_k h_ik^2 + eps).
+
+def rmsnorm_forward(H, gamma, eps: float = 1e-6):
+    """Returns (x [N, d], rstd [N]) in float64."""
+    H = np.asarray(H, np.float64)
+    rstd = 1.0 / np.sqrt(np.mean(H * H, axis=1) + eps)
+    return H * rstd[:, None] * np.asarray(gamma, np.float64)[None, :], rstd
+
+
+def rmsnorm_backward(H, gamma, dX, eps: float = 1e-6):
+    """Chain rule through x = h * rstd(h) * gamma for an upstream gradient dX = dL/dx.
+
+    Returns (dH [N, d], dgamma [d]):  with xh = h * rstd and g = dX * gamma,
+    dH = rstd * (g - xh * mean_k(g * xh)),  dgamma = sum_i dX * xh."""
+    H = np.asarray(H, np.float64)
+    dX = np.asarray(dX, np.float64)
+    gamma = np.asarray(gamma, np.float64)
+    rstd = 1.0 / np.sqrt(np.mean(H * H, axis=1) + eps)
+    xh = H * rstd[:, None]
+    g = dX * gamma[None, :]
+    dH = rstd[:, None] * (g - xh * np.mean(g * xh, axis=1, keepdims=True))
+    return dH, np.sum(dX * xh, axis=0)

@@ -373,3 +373,54 @@ def test_e4m3_encoder():
         assert np.all(err[normal] <= np.abs(r[normal]) * 2.0 ** -4 * 1.0001)
         assert np.all(err[~normal] <= 2.0 ** -10 * 1.0001)
         assert np.all(np.sign(q[np.abs(r) > 2.0 ** -10]) == np.sign(r[np.abs(r) > 2.0 ** -10]))
+
+
+# --------------------------------------------------------------------------- final RMSNorm
+def test_rmsnorm_unit_rms_and_closed_form():
+    rng = np.random.default_rng(5)
+    H = rng.standard_normal((6, 32)) * 3.0
+    x, rstd = oracle.rmsnorm_forward(H, np.ones(32), eps=0.0)
+    np.testing.assert_allclose(np.sqrt(np.mean(x * x, axis=1)), 1.0, rtol=1e-14)
+    # constant row c: rstd = 1/sqrt(c^2 + eps)
+    Hc = np.full((1, 8), 2.0)
+    _, r = oracle.rmsnorm_forward(Hc, np.ones(8), eps=1e-6)
+    assert abs(r[0] - 1.0 / math.sqrt(4.0 + 1e-6)) < 1e-15
+    # gamma scales columns
+    g = rng.standard_normal(32)
+    xg, _ = oracle.rmsnorm_forward(H, g)
+    x1, _ = oracle.rmsnorm_forward(H, np.ones(32))
+    np.testing.assert_allclose(xg, x1 * g, rtol=1e-14)
+
+
+def test_rmsnorm_then_loss_finite_differences():
+    """d loss(rmsnorm(h) W^T) / dh and / dgamma by central differences."""
+    rng = np.random.default_rng(8)
+    N, d, Vr, Vp = 5, 8, 20, 24
+    H = rng.standard_normal((N, d)) * 2.0
+    gamma = 1.0 + 0.3 * rng.standard_normal(d)
+    W = rng.standard_normal((Vp, d)) * 1.5
+    t = rng.integers(0, Vr, N)
+    t[1] = -1
+
+    def L(H_, g_):
+        x, _ = oracle.rmsnorm_forward(H_, g_)
+        return oracle.forward(x, W, t, Vr, 15.0, -1)["loss"]
+
+    x, _ = oracle.rmsnorm_forward(H, gamma)
+    dX, _ = oracle.backward(x, W, t, Vr, 15.0, -1)
+    dH, dg = oracle.rmsnorm_backward(H, gamma, dX)
+    h = 1e-6
+    num_dH = np.zeros_like(H)
+    for idx in np.ndindex(*H.shape):
+        Hp, Hm = H.copy(), H.copy()
+        Hp[idx] += h
+        Hm[idx] -= h
+        num_dH[idx] = (L(Hp, gamma) - L(Hm, gamma)) / (2 * h)
+    num_dg = np.zeros_like(gamma)
+    for k in range(d):
+        gp, gm = gamma.copy(), gamma.copy()
+        gp[k] += h
+        gm[k] -= h
+        num_dg[k] = (L(H, gp) - L(H, gm)) / (2 * h)
+    assert np.linalg.norm(num_dH - dH) <= 1e-6 * np.linalg.norm(dH)
+    assert np.linalg.norm(num_dg - dg) <= 1e-6 * np.linalg.norm(dg)
