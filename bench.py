@@ -56,6 +56,9 @@ def parse_args():
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--ref-rows", type=int, default=128,
                     help="rows per step of the --impl reference arm")
+    ap.add_argument("--norm", action="store_true",
+                    help="time the final-RMSNorm kernels (forward, backward) on the workload's "
+                         "shape against the measured HBM copy bandwidth")
     ap.add_argument("--compare-cublas", action="store_true",
                     help="per-contraction efficiency at the operating clock next to cuBLAS "
                          "(torch.matmul) on the same shapes, with NVML clock/power sampling")
@@ -635,12 +638,56 @@ def compare_cublas(args):
     return 0
 
 
+def norm_bench(args):
+    """RMSNorm forward / backward at N x d of the workload; HBM-bound, so achieved GB/s of the
+    algorithmic bytes against the measured copy bandwidth."""
+    import torch
+    import lm_head_linear_gemm_b200 as flce
+    import synth
+    c = synth.CONFIGS[args.config]
+    N, d = args.rows or c.N, c.d
+    dev = torch.device("cuda", 0)
+    g = torch.Generator(device=dev).manual_seed(0)
+    H = (torch.randn(N, d, device=dev, generator=g) * 2).to(torch.bfloat16)
+    gamma = (1 + 0.1 * torch.randn(d, device=dev, generator=g)).to(torch.bfloat16)
+    dX = (torch.randn(N, d, device=dev, generator=g) * 1e-3).to(torch.bfloat16)
+    X, rstd = flce.rmsnorm_forward(H, gamma)
+    dH, dgamma = flce.rmsnorm_backward(H, gamma, rstd, dX)
+    peaks, src = load_peaks()
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    out = {}
+    for name, fn, nbytes in (
+            ("forward", lambda: flce.rmsnorm_forward(H, gamma, X=X, rstd=rstd), 4 * N * d + 4 * N),
+            ("backward", lambda: flce.rmsnorm_backward(H, gamma, rstd, dX, dH=dH, dgamma=dgamma),
+             10 * N * d + 8 * N)):
+        for _ in range(5):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        reps = 50
+        e0.record()
+        for _ in range(reps):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / reps
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        out[name] = {"ms": ms, "algorithmic_bytes": nbytes, "GB/s": gbs, "frac_of_hbm": gbs / hbm}
+    print(json.dumps({"rmsnorm": out, "N": N, "d": d, "hbm_peak_gbs": hbm, "peak_source": src,
+                      "bytes": "forward: read h, write x (2+2 B per element) + rstd; backward: "
+                               "dH pass reads h, dX, writes dH (6 B), dgamma pass re-reads h, "
+                               "dX (4 B)"}), flush=True)
+    return 0
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
         return run_reference(args)
     if args.compare_cublas:
         return compare_cublas(args)
+    if args.norm:
+        return norm_bench(args)
     return main_gpu(args)
 
 

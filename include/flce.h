@@ -180,6 +180,24 @@ int flce_forward_fp8(const flce_shape* shape, const void* X8, const void* W8,
 int flce_quantize_e4m3(const void* src, int64_t n, void* dst, float* scale_out, void* stream);
 
 /*
+ * The model's final RMSNorm, whose output feeds the head (the write-ups' model is Llama-style
+ * with RMSNorm; config appendix: rms_norm_eps = 1.0e-6):
+ *   x_i = h_i * rstd_i * gamma,  rstd_i = 1 / sqrt(mean_k h_ik^2 + eps)   (fp32 arithmetic)
+ * H [N, d] bf16, gamma [d] bf16, X [N, d] bf16 (out), rstd [N] fp32 (out).  d % 8 == 0.
+ * Backward, for dX = dL/dx from the loss (e.g. flce_forward's dX):
+ *   dH = rstd * (g - xh * mean_k(g * xh)),  dgamma = sum_i dX * xh,  xh = h * rstd, g = dX * gamma
+ * dH [N, d] bf16 (out); dgamma [d] fp32 written, or added to with accumulate_dgamma = 1.  The
+ * dgamma reduction is deterministic (fixed-order partial sums in `workspace`, at least
+ * flce_rmsnorm_workspace_bytes(N, d) bytes, 16-byte aligned).
+ */
+int flce_rmsnorm_forward(const void* H, const void* gamma, float eps, int64_t N, int64_t d,
+                         void* X, float* rstd, void* stream);
+size_t flce_rmsnorm_workspace_bytes(int64_t N, int64_t d);
+int flce_rmsnorm_backward(const void* H, const void* gamma, const float* rstd, const void* dX,
+                          int64_t N, int64_t d, void* dH, float* dgamma, int accumulate_dgamma,
+                          void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Self-test of failure detection (no counterpart on the pages): runs the library's bounded
  * pipeline wait on a barrier that nothing arrives at, with a limit of limit_ns (1 ns .. 10 s).
  * The wait runs out, FLCE_DEV_TIMEOUT is or-ed into the status word of `workspace` (read it with

@@ -93,6 +93,14 @@ def lib() -> ctypes.CDLL:
     L.flce_forward_dp.restype = ctypes.c_int
     L.flce_forward_noalloc.argtypes = [shp, P, P, P, P, P, P]
     L.flce_forward_noalloc.restype = ctypes.c_int
+    L.flce_rmsnorm_forward.argtypes = [P, P, ctypes.c_float, ctypes.c_int64, ctypes.c_int64, P,
+                                       P, P]
+    L.flce_rmsnorm_forward.restype = ctypes.c_int
+    L.flce_rmsnorm_workspace_bytes.argtypes = [ctypes.c_int64, ctypes.c_int64]
+    L.flce_rmsnorm_workspace_bytes.restype = ctypes.c_size_t
+    L.flce_rmsnorm_backward.argtypes = [P, P, P, P, ctypes.c_int64, ctypes.c_int64, P, P,
+                                        ctypes.c_int, P, ctypes.c_size_t, P]
+    L.flce_rmsnorm_backward.restype = ctypes.c_int
     L.flce_selftest_wait_timeout.argtypes = [P, ctypes.c_uint64, P]
     L.flce_selftest_wait_timeout.restype = ctypes.c_int
     L.flce_instrument.argtypes = [ctypes.c_int]
@@ -274,6 +282,42 @@ def forward_dp(X, W, targets, n_valid_total, Vreal: int, cap: float = 15.0,
     if rc != FLCE_OK:
         raise FlceError(rc, "flce_forward_dp")
     return loss, lse, (dX if want_grads else None), (dW if want_grads else None), workspace
+
+
+def rmsnorm_forward(H, gamma, eps: float = 1e-6, X=None, rstd=None, stream=None):
+    """x = h * rstd * gamma (bf16), rstd = 1/sqrt(mean(h^2) + eps) (fp32).  Returns (x, rstd)."""
+    import torch
+    if H.dtype != torch.bfloat16 or gamma.dtype != torch.bfloat16 or not H.is_contiguous():
+        raise TypeError("H and gamma must be contiguous bf16 CUDA tensors")
+    N, d = H.shape
+    if X is None:
+        X = torch.empty_like(H)
+    if rstd is None:
+        rstd = torch.empty(max(N, 1), dtype=torch.float32, device=H.device)[:N]
+    rc = lib().flce_rmsnorm_forward(_ptr(H), _ptr(gamma), float(eps), N, d, _ptr(X), _ptr(rstd),
+                                    _stream(stream))
+    if rc != FLCE_OK:
+        raise FlceError(rc, "flce_rmsnorm_forward")
+    return X, rstd
+
+
+def rmsnorm_backward(H, gamma, rstd, dX, dH=None, dgamma=None, accumulate_dgamma: bool = False,
+                     stream=None):
+    """Chain rule through the RMSNorm for dX = dL/dx.  Returns (dH bf16, dgamma fp32)."""
+    import torch
+    N, d = H.shape
+    if dH is None:
+        dH = torch.empty_like(H)
+    if dgamma is None:
+        dgamma = torch.empty(d, dtype=torch.float32, device=H.device)
+    nbytes = int(lib().flce_rmsnorm_workspace_bytes(N, d))
+    ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=H.device)
+    rc = lib().flce_rmsnorm_backward(_ptr(H), _ptr(gamma), _ptr(rstd), _ptr(dX), N, d, _ptr(dH),
+                                     _ptr(dgamma), int(accumulate_dgamma), _ptr(ws), ws.numel(),
+                                     _stream(stream))
+    if rc != FLCE_OK:
+        raise FlceError(rc, "flce_rmsnorm_backward")
+    return dH, dgamma
 
 
 def quantize_e4m3(x, out=None, scale=None, stream=None):

@@ -41,3 +41,24 @@ def fused_linear_cross_entropy(X, W, targets, Vreal: int, cap: float = 15.0,
                                ignore_index: int = -1, chunk_rows: int = 0):
     """Mean softcapped cross entropy of ``X W^T`` over rows whose target is not ignore_index."""
     return FusedLinearCrossEntropy.apply(X, W, targets, Vreal, cap, ignore_index, chunk_rows)
+
+
+class RMSNorm(torch.autograd.Function):
+    """The model's final RMSNorm in front of the head, in the library's kernels."""
+
+    @staticmethod
+    def forward(ctx, H, gamma, eps):
+        X, rstd = _abi.rmsnorm_forward(H.contiguous(), gamma.contiguous(), eps)
+        ctx.save_for_backward(H, gamma, rstd)
+        return X
+
+    @staticmethod
+    def backward(ctx, dX):
+        H, gamma, rstd = ctx.saved_tensors
+        dH, dgamma = _abi.rmsnorm_backward(H, gamma, rstd, dX.contiguous())
+        return dH, dgamma, None
+
+
+def rmsnorm(H, gamma, eps: float = 1e-6):
+    """x = h / sqrt(mean(h^2) + eps) * gamma, with a backward into H and gamma."""
+    return RMSNorm.apply(H, gamma, eps)

@@ -694,6 +694,72 @@ int flce_forward_noalloc(const flce_shape* shape, const void* X, const void* W,
                       FLCE_NOALLOC_SCRATCH_BYTES, stream);
 }
 
+constexpr int kRmsRowsPerPart = 128;
+
+int rms_args_ok(const void* H, const void* gamma, int64_t N, int64_t d) {
+  if (N < 0 || d <= 0 || d > (int64_t(1) << 24) || gamma == nullptr || (N > 0 && H == nullptr))
+    return FLCE_ERR_ARG;
+  if ((d % 8) != 0 || !aligned16(H) || !aligned16(gamma)) return FLCE_ERR_ALIGN;
+  return FLCE_OK;
+}
+
+int flce_rmsnorm_forward(const void* H, const void* gamma, float eps, int64_t N, int64_t d,
+                         void* X, float* rstd, void* stream) {
+  FLCE_TRY(rms_args_ok(H, gamma, N, d));
+  if (!(eps >= 0.f) || (N > 0 && (X == nullptr || rstd == nullptr))) return FLCE_ERR_ARG;
+  if (!aligned16(X)) return FLCE_ERR_ALIGN;
+  DeviceInfo* di = nullptr;
+  FLCE_TRY(device_info(&di));
+  if (N == 0) return FLCE_OK;
+  rmsnorm_fwd_kernel<<<static_cast<unsigned>((N + 7) / 8), 256, 0,
+                       static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const __nv_bfloat16*>(H), static_cast<const __nv_bfloat16*>(gamma), eps, N,
+      static_cast<int>(d), static_cast<__nv_bfloat16*>(X), rstd);
+  return launch_ok();
+}
+
+size_t flce_rmsnorm_workspace_bytes(int64_t N, int64_t d) {
+  if (N < 0 || d <= 0) return 0;
+  const int64_t parts = N > 0 ? (N + kRmsRowsPerPart - 1) / kRmsRowsPerPart : 1;
+  return align_up(static_cast<size_t>(parts) * static_cast<size_t>(d) * sizeof(float));
+}
+
+int flce_rmsnorm_backward(const void* H, const void* gamma, const float* rstd, const void* dX,
+                          int64_t N, int64_t d, void* dH, float* dgamma, int accumulate_dgamma,
+                          void* workspace, size_t workspace_bytes, void* stream) {
+  FLCE_TRY(rms_args_ok(H, gamma, N, d));
+  if (dgamma == nullptr || workspace == nullptr ||
+      (N > 0 && (rstd == nullptr || dX == nullptr || dH == nullptr)))
+    return FLCE_ERR_ARG;
+  if (!aligned16(dX) || !aligned16(dH) || (reinterpret_cast<uintptr_t>(dgamma) & 3u) != 0 ||
+      (reinterpret_cast<uintptr_t>(workspace) & 15u) != 0)
+    return FLCE_ERR_ALIGN;
+  if (workspace_bytes < flce_rmsnorm_workspace_bytes(N, d)) return FLCE_ERR_WORKSPACE;
+  DeviceInfo* di = nullptr;
+  FLCE_TRY(device_info(&di));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const auto* Hb = static_cast<const __nv_bfloat16*>(H);
+  const auto* dXb = static_cast<const __nv_bfloat16*>(dX);
+  const int di32 = static_cast<int>(d);
+  float* partial = static_cast<float*>(workspace);
+  int parts = 1;
+  if (N > 0) {
+    rmsnorm_bwd_rows_kernel<<<static_cast<unsigned>((N + 7) / 8), 256, 0, st>>>(
+        Hb, static_cast<const __nv_bfloat16*>(gamma), rstd, dXb, N, di32,
+        static_cast<__nv_bfloat16*>(dH));
+    FLCE_TRY(launch_ok());
+    parts = static_cast<int>((N + kRmsRowsPerPart - 1) / kRmsRowsPerPart);
+    rmsnorm_dgamma_partial_kernel<<<dim3((di32 + 255) / 256, parts), 256, 0, st>>>(
+        Hb, rstd, dXb, N, di32, kRmsRowsPerPart, partial);
+    FLCE_TRY(launch_ok());
+  } else {
+    parts = 0;
+  }
+  rmsnorm_dgamma_final_kernel<<<(di32 + 255) / 256, 256, 0, st>>>(partial, parts, di32, dgamma,
+                                                                    accumulate_dgamma);
+  return launch_ok();
+}
+
 int flce_selftest_wait_timeout(void* workspace, uint64_t limit_ns, void* stream) {
   if (workspace == nullptr) return FLCE_ERR_ARG;
   if ((reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0) return FLCE_ERR_ALIGN;

@@ -256,6 +256,128 @@ __global__ void __launch_bounds__(1024) count_valid_kernel(const long long* __re
   }
 }
 
+// ---------------------------------------------------------------- final RMSNorm before the head
+// x_i = h_i * rstd_i * gamma, rstd_i = 1 / sqrt(mean_k h_ik^2 + eps); fp32 arithmetic, bf16 x.
+// One warp per row; every lane handles 8 contiguous columns per step (d % 8 == 0).
+__global__ void __launch_bounds__(256) rmsnorm_fwd_kernel(const __nv_bfloat16* __restrict__ H,
+                                                          const __nv_bfloat16* __restrict__ gamma,
+                                                          float eps, long long N, int d,
+                                                          __nv_bfloat16* __restrict__ X,
+                                                          float* __restrict__ rstd_out) {
+  const long long row = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (row >= N) return;
+  const __nv_bfloat16* h = H + row * d;
+  float ss = 0.f;
+  for (int k = lane * 8; k < d; k += 256) {
+    const uint4 raw = *reinterpret_cast<const uint4*>(h + k);
+    const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float2 f = __bfloat1622float2(p2[q]);
+      ss = fmaf(f.x, f.x, fmaf(f.y, f.y, ss));
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  const float rstd = 1.0f / sqrtf(ss / static_cast<float>(d) + eps);
+  if (lane == 0) rstd_out[row] = rstd;
+  __nv_bfloat16* x = X + row * d;
+  for (int k = lane * 8; k < d; k += 256) {
+    const uint4 raw = *reinterpret_cast<const uint4*>(h + k);
+    const uint4 graw = *reinterpret_cast<const uint4*>(gamma + k);
+    const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+    const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&graw);
+    uint4 w;
+    uint32_t* wo = reinterpret_cast<uint32_t*>(&w);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float2 f = __bfloat1622float2(p2[q]);
+      const float2 g = __bfloat1622float2(g2[q]);
+      wo[q] = pack_bf16x2(f.x * rstd * g.x, f.y * rstd * g.y);
+    }
+    *reinterpret_cast<uint4*>(x + k) = w;
+  }
+}
+
+// dH_i = rstd_i (g_i - xh_i mean_k(g_ik xh_ik)) with xh = h * rstd and g = dX * gamma.
+__global__ void __launch_bounds__(256) rmsnorm_bwd_rows_kernel(
+    const __nv_bfloat16* __restrict__ H, const __nv_bfloat16* __restrict__ gamma,
+    const float* __restrict__ rstd_in, const __nv_bfloat16* __restrict__ dX, long long N, int d,
+    __nv_bfloat16* __restrict__ dH) {
+  const long long row = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (row >= N) return;
+  const float rstd = rstd_in[row];
+  const __nv_bfloat16* h = H + row * d;
+  const __nv_bfloat16* dx = dX + row * d;
+  float dot = 0.f;
+  for (int k = lane * 8; k < d; k += 256) {
+    const uint4 hr = *reinterpret_cast<const uint4*>(h + k);
+    const uint4 dr = *reinterpret_cast<const uint4*>(dx + k);
+    const uint4 gr = *reinterpret_cast<const uint4*>(gamma + k);
+    const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&hr);
+    const __nv_bfloat162* d2 = reinterpret_cast<const __nv_bfloat162*>(&dr);
+    const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&gr);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float2 hf = __bfloat1622float2(h2[q]);
+      const float2 df = __bfloat1622float2(d2[q]);
+      const float2 gf = __bfloat1622float2(g2[q]);
+      dot = fmaf(df.x * gf.x, hf.x * rstd, dot);
+      dot = fmaf(df.y * gf.y, hf.y * rstd, dot);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+  const float mean_dot = dot / static_cast<float>(d);
+  __nv_bfloat16* out = dH + row * d;
+  for (int k = lane * 8; k < d; k += 256) {
+    const uint4 hr = *reinterpret_cast<const uint4*>(h + k);
+    const uint4 dr = *reinterpret_cast<const uint4*>(dx + k);
+    const uint4 gr = *reinterpret_cast<const uint4*>(gamma + k);
+    const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&hr);
+    const __nv_bfloat162* d2 = reinterpret_cast<const __nv_bfloat162*>(&dr);
+    const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&gr);
+    uint4 w;
+    uint32_t* wo = reinterpret_cast<uint32_t*>(&w);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float2 hf = __bfloat1622float2(h2[q]);
+      const float2 df = __bfloat1622float2(d2[q]);
+      const float2 gf = __bfloat1622float2(g2[q]);
+      wo[q] = pack_bf16x2(rstd * (df.x * gf.x - hf.x * rstd * mean_dot),
+                          rstd * (df.y * gf.y - hf.y * rstd * mean_dot));
+    }
+    *reinterpret_cast<uint4*>(out + k) = w;
+  }
+}
+
+// dgamma_k = sum_i dX_ik h_ik rstd_i in two deterministic stages: per block of `rows_per_part`
+// rows a partial sum per column, then the partials summed in order.
+__global__ void __launch_bounds__(256) rmsnorm_dgamma_partial_kernel(
+    const __nv_bfloat16* __restrict__ H, const float* __restrict__ rstd_in,
+    const __nv_bfloat16* __restrict__ dX, long long N, int d, int rows_per_part,
+    float* __restrict__ partial) {
+  const int k = blockIdx.x * blockDim.x + threadIdx.x;
+  if (k >= d) return;
+  const long long r0 = static_cast<long long>(blockIdx.y) * rows_per_part;
+  const long long r1 = r0 + rows_per_part < N ? r0 + rows_per_part : N;
+  float acc = 0.f;
+  for (long long i = r0; i < r1; ++i)
+    acc = fmaf(__bfloat162float(dX[i * d + k]), __bfloat162float(H[i * d + k]) * rstd_in[i], acc);
+  partial[static_cast<long long>(blockIdx.y) * d + k] = acc;
+}
+
+__global__ void rmsnorm_dgamma_final_kernel(const float* __restrict__ partial, int parts, int d,
+                                            float* __restrict__ dgamma, int accumulate) {
+  const int k = blockIdx.x * blockDim.x + threadIdx.x;
+  if (k >= d) return;
+  float acc = 0.f;
+  for (int b = 0; b < parts; ++b) acc += partial[static_cast<long long>(b) * d + k];
+  dgamma[k] = accumulate ? dgamma[k] + acc : acc;
+}
+
 // Self-test of the bounded wait used by every pipeline barrier: one thread initialises an
 // mbarrier that expects one arrival, never arrives, and waits on it with the given limit.  The
 // wait gives up, raises DEV_TIMEOUT in *status and the kernel returns normally.
