@@ -4,10 +4,12 @@
 // Launch sequence of one fused forward + backward (flce_forward with want_grads = 1):
 //   prep_targets                                  targets -> effective ids, Nv, status
 //   for each chunk of Nc rows:
-//     logits GEMM   z = X_c W^T  (tcgen05, fused softcap / sum-exp / target / A' epilogue)
+//     logits GEMM   z = X_c W^T  (tcgen05 on SM pairs, fused softcap / sum-exp / target /
+//                   gradient-operand epilogue)
 //     row_finish    lse, per-row loss, r = 1/(Nv S), target patch of A', Xs = r . X_c
-//     dX GEMM       dX_c = r . (A' W)              (A' K-major, W MN-major)
-//     dW GEMM       dW (+)= A'^T Xs                (both MN-major)
+//     grad GEMMs    one balanced launch of both contractions:
+//                     dX_c = r . (A' W)     (A' K-major, W MN-major)
+//                     dW (+)= A'^T Xs       (both MN-major)
 //   loss          deterministic mean over rows in the loss
 // The logits of a chunk exist only as the bf16 operand A' [Nc, Vpad]; nothing of size N x Vpad
 // is ever allocated.
@@ -28,15 +30,31 @@ using namespace flce;
 
 namespace {
 
-// Contraction tiles: pairs of SMs (cta_group::2), 256 x 256 tiles, 6-stage shared-memory ring.
-using Cfg = PairCfg<256, 6, 8>;
+// Contraction tiles: pairs of SMs (cta_group::2), 256-row tiles, shared-memory rings of
+// 32 KB stages.  Build-time tuning constants (measured defaults).
+#ifndef FLCE_LOGITS_BN
+#define FLCE_LOGITS_BN 256
+#endif
+#ifndef FLCE_LOGITS_STAGES
+#define FLCE_LOGITS_STAGES 6
+#endif
+#ifndef FLCE_GRAD_STAGES
+#define FLCE_GRAD_STAGES 6
+#endif
+#ifndef FLCE_EPI_WARPS
+#define FLCE_EPI_WARPS 8
+#endif
+using Cfg = PairCfg<256, FLCE_GRAD_STAGES, FLCE_EPI_WARPS>;
+using CfgL = PairCfg<FLCE_LOGITS_BN, FLCE_LOGITS_STAGES, FLCE_EPI_WARPS>;
 // logits: A = X (K-major), B = W (K-major)
 constexpr auto kLogitsKernel =
-    gemm_pair_kernel<Cfg, LogitsEpi, LogitsEpi, Major::K, Major::K, Major::K, Major::K>;
+    gemm_pair_kernel<CfgL, LogitsEpi, LogitsEpi, Major::K, Major::K, Major::K, Major::K>;
 // logits from e4m3 operands (kind::f8f6f4, tensorwise scales applied in the epilogue)
-using Cfg8 = PairCfg<256, 6, 8, 1>;
+using Cfg8 = PairCfg<FLCE_LOGITS_BN, FLCE_LOGITS_STAGES, FLCE_EPI_WARPS, 1>;
 constexpr auto kLogitsKernel8 =
     gemm_pair_kernel<Cfg8, LogitsEpi, LogitsEpi, Major::K, Major::K, Major::K, Major::K>;
+static_assert(CfgL::BN == Cfg8::BN && CfgL::COL_SPLIT == Cfg8::COL_SPLIT,
+              "both logits kernels fill the same per-row partial slots");
 // gradients in one launch: dX = A' W (A' K-major, W MN-major), dW = A'^T Xs (both MN-major)
 constexpr auto kGradKernel =
     gemm_pair_kernel<Cfg, DxEpi, DwEpi, Major::K, Major::MN, Major::MN, Major::MN>;
@@ -74,8 +92,8 @@ Layout make_layout(const flce_shape* s, int want_grads) {
   if (nc < 1) nc = 1;
   L.chunk = nc;
   L.fixed_ref = s->cap > 0.f && s->cap <= kFixedRefMaxCap;
-  const int64_t vtiles = (s->Vpad + Cfg::BN - 1) / Cfg::BN;
-  L.n_slabs = static_cast<int>(vtiles * Cfg::COL_SPLIT);
+  const int64_t vtiles = (s->Vpad + CfgL::BN - 1) / CfgL::BN;
+  L.n_slabs = static_cast<int>(vtiles * CfgL::COL_SPLIT);
   size_t off = 0;
   auto take = [&](size_t bytes) {
     const size_t at = off;
@@ -128,7 +146,7 @@ int device_info(DeviceInfo** out) {
   if (!di.ok) return FLCE_ERR_DEVICE;
   if (!di.attrs_set) {
     if (cudaFuncSetAttribute(kLogitsKernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             Cfg::SMEM_BYTES) != cudaSuccess ||
+                             CfgL::SMEM_BYTES) != cudaSuccess ||
         cudaFuncSetAttribute(kGradKernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              Cfg::SMEM_BYTES) != cudaSuccess ||
         cudaFuncSetAttribute(kLogitsKernel8, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -210,9 +228,10 @@ cudaEvent_t pooled_event() {
   return e;
 }
 
+template <class CF>
 long long pair_tiles(const PairProblem& p) {
   if (p.M <= 0 || p.N <= 0) return 0;
-  return static_cast<long long>((p.M + Cfg::BM - 1) / Cfg::BM) * ((p.N + Cfg::BN - 1) / Cfg::BN);
+  return static_cast<long long>((p.M + CF::BM - 1) / CF::BM) * ((p.N + CF::BN - 1) / CF::BN);
 }
 
 // Launch one persistent pair kernel over one or two problems; `kind` labels the launch for the
@@ -222,7 +241,7 @@ int launch_pair(K kernel, const DeviceInfo* di, const CUtensorMap& a0, const CUt
                 const CUtensorMap& a1, const CUtensorMap& b1, const PairProblem& p0,
                 const PairProblem& p1, uint32_t* status, const typename E0::Params& e0,
                 const typename E1::Params& e1, cudaStream_t st, int kind) {
-  const long long tiles = pair_tiles(p0) + pair_tiles(p1);
+  const long long tiles = pair_tiles<CF>(p0) + pair_tiles<CF>(p1);
   if (tiles <= 0) return FLCE_OK;
   const long long units = di->sms / 2;   // one CTA pair per SM pair, persistent
   const int grid = static_cast<int>(2 * (tiles < units ? tiles : units));
@@ -301,14 +320,15 @@ int launch_logits(const Ctx& c, int64_t row0, int rows, const __nv_bfloat16* X,
     return launch_pair<LogitsEpi, LogitsEpi, Cfg8>(kLogitsKernel8, c.di, mX, mW, mX, mW, logits,
                                                     none, &c.hdr->status, lp, lp, c.st, 0);
   }
-  FLCE_TRY(make_map(&mX, X + row0 * s->d, d, rows, d, Cfg::BM_CTA));
-  FLCE_TRY(make_map(&mW, W, d, Vpad, d, Cfg::BN_CTA));
+  FLCE_TRY(make_map(&mX, X + row0 * s->d, d, rows, d, CfgL::BM_CTA));
+  FLCE_TRY(make_map(&mW, W, d, Vpad, d, CfgL::BN_CTA));
   lp.scale_a = lp.scale_b = nullptr;
-  return launch_pair<LogitsEpi, LogitsEpi>(kLogitsKernel, c.di, mX, mW, mX, mW, logits, none,
-                                           &c.hdr->status, lp, lp, c.st, 0);
+  return launch_pair<LogitsEpi, LogitsEpi, CfgL>(kLogitsKernel, c.di, mX, mW, mX, mW, logits,
+                                                  none, &c.hdr->status, lp, lp, c.st, 0);
 }
 
-// One chunk of the gradient path: logits GEMM (mode FUSED or RECOMPUTE), row finish, dX, dW.
+// One chunk of the gradient path: logits GEMM (mode FUSED or RECOMPUTE), row finish, and the
+// dX / dW contractions in one launch.
 int grad_chunk(const Ctx& c, int64_t row0, int rows, const __nv_bfloat16* X,
                const __nv_bfloat16* W, const float* lse_in, float* lse_out, const float* grad_out,
                __nv_bfloat16* dX, float* dW, int accumulate, int mode) {

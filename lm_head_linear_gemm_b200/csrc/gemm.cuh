@@ -1,12 +1,12 @@
 // Persistent, warp-specialised tcgen05 GEMM for sm_100a with fused epilogues.
 //
-//   D[M, N] = A[M, K] * B[N, K]^T, bf16 operands, fp32 accumulation in TMEM.
+//   D[M, N] = A[M, K] * B[N, K]^T, bf16 (or e4m3) operands, fp32 accumulation in TMEM.
 //
 // Runs on pairs of SMs (2-CTA clusters, tcgen05 cta_group::2).  Roles in each CTA
 // (64 + 32*EPI_WARPS threads, one CTA per SM):
 //   warp 0 lane 0 : TMA producer, STAGES-deep shared-memory ring of (A, B) k-blocks;
 //   warp 1        : TMEM allocator; lane 0 of the leader CTA issues tcgen05.mma
-//                   (M=256 across the pair, N=BN, K=16);
+//                   (M=256 across the pair, N=BN, K = 32 bytes of each operand row);
 //   warps 2..     : epilogue; two TMEM accumulators so the epilogue of one tile
 //                   overlaps the main loop of the next.
 // Operands may be K-major (rows of K contiguous) or MN-major (rows of M/N
@@ -60,9 +60,10 @@ __device__ __forceinline__ uint64_t operand_desc(uint32_t base, int k) {
 // BN/2 x 128 B of B, against 16 KB + BN x 128 B on a single SM.
 //
 // One launch may carry two problems (e.g. dX = A'W and dW = A'^T Xs, whose tiles differ in
-// length by 12x): each pair first takes its round-robin share of problem 0's tiles, then a
-// contiguous run of problem 1's tiles sized so that every pair ends with about the same number
-// of k-blocks.  A launch with one problem is the plain round-robin persistent schedule.
+// length by 12x): each pair first takes its round-robin share of problem 0's tiles, then its
+// share of problem 1's tiles, handed out so that every pair ends with about the same number of
+// k-blocks while concurrently running tiles stay neighbours (pair_schedule).  A launch with one
+// problem is the plain round-robin persistent schedule.
 template <int BN_, int STAGES_, int EPI_WARPS_, int ELEM_BYTES_ = 2>
 struct PairCfg {
   static constexpr bool PAIR = true;
@@ -86,7 +87,7 @@ struct PairCfg {
   static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
   static_assert(EPI_WARPS % 4 == 0, "epilogue warps must cover the four TMEM lane quarters");
   static_assert(COLS_PER_WARP % 32 == 0, "epilogue works in 32-column TMEM loads");
-  static_assert(BN_CTA % 64 == 0, "MN-major tiles are whole 64-wide blocks");
+  static_assert(BN_CTA % 32 == 0, "B halves are whole 32-row groups (64-wide when MN-major)");
   static_assert(BN % 32 == 0 && BN >= 64 && BN <= 256, "cta_group::2 M=256 needs N % 16 == 0");
   static_assert(A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "swizzle atoms need 1 KB alignment");
   static_assert((2 * STAGES + 5) * 8 + 32 <= BAR_BYTES, "barrier area too small");
@@ -289,6 +290,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
   } else if (warp == 1) {
     if (lane == 0 && leader) {
       // ------------------------------------------------------------ MMA issuer (leader only)
+      static_assert((B0 == Major::K || C::BN_CTA % 64 == 0) && (B1 == Major::K || C::BN_CTA % 64 == 0),
+                    "MN-major B halves are whole 64-wide blocks");
       static_assert(C::ELEM_BYTES == 2 || (A0 == Major::K && B0 == Major::K && A1 == Major::K &&
                                            B1 == Major::K),
                     "e4m3 operands are staged K-major");
