@@ -47,6 +47,8 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-unfused", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--graph", action="store_true",
+                    help="device-timed steps replay one captured CUDA graph of the step")
     ap.add_argument("--accum-steps", type=int, default=7,
                     help="N>1: micro-batches per optimizer step; dW is accumulated over them and "
                          "all-reduced after the last (the write-ups: 7)")
@@ -308,6 +310,26 @@ def main_gpu(args):
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
+    timed_step = step
+    launches_per_graph_step = None
+    if args.graph and world == 1:
+        flce.instrument(True)
+        step()
+        launches_per_graph_step = flce.instrument_read()["launches_total"]
+        flce.instrument(False)
+        # one step captured into a CUDA graph (same buffers, so replays redo the whole step)
+        cap_stream = torch.cuda.Stream(device=dev)
+        cap_stream.wait_stream(torch.cuda.current_stream())
+        graph = torch.cuda.CUDAGraph()
+        holder = {}
+        with torch.cuda.graph(graph, stream=cap_stream):
+            holder["loss"] = step()
+        graph.replay()
+        torch.cuda.synchronize()
+
+        def timed_step():
+            graph.replay()
+            return holder["loss"]
     status, nv = flce.read_status(ws)
     # everything the fused step holds beyond its inputs: dX, dW, workspace, lse, loss
     peak_fused = torch.cuda.max_memory_allocated(dev) - mem_inputs
@@ -330,7 +352,7 @@ def main_gpu(args):
     torch.cuda.synchronize()
     e0.record(stream)
     for _ in range(args.steps):
-        loss = step()
+        loss = timed_step()
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
@@ -459,7 +481,9 @@ def main_gpu(args):
             "pct_of_measured_bf16_sustained": tflops / world / sustained,
             "credited_flop_per_step": credited, "executed_flop_per_step": credited,
             "roofline": roofline, "kernels": kinds, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": kstats["launches_total"],
+            "gpu_launches": kstats["launches_total"] if launches_per_graph_step is None else
+                            launches_per_graph_step * args.steps,
+            "graph_replay": bool(args.graph and world == 1),
             "gpu_launches_per_step": kstats["launches_total"] / args.steps,
             "clocks": clk,
             "clocks_nvml_10ms": nvml_clk,

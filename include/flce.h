@@ -25,8 +25,9 @@
  *     frees memory.  Scratch space is the caller's `workspace` (see flce_workspace_bytes).
  *   - Layouts are row-major and dense: X [N, d] bf16, W [Vpad, d] bf16, targets [N] int64,
  *     lse [N] fp32, loss [1] fp32, dX [N, d] bf16, dW [Vpad, d] fp32.
- *   - Every data pointer must be 16-byte aligned; d and Vpad must be multiples of 8 (the
- *     tensor-memory-accelerator row stride must be a multiple of 16 bytes).
+ *   - Every array pointer must be 16-byte aligned except loss and lse (4-byte aligned); d and
+ *     Vpad must be multiples of 8 (the tensor-memory-accelerator row stride must be a multiple
+ *     of 16 bytes).
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).  Calls are
  *     stream-ordered and asynchronous; calls on different streams are independent when their
  *     workspaces and outputs differ.

@@ -268,6 +268,7 @@ int launch_pair(K kernel, const DeviceInfo* di, const CUtensorMap& a0, const CUt
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
 #define FLCE_TRY(expr)             \
   do {                             \
@@ -502,7 +503,7 @@ int forward_impl(const flce_shape* s, const void* X, const void* W, const Fp8Log
                  void* stream, const int64_t* nv_total = nullptr) {
   want_grads = want_grads ? 1 : 0;
   if (loss == nullptr || (s->N > 0 && lse == nullptr)) return FLCE_ERR_ARG;
-  if (!aligned16(loss) || !aligned16(lse)) return FLCE_ERR_ALIGN;
+  if (!aligned4(loss) || !aligned4(lse)) return FLCE_ERR_ALIGN;
   if (want_grads) {
     if ((s->N > 0 && dX == nullptr) || dW == nullptr) return FLCE_ERR_ARG;
     if (!aligned16(dX) || !aligned16(dW)) return FLCE_ERR_ALIGN;
@@ -663,7 +664,7 @@ int flce_backward(const flce_shape* s, const void* X, const void* W, const int64
   }
   FLCE_TRY(common_checks(s, X, W, targets, workspace, workspace_bytes, 1));
   if (s->N > 0 && lse == nullptr) return FLCE_ERR_ARG;
-  if (!aligned16(lse)) return FLCE_ERR_ALIGN;
+  if (!aligned4(lse)) return FLCE_ERR_ALIGN;
   DeviceInfo* di = nullptr;
   FLCE_TRY(device_info(&di));
   Ctx c{};

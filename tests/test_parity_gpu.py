@@ -323,3 +323,42 @@ def test_concurrent_calls_on_two_streams(cuda_device):
     for q, p in zip(seq, par):
         assert torch.equal(q[0], p[0]) and torch.equal(q[1], p[1])
         assert torch.equal(q[2], p[2]) and torch.equal(q[3], p[3])
+
+
+def test_fused_step_captures_into_a_cuda_graph(cuda_device):
+    """The library makes no synchronising or host-reading call on the launch path, so a fused
+    forward + backward can be captured once and replayed; replays match eager results."""
+    import lm_head_linear_gemm_b200 as flce
+    torch = _torch()
+    inp = synth.make_inputs(RAGGED)
+    c = inp["cfg"]
+    X, W, t = to_dev(inp["X"]), to_dev(inp["W"]), to_dev(inp["targets"])
+    dX = torch.empty_like(X)
+    dW = torch.empty(W.shape, dtype=torch.float32, device="cuda")
+    g = torch.tensor(0.5, device="cuda")
+    ws = flce.alloc_workspace(flce.make_shape(c.N, c.d, c.Vpad, c.Vreal, c.cap, -1, 128), True,
+                              X.device)
+    out = {}
+
+    def step():
+        loss, lse, _, _, _ = flce.forward(X, W, t, c.Vreal, c.cap, -1, True, dX=dX, dW=dW,
+                                          workspace=ws, chunk_rows=128)
+        flce.backward(X, W, t, lse, c.Vreal, c.cap, -1, grad_out=g, dX=dX, dW=dW,
+                      grads_precomputed=True)
+        out["loss"] = loss
+
+    step()                                     # eager (also sets kernel attributes once)
+    torch.cuda.synchronize()
+    ref = (out["loss"].clone(), dX.clone(), dW.clone())
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=s):
+        step()
+    for _ in range(2):
+        dX.zero_()
+        dW.zero_()
+        graph.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(out["loss"], ref[0])
+        assert torch.equal(dX, ref[1]) and torch.equal(dW, ref[2])
