@@ -770,7 +770,7 @@ int flce_rmsnorm_backward(const void* H, const void* gamma, const float* rstd, c
         static_cast<__nv_bfloat16*>(dH));
     FLCE_TRY(launch_ok());
     parts = static_cast<int>((N + kRmsRowsPerPart - 1) / kRmsRowsPerPart);
-    rmsnorm_dgamma_partial_kernel<<<dim3((di32 + 255) / 256, parts), 256, 0, st>>>(
+    rmsnorm_dgamma_partial_kernel<<<dim3((di32 / 2 + 255) / 256, parts), 256, 0, st>>>(
         Hb, rstd, dXb, N, di32, kRmsRowsPerPart, partial);
     FLCE_TRY(launch_ok());
   } else {

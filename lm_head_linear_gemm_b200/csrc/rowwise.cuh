@@ -354,19 +354,27 @@ __global__ void __launch_bounds__(256) rmsnorm_bwd_rows_kernel(
 }
 
 // dgamma_k = sum_i dX_ik h_ik rstd_i in two deterministic stages: per block of `rows_per_part`
-// rows a partial sum per column, then the partials summed in order.
+// rows a partial sum per column, then the partials summed in order.  Each thread owns two
+// adjacent columns, so a warp reads whole 128-byte lines of each row.
 __global__ void __launch_bounds__(256) rmsnorm_dgamma_partial_kernel(
     const __nv_bfloat16* __restrict__ H, const float* __restrict__ rstd_in,
     const __nv_bfloat16* __restrict__ dX, long long N, int d, int rows_per_part,
     float* __restrict__ partial) {
-  const int k = blockIdx.x * blockDim.x + threadIdx.x;
+  const int k = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
   if (k >= d) return;
   const long long r0 = static_cast<long long>(blockIdx.y) * rows_per_part;
   const long long r1 = r0 + rows_per_part < N ? r0 + rows_per_part : N;
-  float acc = 0.f;
-  for (long long i = r0; i < r1; ++i)
-    acc = fmaf(__bfloat162float(dX[i * d + k]), __bfloat162float(H[i * d + k]) * rstd_in[i], acc);
-  partial[static_cast<long long>(blockIdx.y) * d + k] = acc;
+  float acc0 = 0.f, acc1 = 0.f;
+  for (long long i = r0; i < r1; ++i) {
+    const float2 h = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(H + i * d + k));
+    const float2 g = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(dX + i * d + k));
+    const float r = rstd_in[i];
+    acc0 = fmaf(g.x, h.x * r, acc0);
+    acc1 = fmaf(g.y, h.y * r, acc1);
+  }
+  float* prow = partial + static_cast<long long>(blockIdx.y) * d;
+  prow[k] = acc0;
+  prow[k + 1] = acc1;
 }
 
 __global__ void rmsnorm_dgamma_final_kernel(const float* __restrict__ partial, int parts, int d,

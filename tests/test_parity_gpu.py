@@ -362,3 +362,25 @@ def test_fused_step_captures_into_a_cuda_graph(cuda_device):
         torch.cuda.synchronize()
         assert torch.equal(out["loss"], ref[0])
         assert torch.equal(dX, ref[1]) and torch.equal(dW, ref[2])
+
+
+def test_targets_in_the_padded_tail_tile(cuda_device):
+    """Targets in the last real columns of the pages' vocabulary (50240..50256 share a 32-column
+    epilogue chunk with padded columns; 50176.. is the half-padded last 256-column tile), the
+    first column, and rows at chunk boundaries."""
+    c = synth.custom_config("tail", N=260, d=128, Vreal=50257, Vpad=50304, x_dist="normal",
+                            w_std=0.05, target_dist="uniform", ignore_count=0)
+    inp = synth.make_inputs(c)
+    t = inp["targets"].copy()
+    special = [50256, 50255, 50240, 50239, 50176, 50175, 0, 1, 31, 32]
+    t[:len(special)] = special
+    t[127], t[128], t[255], t[256] = 50256, 50240, 0, 50255      # around 128-row chunk edges
+    inp = dict(inp, targets=t)
+    ref = oracle_full(inp)
+    for chunk in (0, 128):
+        got = run_gpu(inp, chunk_rows=chunk)
+        compare_full(got, ref)
+        assert np.abs(got["dW"][50257:]).max() == 0.0
+        # the target rows of dW carry the -1 of the one-hot: check them element by element
+        rows = np.array(sorted(set(special)))
+        check_tensor("dW target rows", got["dW"][rows], ref["dW"][rows])
