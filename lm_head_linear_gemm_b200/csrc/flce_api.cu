@@ -44,6 +44,10 @@ namespace {
 #ifndef FLCE_EPI_WARPS
 #define FLCE_EPI_WARPS 8
 #endif
+// dX in wide tiles (256 x 512 per SM pair, two accumulators sharing each staged A' k-block)
+#ifndef FLCE_DX_WIDE
+#define FLCE_DX_WIDE 1
+#endif
 using Cfg = PairCfg<256, FLCE_GRAD_STAGES, FLCE_EPI_WARPS>;
 using CfgL = PairCfg<FLCE_LOGITS_BN, FLCE_LOGITS_STAGES, FLCE_EPI_WARPS>;
 // logits: A = X (K-major), B = W (K-major)
@@ -56,8 +60,8 @@ constexpr auto kLogitsKernel8 =
 static_assert(CfgL::BN == Cfg8::BN && CfgL::COL_SPLIT == Cfg8::COL_SPLIT,
               "both logits kernels fill the same per-row partial slots");
 // gradients in one launch: dX = A' W (A' K-major, W MN-major), dW = A'^T Xs (both MN-major)
-constexpr auto kGradKernel =
-    gemm_pair_kernel<Cfg, DxEpi, DwEpi, Major::K, Major::MN, Major::MN, Major::MN>;
+constexpr auto kGradKernel = gemm_pair_kernel<Cfg, DxEpi, DwEpi, Major::K, Major::MN, Major::MN,
+                                             Major::MN, FLCE_DX_WIDE != 0>;
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s bound on every in-kernel wait
 constexpr float kFixedRefMaxCap = 32.f;           // exp(s - cap) >= e^{-64}: no underflow in fp32
@@ -311,7 +315,7 @@ int launch_logits(const Ctx& c, int64_t row0, int rows, const __nv_bfloat16* X,
                   const __nv_bfloat16* W, LogitsParams lp) {
   const flce_shape* s = c.s;
   const int d = static_cast<int>(s->d), Vpad = static_cast<int>(s->Vpad);
-  const PairProblem logits{rows, Vpad, d, 1}, none{0, 0, 0, 0};
+  const PairProblem logits{rows, Vpad, d, 1, 0}, none{0, 0, 0, 0, 0};
   CUtensorMap mX, mW;
   if (c.fp8.X8 != nullptr) {
     FLCE_TRY(make_map(&mX, c.fp8.X8 + row0 * s->d, d, rows, d, Cfg8::BM_CTA, 1));
@@ -395,7 +399,7 @@ int grad_chunk(const Ctx& c, int64_t row0, int rows, const __nv_bfloat16* X,
   // dX (long tiles: K = Vpad) and dW (short tiles: K = rows) share one balanced launch
   DxParams xp{rows, d, r, dX + row0 * s->d};
   DwParams wp{Vpad, d, accumulate, dW};
-  const PairProblem pdx{rows, d, Vpad, 0}, pdw{Vpad, d, rows, 0};
+  const PairProblem pdx{rows, d, Vpad, 0, FLCE_DX_WIDE}, pdw{Vpad, d, rows, 0, 0};
   FLCE_TRY((launch_pair<DxEpi, DwEpi>(kGradKernel, c.di, mA_k, mW_mn, mA_mn, mXs_mn, pdx, pdw,
                                        &c.hdr->status, xp, wp, c.st, 1)));
   return FLCE_OK;

@@ -94,9 +94,15 @@ struct PairCfg {
   static_assert(SMEM_BYTES <= 232448, "more than 227 KB of shared memory");
 };
 
+template <int V>
+struct IntC {
+  static constexpr int value = V;
+};
+
 struct PairProblem {
   int M, N, K;          // extents; M == 0 marks an absent second problem
   int m_fastest;        // tile order: 1 = consecutive tiles walk M first
+  int wide;             // problem 0 only: 1 = wide tiles (see below)
 };
 
 struct PairArgs {
@@ -137,7 +143,7 @@ __device__ inline PairSchedule pair_schedule(int pair, int P, int T0, int c0, in
   return s;
 }
 
-template <class C, class E0, class E1, Major A0, Major B0, Major A1, Major B1>
+template <class C, class E0, class E1, Major A0, Major B0, Major A1, Major B1, bool WIDE0 = false>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
                      const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
@@ -169,6 +175,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
   const int m_tiles1 = (args.prob[1].M + C::BM - 1) / C::BM;
   const int n_tiles1 = (args.prob[1].N + C::BN - 1) / C::BN;
   const int nkb1 = (args.prob[1].K + C::BK - 1) / C::BK;
+  // Wide tiles (problem 0, bf16): two adjacent BN-column blocks share every staged k-block of
+  // A, one TMEM accumulator each, so a pair stages 256 + 512 operand rows per k-block instead
+  // of 2 x (256 + 256).  The second B block goes into the next ring slot (its A area unused),
+  // so a wide k-block takes two slots and the ring stays in step as long as the slot count and
+  // the number of N blocks are even.  Meant for long-K problems: while a wide tile runs, no
+  // accumulator is free for the epilogue of the previous tile to overlap with.
+  const bool wide0 = WIDE0 && args.prob[0].wide != 0 && C::ELEM_BYTES == 2 &&
+                     (C::STAGES % 2) == 0 && (n_tiles0 % 2) == 0;
+  const int w_tiles0 = wide0 ? n_tiles0 / 2 : n_tiles0;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
@@ -181,7 +196,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
-    const PairSchedule ps = pair_schedule(pair, npairs, m_tiles0 * n_tiles0, nkb0,
+    const PairSchedule ps = pair_schedule(pair, npairs, m_tiles0 * w_tiles0,
+                                          wide0 ? 2 * nkb0 : nkb0,
                                           args.prob[1].M > 0 ? m_tiles1 * n_tiles1 : 0,
                                           nkb1 > 0 ? nkb1 : 1);
     sched[0] = ps.n0;
@@ -211,14 +227,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
   const uint32_t leader_full = mapa_shared(smem_u32(full), 0);
   const uint32_t leader_tempty = mapa_shared(smem_u32(tempty), 0);
 
-  // i-th tile of this pair -> (problem, m block, n block, k-blocks)
+  // i-th tile of this pair -> (problem, m block, n block, k-blocks); in a wide problem 0,
+  // nb indexes pairs of N blocks (2 nb and 2 nb + 1).
   auto tile_of = [&](int i, int& prob, int& mb, int& nb, int& kbs) {
     int t, mt, nt, mf;
     if (i < n0) {
       prob = 0;
       t = pair + i * npairs;
       mt = m_tiles0;
-      nt = n_tiles0;
+      nt = w_tiles0;
       mf = args.prob[0].m_fastest;
       kbs = nkb0;
     } else {
@@ -238,6 +255,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
       mb = t / nt;
     }
   };
+  // Every role walks this pair's tiles in order; the wide tiles (all of problem 0, when wide0)
+  // come first and run with NSUB = 2 known at compile time, everything else with NSUB = 1.
+  auto for_each_run = [&](auto&& run) {
+    if constexpr (WIDE0) {
+      if (wide0) {
+        run(IntC<2>{}, 0, n0);
+        run(IntC<1>{}, n0, total);
+        return;
+      }
+    }
+    run(IntC<1>{}, 0, total);
+  };
 
   if (warp == 0) {
     if (lane == 0) {
@@ -245,34 +274,51 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
       int stage = 0;
       uint32_t phase = 0;
       long long arms = 0;
-      for (int i = 0; i < total && !*abort_flag; ++i) {
-        int prob, mb, nb, kbs;
-        tile_of(i, prob, mb, nb, kbs);
-        const int a_row = mb * C::BM + static_cast<int>(rank) * C::BM_CTA;
-        const int b_row = nb * C::BN + static_cast<int>(rank) * C::BN_CTA;
-        for (int kb = 0; kb < kbs; ++kb) {
-          if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, args.status, args.limit_ns)) {
-            *abort_flag = 1;
-            break;
-          }
-          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * C::STAGE_BYTES);
-          uint8_t* sA = smem + stage * C::STAGE_BYTES;
-          uint8_t* sB = sA + C::A_BYTES;
-          const uint32_t bar = leader_full + 8u * stage;
-          if (prob == 0) {
-            load_operand_pair<A0, C::BM_CTA>(sA, &tmA0, bar, a_row, kb * C::BK);
-            load_operand_pair<B0, C::BN_CTA>(sB, &tmB0, bar, b_row, kb * C::BK);
-          } else {
-            load_operand_pair<A1, C::BM_CTA>(sA, &tmA1, bar, a_row, kb * C::BK);
-            load_operand_pair<B1, C::BN_CTA>(sB, &tmB1, bar, b_row, kb * C::BK);
-          }
-          ++arms;
-          if (++stage == C::STAGES) {
-            stage = 0;
-            phase ^= 1u;
+      for_each_run([&](auto nsub_c, int i0, int i1) {
+        constexpr int NSUB = decltype(nsub_c)::value;
+        for (int i = i0; i < i1 && !*abort_flag; ++i) {
+          int prob, mb, nb, kbs;
+          tile_of(i, prob, mb, nb, kbs);
+          const int a_row = mb * C::BM + static_cast<int>(rank) * C::BM_CTA;
+          const int b_row = nb * NSUB * C::BN + static_cast<int>(rank) * C::BN_CTA;
+          for (int kb = 0; kb < kbs; ++kb) {
+            // a wide k-block starts on an even slot, so stage + 1 is in the same ring phase
+            if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, args.status, args.limit_ns)) {
+              *abort_flag = 1;
+              break;
+            }
+            if constexpr (NSUB == 2) {
+              if (!mbar_wait_bounded(&empty[stage + 1], phase ^ 1u, args.status, args.limit_ns)) {
+                *abort_flag = 1;
+                break;
+              }
+            }
+            if (leader) {
+              mbar_arrive_expect_tx(&full[stage], 2 * C::STAGE_BYTES);
+              if constexpr (NSUB == 2) mbar_arrive_expect_tx(&full[stage + 1], 2 * C::B_BYTES);
+            }
+            uint8_t* sA = smem + stage * C::STAGE_BYTES;
+            uint8_t* sB = sA + C::A_BYTES;
+            const uint32_t bar = leader_full + 8u * stage;
+            if (prob == 0) {
+              load_operand_pair<A0, C::BM_CTA>(sA, &tmA0, bar, a_row, kb * C::BK);
+              load_operand_pair<B0, C::BN_CTA>(sB, &tmB0, bar, b_row, kb * C::BK);
+              if constexpr (NSUB == 2)
+                load_operand_pair<B0, C::BN_CTA>(sB + C::STAGE_BYTES, &tmB0, bar + 8u,
+                                                 b_row + C::BN, kb * C::BK);
+            } else {
+              load_operand_pair<A1, C::BM_CTA>(sA, &tmA1, bar, a_row, kb * C::BK);
+              load_operand_pair<B1, C::BN_CTA>(sB, &tmB1, bar, b_row, kb * C::BK);
+            }
+            arms += NSUB;
+            stage += NSUB;
+            if (stage == C::STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
           }
         }
-      }
+      });
       if (leader) {
         // Drain: the last phases of every stage include both CTAs' copies.
         const long long first = arms > C::STAGES ? arms - C::STAGES : 0;
@@ -306,56 +352,90 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
       int acc = 0;
       uint32_t acc_phase = 0;
       bool issued = false;
-      for (int i = 0; i < total && !*abort_flag; ++i) {
-        int prob, mb, nb, kbs;
-        tile_of(i, prob, mb, nb, kbs);
-        if (!mbar_wait_bounded_cluster(&tempty[acc], acc_phase ^ 1u, args.status, args.limit_ns)) {
-          *abort_flag = 1;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * C::BN);
-        bool ok = true;
-        for (int kb = 0; kb < kbs; ++kb) {
-          if (!mbar_wait_bounded(&full[stage], phase, args.status, args.limit_ns)) {
+      for_each_run([&](auto nsub_c, int i0, int i1) {
+        constexpr int NSUB = decltype(nsub_c)::value;
+        for (int i = i0; i < i1 && !*abort_flag; ++i) {
+          int prob, mb, nb, kbs;
+          tile_of(i, prob, mb, nb, kbs);
+          // a wide tile takes both accumulators: acc, then the other one
+          const int acc2 = acc ^ 1;
+          const uint32_t acc2_phase = acc == 1 ? acc_phase ^ 1u : acc_phase;
+          if (!mbar_wait_bounded_cluster(&tempty[acc], acc_phase ^ 1u, args.status,
+                                         args.limit_ns)) {
             *abort_flag = 1;
-            ok = false;
-            break;
+            return;
+          }
+          if constexpr (NSUB == 2) {
+            if (!mbar_wait_bounded_cluster(&tempty[acc2], acc2_phase ^ 1u, args.status,
+                                           args.limit_ns)) {
+              *abort_flag = 1;
+              return;
+            }
           }
           tc_fence_after();
-          const uint32_t a_base = smem_u32(smem + stage * C::STAGE_BYTES);
-          const uint32_t b_base = a_base + C::A_BYTES;
-          if constexpr (C::ELEM_BYTES == 1) {
+          const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * C::BN);
+          for (int kb = 0; kb < kbs; ++kb) {
+            if (!mbar_wait_bounded(&full[stage], phase, args.status, args.limit_ns)) {
+              *abort_flag = 1;
+              return;
+            }
+            if constexpr (NSUB == 2) {
+              if (!mbar_wait_bounded(&full[stage + 1], phase, args.status, args.limit_ns)) {
+                *abort_flag = 1;
+                return;
+              }
+            }
+            tc_fence_after();
+            const uint32_t a_base = smem_u32(smem + stage * C::STAGE_BYTES);
+            const uint32_t b_base = a_base + C::A_BYTES;
+            if constexpr (C::ELEM_BYTES == 1) {
 #pragma unroll
-            for (int k = 0; k < C::BK / C::MMA_K; ++k)
-              mma_e4m3_ss_pair(d_tmem, operand_desc<Major::K>(a_base, k),
-                               operand_desc<Major::K>(b_base, k), prob == 0 ? idesc0 : idesc1,
-                               (kb | k) != 0 ? 1u : 0u);
-          } else if (prob == 0) {
+              for (int k = 0; k < C::BK / C::MMA_K; ++k)
+                mma_e4m3_ss_pair(d_tmem, operand_desc<Major::K>(a_base, k),
+                                 operand_desc<Major::K>(b_base, k), prob == 0 ? idesc0 : idesc1,
+                                 (kb | k) != 0 ? 1u : 0u);
+            } else if constexpr (NSUB == 2) {
+              // both N blocks from one staged A k-block; the second B block is in the next slot
+              const uint32_t d_tmem2 = tmem_base + static_cast<uint32_t>(acc2 * C::BN);
+              const uint32_t b_base2 = b_base + C::STAGE_BYTES;
 #pragma unroll
-            for (int k = 0; k < C::BK / C::MMA_K; ++k)
-              mma_bf16_ss_pair(d_tmem, operand_desc<A0>(a_base, k), operand_desc<B0>(b_base, k),
-                               idesc0, (kb | k) != 0 ? 1u : 0u);
-          } else {
+              for (int k = 0; k < C::BK / C::MMA_K; ++k) {
+                mma_bf16_ss_pair(d_tmem, operand_desc<A0>(a_base, k), operand_desc<B0>(b_base, k),
+                                 idesc0, (kb | k) != 0 ? 1u : 0u);
+                mma_bf16_ss_pair(d_tmem2, operand_desc<A0>(a_base, k),
+                                 operand_desc<B0>(b_base2, k), idesc0, (kb | k) != 0 ? 1u : 0u);
+              }
+            } else if (prob == 0) {
 #pragma unroll
-            for (int k = 0; k < C::BK / C::MMA_K; ++k)
-              mma_bf16_ss_pair(d_tmem, operand_desc<A1>(a_base, k), operand_desc<B1>(b_base, k),
-                               idesc1, (kb | k) != 0 ? 1u : 0u);
+              for (int k = 0; k < C::BK / C::MMA_K; ++k)
+                mma_bf16_ss_pair(d_tmem, operand_desc<A0>(a_base, k), operand_desc<B0>(b_base, k),
+                                 idesc0, (kb | k) != 0 ? 1u : 0u);
+            } else {
+#pragma unroll
+              for (int k = 0; k < C::BK / C::MMA_K; ++k)
+                mma_bf16_ss_pair(d_tmem, operand_desc<A1>(a_base, k), operand_desc<B1>(b_base, k),
+                                 idesc1, (kb | k) != 0 ? 1u : 0u);
+            }
+            issued = true;
+            mma_commit_pair_both(&empty[stage]);
+            if constexpr (NSUB == 2) mma_commit_pair_both(&empty[stage + 1]);
+            stage += NSUB;
+            if (stage == C::STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
           }
-          issued = true;
-          mma_commit_pair_both(&empty[stage]);
-          if (++stage == C::STAGES) {
-            stage = 0;
-            phase ^= 1u;
+          mma_commit_pair_both(&tfull[acc]);
+          if constexpr (NSUB == 2) mma_commit_pair_both(&tfull[acc2]);
+#pragma unroll
+          for (int sub = 0; sub < NSUB; ++sub) {
+            if (++acc == 2) {
+              acc = 0;
+              acc_phase ^= 1u;
+            }
           }
         }
-        if (!ok) break;
-        mma_commit_pair_both(&tfull[acc]);
-        if (++acc == 2) {
-          acc = 0;
-          acc_phase ^= 1u;
-        }
-      }
+      });
       if (issued) {
         mma_commit_pair_both(drain);
         mbar_wait_bounded(drain, 0, args.status, args.limit_ns);
@@ -369,30 +449,37 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
     const int row_in_cta = quarter * 32 + lane;
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int i = 0; i < total && !*abort_flag; ++i) {
-      int prob, mb, nb, kbs;
-      tile_of(i, prob, mb, nb, kbs);
-      if (!mbar_wait_bounded(&tfull[acc], acc_phase, args.status, args.limit_ns)) {
-        *abort_flag = 1;
-        break;
+    for_each_run([&](auto nsub_c, int i0, int i1) {
+      constexpr int NSUB = decltype(nsub_c)::value;
+      for (int i = i0; i < i1 && !*abort_flag; ++i) {
+        int prob, mb, nb, kbs;
+        tile_of(i, prob, mb, nb, kbs);
+#pragma unroll
+        for (int sub = 0; sub < NSUB; ++sub) {   // a wide tile: its two N blocks in turn
+          if (!mbar_wait_bounded(&tfull[acc], acc_phase, args.status, args.limit_ns)) {
+            *abort_flag = 1;
+            return;
+          }
+          tc_fence_after();
+          const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
+                                 static_cast<uint32_t>(acc * C::BN + slab * C::COLS_PER_WARP);
+          const int nbs = nb * NSUB + sub;
+          const int row = mb * C::BM + static_cast<int>(rank) * C::BM_CTA + row_in_cta;
+          const int col0 = nbs * C::BN + slab * C::COLS_PER_WARP;
+          if (prob == 0)
+            E0::template apply<C::COLS_PER_WARP>(ep0, row, col0, taddr, nbs * C::COL_SPLIT + slab);
+          else
+            E1::template apply<C::COLS_PER_WARP>(ep1, row, col0, taddr, nbs * C::COL_SPLIT + slab);
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(leader_tempty + 8u * acc);
+          if (++acc == 2) {
+            acc = 0;
+            acc_phase ^= 1u;
+          }
+        }
       }
-      tc_fence_after();
-      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) +
-                             static_cast<uint32_t>(acc * C::BN + slab * C::COLS_PER_WARP);
-      const int row = mb * C::BM + static_cast<int>(rank) * C::BM_CTA + row_in_cta;
-      const int col0 = nb * C::BN + slab * C::COLS_PER_WARP;
-      if (prob == 0)
-        E0::template apply<C::COLS_PER_WARP>(ep0, row, col0, taddr, nb * C::COL_SPLIT + slab);
-      else
-        E1::template apply<C::COLS_PER_WARP>(ep1, row, col0, taddr, nb * C::COL_SPLIT + slab);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(leader_tempty + 8u * acc);
-      if (++acc == 2) {
-        acc = 0;
-        acc_phase ^= 1u;
-      }
-    }
+    });
   }
 
   __syncwarp();

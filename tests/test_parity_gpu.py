@@ -125,6 +125,21 @@ def test_ragged_multi_tile(cuda_device, chunk_rows):
     compare_full(run_gpu(inp, chunk_rows=chunk_rows, recompute=True), ref)
 
 
+WIDE = synth.custom_config("wide", N=600, d=1024, Vreal=3000, Vpad=3008, x_dist="normal",
+                           w_std=0.05, target_dist="uniform", ignore_count=9)
+
+
+@pytest.mark.parametrize("chunk_rows", [0, 256])
+def test_wide_dx_tiles_every_element(cuda_device, chunk_rows):
+    """d = 1024: four 256-column blocks, so dX runs in wide tiles (two accumulators sharing
+    each staged A' k-block); 600 rows give ragged row tiles and, with 256-row chunks, a ragged
+    last chunk.  Every element of dX and dW against the oracle."""
+    inp = synth.make_inputs(WIDE)
+    ref = oracle_full(inp)
+    compare_full(run_gpu(inp, chunk_rows=chunk_rows), ref)
+    compare_full(run_gpu(inp, chunk_rows=chunk_rows, recompute=True), ref)
+
+
 @pytest.mark.parametrize("cap,w_std", [(0.0, 0.05), (2.0, 0.3), (50.0, 0.3), (15.0, 1.0)])
 def test_softcap_variants(cuda_device, cap, w_std):
     """No softcap (online max path), a small cap (deep saturation), a large cap (softcap
