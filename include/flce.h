@@ -208,6 +208,18 @@ int flce_rmsnorm_backward(const void* H, const void* gamma, const float* rstd, c
 int flce_selftest_wait_timeout(void* workspace, uint64_t limit_ns, void* stream);
 
 /*
+ * Host-side check of the persistent tile schedule (no counterpart on the pages; runs on the CPU,
+ * no GPU needed): `pairs` SM pairs share T0 tiles of cost c0 and T1 tiles of cost c1 (costs in
+ * k-blocks) with the same assignment the contraction kernels use.  Returns FLCE_OK when every
+ * tile of both problems goes to exactly one (pair, slot); FLCE_ERR_ARG for bad sizes
+ * (pairs < 1 or > 4096, T0, T1 < 0 or above 2^24, c0, c1 < 1) or a tile that is missing,
+ * repeated or out of range.  max_cost / min_cost (either may be NULL) receive the largest
+ * and smallest per-pair sum of tile costs.
+ */
+int flce_check_pair_schedule(int pairs, int T0, int c0, int T1, int c1, int64_t* max_cost,
+                             int64_t* min_cost);
+
+/*
  * Reads the device status word (FLCE_DEV_* bits) and the number of rows in the loss from the
  * workspace of the last call on `stream`.  Synchronises that stream.  Either output may be
  * NULL.

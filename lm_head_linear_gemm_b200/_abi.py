@@ -103,6 +103,9 @@ def lib() -> ctypes.CDLL:
     L.flce_rmsnorm_backward.restype = ctypes.c_int
     L.flce_selftest_wait_timeout.argtypes = [P, ctypes.c_uint64, P]
     L.flce_selftest_wait_timeout.restype = ctypes.c_int
+    L.flce_check_pair_schedule.argtypes = [ctypes.c_int] * 5 + [
+        ctypes.POINTER(ctypes.c_int64), ctypes.POINTER(ctypes.c_int64)]
+    L.flce_check_pair_schedule.restype = ctypes.c_int
     L.flce_instrument.argtypes = [ctypes.c_int]
     L.flce_instrument.restype = ctypes.c_int
     L.flce_instrument_read.argtypes = [ctypes.POINTER(flce_kernel_stats)]
@@ -172,6 +175,17 @@ def read_status(workspace, stream=None) -> tuple[int, int]:
     if rc != FLCE_OK:
         raise FlceError(rc, "flce_read_status")
     return int(st.value), int(nv.value)
+
+
+def check_pair_schedule(pairs: int, T0: int, c0: int, T1: int, c1: int):
+    """Host-side check of the contraction kernels' tile schedule: raises FlceError unless every
+    tile of both problems goes to exactly one pair; returns (max, min) per-pair cost."""
+    hi, lo = ctypes.c_int64(0), ctypes.c_int64(0)
+    rc = lib().flce_check_pair_schedule(int(pairs), int(T0), int(c0), int(T1), int(c1),
+                                        ctypes.byref(hi), ctypes.byref(lo))
+    if rc != FLCE_OK:
+        raise FlceError(rc, "flce_check_pair_schedule")
+    return hi.value, lo.value
 
 
 def selftest_wait_timeout(workspace, limit_ns: int, stream=None) -> None:

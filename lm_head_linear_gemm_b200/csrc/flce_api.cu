@@ -796,6 +796,37 @@ int flce_selftest_wait_timeout(void* workspace, uint64_t limit_ns, void* stream)
   return launch_ok();
 }
 
+int flce_check_pair_schedule(int pairs, int T0, int c0, int T1, int c1, int64_t* max_cost,
+                             int64_t* min_cost) {
+  if (pairs < 1 || pairs > 4096 || T0 < 0 || T1 < 0 || T0 > (1 << 24) || T1 > (1 << 24) ||
+      c0 < 1 || c1 < 1)
+    return FLCE_ERR_ARG;
+  std::vector<uint8_t> seen0(static_cast<size_t>(T0), 0), seen1(static_cast<size_t>(T1), 0);
+  int64_t hi = 0, lo = INT64_MAX;
+  for (int p = 0; p < pairs; ++p) {
+    const PairSchedule ps = pair_schedule(p, pairs, T0, c0, T1, c1);
+    if (ps.n0 < 0 || ps.qa < 0 || ps.qb < 0) return FLCE_ERR_ARG;
+    const int total = ps.n0 + ps.qa + ps.qb;
+    int64_t cost = 0;
+    for (int i = 0; i < total; ++i) {
+      const PairTile pt = pair_tile(ps, p, pairs, i);
+      std::vector<uint8_t>& seen = pt.prob == 0 ? seen0 : seen1;
+      if (pt.t < 0 || pt.t >= static_cast<int>(seen.size()) || seen[pt.t]) return FLCE_ERR_ARG;
+      seen[pt.t] = 1;
+      cost += pt.prob == 0 ? c0 : c1;
+    }
+    hi = cost > hi ? cost : hi;
+    lo = cost < lo ? cost : lo;
+  }
+  for (uint8_t v : seen0)
+    if (!v) return FLCE_ERR_ARG;
+  for (uint8_t v : seen1)
+    if (!v) return FLCE_ERR_ARG;
+  if (max_cost) *max_cost = hi;
+  if (min_cost) *min_cost = lo;
+  return FLCE_OK;
+}
+
 int flce_read_status(const void* workspace, uint32_t* dev_status_out, int64_t* n_valid_out,
                      void* stream) {
   if (workspace == nullptr) return FLCE_ERR_ARG;

@@ -127,7 +127,8 @@ struct PairSchedule {
   int ta;        // problem-1 tiles handed out in phase A
 };
 
-__device__ inline PairSchedule pair_schedule(int pair, int P, int T0, int c0, int T1, int c1) {
+__host__ __device__ inline PairSchedule pair_schedule(int pair, int P, int T0, int c0, int T1,
+                                                     int c1) {
   PairSchedule s{0, 0, 0, 0, 1, 0};
   const int a = T0 / P, n_hi = T0 % P;
   s.n0 = a + (pair < n_hi ? 1 : 0);
@@ -141,6 +142,18 @@ __device__ inline PairSchedule pair_schedule(int pair, int P, int T0, int c0, in
   const int rest = T1 - s.ta;
   s.qb = pair < rest ? (rest - pair + P - 1) / P : 0;
   return s;
+}
+
+// The i-th tile (0 <= i < n0 + qa + qb) of pair `pair`: its problem and its index t within that
+// problem's tiles.  Compiled for the host too, where the library checks that every tile of both
+// problems goes to exactly one (pair, i).
+struct PairTile {
+  int prob, t;
+};
+__host__ __device__ inline PairTile pair_tile(const PairSchedule& s, int pair, int P, int i) {
+  if (i < s.n0) return PairTile{0, pair + i * P};
+  const int j = i - s.n0;
+  return PairTile{1, j < s.qa ? s.la + j * s.p_light : s.ta + pair + (j - s.qa) * P};
 }
 
 template <class C, class E0, class E1, Major A0, Major B0, Major A1, Major B1, bool WIDE0 = false>
@@ -196,16 +209,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
-    const PairSchedule ps = pair_schedule(pair, npairs, m_tiles0 * w_tiles0,
-                                          wide0 ? 2 * nkb0 : nkb0,
-                                          args.prob[1].M > 0 ? m_tiles1 * n_tiles1 : 0,
-                                          nkb1 > 0 ? nkb1 : 1);
-    sched[0] = ps.n0;
-    sched[1] = ps.qa;
-    sched[2] = ps.qb;
-    sched[3] = ps.la;
-    sched[4] = ps.p_light;
-    sched[5] = ps.ta;
+    const PairSchedule mine = pair_schedule(pair, npairs, m_tiles0 * w_tiles0,
+                                            wide0 ? 2 * nkb0 : nkb0,
+                                            args.prob[1].M > 0 ? m_tiles1 * n_tiles1 : 0,
+                                            nkb1 > 0 ? nkb1 : 1);
+    sched[0] = mine.n0;
+    sched[1] = mine.qa;
+    sched[2] = mine.qb;
+    sched[3] = mine.la;
+    sched[4] = mine.p_light;
+    sched[5] = mine.ta;
     fence_barrier_init();
   }
   if (warp == 0 && lane == 0) {
@@ -222,26 +235,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
   cluster_sync_all();   // both CTAs' barriers initialised, schedule written, TMEM allocated
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const int n0 = sched[0], qa = sched[1], total = sched[0] + sched[1] + sched[2];
-  const int la = sched[3], p_light = sched[4], ta = sched[5];
+  PairSchedule ps;
+  ps.n0 = sched[0];
+  ps.qa = sched[1];
+  ps.qb = sched[2];
+  ps.la = sched[3];
+  ps.p_light = sched[4];
+  ps.ta = sched[5];
+  const int n0 = ps.n0, total = ps.n0 + ps.qa + ps.qb;
   const uint32_t leader_full = mapa_shared(smem_u32(full), 0);
   const uint32_t leader_tempty = mapa_shared(smem_u32(tempty), 0);
 
   // i-th tile of this pair -> (problem, m block, n block, k-blocks); in a wide problem 0,
   // nb indexes pairs of N blocks (2 nb and 2 nb + 1).
   auto tile_of = [&](int i, int& prob, int& mb, int& nb, int& kbs) {
-    int t, mt, nt, mf;
-    if (i < n0) {
-      prob = 0;
-      t = pair + i * npairs;
+    const PairTile pt = pair_tile(ps, pair, npairs, i);
+    const int t = pt.t;
+    int mt, nt, mf;
+    prob = pt.prob;
+    if (prob == 0) {
       mt = m_tiles0;
       nt = w_tiles0;
       mf = args.prob[0].m_fastest;
       kbs = nkb0;
     } else {
-      prob = 1;
-      const int j = i - n0;
-      t = j < qa ? la + j * p_light : ta + pair + (j - qa) * npairs;
       mt = m_tiles1;
       nt = n_tiles1;
       mf = args.prob[1].m_fastest;

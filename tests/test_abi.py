@@ -27,7 +27,8 @@ def test_exports_every_declared_symbol(L):
                           "flce_instrument_read", "flce_forward_noalloc", "flce_forward_fp8",
                           "flce_quantize_e4m3", "flce_selftest_wait_timeout",
                           "flce_count_valid", "flce_forward_dp", "flce_rmsnorm_forward",
-                          "flce_rmsnorm_workspace_bytes", "flce_rmsnorm_backward"}
+                          "flce_rmsnorm_workspace_bytes", "flce_rmsnorm_backward",
+                          "flce_check_pair_schedule"}
     for n in names:
         assert hasattr(L, n), n
     out = subprocess.run(["nm", "-D", "--defined-only", _abi.LIB_PATH], capture_output=True,
