@@ -34,6 +34,9 @@ DATASHEET_BF16_TFLOPS = 2250.0
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
+# rows per chunk the library picks when chunk_rows = 0 (only used to label the JSON line)
+AUTO_CHUNK_ROWS = 8192
+
 def parse_args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -470,7 +473,7 @@ def main_gpu(args):
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None,
             "dtype": "e4m3 logits + bf16 gradients" if fp8 else "bf16", "data": "synthetic",
-            "config": dict(workload_desc(c, shape.chunk_rows or min(N, 4096)),
+            "config": dict(workload_desc(c, shape.chunk_rows or min(N, AUTO_CHUNK_ROWS)),
                            parallelism=(f"data parallel x{world}: global-count loss, dW "
                                         f"all-reduce every {args.accum_steps} micro-batches"
                                         if dp else
@@ -603,7 +606,7 @@ def compare_cublas(args):
     import synth
     dev = torch.device("cuda", 0)
     cfg = synth.CONFIGS[args.config]
-    Nc = args.rows or 4096
+    Nc = args.rows or AUTO_CHUNK_ROWS
     inp = synth.make_inputs(cfg, N=Nc)
     c = inp["cfg"]
     sms = torch.cuda.get_device_properties(dev).multi_processor_count

@@ -44,6 +44,27 @@ namespace {
 #ifndef FLCE_EPI_WARPS
 #define FLCE_EPI_WARPS 8
 #endif
+// L2 priorities of the operand streams (0 normal, 1 evict first, 2 evict last): the logits
+// keep their X rows, which every W slab meets (last); the gradient launch keeps Xs, which
+// every dW tile re-reads (last).  Marking W or A' evict-first measured slower.
+#ifndef FLCE_L2_LOGITS_X
+#define FLCE_L2_LOGITS_X 2
+#endif
+#ifndef FLCE_L2_LOGITS_W
+#define FLCE_L2_LOGITS_W 0
+#endif
+#ifndef FLCE_L2_DX_A
+#define FLCE_L2_DX_A 0
+#endif
+#ifndef FLCE_L2_DX_W
+#define FLCE_L2_DX_W 0
+#endif
+#ifndef FLCE_L2_DW_A
+#define FLCE_L2_DW_A 0
+#endif
+#ifndef FLCE_L2_DW_XS
+#define FLCE_L2_DW_XS 2
+#endif
 // dX in wide tiles (256 x 512 per SM pair, two accumulators sharing each staged A' k-block)
 #ifndef FLCE_DX_WIDE
 #define FLCE_DX_WIDE 1
@@ -65,7 +86,8 @@ constexpr auto kGradKernel = gemm_pair_kernel<Cfg, DxEpi, DwEpi, Major::K, Major
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s bound on every in-kernel wait
 constexpr float kFixedRefMaxCap = 32.f;           // exp(s - cap) >= e^{-64}: no underflow in fp32
-constexpr int64_t kAutoChunkRows = 4096;
+constexpr int64_t kAutoChunkRows = 8192;   // rows per chunk when chunk_rows = 0
+constexpr int kLogitsRows = 4096;          // rows per logits launch (launch_logits)
 constexpr size_t kAlign = 256;
 
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
@@ -311,11 +333,12 @@ struct Ctx {
 
 // Logits contraction of rows [row0, row0 + rows) with the given epilogue parameters, from the
 // bf16 X/W or, when the context carries them, from the e4m3 operands.
-int launch_logits(const Ctx& c, int64_t row0, int rows, const __nv_bfloat16* X,
-                  const __nv_bfloat16* W, LogitsParams lp) {
+int launch_logits_rows(const Ctx& c, int64_t row0, int rows, const __nv_bfloat16* X,
+                       const __nv_bfloat16* W, LogitsParams lp) {
   const flce_shape* s = c.s;
   const int d = static_cast<int>(s->d), Vpad = static_cast<int>(s->Vpad);
-  const PairProblem logits{rows, Vpad, d, 1, 0}, none{0, 0, 0, 0, 0};
+  const PairProblem logits{rows, Vpad, d, 1, 0, FLCE_L2_LOGITS_X, FLCE_L2_LOGITS_W};
+  const PairProblem none{0, 0, 0, 0, 0, 0, 0};
   CUtensorMap mX, mW;
   if (c.fp8.X8 != nullptr) {
     FLCE_TRY(make_map(&mX, c.fp8.X8 + row0 * s->d, d, rows, d, Cfg8::BM_CTA, 1));
@@ -330,6 +353,28 @@ int launch_logits(const Ctx& c, int64_t row0, int rows, const __nv_bfloat16* X,
   lp.scale_a = lp.scale_b = nullptr;
   return launch_pair<LogitsEpi, LogitsEpi, CfgL>(kLogitsKernel, c.di, mX, mW, mX, mW, logits,
                                                   none, &c.hdr->status, lp, lp, c.st, 0);
+}
+
+// The logits of rows [row0, row0 + rows) in launches of at most kLogitsRows rows: a launch walks
+// the row blocks of one W slab before the next, so its X rows must stay in L2 next to the W
+// slabs and the A' stream; past 4096 rows (25 MB of X at d = 3072) they start to fall out.
+int launch_logits(const Ctx& c, int64_t row0, int rows, const __nv_bfloat16* X,
+                  const __nv_bfloat16* W, const LogitsParams& lp) {
+  const int per_row = lp.fixed_ref ? 1 : 2;   // partial words per (row, slab)
+  for (int r0 = 0; r0 < rows; r0 += kLogitsRows) {
+    const int rr = rows - r0 < kLogitsRows ? rows - r0 : kLogitsRows;
+    LogitsParams q = lp;
+    q.rows = rr;
+    q.tgt = lp.tgt + r0;
+    q.ref = lp.ref != nullptr ? lp.ref + r0 : nullptr;
+    q.partial = lp.partial + static_cast<size_t>(r0) * lp.n_slabs * per_row;
+    q.s_t = lp.s_t + r0;
+    q.der_t = lp.der_t + r0;
+    q.e_t = lp.e_t + r0;
+    q.A = lp.A != nullptr ? lp.A + static_cast<size_t>(r0) * lp.Vpad : nullptr;
+    FLCE_TRY(launch_logits_rows(c, row0 + r0, rr, X, W, q));
+  }
+  return FLCE_OK;
 }
 
 // One chunk of the gradient path: logits GEMM (mode FUSED or RECOMPUTE), row finish, and the
@@ -399,7 +444,8 @@ int grad_chunk(const Ctx& c, int64_t row0, int rows, const __nv_bfloat16* X,
   // dX (long tiles: K = Vpad) and dW (short tiles: K = rows) share one balanced launch
   DxParams xp{rows, d, r, dX + row0 * s->d};
   DwParams wp{Vpad, d, accumulate, dW};
-  const PairProblem pdx{rows, d, Vpad, 0, FLCE_DX_WIDE}, pdw{Vpad, d, rows, 0, 0};
+  const PairProblem pdx{rows, d, Vpad, 0, FLCE_DX_WIDE, FLCE_L2_DX_A, FLCE_L2_DX_W};
+  const PairProblem pdw{Vpad, d, rows, 0, 0, FLCE_L2_DW_A, FLCE_L2_DW_XS};
   FLCE_TRY((launch_pair<DxEpi, DwEpi>(kGradKernel, c.di, mA_k, mW_mn, mA_mn, mXs_mn, pdx, pdw,
                                        &c.hdr->status, xp, wp, c.st, 1)));
   return FLCE_OK;

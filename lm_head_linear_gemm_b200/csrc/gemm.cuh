@@ -28,13 +28,14 @@ enum class Major : int { K = 0, MN = 1 };
 // The copy completes on the pair leader's barrier (shared::cluster address).
 template <Major MAJ, int ROWS>
 __device__ __forceinline__ void load_operand_pair(uint8_t* dst, const CUtensorMap* map,
-                                                  uint32_t leader_bar, int row0, int k0) {
+                                                  uint32_t leader_bar, int row0, int k0,
+                                                  uint64_t policy) {
   if constexpr (MAJ == Major::K) {
-    tma_load_2d_pair(dst, map, leader_bar, k0, row0);
+    tma_load_2d_pair_hint(dst, map, leader_bar, k0, row0, policy);
   } else {
 #pragma unroll
     for (int q = 0; q < ROWS / 64; ++q)
-      tma_load_2d_pair(dst + q * 8192, map, leader_bar, row0 + 64 * q, k0);
+      tma_load_2d_pair_hint(dst + q * 8192, map, leader_bar, row0 + 64 * q, k0, policy);
   }
 }
 
@@ -103,6 +104,7 @@ struct PairProblem {
   int M, N, K;          // extents; M == 0 marks an absent second problem
   int m_fastest;        // tile order: 1 = consecutive tiles walk M first
   int wide;             // problem 0 only: 1 = wide tiles (see below)
+  int l2_a, l2_b;       // L2 priority of the A / B operand reads (l2_policy: 0, 1 first, 2 last)
 };
 
 struct PairArgs {
@@ -291,6 +293,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
       int stage = 0;
       uint32_t phase = 0;
       long long arms = 0;
+      const uint64_t pol_a0 = l2_policy(args.prob[0].l2_a), pol_b0 = l2_policy(args.prob[0].l2_b);
+      const uint64_t pol_a1 = l2_policy(args.prob[1].l2_a), pol_b1 = l2_policy(args.prob[1].l2_b);
       for_each_run([&](auto nsub_c, int i0, int i1) {
         constexpr int NSUB = decltype(nsub_c)::value;
         for (int i = i0; i < i1 && !*abort_flag; ++i) {
@@ -318,14 +322,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
             uint8_t* sB = sA + C::A_BYTES;
             const uint32_t bar = leader_full + 8u * stage;
             if (prob == 0) {
-              load_operand_pair<A0, C::BM_CTA>(sA, &tmA0, bar, a_row, kb * C::BK);
-              load_operand_pair<B0, C::BN_CTA>(sB, &tmB0, bar, b_row, kb * C::BK);
+              load_operand_pair<A0, C::BM_CTA>(sA, &tmA0, bar, a_row, kb * C::BK, pol_a0);
+              load_operand_pair<B0, C::BN_CTA>(sB, &tmB0, bar, b_row, kb * C::BK, pol_b0);
               if constexpr (NSUB == 2)
                 load_operand_pair<B0, C::BN_CTA>(sB + C::STAGE_BYTES, &tmB0, bar + 8u,
-                                                 b_row + C::BN, kb * C::BK);
+                                                 b_row + C::BN, kb * C::BK, pol_b0);
             } else {
-              load_operand_pair<A1, C::BM_CTA>(sA, &tmA1, bar, a_row, kb * C::BK);
-              load_operand_pair<B1, C::BN_CTA>(sB, &tmB1, bar, b_row, kb * C::BK);
+              load_operand_pair<A1, C::BM_CTA>(sA, &tmA1, bar, a_row, kb * C::BK, pol_a1);
+              load_operand_pair<B1, C::BN_CTA>(sB, &tmB1, bar, b_row, kb * C::BK, pol_b1);
             }
             arms += NSUB;
             stage += NSUB;

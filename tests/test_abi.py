@@ -49,18 +49,18 @@ def test_status_strings(L):
 
 
 def test_workspace_has_no_tokens_by_vocab_term(L):
-    s = flce.make_shape(16384, 3072, 50304, 50257, 15.0, -1, 0)
+    s = flce.make_shape(65536, 3072, 50304, 50257, 15.0, -1, 0)
     fwd = flce.workspace_bytes(s, False)
     grads = flce.workspace_bytes(s, True)
-    logits_bytes = 16384 * 50304 * 2                     # one bf16 N x Vpad buffer
+    logits_bytes = 65536 * 50304 * 2                     # one bf16 N x Vpad buffer
     W_bytes = 50304 * 3072 * 2
-    assert 0 < fwd < grads < logits_bytes / 3
-    assert grads < 2 * W_bytes                            # O(Vpad * chunk) with chunk <= 4096
+    assert 0 < fwd < grads < logits_bytes / 6
+    assert grads < 3 * W_bytes                            # O(Vpad * chunk) with chunk <= 8192
     # doubling N grows the scratch only by O(N) per-row words, not by Vpad per row
-    s2 = flce.make_shape(32768, 3072, 50304, 50257, 15.0, -1, 0)
-    assert flce.workspace_bytes(s2, True) - grads < 32 * 16384
+    s2 = flce.make_shape(131072, 3072, 50304, 50257, 15.0, -1, 0)
+    assert flce.workspace_bytes(s2, True) - grads < 32 * 65536
     # the chunk bounds the gradient operand
-    s3 = flce.make_shape(16384, 3072, 50304, 50257, 15.0, -1, 1024)
+    s3 = flce.make_shape(65536, 3072, 50304, 50257, 15.0, -1, 1024)
     assert flce.workspace_bytes(s3, True) < grads / 3
 
 

@@ -140,6 +140,24 @@ def test_wide_dx_tiles_every_element(cuda_device, chunk_rows):
     compare_full(run_gpu(inp, chunk_rows=chunk_rows, recompute=True), ref)
 
 
+SUBLAUNCH = synth.custom_config("sublaunch", N=4200, d=128, Vreal=1000, Vpad=1024,
+                                x_dist="normal", w_std=0.05, target_dist="uniform",
+                                ignore_count=40)
+
+
+@pytest.mark.parametrize("cap", [15.0, 0.0])
+def test_logits_in_sub_launches_every_element(cuda_device, cap):
+    """4200 rows in one chunk: the logits run as two launches (4096 rows + a ragged 104) that
+    fill one chunk's partial sums and gradient operand; with and without the softcap (fixed
+    reference vs (max, sum-exp) pairs).  Every element against the oracle."""
+    inp = synth.make_inputs(SUBLAUNCH)
+    ref = oracle_full(inp, cap=cap)
+    compare_full(run_gpu(inp, cap=cap), ref)
+    compare_full(run_gpu(inp, cap=cap, recompute=True), ref)
+    stats = run_gpu(inp, cap=cap, want_grads=False)
+    compare_full(stats, ref, grads=False)
+
+
 @pytest.mark.parametrize("cap,w_std", [(0.0, 0.05), (2.0, 0.3), (50.0, 0.3), (15.0, 1.0)])
 def test_softcap_variants(cuda_device, cap, w_std):
     """No softcap (online max path), a small cap (deep saturation), a large cap (softcap
@@ -311,6 +329,40 @@ def test_full_size_2k_context(cuda_device):
     the softcap's curved range."""
     got, f = _sampled_full_size("3.8b-2k")
     assert math.isfinite(got["loss"])
+
+
+def test_rows_beyond_32bit_element_offsets(cuda_device):
+    """N = 1400 x 512 = 716,800 rows at d = 3072: X and dX hold 2.2e9 elements each, past 32-bit
+    element offsets, in 175 chunks whose dW contributions accumulate.  The rows are 1400 copies
+    of a 512-row base problem (the 3.8b head's shapes and distributions), so the oracle on the
+    base fixes every result: the loss and each row's lse equal the base's, each dX row is the
+    base row's divided by 1400 (the count of rows in the loss is 1400 times larger), and dW
+    equals the base's.  Copies of a row go through the same arithmetic, so they must agree
+    bit for bit."""
+    import lm_head_linear_gemm_b200 as flce
+    torch = _torch()
+    k = 1400
+    inp = synth.make_inputs("3.8b", N=512)
+    c = inp["cfg"]
+    ref = oracle_full(inp)
+    Xb, W, tb = to_dev(inp["X"]), to_dev(inp["W"]), to_dev(inp["targets"])
+    X = Xb.repeat(k, 1)
+    t = tb.repeat(k)
+    assert X.numel() > 2**31
+    loss, lse, dX, dW, ws = flce.forward(X, W, t, c.Vreal, c.cap, c.ignore_index, True)
+    torch.cuda.synchronize()
+    status, nv = flce.read_status(ws)
+    assert status == 0 and nv == k * ref["n_valid"]
+    del X
+    assert abs(float(loss.item()) - ref["loss"]) <= LOSS_TOL
+    lse_k = lse.view(k, 512)
+    assert torch.equal(lse_k, lse_k[:1].expand(k, 512))
+    assert np.abs(lse_k[0].double().cpu().numpy() - ref["lse"]).max() <= LSE_TOL
+    dX_k = dX.view(k, 512, c.d)
+    for i0 in range(0, k, 100):
+        assert torch.equal(dX_k[i0:i0 + 100], dX_k[:1].expand(min(100, k - i0), 512, c.d)), i0
+    check_tensor("dX rows (x copies)", dX_k[0].double().cpu().numpy() * k, ref["dX"])
+    check_tensor("dW", dW.double().cpu().numpy(), ref["dW"])
 
 
 def test_concurrent_calls_on_two_streams(cuda_device):
