@@ -689,12 +689,26 @@ struct LogitsEpi {
         uint32_t packed[16];
 #pragma unroll
         for (int k = 0; k < 16; ++k) packed[k] = pack_bf16x2(v[2 * k], v[2 * k + 1]);
+        if ((p.Vpad & 15) == 0) {
+          // rows start on 32-byte boundaries: two full-sector stores per 32 columns
 #pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          const int col = cbase + 8 * g;
-          if (col < p.Vpad) {
-            *reinterpret_cast<uint4*>(arow + col) =
-                make_uint4(packed[4 * g], packed[4 * g + 1], packed[4 * g + 2], packed[4 * g + 3]);
+          for (int g = 0; g < 2; ++g) {
+            const int col = cbase + 16 * g;
+            if (col < p.Vpad) {
+              const uint32_t w[8] = {packed[8 * g],     packed[8 * g + 1], packed[8 * g + 2],
+                                     packed[8 * g + 3], packed[8 * g + 4], packed[8 * g + 5],
+                                     packed[8 * g + 6], packed[8 * g + 7]};
+              st_global_v8(arow + col, w);
+            }
+          }
+        } else {
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            const int col = cbase + 8 * g;
+            if (col < p.Vpad) {
+              *reinterpret_cast<uint4*>(arow + col) = make_uint4(
+                  packed[4 * g], packed[4 * g + 1], packed[4 * g + 2], packed[4 * g + 3]);
+            }
           }
         }
       }
