@@ -73,11 +73,11 @@ using Cfg = PairCfg<256, FLCE_GRAD_STAGES, FLCE_EPI_WARPS>;
 using CfgL = PairCfg<FLCE_LOGITS_BN, FLCE_LOGITS_STAGES, FLCE_EPI_WARPS>;
 // logits: A = X (K-major), B = W (K-major)
 constexpr auto kLogitsKernel =
-    gemm_pair_kernel<CfgL, LogitsEpi, LogitsEpi, Major::K, Major::K, Major::K, Major::K>;
+    gemm_pair_kernel<CfgL, LogitsEpi, LogitsEpi, Major::K, Major::K, Major::K, Major::K, false, 2>;
 // logits from e4m3 operands (kind::f8f6f4, tensorwise scales applied in the epilogue)
 using Cfg8 = PairCfg<FLCE_LOGITS_BN, FLCE_LOGITS_STAGES, FLCE_EPI_WARPS, 1>;
 constexpr auto kLogitsKernel8 =
-    gemm_pair_kernel<Cfg8, LogitsEpi, LogitsEpi, Major::K, Major::K, Major::K, Major::K>;
+    gemm_pair_kernel<Cfg8, LogitsEpi, LogitsEpi, Major::K, Major::K, Major::K, Major::K, false, 2>;
 static_assert(CfgL::BN == Cfg8::BN && CfgL::COL_SPLIT == Cfg8::COL_SPLIT,
               "both logits kernels fill the same per-row partial slots");
 // gradients in one launch: dX = A' W (A' K-major, W MN-major), dW = A'^T Xs (both MN-major)

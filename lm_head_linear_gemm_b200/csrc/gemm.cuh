@@ -39,6 +39,13 @@ __device__ __forceinline__ void load_operand_pair(uint8_t* dst, const CUtensorMa
   }
 }
 
+// Descriptor increment between consecutive MMA slices (start address field, 16-byte units);
+// staged tiles sit below 256 KB, so adding to the 14-bit field never carries out of it.
+template <Major MAJ>
+__device__ __forceinline__ constexpr uint64_t desc_step() {
+  return MAJ == Major::K ? 2u : 128u;
+}
+
 // Descriptor of the k-th MMA slice of a staged operand tile (32 bytes of K: 16 bf16 or 32 e4m3
 // elements; MN-major slices are bf16 only: 16 K rows = two 1 KB swizzle atoms).
 template <Major MAJ>
@@ -158,7 +165,10 @@ __host__ __device__ inline PairTile pair_tile(const PairSchedule& s, int pair, i
   return PairTile{1, j < s.qa ? s.la + j * s.p_light : s.ta + pair + (j - s.qa) * P};
 }
 
-template <class C, class E0, class E1, Major A0, Major B0, Major A1, Major B1, bool WIDE0 = false>
+// WIDE0: problem 0 may run in wide tiles (below).  ROUND: k-blocks per MMA-issue round of
+// the other tiles (1 or 2).
+template <class C, class E0, class E1, Major A0, Major B0, Major A1, Major B1, bool WIDE0 = false,
+          int ROUND = 1>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
                      const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
@@ -395,55 +405,88 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
           }
           tc_fence_after();
           const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * C::BN);
-          for (int kb = 0; kb < kbs; ++kb) {
-            if (!mbar_wait_bounded(&full[stage], phase, args.status, args.limit_ns)) {
-              *abort_flag = 1;
-              return;
-            }
-            if constexpr (NSUB == 2) {
-              if (!mbar_wait_bounded(&full[stage + 1], phase, args.status, args.limit_ns)) {
+          if constexpr (NSUB == 2) {
+            for (int kb = 0; kb < kbs; ++kb) {
+              if (!mbar_wait_bounded(&full[stage], phase, args.status, args.limit_ns) ||
+                  !mbar_wait_bounded(&full[stage + 1], phase, args.status, args.limit_ns)) {
                 *abort_flag = 1;
                 return;
               }
-            }
-            tc_fence_after();
-            const uint32_t a_base = smem_u32(smem + stage * C::STAGE_BYTES);
-            const uint32_t b_base = a_base + C::A_BYTES;
-            if constexpr (C::ELEM_BYTES == 1) {
-#pragma unroll
-              for (int k = 0; k < C::BK / C::MMA_K; ++k)
-                mma_e4m3_ss_pair(d_tmem, operand_desc<Major::K>(a_base, k),
-                                 operand_desc<Major::K>(b_base, k), prob == 0 ? idesc0 : idesc1,
-                                 (kb | k) != 0 ? 1u : 0u);
-            } else if constexpr (NSUB == 2) {
+              tc_fence_after();
+              const uint32_t a_base = smem_u32(smem + stage * C::STAGE_BYTES);
+              const uint32_t b_base = a_base + C::A_BYTES;
               // both N blocks from one staged A k-block; the second B block is in the next slot
               const uint32_t d_tmem2 = tmem_base + static_cast<uint32_t>(acc2 * C::BN);
               const uint32_t b_base2 = b_base + C::STAGE_BYTES;
+              const uint64_t da = operand_desc<A0>(a_base, 0), db = operand_desc<B0>(b_base, 0);
+              const uint64_t db2 = operand_desc<B0>(b_base2, 0);
 #pragma unroll
               for (int k = 0; k < C::BK / C::MMA_K; ++k) {
-                mma_bf16_ss_pair(d_tmem, operand_desc<A0>(a_base, k), operand_desc<B0>(b_base, k),
+                mma_bf16_ss_pair(d_tmem, da + desc_step<A0>() * k, db + desc_step<B0>() * k,
                                  idesc0, (kb | k) != 0 ? 1u : 0u);
-                mma_bf16_ss_pair(d_tmem2, operand_desc<A0>(a_base, k),
-                                 operand_desc<B0>(b_base2, k), idesc0, (kb | k) != 0 ? 1u : 0u);
+                mma_bf16_ss_pair(d_tmem2, da + desc_step<A0>() * k, db2 + desc_step<B0>() * k,
+                                 idesc0, (kb | k) != 0 ? 1u : 0u);
               }
-            } else if (prob == 0) {
-#pragma unroll
-              for (int k = 0; k < C::BK / C::MMA_K; ++k)
-                mma_bf16_ss_pair(d_tmem, operand_desc<A0>(a_base, k), operand_desc<B0>(b_base, k),
-                                 idesc0, (kb | k) != 0 ? 1u : 0u);
-            } else {
-#pragma unroll
-              for (int k = 0; k < C::BK / C::MMA_K; ++k)
-                mma_bf16_ss_pair(d_tmem, operand_desc<A1>(a_base, k), operand_desc<B1>(b_base, k),
-                                 idesc1, (kb | k) != 0 ? 1u : 0u);
+              issued = true;
+              mma_commit_pair_both(&empty[stage]);
+              mma_commit_pair_both(&empty[stage + 1]);
+              stage += 2;
+              if (stage == C::STAGES) {
+                stage = 0;
+                phase ^= 1u;
+              }
             }
-            issued = true;
-            mma_commit_pair_both(&empty[stage]);
-            if constexpr (NSUB == 2) mma_commit_pair_both(&empty[stage + 1]);
-            stage += NSUB;
-            if (stage == C::STAGES) {
-              stage = 0;
-              phase ^= 1u;
+          } else {
+            // the MMAs of one staged k-block into d_tmem
+            auto issue = [&](int st, int kb) {
+              const uint32_t a_base = smem_u32(smem + st * C::STAGE_BYTES);
+              const uint32_t b_base = a_base + C::A_BYTES;
+              const uint64_t da = operand_desc<A0>(a_base, 0), db = operand_desc<B0>(b_base, 0);
+              const uint64_t da1 = operand_desc<A1>(a_base, 0), db1 = operand_desc<B1>(b_base, 0);
+              if constexpr (C::ELEM_BYTES == 1) {
+#pragma unroll
+                for (int k = 0; k < C::BK / C::MMA_K; ++k)
+                  mma_e4m3_ss_pair(d_tmem, operand_desc<Major::K>(a_base, k),
+                                   operand_desc<Major::K>(b_base, k), prob == 0 ? idesc0 : idesc1,
+                                   (kb | k) != 0 ? 1u : 0u);
+              } else if (prob == 0) {
+#pragma unroll
+                for (int k = 0; k < C::BK / C::MMA_K; ++k)
+                  mma_bf16_ss_pair(d_tmem, da + desc_step<A0>() * k, db + desc_step<B0>() * k,
+                                   idesc0, (kb | k) != 0 ? 1u : 0u);
+              } else {
+#pragma unroll
+                for (int k = 0; k < C::BK / C::MMA_K; ++k)
+                  mma_bf16_ss_pair(d_tmem, da1 + desc_step<A1>() * k, db1 + desc_step<B1>() * k,
+                                   idesc1, (kb | k) != 0 ? 1u : 0u);
+              }
+            };
+            // ROUND = 2: two k-blocks per round, one fence and one loop step per eight MMAs.
+            // The single MMA-issuing thread is what limits these 4-MMA k-blocks (its waits,
+            // fence and commit take about as long as the MMAs run); this measured faster for the
+            // logits and slower for the dW tiles, whose MN-major loads arrive later.
+            static_assert(ROUND == 1 || ROUND == 2, "one or two k-blocks per round");
+            for (int kb = 0; kb < kbs; kb += ROUND) {
+              const bool two = ROUND == 2 && kb + 1 < kbs;
+              const int st2 = stage + 1 == C::STAGES ? 0 : stage + 1;
+              const uint32_t ph2 = stage + 1 == C::STAGES ? phase ^ 1u : phase;
+              if (!mbar_wait_bounded(&full[stage], phase, args.status, args.limit_ns) ||
+                  (two && !mbar_wait_bounded(&full[st2], ph2, args.status, args.limit_ns))) {
+                *abort_flag = 1;
+                return;
+              }
+              tc_fence_after();
+              issue(stage, kb);
+              if (two) issue(st2, kb + 1);
+              issued = true;
+              mma_commit_pair_both(&empty[stage]);
+              if (two) mma_commit_pair_both(&empty[st2]);
+              stage = two ? st2 : stage;
+              phase = two ? ph2 : phase;
+              if (++stage == C::STAGES) {
+                stage = 0;
+                phase ^= 1u;
+              }
             }
           }
           mma_commit_pair_both(&tfull[acc]);
