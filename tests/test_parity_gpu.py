@@ -334,11 +334,11 @@ def test_full_size_2k_context(cuda_device):
 def test_rows_beyond_32bit_element_offsets(cuda_device):
     """N = 1400 x 512 = 716,800 rows at d = 3072: X and dX hold 2.2e9 elements each, past 32-bit
     element offsets, in 88 chunks (the last one half full) whose dW contributions accumulate.
-    The rows are 1400 copies of a 512-row base problem (the 3.8b head's shapes and distributions), so the oracle on the
-    base fixes every result: the loss and each row's lse equal the base's, each dX row is the
-    base row's divided by 1400 (the count of rows in the loss is 1400 times larger), and dW
-    equals the base's.  Copies of a row go through the same arithmetic, so they must agree
-    bit for bit."""
+    The rows are 1400 copies of a 512-row base problem (the 3.8b head's shapes and
+    distributions), so the oracle on the base fixes every result: the loss and each row's lse
+    equal the base's, each dX row is the base row's divided by 1400 (the count of rows in the
+    loss is 1400 times larger), and dW equals the base's.  Copies of a row go through the same
+    arithmetic, so they must agree bit for bit."""
     import lm_head_linear_gemm_b200 as flce
     torch = _torch()
     k = 1400
