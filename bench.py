@@ -34,8 +34,10 @@ DATASHEET_BF16_TFLOPS = 2250.0
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
-# rows per chunk the library picks when chunk_rows = 0 (only used to label the JSON line)
+# rows per chunk the library picks when chunk_rows = 0, and the most rows one logits launch
+# covers (used to label the JSON line and to match recorded DRAM traffic to launch sizes)
 AUTO_CHUNK_ROWS = 8192
+LOGITS_LAUNCH_ROWS = 4096
 
 def parse_args():
     ap = argparse.ArgumentParser()
@@ -446,7 +448,10 @@ def main_gpu(args):
     if dom and os.path.exists(tpath):
         tj = json.load(open(tpath))
         ent = tj.get(dom)
-        if ent and ent.get("kernel_rev") == kernel_rev() and ent.get("config") == c.name:
+        chunk = min(N, shape.chunk_rows or AUTO_CHUNK_ROWS)
+        launch_rows = {"dX+dW": chunk, "logits": min(chunk, LOGITS_LAUNCH_ROWS)}.get(dom)
+        if (ent and ent.get("kernel_rev") == kernel_rev() and ent.get("config") == c.name
+                and ent.get("rows_per_launch") == launch_rows):
             traffic = ent.get("bytes_per_launch")
     roofline = None
     if dom:
