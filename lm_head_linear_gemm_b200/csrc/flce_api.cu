@@ -36,7 +36,11 @@ namespace {
 #define FLCE_LOGITS_BN 256
 #endif
 #ifndef FLCE_LOGITS_STAGES
-#define FLCE_LOGITS_STAGES 6
+#define FLCE_LOGITS_STAGES 3
+#endif
+// k-blocks per ring slot of the logits kernels (slots of 64 KB)
+#ifndef FLCE_LOGITS_KSUB
+#define FLCE_LOGITS_KSUB 2
 #endif
 #ifndef FLCE_GRAD_STAGES
 #define FLCE_GRAD_STAGES 6
@@ -65,19 +69,25 @@ namespace {
 #ifndef FLCE_L2_DW_XS
 #define FLCE_L2_DW_XS 2
 #endif
+// ring slots per MMA-issue round in the logits kernels
+#ifndef FLCE_LOGITS_ROUND
+#define FLCE_LOGITS_ROUND 1
+#endif
 // dX in wide tiles (256 x 512 per SM pair, two accumulators sharing each staged A' k-block)
 #ifndef FLCE_DX_WIDE
 #define FLCE_DX_WIDE 1
 #endif
 using Cfg = PairCfg<256, FLCE_GRAD_STAGES, FLCE_EPI_WARPS>;
-using CfgL = PairCfg<FLCE_LOGITS_BN, FLCE_LOGITS_STAGES, FLCE_EPI_WARPS>;
+using CfgL = PairCfg<FLCE_LOGITS_BN, FLCE_LOGITS_STAGES, FLCE_EPI_WARPS, 2, FLCE_LOGITS_KSUB>;
 // logits: A = X (K-major), B = W (K-major)
 constexpr auto kLogitsKernel =
-    gemm_pair_kernel<CfgL, LogitsEpi, LogitsEpi, Major::K, Major::K, Major::K, Major::K, false, 2>;
+    gemm_pair_kernel<CfgL, LogitsEpi, LogitsEpi, Major::K, Major::K, Major::K, Major::K, false,
+                     FLCE_LOGITS_ROUND>;
 // logits from e4m3 operands (kind::f8f6f4, tensorwise scales applied in the epilogue)
-using Cfg8 = PairCfg<FLCE_LOGITS_BN, FLCE_LOGITS_STAGES, FLCE_EPI_WARPS, 1>;
+using Cfg8 = PairCfg<FLCE_LOGITS_BN, FLCE_LOGITS_STAGES, FLCE_EPI_WARPS, 1, FLCE_LOGITS_KSUB>;
 constexpr auto kLogitsKernel8 =
-    gemm_pair_kernel<Cfg8, LogitsEpi, LogitsEpi, Major::K, Major::K, Major::K, Major::K, false, 2>;
+    gemm_pair_kernel<Cfg8, LogitsEpi, LogitsEpi, Major::K, Major::K, Major::K, Major::K, false,
+                     FLCE_LOGITS_ROUND>;
 static_assert(CfgL::BN == Cfg8::BN && CfgL::COL_SPLIT == Cfg8::COL_SPLIT,
               "both logits kernels fill the same per-row partial slots");
 // gradients in one launch: dX = A' W (A' K-major, W MN-major), dW = A'^T Xs (both MN-major)

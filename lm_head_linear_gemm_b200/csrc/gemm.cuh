@@ -72,7 +72,9 @@ __device__ __forceinline__ uint64_t operand_desc(uint32_t base, int k) {
 // share of problem 1's tiles, handed out so that every pair ends with about the same number of
 // k-blocks while concurrently running tiles stay neighbours (pair_schedule).  A launch with one
 // problem is the plain round-robin persistent schedule.
-template <int BN_, int STAGES_, int EPI_WARPS_, int ELEM_BYTES_ = 2>
+// KSUB: k-blocks (128-byte swizzle rows of K) per ring slot.  Two per slot halve the barrier
+// waits, fences and commits of the single MMA-issuing thread per MMA.
+template <int BN_, int STAGES_, int EPI_WARPS_, int ELEM_BYTES_ = 2, int KSUB_ = 1>
 struct PairCfg {
   static constexpr bool PAIR = true;
   static constexpr int ELEM_BYTES = ELEM_BYTES_;  // 2: bf16 (kind::f16), 1: e4m3 (kind::f8f6f4)
@@ -81,12 +83,16 @@ struct PairCfg {
   static constexpr int BN = BN_;         // columns per pair tile
   static constexpr int BN_CTA = BN_ / 2; // B rows staged by each CTA
   static constexpr int BK = 128 / ELEM_BYTES;  // one 128-byte swizzle row of K per k-block
+  static constexpr int KSUB = KSUB_;           // k-blocks per ring slot
+  static constexpr int KSLOT = BK * KSUB;      // K per ring slot
   static constexpr int MMA_K = 32 / ELEM_BYTES; // K per tcgen05.mma: 32 bytes of each row
   static constexpr int STAGES = STAGES_;
   static constexpr int EPI_WARPS = EPI_WARPS_;
   static constexpr int THREADS = 64 + 32 * EPI_WARPS;
-  static constexpr int A_BYTES = BM_CTA * 128;
-  static constexpr int B_BYTES = BN_CTA * 128;
+  static constexpr int A_SUB = BM_CTA * 128;   // one k-block of A (this CTA's rows)
+  static constexpr int B_SUB = BN_CTA * 128;
+  static constexpr int A_BYTES = A_SUB * KSUB;
+  static constexpr int B_BYTES = B_SUB * KSUB;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int TMEM_COLS = (2 * BN <= 256) ? 256 : 512;
   static constexpr int COL_SPLIT = EPI_WARPS / 4;
@@ -100,6 +106,7 @@ struct PairCfg {
   static_assert(A_BYTES % 1024 == 0 && B_BYTES % 1024 == 0, "swizzle atoms need 1 KB alignment");
   static_assert((2 * STAGES + 5) * 8 + 32 <= BAR_BYTES, "barrier area too small");
   static_assert(SMEM_BYTES <= 232448, "more than 227 KB of shared memory");
+  static_assert(KSUB >= 1 && KSUB <= 4, "1 to 4 k-blocks per slot");
 };
 
 template <int V>
@@ -165,7 +172,7 @@ __host__ __device__ inline PairTile pair_tile(const PairSchedule& s, int pair, i
   return PairTile{1, j < s.qa ? s.la + j * s.p_light : s.ta + pair + (j - s.qa) * P};
 }
 
-// WIDE0: problem 0 may run in wide tiles (below).  ROUND: k-blocks per MMA-issue round of
+// WIDE0: problem 0 may run in wide tiles (below).  ROUND: ring slots per MMA-issue round of
 // the other tiles (1 or 2).
 template <class C, class E0, class E1, Major A0, Major B0, Major A1, Major B1, bool WIDE0 = false,
           int ROUND = 1>
@@ -196,17 +203,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
 
   const int m_tiles0 = (args.prob[0].M + C::BM - 1) / C::BM;
   const int n_tiles0 = (args.prob[0].N + C::BN - 1) / C::BN;
-  const int nkb0 = (args.prob[0].K + C::BK - 1) / C::BK;
+  const int nkb0 = (args.prob[0].K + C::KSLOT - 1) / C::KSLOT;   // ring slots per tile
   const int m_tiles1 = (args.prob[1].M + C::BM - 1) / C::BM;
   const int n_tiles1 = (args.prob[1].N + C::BN - 1) / C::BN;
-  const int nkb1 = (args.prob[1].K + C::BK - 1) / C::BK;
+  const int nkb1 = (args.prob[1].K + C::KSLOT - 1) / C::KSLOT;
   // Wide tiles (problem 0, bf16): two adjacent BN-column blocks share every staged k-block of
   // A, one TMEM accumulator each, so a pair stages 256 + 512 operand rows per k-block instead
   // of 2 x (256 + 256).  The second B block goes into the next ring slot (its A area unused),
   // so a wide k-block takes two slots and the ring stays in step as long as the slot count and
   // the number of N blocks are even.  Meant for long-K problems: while a wide tile runs, no
   // accumulator is free for the epilogue of the previous tile to overlap with.
-  const bool wide0 = WIDE0 && args.prob[0].wide != 0 && C::ELEM_BYTES == 2 &&
+  const bool wide0 = WIDE0 && args.prob[0].wide != 0 && C::ELEM_BYTES == 2 && C::KSUB == 1 &&
                      (C::STAGES % 2) == 0 && (n_tiles0 % 2) == 0;
   const int w_tiles0 = wide0 ? n_tiles0 / 2 : n_tiles0;
 
@@ -331,15 +338,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
             uint8_t* sA = smem + stage * C::STAGE_BYTES;
             uint8_t* sB = sA + C::A_BYTES;
             const uint32_t bar = leader_full + 8u * stage;
-            if (prob == 0) {
-              load_operand_pair<A0, C::BM_CTA>(sA, &tmA0, bar, a_row, kb * C::BK, pol_a0);
-              load_operand_pair<B0, C::BN_CTA>(sB, &tmB0, bar, b_row, kb * C::BK, pol_b0);
-              if constexpr (NSUB == 2)
-                load_operand_pair<B0, C::BN_CTA>(sB + C::STAGE_BYTES, &tmB0, bar + 8u,
-                                                 b_row + C::BN, kb * C::BK, pol_b0);
-            } else {
-              load_operand_pair<A1, C::BM_CTA>(sA, &tmA1, bar, a_row, kb * C::BK, pol_a1);
-              load_operand_pair<B1, C::BN_CTA>(sB, &tmB1, bar, b_row, kb * C::BK, pol_b1);
+#pragma unroll
+            for (int j = 0; j < C::KSUB; ++j) {
+              const int k0 = kb * C::KSLOT + j * C::BK;
+              if (prob == 0) {
+                load_operand_pair<A0, C::BM_CTA>(sA + j * C::A_SUB, &tmA0, bar, a_row, k0, pol_a0);
+                load_operand_pair<B0, C::BN_CTA>(sB + j * C::B_SUB, &tmB0, bar, b_row, k0, pol_b0);
+                if constexpr (NSUB == 2)
+                  load_operand_pair<B0, C::BN_CTA>(sB + C::STAGE_BYTES, &tmB0, bar + 8u,
+                                                   b_row + C::BN, k0, pol_b0);
+              } else {
+                load_operand_pair<A1, C::BM_CTA>(sA + j * C::A_SUB, &tmA1, bar, a_row, k0, pol_a1);
+                load_operand_pair<B1, C::BN_CTA>(sB + j * C::B_SUB, &tmB1, bar, b_row, k0, pol_b1);
+              }
             }
             arms += NSUB;
             stage += NSUB;
@@ -438,34 +449,41 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
             }
           } else {
             // the MMAs of one staged k-block into d_tmem
+            // the MMAs of one ring slot (KSUB k-blocks) into d_tmem
             auto issue = [&](int st, int kb) {
-              const uint32_t a_base = smem_u32(smem + st * C::STAGE_BYTES);
-              const uint32_t b_base = a_base + C::A_BYTES;
-              const uint64_t da = operand_desc<A0>(a_base, 0), db = operand_desc<B0>(b_base, 0);
-              const uint64_t da1 = operand_desc<A1>(a_base, 0), db1 = operand_desc<B1>(b_base, 0);
-              if constexpr (C::ELEM_BYTES == 1) {
 #pragma unroll
-                for (int k = 0; k < C::BK / C::MMA_K; ++k)
-                  mma_e4m3_ss_pair(d_tmem, operand_desc<Major::K>(a_base, k),
-                                   operand_desc<Major::K>(b_base, k), prob == 0 ? idesc0 : idesc1,
-                                   (kb | k) != 0 ? 1u : 0u);
-              } else if (prob == 0) {
+              for (int j = 0; j < C::KSUB; ++j) {
+                const uint32_t a_base = smem_u32(smem + st * C::STAGE_BYTES + j * C::A_SUB);
+                const uint32_t b_base = smem_u32(smem + st * C::STAGE_BYTES + C::A_BYTES +
+                                                 j * C::B_SUB);
+                const uint64_t da = operand_desc<A0>(a_base, 0), db = operand_desc<B0>(b_base, 0);
+                const uint64_t da1 = operand_desc<A1>(a_base, 0), db1 = operand_desc<B1>(b_base, 0);
+                const int first = kb | j;   // 0 only for the first k-block of the tile
+                if constexpr (C::ELEM_BYTES == 1) {
 #pragma unroll
-                for (int k = 0; k < C::BK / C::MMA_K; ++k)
-                  mma_bf16_ss_pair(d_tmem, da + desc_step<A0>() * k, db + desc_step<B0>() * k,
-                                   idesc0, (kb | k) != 0 ? 1u : 0u);
-              } else {
+                  for (int k = 0; k < C::BK / C::MMA_K; ++k)
+                    mma_e4m3_ss_pair(d_tmem, operand_desc<Major::K>(a_base, k),
+                                     operand_desc<Major::K>(b_base, k), prob == 0 ? idesc0 : idesc1,
+                                     (first | k) != 0 ? 1u : 0u);
+                } else if (prob == 0) {
 #pragma unroll
-                for (int k = 0; k < C::BK / C::MMA_K; ++k)
-                  mma_bf16_ss_pair(d_tmem, da1 + desc_step<A1>() * k, db1 + desc_step<B1>() * k,
-                                   idesc1, (kb | k) != 0 ? 1u : 0u);
+                  for (int k = 0; k < C::BK / C::MMA_K; ++k)
+                    mma_bf16_ss_pair(d_tmem, da + desc_step<A0>() * k, db + desc_step<B0>() * k,
+                                     idesc0, (first | k) != 0 ? 1u : 0u);
+                } else {
+#pragma unroll
+                  for (int k = 0; k < C::BK / C::MMA_K; ++k)
+                    mma_bf16_ss_pair(d_tmem, da1 + desc_step<A1>() * k, db1 + desc_step<B1>() * k,
+                                     idesc1, (first | k) != 0 ? 1u : 0u);
+                }
               }
             };
-            // ROUND = 2: two k-blocks per round, one fence and one loop step per eight MMAs.
-            // The single MMA-issuing thread is what limits these 4-MMA k-blocks (its waits,
-            // fence and commit take about as long as the MMAs run); this measured faster for the
-            // logits and slower for the dW tiles, whose MN-major loads arrive later.
-            static_assert(ROUND == 1 || ROUND == 2, "one or two k-blocks per round");
+            // ROUND = 2: two ring slots per round, one fence and one loop step for both.  The
+            // single MMA-issuing thread is what limits slots of one k-block (4 MMAs): its waits,
+            // fence and commit take about as long as the MMAs run.  The logits use slots of two
+            // k-blocks instead (KSUB = 2: one wait and one commit per 8 MMAs); the dW tiles keep
+            // one (two per round measured slower there: their MN-major loads arrive later).
+            static_assert(ROUND == 1 || ROUND == 2, "one or two ring slots per round");
             for (int kb = 0; kb < kbs; kb += ROUND) {
               const bool two = ROUND == 2 && kb + 1 < kbs;
               const int st2 = stage + 1 == C::STAGES ? 0 : stage + 1;
