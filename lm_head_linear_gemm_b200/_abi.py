@@ -213,10 +213,47 @@ def instrument_read() -> dict:
     return dict(launches_total=int(st.launches_total), gemm=kinds)
 
 
+def _check_buffer(t, name, dtype, shape, device):
+    """A caller-supplied tensor the library reads or writes through a raw pointer: it must be a
+    contiguous CUDA tensor on ``device`` with exactly this dtype and shape (a wrong one would
+    let a kernel write past its end)."""
+    if t is None:
+        return
+    if not t.is_cuda or t.device != device:
+        raise ValueError(f"{name} must be a CUDA tensor on {device}")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _check_scalar(t, name, dtype, device):
+    """A one-element device tensor (count, scale, upstream gradient)."""
+    if t is None:
+        return
+    if not t.is_cuda or t.device != device:
+        raise ValueError(f"{name} must be a CUDA tensor on {device}")
+    if t.dtype != dtype or t.numel() != 1:
+        raise TypeError(f"{name} must be a one-element {dtype} tensor")
+
+
+def _check_workspace(ws, device):
+    import torch
+    if ws is None:
+        return
+    if not ws.is_cuda or ws.device != device or ws.dtype != torch.uint8 or ws.dim() != 1 \
+            or not ws.is_contiguous():
+        raise ValueError(f"workspace must be a contiguous 1-D uint8 CUDA tensor on {device}")
+
+
 def _check(X, W, targets):
     import torch
     if not (X.is_cuda and W.is_cuda and targets.is_cuda):
         raise ValueError("X, W and targets must be CUDA tensors")
+    if not (X.device == W.device == targets.device):
+        raise ValueError("X, W and targets must be on the same device")
     if X.dtype != torch.bfloat16 or W.dtype != torch.bfloat16:
         raise TypeError("X and W must be bfloat16")
     if targets.dtype != torch.int64:
@@ -247,8 +284,12 @@ def forward(X, W, targets, Vreal: int, cap: float = 15.0, ignore_index: int = -1
     import torch
     _check(X, W, targets)
     N, d = X.shape
-    shape = make_shape(N, d, W.shape[0], Vreal, cap, ignore_index, chunk_rows)
     dev = X.device
+    if want_grads:
+        _check_buffer(dX, "dX", torch.bfloat16, X.shape, dev)
+        _check_buffer(dW, "dW", torch.float32, W.shape, dev)
+    _check_workspace(workspace, dev)
+    shape = make_shape(N, d, W.shape[0], Vreal, cap, ignore_index, chunk_rows)
     loss = torch.empty((), dtype=torch.float32, device=dev)
     lse = torch.empty(max(N, 1), dtype=torch.float32, device=dev)[:N]
     if want_grads:
@@ -274,11 +315,16 @@ def forward_dp(X, W, targets, n_valid_total, Vreal: int, cap: float = 15.0,
     data-parallel ranks.  Returns (loss share, lse, dX, dW, workspace)."""
     import torch
     _check(X, W, targets)
-    if not n_valid_total.is_cuda or n_valid_total.dtype != torch.int64:
-        raise TypeError("n_valid_total must be a CUDA int64 tensor")
     N, d = X.shape
-    shape = make_shape(N, d, W.shape[0], Vreal, cap, ignore_index, chunk_rows)
     dev = X.device
+    if n_valid_total is None:
+        raise TypeError("n_valid_total must be a CUDA int64 tensor")
+    _check_scalar(n_valid_total, "n_valid_total", torch.int64, dev)
+    if want_grads:
+        _check_buffer(dX, "dX", torch.bfloat16, X.shape, dev)
+        _check_buffer(dW, "dW", torch.float32, W.shape, dev)
+    _check_workspace(workspace, dev)
+    shape = make_shape(N, d, W.shape[0], Vreal, cap, ignore_index, chunk_rows)
     loss = torch.empty((), dtype=torch.float32, device=dev)
     lse = torch.empty(max(N, 1), dtype=torch.float32, device=dev)[:N]
     if want_grads:
@@ -301,9 +347,14 @@ def forward_dp(X, W, targets, n_valid_total, Vreal: int, cap: float = 15.0,
 def rmsnorm_forward(H, gamma, eps: float = 1e-6, X=None, rstd=None, stream=None):
     """x = h * rstd * gamma (bf16), rstd = 1/sqrt(mean(h^2) + eps) (fp32).  Returns (x, rstd)."""
     import torch
-    if H.dtype != torch.bfloat16 or gamma.dtype != torch.bfloat16 or not H.is_contiguous():
-        raise TypeError("H and gamma must be contiguous bf16 CUDA tensors")
+    if not H.is_cuda or H.dim() != 2:
+        raise ValueError("H must be a 2-D CUDA tensor [N, d]")
     N, d = H.shape
+    dev = H.device
+    _check_buffer(H, "H", torch.bfloat16, (N, d), dev)
+    _check_buffer(gamma, "gamma", torch.bfloat16, (d,), dev)
+    _check_buffer(X, "X", torch.bfloat16, (N, d), dev)
+    _check_buffer(rstd, "rstd", torch.float32, (N,), dev)
     if X is None:
         X = torch.empty_like(H)
     if rstd is None:
@@ -319,7 +370,16 @@ def rmsnorm_backward(H, gamma, rstd, dX, dH=None, dgamma=None, accumulate_dgamma
                      stream=None):
     """Chain rule through the RMSNorm for dX = dL/dx.  Returns (dH bf16, dgamma fp32)."""
     import torch
+    if not H.is_cuda or H.dim() != 2:
+        raise ValueError("H must be a 2-D CUDA tensor [N, d]")
     N, d = H.shape
+    dev = H.device
+    _check_buffer(H, "H", torch.bfloat16, (N, d), dev)
+    _check_buffer(gamma, "gamma", torch.bfloat16, (d,), dev)
+    _check_buffer(rstd, "rstd", torch.float32, (N,), dev)
+    _check_buffer(dX, "dX", torch.bfloat16, (N, d), dev)
+    _check_buffer(dH, "dH", torch.bfloat16, (N, d), dev)
+    _check_buffer(dgamma, "dgamma", torch.float32, (d,), dev)
     if dH is None:
         dH = torch.empty_like(H)
     if dgamma is None:
@@ -340,6 +400,8 @@ def quantize_e4m3(x, out=None, scale=None, stream=None):
     import torch
     if not x.is_cuda or x.dtype != torch.bfloat16 or not x.is_contiguous():
         raise TypeError("x must be a contiguous bf16 CUDA tensor")
+    _check_buffer(out, "out", torch.uint8, x.shape, x.device)
+    _check_scalar(scale, "scale", torch.float32, x.device)
     if out is None:
         out = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
     if scale is None:
@@ -361,13 +423,29 @@ def forward_fp8(X8, W8, scale_x, scale_w, X, W, targets, Vreal: int, cap: float 
             raise TypeError(f"{name} must be a CUDA uint8 / float8_e4m3fn tensor")
         if not t.is_contiguous():
             raise ValueError(f"{name} must be contiguous")
+    if X8.dim() != 2 or W8.dim() != 2 or X8.shape[1] != W8.shape[1]:
+        raise ValueError(f"expected X8 [N, d], W8 [Vpad, d]; got {tuple(X8.shape)}, "
+                         f"{tuple(W8.shape)}")
     N, d = X8.shape
-    shape = make_shape(N, d, W8.shape[0], Vreal, cap, ignore_index, chunk_rows)
     dev = X8.device
+    if W8.device != dev:
+        raise ValueError("X8 and W8 must be on the same device")
+    _check_scalar(scale_x, "scale_x", torch.float32, dev)
+    _check_scalar(scale_w, "scale_w", torch.float32, dev)
+    if scale_x is None or scale_w is None:
+        raise TypeError("scale_x and scale_w must be one-element float32 CUDA tensors")
+    _check_buffer(targets, "targets", torch.int64, (N,), dev)
+    if want_grads:
+        _check(X, W, targets)
+        _check_buffer(X, "X", torch.bfloat16, (N, d), dev)
+        _check_buffer(W, "W", torch.bfloat16, tuple(W8.shape), dev)
+        _check_buffer(dX, "dX", torch.bfloat16, (N, d), dev)
+        _check_buffer(dW, "dW", torch.float32, tuple(W8.shape), dev)
+    _check_workspace(workspace, dev)
+    shape = make_shape(N, d, W8.shape[0], Vreal, cap, ignore_index, chunk_rows)
     loss = torch.empty((), dtype=torch.float32, device=dev)
     lse = torch.empty(max(N, 1), dtype=torch.float32, device=dev)[:N]
     if want_grads:
-        _check(X, W, targets)
         if dX is None:
             dX = torch.empty_like(X)
         if dW is None:
@@ -392,14 +470,17 @@ def backward(X, W, targets, lse, Vreal: int, cap: float = 15.0, ignore_index: in
     import torch
     _check(X, W, targets)
     N, d = X.shape
-    shape = make_shape(N, d, W.shape[0], Vreal, cap, ignore_index, chunk_rows)
     dev = X.device
+    _check_buffer(lse, "lse", torch.float32, (N,), dev)
+    _check_buffer(dX, "dX", torch.bfloat16, X.shape, dev)
+    _check_buffer(dW, "dW", torch.float32, W.shape, dev)
+    _check_scalar(grad_out, "grad_out", torch.float32, dev)
+    _check_workspace(workspace, dev)
+    shape = make_shape(N, d, W.shape[0], Vreal, cap, ignore_index, chunk_rows)
     if dX is None:
         dX = torch.empty_like(X)
     if dW is None:
         dW = torch.empty(W.shape, dtype=torch.float32, device=dev)
-    if grad_out is not None and (grad_out.dtype != torch.float32 or not grad_out.is_cuda):
-        raise TypeError("grad_out must be a float32 CUDA scalar")
     if workspace is None and not grads_precomputed:
         workspace = alloc_workspace(shape, True, dev)
     rc = raw_backward(shape, _ptr(X), _ptr(W), _ptr(targets), _ptr(lse), _ptr(grad_out),
