@@ -1,7 +1,7 @@
 """Data-parallel fused linear cross-entropy: one process per GPU, ``torch.distributed``.
 
-The write-ups train the 3.8B model with plain DDP on one 8-GPU node (gradient all-reduce;
-"the distributed strategy is plain DDP"). Every rank holds the LM head W and its own token
+The write-ups train the 3.8B model with plain DDP on one 8-GPU node (a gradient all-reduce;
+their "distributed strategy" paragraph). Every rank holds the LM head W and its own token
 rows. One step here gives exactly the result of a single call on the union of all ranks'
 rows:
 
