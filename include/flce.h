@@ -3,8 +3,8 @@
  *
  * The operation (little-lm 3.8B write-ups):
  *   - the untied LM head W [Vpad, d] (154.5M = 50304 x 3072 parameters; "Setup" table);
- *   - logits z = X W^T with a logit softcap s = cap * tanh(z / cap), cap = 15 (config appendix:
- *     logit_softcap: 15.0, LigerFusedLinearCrossEntropyLoss(softcap=15.0); the pages print no
+ *   - logits z = X W^T with a logit softcap s = cap * tanh(z / cap), cap = 15 (the config
+ *     appendix sets a softcap of 15 for the model and its fused loss; the pages print no
  *     formula, cap*tanh(z/cap) is the reading used);
  *   - a vocabulary of Vreal = 50257 tokens padded to Vpad = 50304, a multiple of 64, for the
  *     tensor cores ("Increasing throughput", vocabulary padding; config appendix).  Padded

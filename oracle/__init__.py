@@ -10,8 +10,8 @@ inputs (the GPU path reads the same bf16 values):
 
 * logits of the untied LM head, ``z = X W^T`` over all ``Vpad`` rows of ``W``
   (little-lm 3.8B write-up, "Setup": LM head of 154.5M = 50304 x 3072 parameters);
-* the logit softcap ``s = cap * tanh(z / cap)`` with ``cap = 15`` (config
-  appendix: ``logit_softcap: 15.0``; loss ``LigerFusedLinearCrossEntropyLoss(softcap=15.0)``).
+* the logit softcap ``s = cap * tanh(z / cap)`` with ``cap = 15`` (the config appendix sets a
+  logit softcap of 15 and passes the same value to its third-party fused loss).
   The pages name the softcap but print no formula; ``cap*tanh(z/cap)`` is the
   reading adopted.  ``cap <= 0`` means no softcap (``s = z``);
 * the padded vocabulary (50257 real tokens padded to 50304 for the tensor cores,

@@ -8,8 +8,7 @@ Workload shapes follow the little-lm 3.8B write-ups: the untied LM head is
 ``[50304, 3072]`` (154.5M parameters, "Setup" table of the write-up and the
 config appendix), the GPT-2 vocabulary of 50257 tokens is padded to 50304, a
 multiple of 64 (config appendix, "Increasing throughput"), and the logit softcap
-is 15.0 (config appendix: ``logit_softcap: 15.0``,
-``LigerFusedLinearCrossEntropyLoss(softcap=15.0)``).  The pages train on
+is 15.0 (the config appendix sets it for the model and for its fused loss).  The pages train on
 ClimbMix text through the GPT-2 tokenizer; that data is not available, so
 targets are drawn from a truncated Zipf law over the real vocabulary as a
 stand-in for natural-text token frequencies.
