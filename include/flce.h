@@ -185,6 +185,7 @@ int flce_quantize_e4m3(const void* src, int64_t n, void* dst, float* scale_out, 
  * with RMSNorm; config appendix: rms_norm_eps = 1.0e-6):
  *   x_i = h_i * rstd_i * gamma,  rstd_i = 1 / sqrt(mean_k h_ik^2 + eps)   (fp32 arithmetic)
  * H [N, d] bf16, gamma [d] bf16, X [N, d] bf16 (out), rstd [N] fp32 (out).  d % 8 == 0.
+ * H, gamma, X, dX, dH 16-byte aligned; rstd and dgamma 4-byte aligned.
  * Backward, for dX = dL/dx from the loss (e.g. flce_forward's dX):
  *   dH = rstd * (g - xh * mean_k(g * xh)),  dgamma = sum_i dX * xh,  xh = h * rstd, g = dX * gamma
  * dH [N, d] bf16 (out); dgamma [d] fp32 written, or added to with accumulate_dgamma = 1.  The

@@ -788,7 +788,7 @@ int flce_rmsnorm_forward(const void* H, const void* gamma, float eps, int64_t N,
                          void* X, float* rstd, void* stream) {
   FLCE_TRY(rms_args_ok(H, gamma, N, d));
   if (!(eps >= 0.f) || (N > 0 && (X == nullptr || rstd == nullptr))) return FLCE_ERR_ARG;
-  if (!aligned16(X)) return FLCE_ERR_ALIGN;
+  if (!aligned16(X) || (reinterpret_cast<uintptr_t>(rstd) & 3u) != 0) return FLCE_ERR_ALIGN;
   DeviceInfo* di = nullptr;
   FLCE_TRY(device_info(&di));
   if (N == 0) return FLCE_OK;
@@ -813,6 +813,7 @@ int flce_rmsnorm_backward(const void* H, const void* gamma, const float* rstd, c
       (N > 0 && (rstd == nullptr || dX == nullptr || dH == nullptr)))
     return FLCE_ERR_ARG;
   if (!aligned16(dX) || !aligned16(dH) || (reinterpret_cast<uintptr_t>(dgamma) & 3u) != 0 ||
+      (reinterpret_cast<uintptr_t>(rstd) & 3u) != 0 ||
       (reinterpret_cast<uintptr_t>(workspace) & 15u) != 0)
     return FLCE_ERR_ALIGN;
   if (workspace_bytes < flce_rmsnorm_workspace_bytes(N, d)) return FLCE_ERR_WORKSPACE;

@@ -121,3 +121,25 @@ def test_shape_struct_matches_header():
     # int64 N, d, Vpad, Vreal; float cap (+4 padding); int64 ignore_index, chunk_rows
     assert ctypes.sizeof(_abi.flce_shape) == 56
     assert _abi.flce_shape.cap.offset == 32 and _abi.flce_shape.ignore_index.offset == 40
+
+
+def test_rmsnorm_and_quantiser_reject_bad_arguments_before_launch(L):
+    p = 0x10000000      # never dereferenced: argument checks come first
+    fwd = L.flce_rmsnorm_forward
+    fwd.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_float, ctypes.c_int64,
+                    ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
+    assert fwd(p, None, 1e-6, 4, 64, p, p, None) == -1          # gamma missing
+    assert fwd(p, p, -1.0, 4, 64, p, p, None) == -1             # negative eps
+    assert fwd(p, p, 1e-6, 4, 60, p, p, None) == -2             # d % 8 != 0
+    assert fwd(p + 8, p, 1e-6, 4, 64, p, p, None) == -2         # H not 16-byte aligned
+    assert fwd(p, p, 1e-6, 4, 64, p, p + 2, None) == -2         # rstd not 4-byte aligned
+    bwd = L.flce_rmsnorm_backward
+    ws = flce.lib().flce_rmsnorm_workspace_bytes(300, 64)
+    assert ws >= 3 * 64 * 4
+    assert bwd(p, p, p, p, 300, 64, p, p, 0, p, ws - 1, None) == -3
+    assert bwd(p, p, p + 2, p, 300, 64, p, p, 0, p, ws, None) == -2
+    assert bwd(p, p, p, p, 300, 64, p, None, 0, p, ws, None) == -1
+    q = L.flce_quantize_e4m3
+    assert q(p, -1, p, p, None) == -1
+    assert q(p, 16, None, p, None) == -1
+    assert q(p, 16, p, p + 2, None) == -2
