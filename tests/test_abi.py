@@ -143,3 +143,29 @@ def test_rmsnorm_and_quantiser_reject_bad_arguments_before_launch(L):
     assert q(p, -1, p, p, None) == -1
     assert q(p, 16, None, p, None) == -1
     assert q(p, 16, p, p + 2, None) == -2
+
+
+def test_fp8_dp_and_count_entry_points_reject_bad_arguments_before_launch(L):
+    p = 0x10000000      # never dereferenced: argument checks come first
+    s = flce.make_shape(8, 64, 128, 100)
+    ws = flce.workspace_bytes(s, True)
+    sp = ctypes.byref(s)
+    f8 = L.flce_forward_fp8
+    # X8, W8, sx, sw, X, W, t, loss, lse, want_grads, dX, dW, acc, ws, ws_bytes, stream
+    assert f8(sp, p, p, None, p, p, p, p, p, p, 1, p, p, 0, p, ws, None) == -1    # scale_x
+    assert f8(sp, p, p, p, p, None, p, p, p, p, 1, p, p, 0, p, ws, None) == -1    # X for grads
+    assert f8(sp, p, p, p + 2, p, p, p, p, p, p, 1, p, p, 0, p, ws, None) == -2   # scale align
+    assert f8(sp, p + 8, p, p, p, p, p, p, p, p, 1, p, p, 0, p, ws, None) == -2   # X8 align
+    assert f8(sp, p, p, p, p, p, p, p, p, p, 1, p, p, 0, p, ws - 1, None) == -3
+    s48 = flce.make_shape(8, 72, 128, 100)          # d % 16 != 0: e4m3 rows not 16-byte
+    assert f8(ctypes.byref(s48), p, p, p, p, p, p, p, p, p, 0, None, None, 0, p, 1 << 30,
+              None) == -2
+    dp = L.flce_forward_dp
+    # X, W, t, nv_total, loss, lse, want_grads, dX, dW, acc, ws, ws_bytes, stream
+    assert dp(sp, p, p, p, None, p, p, 1, p, p, 0, p, ws, None) == -1             # count
+    assert dp(sp, p, p, p, p + 4, p, p, 1, p, p, 0, p, ws, None) == -2            # 8-byte
+    cv = L.flce_count_valid
+    assert cv(sp, p, None, None) == -1
+    assert cv(sp, p, p + 4, None) == -2
+    bad = flce.make_shape(8, 64, 128, 200)          # Vreal > Vpad
+    assert cv(ctypes.byref(bad), p, p, None) == -1
