@@ -93,6 +93,15 @@ def workload_desc(c, chunk):
     }
 
 
+def arm_config(c, chunk, world, dp, accum_steps):
+    """The ``config`` object of the JSON line; both arms print the same one for the same
+    arguments."""
+    return dict(workload_desc(c, chunk),
+                parallelism=(f"data parallel x{world}: global-count loss, dW all-reduce every "
+                             f"{accum_steps} micro-batches" if dp else
+                             f"replicas x{world}" if world > 1 else "single GPU"))
+
+
 # ----------------------------------------------------------------------------------- CPU oracle
 def blas_threads() -> int:
     try:
@@ -138,10 +147,11 @@ def cpu_baseline(inp, target_s: float):
 
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
     if rank != 0:
         return 0
     import synth
-    inp = synth.make_inputs(args.config)
+    inp = synth.make_inputs(args.config, N=args.rows or None)
     c = inp["cfg"]
     rows = max(1, min(args.ref_rows, c.N))
     times = []
@@ -157,7 +167,10 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": workload_desc(c, 0),
+        "data": "synthetic",
+        "config": arm_config(c, args.chunk_rows or min(c.N, AUTO_CHUNK_ROWS), world,
+                             world > 1 and not args.no_allreduce and args.config != "fp8",
+                             args.accum_steps),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
                          "sample": f"{rows} contiguous rows per step (fp64 forward + backward "
                                    f"over all Vpad and d, dW contribution included)"},
@@ -478,11 +491,8 @@ def main_gpu(args):
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None,
             "dtype": "e4m3 logits + bf16 gradients" if fp8 else "bf16", "data": "synthetic",
-            "config": dict(workload_desc(c, shape.chunk_rows or min(N, AUTO_CHUNK_ROWS)),
-                           parallelism=(f"data parallel x{world}: global-count loss, dW "
-                                        f"all-reduce every {args.accum_steps} micro-batches"
-                                        if dp else
-                                        f"replicas x{world}" if world > 1 else "single GPU")),
+            "config": arm_config(c, shape.chunk_rows or min(N, AUTO_CHUNK_ROWS), world, dp,
+                                 args.accum_steps),
             "tflops": tflops,
             "pct_of_bf16_datasheet_2250": tflops / world / DATASHEET_BF16_TFLOPS,
             "pct_of_measured_bf16_burst": tflops / world / burst,
