@@ -424,3 +424,35 @@ def test_rmsnorm_then_loss_finite_differences():
         num_dg[k] = (L(H, gp) - L(H, gm)) / (2 * h)
     assert np.linalg.norm(num_dH - dH) <= 1e-6 * np.linalg.norm(dH)
     assert np.linalg.norm(num_dg - dg) <= 1e-6 * np.linalg.norm(dg)
+
+
+# --------------------------------------------------------------------------- randomised library check
+def test_against_torch_on_random_shapes():
+    """The library special case (torch cross_entropy + autograd in fp64, through torch.tanh
+    for the softcap) on many random small shapes, caps, weight scales and ignored counts,
+    including padded vocabularies, all-ignored batches and a single row."""
+    hypothesis = pytest.importorskip("hypothesis")
+    st = hypothesis.strategies
+
+    @hypothesis.settings(max_examples=60, deadline=None, derandomize=True)
+    @hypothesis.given(N=st.integers(1, 9), d=st.integers(1, 10), Vr=st.integers(2, 25),
+                      pad=st.integers(0, 9), cap=st.sampled_from([0.0, 0.5, 3.0, 15.0]),
+                      w_std=st.sampled_from([0.1, 1.0, 4.0]), ign=st.integers(0, 9),
+                      seed=st.integers(0, 10_000))
+    def check(N, d, Vr, pad, cap, w_std, ign, seed):
+        rng = np.random.default_rng(seed)
+        X = rng.standard_normal((N, d))
+        W = rng.standard_normal((Vr + pad, d)) * w_std
+        t = rng.integers(0, Vr, N)
+        t[rng.permutation(N)[:min(ign, N)]] = -1
+        f = oracle.forward_backward(X, W, t, Vr, cap, -1)
+        if (t >= 0).sum() == 0:            # the oracle's reading: loss 0, zero gradients
+            assert f["loss"] == 0.0 and not f["dX"].any() and not f["dW"].any()
+            return
+        ref_loss, ref_dX, ref_dW = _torch_reference(X, W, t, Vr, cap, -1)
+        assert abs(f["loss"] - ref_loss) <= 1e-12 * max(1.0, abs(ref_loss))
+        np.testing.assert_allclose(f["dX"], ref_dX, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(f["dW"], ref_dW, rtol=0, atol=1e-12)
+        assert not f["dW"][Vr:].any()
+
+    check()
