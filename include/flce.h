@@ -69,7 +69,7 @@ typedef struct {
   int64_t Vreal;        /* real vocabulary, 1 <= Vreal <= Vpad */
   float cap;            /* logit softcap; <= 0 disables it */
   int64_t ignore_index; /* target value that leaves a row out of the loss (e.g. -1) */
-  int64_t chunk_rows;   /* rows per fused chunk (bounds the scratch); 0 = automatic */
+  int64_t chunk_rows;   /* rows per fused chunk (bounds the scratch); 0 = automatic: 8192 */
 } flce_shape;
 
 /*
