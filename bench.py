@@ -59,6 +59,10 @@ def parse_args():
                          "all-reduced after the last (the write-ups: 7)")
     ap.add_argument("--no-allreduce", action="store_true",
                     help="N>1: independent replicas with no collective (weak-scaling floor)")
+    ap.add_argument("--buckets", type=int, default=4,
+                    help="N>1: vocabulary buckets of the dW all-reduce, each exchanged as soon "
+                         "as the last chunk's gradient launch for it is done (1: one all-reduce "
+                         "after the step)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--ref-rows", type=int, default=128,
@@ -93,12 +97,13 @@ def workload_desc(c, chunk):
     }
 
 
-def arm_config(c, chunk, world, dp, accum_steps):
+def arm_config(c, chunk, world, dp, accum_steps, buckets=1):
     """The ``config`` object of the JSON line; both arms print the same one for the same
     arguments."""
     return dict(workload_desc(c, chunk),
                 parallelism=(f"data parallel x{world}: global-count loss, dW all-reduce every "
-                             f"{accum_steps} micro-batches" if dp else
+                             f"{accum_steps} micro-batches in {buckets} vocabulary buckets "
+                             f"overlapping the last gradient launches" if dp else
                              f"replicas x{world}" if world > 1 else "single GPU"))
 
 
@@ -170,7 +175,7 @@ def run_reference(args):
         "data": "synthetic",
         "config": arm_config(c, args.chunk_rows or min(c.N, AUTO_CHUNK_ROWS), world,
                              world > 1 and not args.no_allreduce and args.config != "fp8",
-                             args.accum_steps),
+                             args.accum_steps, args.buckets),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
                          "sample": f"{rows} contiguous rows per step (fp64 forward + backward "
                                    f"over all Vpad and d, dW contribution included)"},
@@ -298,6 +303,9 @@ def main_gpu(args):
 
     dp = world > 1 and not args.no_allreduce and not fp8
     micro = [0]
+    # each micro-batch's loss is divided by the number of micro-batches
+    g_accum = torch.tensor(1.0 / max(1, args.accum_steps), dtype=torch.float32, device=dev)
+    dp_ops = flce.data_parallel.LibraryOps() if dp else None
 
     def step(Xd=None, td=None):
         Xd = X if Xd is None else Xd
@@ -310,7 +318,8 @@ def main_gpu(args):
             loss, _, _, _, _ = flce.dp_step(
                 Xd, W, td, Vr, c.cap, c.ignore_index, dW=dW, accumulate_dW=k > 0,
                 allreduce_dW=k == max(1, args.accum_steps) - 1, workspace=ws,
-                chunk_rows=args.chunk_rows)
+                chunk_rows=args.chunk_rows, grad_scale=g_accum, buckets=args.buckets,
+                ops=dp_ops)
             return loss
         if fp8:
             loss, lse, _, _, _ = flce.forward_fp8(X8, W8, sX, sW, Xd, W, td, Vr, c.cap,
@@ -444,7 +453,9 @@ def main_gpu(args):
                "ms_per_step": e2e_ms / args.steps,
                "what": "pinned-host X and targets copied in and the loss copied out every step "
                        "(copies on a side stream, double-buffered, overlapping the previous "
-                       "step); W and dW stay resident (the head's parameter and its gradient)"}
+                       "step); W and dW stay resident (the head's parameter and its gradient), "
+                       "and dX stays on the device, where the backward of the layer below "
+                       "consumes it"}
 
     peaks, peaks_src = load_peaks()
     sustained = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
@@ -492,7 +503,7 @@ def main_gpu(args):
             "scaling": "weak", "vs_baseline": None,
             "dtype": "e4m3 logits + bf16 gradients" if fp8 else "bf16", "data": "synthetic",
             "config": arm_config(c, shape.chunk_rows or min(N, AUTO_CHUNK_ROWS), world, dp,
-                                 args.accum_steps),
+                                 args.accum_steps, args.buckets),
             "tflops": tflops,
             "pct_of_bf16_datasheet_2250": tflops / world / DATASHEET_BF16_TFLOPS,
             "pct_of_measured_bf16_burst": tflops / world / burst,

@@ -24,7 +24,7 @@
  *   - Data pointers are DEVICE pointers owned by the caller; the library never allocates or
  *     frees memory.  Scratch space is the caller's `workspace` (see flce_workspace_bytes).
  *   - Layouts are row-major and dense: X [N, d] bf16, W [Vpad, d] bf16, targets [N] int64,
- *     lse [N] fp32, loss [1] fp32, dX [N, d] bf16, dW [Vpad, d] fp32.
+ *     lse [N] fp32, loss [1] fp32, dX [N, d] bf16, dW [Vpad, d] fp32 or bf16 (dW_dtype).
  *   - Every array pointer must be 16-byte aligned except loss and lse (4-byte aligned); d and
  *     Vpad must be multiples of 8 (the tensor-memory-accelerator row stride must be a multiple
  *     of 16 bytes).
@@ -62,6 +62,9 @@ typedef enum {
 /* Bits of the device status word (flce_read_status). */
 enum { FLCE_DEV_BAD_TARGET = 1u, FLCE_DEV_TIMEOUT = 2u };
 
+/* Element type of the dW output (dW_dtype arguments). */
+enum { FLCE_DTYPE_F32 = 0, FLCE_DTYPE_BF16 = 1 };
+
 typedef struct {
   int64_t N;            /* tokens (rows of X, targets); N = 0 is allowed and gives loss 0 */
   int64_t d;            /* hidden size; multiple of 8 */
@@ -83,32 +86,43 @@ size_t flce_workspace_bytes(const flce_shape* shape, int want_grads);
 
 /*
  * Forward.  Writes loss[0] (mean over rows in the loss) and lse[i] for every row (ignored rows
- * included).  With want_grads = 1 it also forms the gradients of the mean loss (upstream
- * gradient g = 1) in the same pass over the logits: dX [N, d] bf16 is written, and dW [Vpad, d]
- * fp32 is written (accumulate_dW = 0) or added to (accumulate_dW = 1, gradient accumulation over
- * micro-batches as in the pages' 7-step accumulation).  With want_grads = 0, dX and dW may be
- * NULL and are not touched.  When N = 0, X, targets, lse and dX may be NULL.
+ * included).  With want_grads = 1 it also forms, in the same pass over the logits, the
+ * gradients of g * loss for the upstream gradient g = *grad_scale (a device float; NULL means
+ * g = 1): dX [N, d] bf16 is written, and dW [Vpad, d] is written (accumulate_dW = 0) or added to
+ * (accumulate_dW = 1).  Gradient accumulation over micro-batches (the pages accumulate over 7
+ * per optimizer step) with each micro-batch's loss divided by the number of micro-batches m is
+ * accumulate_dW = 1 with *grad_scale = 1/m on every call: each call adds only its own scaled
+ * contribution.
+ *   dW_dtype: FLCE_DTYPE_F32 (fp32 dW) or FLCE_DTYPE_BF16 (bf16 dW, for bf16 master weights;
+ *     each chunk's contribution is added to the stored values in fp32 and rounded to bf16 once).
+ * With want_grads = 0, grad_scale, dX and dW may be NULL and are not touched.  When N = 0, X,
+ * targets, lse and dX may be NULL.
  * workspace: device scratch of at least flce_workspace_bytes(shape, want_grads) bytes,
  * 256-byte aligned; its contents on entry are ignored.
  */
 int flce_forward(const flce_shape* shape, const void* X, const void* W, const int64_t* targets,
-                 float* loss, float* lse, int want_grads, void* dX, float* dW, int accumulate_dW,
-                 void* workspace, size_t workspace_bytes, void* stream);
+                 float* loss, float* lse, int want_grads, const float* grad_scale, void* dX,
+                 void* dW, int dW_dtype, int accumulate_dW, void* workspace,
+                 size_t workspace_bytes, void* stream);
 
 /*
  * Backward.
- *   grads_precomputed = 1: dX and dW were formed by flce_forward(want_grads = 1); they are
- *     multiplied in place by the device scalar *grad_out (nothing runs when grad_out is NULL;
- *     the kernel returns at once when *grad_out == 1).  When the forward accumulated into dW,
- *     the whole dW buffer is scaled.
+ *   grads_precomputed = 1: dX and dW were formed by flce_forward(want_grads = 1) with
+ *     accumulate_dW = 0 and grad_scale NULL; both are multiplied in place by the device scalar
+ *     *grad_out (nothing runs when grad_out is NULL; the kernel returns at once when
+ *     *grad_out == 1).  accumulate_dW must be 0 here (FLCE_ERR_ARG otherwise): a dW that holds
+ *     earlier micro-batches cannot be scaled after the fact -- pass g to the forward as
+ *     grad_scale instead.
  *   grads_precomputed = 0: recomputes the logits chunk by chunk from X and W, using lse from
  *     flce_forward, and forms dX (written) and dW (written, or added to when
  *     accumulate_dW = 1) for upstream gradient *grad_out (1 when grad_out is NULL).
- * workspace: at least flce_workspace_bytes(shape, 1) bytes.
+ * dW_dtype as in flce_forward.  workspace: at least flce_workspace_bytes(shape, 1) bytes
+ * (unused when grads_precomputed = 1).
  */
 int flce_backward(const flce_shape* shape, const void* X, const void* W, const int64_t* targets,
-                  const float* lse, const float* grad_out, void* dX, float* dW, int accumulate_dW,
-                  int grads_precomputed, void* workspace, size_t workspace_bytes, void* stream);
+                  const float* lse, const float* grad_out, void* dX, void* dW, int dW_dtype,
+                  int accumulate_dW, int grads_precomputed, void* workspace,
+                  size_t workspace_bytes, void* stream);
 
 /*
  * Forward without any caller-provided scratch: loss[0] and lse[N] exactly as flce_forward with
@@ -127,8 +141,9 @@ int flce_backward(const flce_shape* shape, const void* X, const void* W, const i
  *   - All calls share the array and it keeps the last call's contents (nothing in it needs to
  *     start at zero).  Calls that overlap on the GPU (different streams, or different host
  *     threads without ordering) race on it and must not be issued.
- *   - The status word of the call stays inside the array and is not reported.
- * Same argument rules as flce_forward otherwise.
+ *   - The device status word and the count of rows in the loss of the last call on the current
+ *     device are read with flce_read_status(NULL, ...), like a workspace's.
+ * Same argument rules as flce_forward with want_grads = 0 otherwise.
  */
 #define FLCE_NOALLOC_SCRATCH_BYTES (16u << 20)
 int flce_forward_noalloc(const flce_shape* shape, const void* X, const void* W,
@@ -151,8 +166,29 @@ int flce_count_valid(const flce_shape* shape, const int64_t* targets, int64_t* n
                      void* stream);
 int flce_forward_dp(const flce_shape* shape, const void* X, const void* W, const int64_t* targets,
                     const int64_t* n_valid_total, float* loss, float* lse, int want_grads,
-                    void* dX, float* dW, int accumulate_dW, void* workspace,
-                    size_t workspace_bytes, void* stream);
+                    const float* grad_scale, void* dX, void* dW, int dW_dtype,
+                    int accumulate_dW, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * flce_forward_dp (want_grads = 1) whose dW becomes final in vocabulary buckets, so that the
+ * caller's dW all-reduce (step 4) can overlap the rest of the computation: the gradient
+ * contractions of the last chunk run as n_buckets launches; launch b completes dW rows
+ * [bucket_bounds[b], bucket_bounds[b + 1]) (whole 256-row vocabulary tiles; the last bucket
+ * also carries dX), after which the library records bucket_events[b] on `stream`.
+ *   n_buckets: 1 .. min(64, ceil(Vpad / 256)).
+ *   bucket_events: n_buckets cudaEvent_t handles created by the caller (none NULL).
+ *   bucket_bounds: host array of n_buckets + 1 int64, written before the call returns.
+ * A caller exchanges bucket b by making its communication stream wait on bucket_events[b] and
+ * all-reducing those dW rows there.  The write-ups train with unmodified DDP ("distributed
+ * strategy" paragraph), which all-reduces gradients in buckets that overlap the backward pass;
+ * this is that overlap for the head's gradient, which the fused forward forms.
+ */
+int flce_forward_dp_bucketed(const flce_shape* shape, const void* X, const void* W,
+                             const int64_t* targets, const int64_t* n_valid_total, float* loss,
+                             float* lse, const float* grad_scale, void* dX, void* dW,
+                             int dW_dtype, int accumulate_dW, int n_buckets,
+                             void* const* bucket_events, int64_t* bucket_bounds,
+                             void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * Forward with FP8 logits: the logits contraction z = X W^T reads e4m3 operands with dynamic
@@ -168,9 +204,9 @@ int flce_forward_dp(const flce_shape* shape, const void* X, const void* W, const
  */
 int flce_forward_fp8(const flce_shape* shape, const void* X8, const void* W8,
                      const float* scale_x, const float* scale_w, const void* X, const void* W,
-                     const int64_t* targets, float* loss, float* lse, int want_grads, void* dX,
-                     float* dW, int accumulate_dW, void* workspace, size_t workspace_bytes,
-                     void* stream);
+                     const int64_t* targets, float* loss, float* lse, int want_grads,
+                     const float* grad_scale, void* dX, void* dW, int dW_dtype,
+                     int accumulate_dW, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * Dynamic tensorwise e4m3 quantisation of n bf16 values: *scale_out = amax(|src|) / 448
@@ -222,8 +258,9 @@ int flce_check_pair_schedule(int pairs, int T0, int c0, int T1, int c1, int64_t*
 
 /*
  * Reads the device status word (FLCE_DEV_* bits) and the number of rows in the loss from the
- * workspace of the last call on `stream`.  Synchronises that stream.  Either output may be
- * NULL.
+ * workspace of the last call on `stream`; workspace = NULL reads those of the last
+ * flce_forward_noalloc call on the current device.  Synchronises that stream.  Either output
+ * may be NULL.
  */
 int flce_read_status(const void* workspace, uint32_t* dev_status_out, int64_t* n_valid_out,
                      void* stream);

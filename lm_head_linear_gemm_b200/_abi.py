@@ -18,6 +18,8 @@ FLCE_OK = 0
 NOALLOC_SCRATCH_BYTES = 16 << 20      # FLCE_NOALLOC_SCRATCH_BYTES in include/flce.h
 DEV_BAD_TARGET = 1
 DEV_TIMEOUT = 2
+DTYPE_F32 = 0                         # FLCE_DTYPE_F32: fp32 dW
+DTYPE_BF16 = 1                        # FLCE_DTYPE_BF16: bf16 dW
 
 
 class FlceError(RuntimeError):
@@ -72,25 +74,28 @@ def lib() -> ctypes.CDLL:
     shp = ctypes.POINTER(flce_shape)
     L.flce_workspace_bytes.argtypes = [shp, ctypes.c_int]
     L.flce_workspace_bytes.restype = ctypes.c_size_t
-    L.flce_forward.argtypes = [shp, P, P, P, P, P, ctypes.c_int, P, P, ctypes.c_int, P,
-                               ctypes.c_size_t, P]
+    I = ctypes.c_int
+    L.flce_forward.argtypes = [shp, P, P, P, P, P, I, P, P, P, I, I, P, ctypes.c_size_t, P]
     L.flce_forward.restype = ctypes.c_int
-    L.flce_backward.argtypes = [shp, P, P, P, P, P, P, P, ctypes.c_int, ctypes.c_int, P,
-                                ctypes.c_size_t, P]
+    L.flce_backward.argtypes = [shp, P, P, P, P, P, P, P, I, I, I, P, ctypes.c_size_t, P]
     L.flce_backward.restype = ctypes.c_int
     L.flce_read_status.argtypes = [P, ctypes.POINTER(ctypes.c_uint32),
                                    ctypes.POINTER(ctypes.c_int64), P]
     L.flce_read_status.restype = ctypes.c_int
-    L.flce_forward_fp8.argtypes = [shp, P, P, P, P, P, P, P, P, P, ctypes.c_int, P, P,
-                                   ctypes.c_int, P, ctypes.c_size_t, P]
+    L.flce_forward_fp8.argtypes = [shp, P, P, P, P, P, P, P, P, P, I, P, P, P, I, I, P,
+                                   ctypes.c_size_t, P]
     L.flce_forward_fp8.restype = ctypes.c_int
     L.flce_quantize_e4m3.argtypes = [P, ctypes.c_int64, P, P, P]
     L.flce_quantize_e4m3.restype = ctypes.c_int
     L.flce_count_valid.argtypes = [shp, P, P, P]
     L.flce_count_valid.restype = ctypes.c_int
-    L.flce_forward_dp.argtypes = [shp, P, P, P, P, P, P, ctypes.c_int, P, P, ctypes.c_int, P,
+    L.flce_forward_dp.argtypes = [shp, P, P, P, P, P, P, I, P, P, P, I, I, P,
                                   ctypes.c_size_t, P]
     L.flce_forward_dp.restype = ctypes.c_int
+    L.flce_forward_dp_bucketed.argtypes = [shp, P, P, P, P, P, P, P, P, P, I, I, I,
+                                           ctypes.POINTER(P), ctypes.POINTER(ctypes.c_int64), P,
+                                           ctypes.c_size_t, P]
+    L.flce_forward_dp_bucketed.restype = ctypes.c_int
     L.flce_forward_noalloc.argtypes = [shp, P, P, P, P, P, P]
     L.flce_forward_noalloc.restype = ctypes.c_int
     L.flce_rmsnorm_forward.argtypes = [P, P, ctypes.c_float, ctypes.c_int64, ctypes.c_int64, P,
@@ -144,12 +149,13 @@ def _stream(stream) -> int | None:
     return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
 
 
-def raw_forward(shape, X_ptr, W_ptr, t_ptr, loss_ptr, lse_ptr, want_grads, dX_ptr, dW_ptr,
-                accumulate_dW, ws_ptr, ws_bytes, stream_handle) -> int:
-    """Direct C-ABI call with integer pointers; returns the flce_status code."""
+def raw_forward(shape, X_ptr, W_ptr, t_ptr, loss_ptr, lse_ptr, want_grads, grad_scale_ptr,
+                dX_ptr, dW_ptr, dW_dtype, accumulate_dW, ws_ptr, ws_bytes, stream_handle) -> int:
+    """Direct C-ABI call with integer pointers (flce_forward's argument order); returns the
+    flce_status code."""
     return lib().flce_forward(ctypes.byref(shape), X_ptr, W_ptr, t_ptr, loss_ptr, lse_ptr,
-                              int(want_grads), dX_ptr, dW_ptr, int(accumulate_dW), ws_ptr,
-                              int(ws_bytes), stream_handle)
+                              int(want_grads), grad_scale_ptr, dX_ptr, dW_ptr, int(dW_dtype),
+                              int(accumulate_dW), ws_ptr, int(ws_bytes), stream_handle)
 
 
 def raw_forward_noalloc(shape, X_ptr, W_ptr, t_ptr, loss_ptr, lse_ptr, stream_handle) -> int:
@@ -159,15 +165,18 @@ def raw_forward_noalloc(shape, X_ptr, W_ptr, t_ptr, loss_ptr, lse_ptr, stream_ha
                                       lse_ptr, stream_handle)
 
 
-def raw_backward(shape, X_ptr, W_ptr, t_ptr, lse_ptr, g_ptr, dX_ptr, dW_ptr, accumulate_dW,
-                 grads_precomputed, ws_ptr, ws_bytes, stream_handle) -> int:
+def raw_backward(shape, X_ptr, W_ptr, t_ptr, lse_ptr, g_ptr, dX_ptr, dW_ptr, dW_dtype,
+                 accumulate_dW, grads_precomputed, ws_ptr, ws_bytes, stream_handle) -> int:
+    """Direct C-ABI call of flce_backward (its argument order); returns the flce_status code."""
     return lib().flce_backward(ctypes.byref(shape), X_ptr, W_ptr, t_ptr, lse_ptr, g_ptr, dX_ptr,
-                               dW_ptr, int(accumulate_dW), int(grads_precomputed), ws_ptr,
-                               int(ws_bytes), stream_handle)
+                               dW_ptr, int(dW_dtype), int(accumulate_dW), int(grads_precomputed),
+                               ws_ptr, int(ws_bytes), stream_handle)
 
 
 def read_status(workspace, stream=None) -> tuple[int, int]:
-    """(device status bits, rows in the loss) of the last call that used ``workspace``."""
+    """(device status bits, rows in the loss) of the last call that used ``workspace``;
+    ``workspace=None`` reads those of the last ``flce_forward_noalloc`` call on the current
+    device."""
     st = ctypes.c_uint32(0)
     nv = ctypes.c_int64(0)
     rc = lib().flce_read_status(_ptr(workspace), ctypes.byref(st), ctypes.byref(nv),
@@ -248,6 +257,29 @@ def _check_workspace(ws, device):
         raise ValueError(f"workspace must be a contiguous 1-D uint8 CUDA tensor on {device}")
 
 
+def _dW_type(dW, dW_dtype):
+    """(torch dtype, FLCE_DTYPE_* code) of the dW output: the given buffer's type, else
+    ``dW_dtype`` (default float32)."""
+    import torch
+    dt = dW.dtype if dW is not None else (dW_dtype if dW_dtype is not None else torch.float32)
+    if dt == torch.float32:
+        return torch.float32, DTYPE_F32
+    if dt == torch.bfloat16:
+        return torch.bfloat16, DTYPE_BF16
+    raise TypeError(f"dW must be float32 or bfloat16, got {dt}")
+
+
+def _grad_scale(grad_scale, device):
+    """The upstream-gradient scalar as a one-element float32 device tensor (or None)."""
+    import torch
+    if grad_scale is None:
+        return None
+    if not isinstance(grad_scale, torch.Tensor):
+        return torch.tensor(float(grad_scale), dtype=torch.float32, device=device)
+    _check_scalar(grad_scale, "grad_scale", torch.float32, device)
+    return grad_scale
+
+
 def _check(X, W, targets):
     import torch
     if not (X.is_cuda and W.is_cuda and targets.is_cuda):
@@ -278,16 +310,20 @@ def alloc_workspace(shape: flce_shape, want_grads: bool, device):
 
 def forward(X, W, targets, Vreal: int, cap: float = 15.0, ignore_index: int = -1,
             want_grads: bool = False, dX=None, dW=None, accumulate_dW: bool = False,
-            workspace=None, chunk_rows: int = 0, stream=None):
+            workspace=None, chunk_rows: int = 0, stream=None, grad_scale=None, dW_dtype=None):
     """Fused forward.  Returns ``(loss [] fp32, lse [N] fp32, dX, dW, workspace)``;
-    dX/dW are None unless ``want_grads``."""
+    dX/dW are None unless ``want_grads``.  With ``want_grads`` the gradients are those of
+    ``grad_scale * loss`` (a float or a one-element float32 device tensor; None = 1), and dW is
+    float32 unless ``dW`` (or ``dW_dtype``) is bfloat16."""
     import torch
     _check(X, W, targets)
     N, d = X.shape
     dev = X.device
+    dw_t, dw_code = _dW_type(dW, dW_dtype)
     if want_grads:
         _check_buffer(dX, "dX", torch.bfloat16, X.shape, dev)
-        _check_buffer(dW, "dW", torch.float32, W.shape, dev)
+        _check_buffer(dW, "dW", dw_t, W.shape, dev)
+        grad_scale = _grad_scale(grad_scale, dev)
     _check_workspace(workspace, dev)
     shape = make_shape(N, d, W.shape[0], Vreal, cap, ignore_index, chunk_rows)
     loss = torch.empty((), dtype=torch.float32, device=dev)
@@ -296,13 +332,13 @@ def forward(X, W, targets, Vreal: int, cap: float = 15.0, ignore_index: int = -1
         if dX is None:
             dX = torch.empty_like(X)
         if dW is None:
-            dW = torch.empty(W.shape, dtype=torch.float32, device=dev)
+            dW = torch.empty(W.shape, dtype=dw_t, device=dev)
     if workspace is None:
         workspace = alloc_workspace(shape, want_grads, dev)
     rc = raw_forward(shape, _ptr(X), _ptr(W), _ptr(targets), _ptr(loss), _ptr(lse),
-                     want_grads, _ptr(dX) if want_grads else None,
-                     _ptr(dW) if want_grads else None, accumulate_dW, _ptr(workspace),
-                     workspace.numel(), _stream(stream))
+                     want_grads, _ptr(grad_scale) if want_grads else None,
+                     _ptr(dX) if want_grads else None, _ptr(dW) if want_grads else None,
+                     dw_code, accumulate_dW, _ptr(workspace), workspace.numel(), _stream(stream))
     if rc != FLCE_OK:
         raise FlceError(rc, "flce_forward")
     return loss, lse, (dX if want_grads else None), (dW if want_grads else None), workspace
@@ -310,7 +346,8 @@ def forward(X, W, targets, Vreal: int, cap: float = 15.0, ignore_index: int = -1
 
 def forward_dp(X, W, targets, n_valid_total, Vreal: int, cap: float = 15.0,
                ignore_index: int = -1, want_grads: bool = True, dX=None, dW=None,
-               accumulate_dW: bool = False, workspace=None, chunk_rows: int = 0, stream=None):
+               accumulate_dW: bool = False, workspace=None, chunk_rows: int = 0, stream=None,
+               grad_scale=None, dW_dtype=None):
     """flce_forward normalised by a device int64 count of rows in the loss over all
     data-parallel ranks.  Returns (loss share, lse, dX, dW, workspace)."""
     import torch
@@ -320,9 +357,11 @@ def forward_dp(X, W, targets, n_valid_total, Vreal: int, cap: float = 15.0,
     if n_valid_total is None:
         raise TypeError("n_valid_total must be a CUDA int64 tensor")
     _check_scalar(n_valid_total, "n_valid_total", torch.int64, dev)
+    dw_t, dw_code = _dW_type(dW, dW_dtype)
     if want_grads:
         _check_buffer(dX, "dX", torch.bfloat16, X.shape, dev)
-        _check_buffer(dW, "dW", torch.float32, W.shape, dev)
+        _check_buffer(dW, "dW", dw_t, W.shape, dev)
+        grad_scale = _grad_scale(grad_scale, dev)
     _check_workspace(workspace, dev)
     shape = make_shape(N, d, W.shape[0], Vreal, cap, ignore_index, chunk_rows)
     loss = torch.empty((), dtype=torch.float32, device=dev)
@@ -331,17 +370,64 @@ def forward_dp(X, W, targets, n_valid_total, Vreal: int, cap: float = 15.0,
         if dX is None:
             dX = torch.empty_like(X)
         if dW is None:
-            dW = torch.empty(W.shape, dtype=torch.float32, device=dev)
+            dW = torch.empty(W.shape, dtype=dw_t, device=dev)
     if workspace is None:
         workspace = alloc_workspace(shape, want_grads, dev)
     rc = lib().flce_forward_dp(ctypes.byref(shape), _ptr(X), _ptr(W), _ptr(targets),
                                _ptr(n_valid_total), _ptr(loss), _ptr(lse),
-                               1 if want_grads else 0, _ptr(dX) if want_grads else None,
-                               _ptr(dW) if want_grads else None, int(accumulate_dW),
+                               1 if want_grads else 0,
+                               _ptr(grad_scale) if want_grads else None,
+                               _ptr(dX) if want_grads else None,
+                               _ptr(dW) if want_grads else None, dw_code, int(accumulate_dW),
                                _ptr(workspace), workspace.numel(), _stream(stream))
     if rc != FLCE_OK:
         raise FlceError(rc, "flce_forward_dp")
     return loss, lse, (dX if want_grads else None), (dW if want_grads else None), workspace
+
+
+def forward_dp_bucketed(X, W, targets, n_valid_total, Vreal: int, cap: float, ignore_index: int,
+                        events, dX=None, dW=None, accumulate_dW: bool = False, workspace=None,
+                        chunk_rows: int = 0, stream=None, grad_scale=None, dW_dtype=None):
+    """forward_dp with gradients whose dW becomes final in len(events) vocabulary buckets:
+    the library records ``events[b]`` (torch.cuda.Event) on the stream once dW rows
+    ``bounds[b]:bounds[b + 1]`` are complete.  Returns (loss share, lse, dX, dW, bounds,
+    workspace)."""
+    import torch
+    _check(X, W, targets)
+    N, d = X.shape
+    dev = X.device
+    if n_valid_total is None:
+        raise TypeError("n_valid_total must be a CUDA int64 tensor")
+    _check_scalar(n_valid_total, "n_valid_total", torch.int64, dev)
+    dw_t, dw_code = _dW_type(dW, dW_dtype)
+    _check_buffer(dX, "dX", torch.bfloat16, X.shape, dev)
+    _check_buffer(dW, "dW", dw_t, W.shape, dev)
+    grad_scale = _grad_scale(grad_scale, dev)
+    _check_workspace(workspace, dev)
+    n = len(events)
+    st = _stream(stream)
+    for ev in events:                       # torch creates the CUDA event on first record
+        if not ev.cuda_event:
+            ev.record(torch.cuda.current_stream(dev) if stream is None else stream)
+    handles = (ctypes.c_void_p * n)(*[ctypes.c_void_p(ev.cuda_event) for ev in events])
+    bounds = (ctypes.c_int64 * (n + 1))()
+    shape = make_shape(N, d, W.shape[0], Vreal, cap, ignore_index, chunk_rows)
+    loss = torch.empty((), dtype=torch.float32, device=dev)
+    lse = torch.empty(max(N, 1), dtype=torch.float32, device=dev)[:N]
+    if dX is None:
+        dX = torch.empty_like(X)
+    if dW is None:
+        dW = torch.empty(W.shape, dtype=dw_t, device=dev)
+    if workspace is None:
+        workspace = alloc_workspace(shape, True, dev)
+    rc = lib().flce_forward_dp_bucketed(ctypes.byref(shape), _ptr(X), _ptr(W), _ptr(targets),
+                                        _ptr(n_valid_total), _ptr(loss), _ptr(lse),
+                                        _ptr(grad_scale), _ptr(dX), _ptr(dW), dw_code,
+                                        int(accumulate_dW), n, handles, bounds, _ptr(workspace),
+                                        workspace.numel(), st)
+    if rc != FLCE_OK:
+        raise FlceError(rc, "flce_forward_dp_bucketed")
+    return loss, lse, dX, dW, [int(b) for b in bounds], workspace
 
 
 def rmsnorm_forward(H, gamma, eps: float = 1e-6, X=None, rstd=None, stream=None):
@@ -414,7 +500,8 @@ def quantize_e4m3(x, out=None, scale=None, stream=None):
 
 def forward_fp8(X8, W8, scale_x, scale_w, X, W, targets, Vreal: int, cap: float = 15.0,
                 ignore_index: int = -1, want_grads: bool = False, dX=None, dW=None,
-                accumulate_dW: bool = False, workspace=None, chunk_rows: int = 0, stream=None):
+                accumulate_dW: bool = False, workspace=None, chunk_rows: int = 0, stream=None,
+                grad_scale=None, dW_dtype=None):
     """Fused forward with e4m3 logits operands (uint8 codes + fp32 device scales) and bf16
     copies X/W for the gradient contractions.  Returns (loss, lse, dX, dW, workspace)."""
     import torch
@@ -435,12 +522,14 @@ def forward_fp8(X8, W8, scale_x, scale_w, X, W, targets, Vreal: int, cap: float 
     if scale_x is None or scale_w is None:
         raise TypeError("scale_x and scale_w must be one-element float32 CUDA tensors")
     _check_buffer(targets, "targets", torch.int64, (N,), dev)
+    dw_t, dw_code = _dW_type(dW, dW_dtype)
     if want_grads:
         _check(X, W, targets)
         _check_buffer(X, "X", torch.bfloat16, (N, d), dev)
         _check_buffer(W, "W", torch.bfloat16, tuple(W8.shape), dev)
         _check_buffer(dX, "dX", torch.bfloat16, (N, d), dev)
-        _check_buffer(dW, "dW", torch.float32, tuple(W8.shape), dev)
+        _check_buffer(dW, "dW", dw_t, tuple(W8.shape), dev)
+        grad_scale = _grad_scale(grad_scale, dev)
     _check_workspace(workspace, dev)
     shape = make_shape(N, d, W8.shape[0], Vreal, cap, ignore_index, chunk_rows)
     loss = torch.empty((), dtype=torch.float32, device=dev)
@@ -449,14 +538,15 @@ def forward_fp8(X8, W8, scale_x, scale_w, X, W, targets, Vreal: int, cap: float 
         if dX is None:
             dX = torch.empty_like(X)
         if dW is None:
-            dW = torch.empty(W.shape, dtype=torch.float32, device=dev)
+            dW = torch.empty(W.shape, dtype=dw_t, device=dev)
     if workspace is None:
         workspace = alloc_workspace(shape, want_grads, dev)
     rc = lib().flce_forward_fp8(ctypes.byref(shape), _ptr(X8), _ptr(W8), _ptr(scale_x),
                                 _ptr(scale_w), _ptr(X), _ptr(W), _ptr(targets), _ptr(loss),
                                 _ptr(lse), 1 if want_grads else 0,
+                                _ptr(grad_scale) if want_grads else None,
                                 _ptr(dX) if want_grads else None,
-                                _ptr(dW) if want_grads else None, int(accumulate_dW),
+                                _ptr(dW) if want_grads else None, dw_code, int(accumulate_dW),
                                 _ptr(workspace), workspace.numel(), _stream(stream))
     if rc != FLCE_OK:
         raise FlceError(rc, "flce_forward_fp8")
@@ -465,27 +555,31 @@ def forward_fp8(X8, W8, scale_x, scale_w, X, W, targets, Vreal: int, cap: float 
 
 def backward(X, W, targets, lse, Vreal: int, cap: float = 15.0, ignore_index: int = -1,
              grad_out=None, dX=None, dW=None, accumulate_dW: bool = False,
-             grads_precomputed: bool = False, workspace=None, chunk_rows: int = 0, stream=None):
-    """Backward.  Returns ``(dX bf16 [N, d], dW fp32 [Vpad, d])``."""
+             grads_precomputed: bool = False, workspace=None, chunk_rows: int = 0, stream=None,
+             dW_dtype=None):
+    """Backward.  Returns ``(dX bf16 [N, d], dW [Vpad, d])``; dW is float32 unless ``dW`` (or
+    ``dW_dtype``) is bfloat16."""
     import torch
     _check(X, W, targets)
     N, d = X.shape
     dev = X.device
+    dw_t, dw_code = _dW_type(dW, dW_dtype)
     _check_buffer(lse, "lse", torch.float32, (N,), dev)
     _check_buffer(dX, "dX", torch.bfloat16, X.shape, dev)
-    _check_buffer(dW, "dW", torch.float32, W.shape, dev)
+    _check_buffer(dW, "dW", dw_t, W.shape, dev)
     _check_scalar(grad_out, "grad_out", torch.float32, dev)
     _check_workspace(workspace, dev)
     shape = make_shape(N, d, W.shape[0], Vreal, cap, ignore_index, chunk_rows)
     if dX is None:
         dX = torch.empty_like(X)
     if dW is None:
-        dW = torch.empty(W.shape, dtype=torch.float32, device=dev)
+        dW = torch.empty(W.shape, dtype=dw_t, device=dev)
     if workspace is None and not grads_precomputed:
         workspace = alloc_workspace(shape, True, dev)
     rc = raw_backward(shape, _ptr(X), _ptr(W), _ptr(targets), _ptr(lse), _ptr(grad_out),
-                      _ptr(dX), _ptr(dW), accumulate_dW, grads_precomputed, _ptr(workspace),
-                      0 if workspace is None else workspace.numel(), _stream(stream))
+                      _ptr(dX), _ptr(dW), dw_code, accumulate_dW, grads_precomputed,
+                      _ptr(workspace), 0 if workspace is None else workspace.numel(),
+                      _stream(stream))
     if rc != FLCE_OK:
         raise FlceError(rc, "flce_backward")
     return dX, dW

@@ -1,46 +1,110 @@
-"""``torch.autograd`` drop-in for the fused linear cross-entropy.
+"""``torch.autograd`` drop-ins for the fused linear cross-entropy and the final RMSNorm.
 
     loss = fused_linear_cross_entropy(hidden, lm_head_weight, targets, Vreal=50257, cap=15.0)
     loss.backward()
 
-When a gradient is needed the forward call already forms dX and dW in the same
-pass over the logits (the gradient of the mean loss); backward only multiplies
-them by the upstream gradient inside the library.  Otherwise the forward keeps
-only the per-row log-sum-exp.
+How the head's gradient is formed depends on what the weight carries:
+
+* plain weight (default): the forward forms dX and dW for g = 1 in the same pass over the
+  logits that gives the loss (dW in the weight's dtype, so bf16 for a bf16 head); backward
+  multiplies both by the upstream gradient g in place and hands them to autograd, which
+  accumulates W.grad across micro-batches in the weight's dtype (bf16 master weights, as the
+  pages train).
+* ``W.main_grad`` (an fp32 tensor of W's shape, the mixed-precision convention): the library
+  adds the gradient into main_grad in fp32 and W.grad is left untouched.  Without a hint the
+  forward keeps only the per-row log-sum-exp and backward recomputes the logits with g known
+  (8 N d Vpad FLOPs instead of 6).
+* ``W.main_grad`` and ``grad_scale=g0``: the forward adds g0 * dW into main_grad in the same
+  pass (6 N d Vpad FLOPs), for a training loop that already knows g (e.g. 1/7 when each of 7
+  micro-batch losses is divided by 7); backward checks on the host that the upstream gradient
+  equals g0 and raises if it does not.
+
+Each backward runs once (``once_differentiable``); a second backward through the same graph
+raises instead of scaling the saved gradients twice.
 """
 from __future__ import annotations
 
 import torch
+from torch.autograd.function import once_differentiable
 
 from . import _abi
 
 
 class FusedLinearCrossEntropy(torch.autograd.Function):
     @staticmethod
-    def forward(ctx, X, W, targets, Vreal, cap, ignore_index, chunk_rows):
+    def forward(ctx, X, W, targets, Vreal, cap, ignore_index, chunk_rows, grad_scale):
         need = ctx.needs_input_grad[0] or ctx.needs_input_grad[1]
-        loss, lse, dX, dW, ws = _abi.forward(X, W, targets, Vreal, cap, ignore_index,
-                                             want_grads=need, chunk_rows=chunk_rows)
+        main_grad = getattr(W, "main_grad", None) if ctx.needs_input_grad[1] else None
         ctx.meta = (Vreal, cap, ignore_index, chunk_rows)
-        if need:
-            ctx.save_for_backward(X, W, targets, lse, dX, dW)
+        ctx.done = False
+        ctx.mode = "none"
+        if not need:
+            loss, _, _, _, _ = _abi.forward(X, W, targets, Vreal, cap, ignore_index,
+                                            chunk_rows=chunk_rows)
+            return loss
+        if main_grad is not None:
+            if main_grad.dtype != torch.float32 or tuple(main_grad.shape) != tuple(W.shape):
+                raise TypeError("W.main_grad must be a float32 tensor of W's shape")
+            if grad_scale is None:
+                # g is not known yet: keep lse, recompute in backward with g
+                loss, lse, _, _, _ = _abi.forward(X, W, targets, Vreal, cap, ignore_index,
+                                                  chunk_rows=chunk_rows)
+                ctx.mode = "recompute"
+                ctx.save_for_backward(X, W, targets, lse)
+                ctx.main_grad = main_grad
+                return loss
+            g0 = torch.tensor(float(grad_scale), dtype=torch.float32, device=X.device)
+            loss, _, dX, _, _ = _abi.forward(X, W, targets, Vreal, cap, ignore_index,
+                                             want_grads=True, dW=main_grad, accumulate_dW=True,
+                                             grad_scale=g0, chunk_rows=chunk_rows)
+            ctx.mode = "hinted"
+            ctx.save_for_backward(dX, g0)
+            return loss
+        dW_dtype = W.dtype if W.dtype in (torch.float32, torch.bfloat16) else torch.float32
+        loss, lse, dX, dW, _ = _abi.forward(X, W, targets, Vreal, cap, ignore_index,
+                                            want_grads=True, chunk_rows=chunk_rows,
+                                            dW_dtype=dW_dtype)
+        ctx.mode = "fused"
+        ctx.save_for_backward(X, W, targets, lse, dX, dW)
         return loss
 
     @staticmethod
+    @once_differentiable
     def backward(ctx, g):
-        X, W, targets, lse, dX, dW = ctx.saved_tensors
+        if ctx.done:
+            raise RuntimeError("fused_linear_cross_entropy: backward already ran for this graph "
+                               "(its gradients were formed in place)")
+        ctx.done = True
         Vreal, cap, ignore_index, chunk_rows = ctx.meta
         g = g.detach().to(torch.float32).contiguous()
-        _abi.backward(X, W, targets, lse, Vreal, cap, ignore_index, grad_out=g, dX=dX, dW=dW,
-                      grads_precomputed=True)
-        return (dX if ctx.needs_input_grad[0] else None,
-                dW if ctx.needs_input_grad[1] else None, None, None, None, None, None)
+        wants = ctx.needs_input_grad
+        if ctx.mode == "fused":
+            X, W, targets, lse, dX, dW = ctx.saved_tensors
+            _abi.backward(X, W, targets, lse, Vreal, cap, ignore_index, grad_out=g, dX=dX, dW=dW,
+                          grads_precomputed=True)
+            return (dX if wants[0] else None, dW if wants[1] else None,
+                    None, None, None, None, None, None)
+        if ctx.mode == "recompute":
+            X, W, targets, lse = ctx.saved_tensors
+            dX, _ = _abi.backward(X, W, targets, lse, Vreal, cap, ignore_index, grad_out=g,
+                                  dW=ctx.main_grad, accumulate_dW=True, chunk_rows=chunk_rows)
+            return (dX if wants[0] else None, None, None, None, None, None, None, None)
+        dX, g0 = ctx.saved_tensors                                   # "hinted"
+        if not torch.equal(g, g0):
+            raise RuntimeError(f"fused_linear_cross_entropy: upstream gradient {g.item()} differs "
+                               f"from grad_scale {g0.item()} already applied to W.main_grad")
+        return (dX if wants[0] else None, None, None, None, None, None, None, None)
 
 
 def fused_linear_cross_entropy(X, W, targets, Vreal: int, cap: float = 15.0,
-                               ignore_index: int = -1, chunk_rows: int = 0):
-    """Mean softcapped cross entropy of ``X W^T`` over rows whose target is not ignore_index."""
-    return FusedLinearCrossEntropy.apply(X, W, targets, Vreal, cap, ignore_index, chunk_rows)
+                               ignore_index: int = -1, chunk_rows: int = 0,
+                               grad_scale: float | None = None):
+    """Mean softcapped cross entropy of ``X W^T`` over rows whose target is not ignore_index.
+
+    ``grad_scale`` only matters when W carries ``main_grad``: it is the upstream gradient the
+    caller will back-propagate (the forward then accumulates into main_grad in the same pass)."""
+    return FusedLinearCrossEntropy.apply(X, W, targets, Vreal, cap, ignore_index, chunk_rows,
+                                         grad_scale)
 
 
 class RMSNorm(torch.autograd.Function):

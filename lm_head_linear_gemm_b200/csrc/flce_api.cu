@@ -73,9 +73,17 @@ namespace {
 #ifndef FLCE_LOGITS_ROUND
 #define FLCE_LOGITS_ROUND 1
 #endif
+// the gradient contractions run over each chunk's rows in the loss only (compacted)
+#ifndef FLCE_COMPACT
+#define FLCE_COMPACT 1
+#endif
 // dX in wide tiles (256 x 512 per SM pair, two accumulators sharing each staged A' k-block)
 #ifndef FLCE_DX_WIDE
 #define FLCE_DX_WIDE 1
+#endif
+// gradient epilogues write (and, accumulating dW, read) whole 32-byte sectors when aligned
+#ifndef FLCE_EPI_SECTOR32
+#define FLCE_EPI_SECTOR32 1
 #endif
 using Cfg = PairCfg<256, FLCE_GRAD_STAGES, FLCE_EPI_WARPS>;
 using CfgL = PairCfg<FLCE_LOGITS_BN, FLCE_LOGITS_STAGES, FLCE_EPI_WARPS, 2, FLCE_LOGITS_KSUB>;
@@ -104,9 +112,11 @@ size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 struct Layout {
   int64_t chunk;      // rows per pass
+  int n_chunks;
   int n_slabs;        // per-row partial slots of the logits pass
   bool fixed_ref;
-  size_t hdr, tgt, s_t, der_t, e_t, row_loss, partial, r, A, Xs, total;
+  bool compact;       // gradients over each chunk's rows in the loss only
+  size_t hdr, tgt, s_t, der_t, e_t, row_loss, partial, r, A, Xs, pos, orig, cnt, bad, total;
 };
 
 bool shape_ok(const flce_shape* s) {
@@ -127,7 +137,9 @@ Layout make_layout(const flce_shape* s, int want_grads) {
   if (nc > N) nc = N;
   if (nc < 1) nc = 1;
   L.chunk = nc;
+  L.n_chunks = static_cast<int>(N > 0 ? (N + nc - 1) / nc : 1);
   L.fixed_ref = s->cap > 0.f && s->cap <= kFixedRefMaxCap;
+  L.compact = want_grads && FLCE_COMPACT;
   const int64_t vtiles = (s->Vpad + CfgL::BN - 1) / CfgL::BN;
   L.n_slabs = static_cast<int>(vtiles * CfgL::COL_SPLIT);
   size_t off = 0;
@@ -148,6 +160,12 @@ Layout make_layout(const flce_shape* s, int want_grads) {
     L.r = take(static_cast<size_t>(nc) * sizeof(float));
     L.A = take(static_cast<size_t>(nc) * s->Vpad * sizeof(__nv_bfloat16));
     L.Xs = take(static_cast<size_t>(nc) * s->d * sizeof(__nv_bfloat16));
+    if (L.compact) {
+      L.pos = take(n * sizeof(int));
+      L.orig = take(n * sizeof(int));
+      L.cnt = take(static_cast<size_t>(L.n_chunks) * sizeof(int));
+      L.bad = take(static_cast<size_t>(L.n_chunks) * sizeof(int));
+    }
   }
   L.total = off;
   return L;
@@ -276,12 +294,13 @@ template <class E0, class E1, class CF = Cfg, class K>
 int launch_pair(K kernel, const DeviceInfo* di, const CUtensorMap& a0, const CUtensorMap& b0,
                 const CUtensorMap& a1, const CUtensorMap& b1, const PairProblem& p0,
                 const PairProblem& p1, uint32_t* status, const typename E0::Params& e0,
-                const typename E1::Params& e1, cudaStream_t st, int kind) {
+                const typename E1::Params& e1, cudaStream_t st, int kind,
+                const int* dyn = nullptr) {
   const long long tiles = pair_tiles<CF>(p0) + pair_tiles<CF>(p1);
   if (tiles <= 0) return FLCE_OK;
   const long long units = di->sms / 2;   // one CTA pair per SM pair, persistent
   const int grid = static_cast<int>(2 * (tiles < units ? tiles : units));
-  PairArgs args{{p0, p1}, status, kWaitLimitNs};
+  PairArgs args{{p0, p1}, status, kWaitLimitNs, dyn};
   cudaEvent_t ev0 = nullptr, ev1 = nullptr;
   const bool timed = g_instr.load(std::memory_order_relaxed) != 0;
   if (timed) {
@@ -305,6 +324,7 @@ int launch_pair(K kernel, const DeviceInfo* di, const CUtensorMap& a0, const CUt
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+bool aligned32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
 
 #define FLCE_TRY(expr)             \
   do {                             \
@@ -330,6 +350,7 @@ struct Ctx {
   const flce_shape* s;
   Fp8Logits fp8;
   const long long* nv_total = nullptr;   // data-parallel normaliser (null: this call's rows)
+  int dW_bf16 = 0;                       // dW element type: 0 fp32, 1 bf16
   Layout L;
   uint8_t* ws;
   DevHeader* hdr;
@@ -381,7 +402,9 @@ int launch_logits(const Ctx& c, int64_t row0, int rows, const __nv_bfloat16* X,
     q.s_t = lp.s_t + r0;
     q.der_t = lp.der_t + r0;
     q.e_t = lp.e_t + r0;
-    q.A = lp.A != nullptr ? lp.A + static_cast<size_t>(r0) * lp.Vpad : nullptr;
+    // compacted rows index A from the chunk's first row: only pos moves with the launch
+    q.pos = lp.pos != nullptr ? lp.pos + r0 : nullptr;
+    q.A = lp.A != nullptr && lp.pos == nullptr ? lp.A + static_cast<size_t>(r0) * lp.Vpad : lp.A;
     FLCE_TRY(launch_logits_rows(c, row0 + r0, rr, X, W, q));
   }
   return FLCE_OK;
@@ -389,9 +412,19 @@ int launch_logits(const Ctx& c, int64_t row0, int rows, const __nv_bfloat16* X,
 
 // One chunk of the gradient path: logits GEMM (mode FUSED or RECOMPUTE), row finish, and the
 // dX / dW contractions in one launch.
+// Vocabulary buckets of a chunk's dW (data-parallel exchange): after the launch that completes
+// bucket b the library records events[b] (when not NULL) on the call's stream and writes the
+// bucket's dW rows [bounds[b], bounds[b + 1]).
+struct Buckets {
+  int n;
+  void* const* events;
+  int64_t* bounds;
+};
+
 int grad_chunk(const Ctx& c, int64_t row0, int rows, const __nv_bfloat16* X,
                const __nv_bfloat16* W, const float* lse_in, float* lse_out, const float* grad_out,
-               __nv_bfloat16* dX, float* dW, int accumulate, int mode) {
+               __nv_bfloat16* dX, void* dW, int accumulate, int mode,
+               const Buckets* buckets = nullptr) {
   const flce_shape* s = c.s;
   const int d = static_cast<int>(s->d), Vpad = static_cast<int>(s->Vpad);
   const __nv_bfloat16* Xc = X + row0 * s->d;
@@ -422,6 +455,9 @@ int grad_chunk(const Ctx& c, int64_t row0, int rows, const __nv_bfloat16* X,
   lp.der_t = c.at<float>(c.L.der_t) + row0;
   lp.e_t = c.at<float>(c.L.e_t) + row0;
   lp.A = Abuf;
+  const int chunk_index = static_cast<int>(row0 / c.L.chunk);
+  const int* cnt = c.L.compact ? c.at<int>(c.L.cnt) + chunk_index : nullptr;
+  lp.pos = c.L.compact ? c.at<int>(c.L.pos) + row0 : nullptr;
   FLCE_TRY(launch_logits(c, row0, rows, X, W, lp));
 
   RowFinishParams rp{};
@@ -448,16 +484,51 @@ int grad_chunk(const Ctx& c, int64_t row0, int rows, const __nv_bfloat16* X,
   rp.A = Abuf;
   rp.X = Xc;
   rp.Xs = Xs;
-  row_finish_kernel<<<(rows + 7) / 8, 256, 0, c.st>>>(rp);
+  __nv_bfloat16* dXc = dX + row0 * s->d;
+  rp.pos = lp.pos;
+  rp.cnt = cnt;
+  rp.dX = dXc;
+  const int finish_warps = rows + (c.L.compact ? 64 : 0);
+  row_finish_kernel<<<(finish_warps + 7) / 8, 256, 0, c.st>>>(rp);
   FLCE_TRY(launch_ok());
 
-  // dX (long tiles: K = Vpad) and dW (short tiles: K = rows) share one balanced launch
-  DxParams xp{rows, d, r, dX + row0 * s->d};
-  DwParams wp{Vpad, d, accumulate, dW};
-  const PairProblem pdx{rows, d, Vpad, 0, FLCE_DX_WIDE, FLCE_L2_DX_A, FLCE_L2_DX_W};
-  const PairProblem pdw{Vpad, d, rows, 0, 0, FLCE_L2_DW_A, FLCE_L2_DW_XS};
-  FLCE_TRY((launch_pair<DxEpi, DwEpi>(kGradKernel, c.di, mA_k, mW_mn, mA_mn, mXs_mn, pdx, pdw,
-                                       &c.hdr->status, xp, wp, c.st, 1)));
+  // dX (long tiles: K = Vpad) and dW (short tiles: K = rows) share one balanced launch; with
+  // compaction both run over the chunk's rows in the loss only (a device-side count: dX's M
+  // and dW's K), dX rows scattered back to their places
+  const int dx32 = FLCE_EPI_SECTOR32 && (d % 16) == 0 && aligned32(dXc);
+  DxParams xp{rows, d, dx32, r, dXc, c.L.compact ? c.at<int>(c.L.orig) + row0 : nullptr, cnt};
+  const int dyn_x = c.L.compact ? DYN_M : 0, dyn_w = c.L.compact ? DYN_K : 0;
+  const PairProblem pdx{rows, d, Vpad, 0, FLCE_DX_WIDE, FLCE_L2_DX_A, FLCE_L2_DX_W, dyn_x};
+  const PairProblem none{0, 0, 0, 0, 0, 0, 0, 0};
+  const int nb = buckets != nullptr ? buckets->n : 1;
+  const int vtiles = (Vpad + Cfg::BM - 1) / Cfg::BM;
+  for (int b = 0; b < nb; ++b) {
+    // Bucket b: the dW rows of vocabulary tiles [b vtiles / nb, (b + 1) vtiles / nb); the dX
+    // tiles ride with the last bucket, so earlier buckets are final (and can be exchanged)
+    // while dX still runs.  One bucket is the plain combined launch.
+    const int v0 = static_cast<int>(static_cast<int64_t>(b) * vtiles / nb) * Cfg::BM;
+    const int v1 = b + 1 == nb ? Vpad
+                               : static_cast<int>(static_cast<int64_t>(b + 1) * vtiles / nb) * Cfg::BM;
+    void* dWb = static_cast<uint8_t*>(dW) +
+                static_cast<size_t>(v0) * s->d * (c.dW_bf16 ? 2 : 4);
+    const int dw32 = FLCE_EPI_SECTOR32 && aligned32(dWb) && (!c.dW_bf16 || (d % 16) == 0);
+    DwParams wp{v1 - v0, d, accumulate, dw32, c.dW_bf16, dWb};
+    const PairProblem pdw{v1 - v0, d, rows, 0, 0, FLCE_L2_DW_A, FLCE_L2_DW_XS, dyn_w};
+    CUtensorMap mA_mn_b = mA_mn;
+    if (v0 > 0) FLCE_TRY(make_map(&mA_mn_b, Abuf + v0, Vpad - v0, rows, Vpad, 64));
+    if (v1 > v0 || b + 1 == nb)
+      FLCE_TRY((launch_pair<DxEpi, DwEpi>(kGradKernel, c.di, mA_k, mW_mn, mA_mn_b, mXs_mn,
+                                           b + 1 == nb ? pdx : none, v1 > v0 ? pdw : none,
+                                           &c.hdr->status, xp, wp, c.st, 1, cnt)));
+    if (buckets != nullptr && buckets->events[b] != nullptr) {
+      if (cudaEventRecord(static_cast<cudaEvent_t>(buckets->events[b]), c.st) != cudaSuccess)
+        return FLCE_ERR_CUDA;
+    }
+    if (buckets != nullptr && buckets->bounds != nullptr) {
+      buckets->bounds[b] = v0;
+      buckets->bounds[b + 1] = v1;
+    }
+  }
   return FLCE_OK;
 }
 
@@ -513,9 +584,29 @@ __global__ void fill_zero_f32_kernel(float* p, long long n) {
     p[i] = 0.f;
 }
 
-int zero_dW(const Ctx& c, float* dW) {
-  const long long n = c.s->Vpad * c.s->d;
-  fill_zero_f32_kernel<<<4 * c.di->sms, 256, 0, c.st>>>(dW, n);
+int zero_dW(const Ctx& c, void* dW) {
+  // fp32: Vpad * d words; bf16: half as many (d is even)
+  const long long n = c.s->Vpad * c.s->d / (c.dW_bf16 ? 2 : 1);
+  fill_zero_f32_kernel<<<4 * c.di->sms, 256, 0, c.st>>>(static_cast<float*>(dW), n);
+  return launch_ok();
+}
+
+// Targets -> effective ids, the count of rows in the loss and the status word; with compaction
+// also each chunk's positions of its rows in the loss (prep_chunks_kernel).
+int prep(const Ctx& c, const int64_t* targets) {
+  const flce_shape* s = c.s;
+  const auto* t = reinterpret_cast<const long long*>(targets);
+  if (!c.L.compact) {
+    prep_targets_kernel<<<1, 1024, 0, c.st>>>(t, s->N, s->Vreal, s->ignore_index,
+                                              c.at<int>(c.L.tgt), c.hdr);
+    return launch_ok();
+  }
+  prep_chunks_kernel<<<c.L.n_chunks, 1024, 0, c.st>>>(
+      t, s->N, c.L.chunk, s->Vreal, s->ignore_index, c.at<int>(c.L.tgt), c.at<int>(c.L.pos),
+      c.at<int>(c.L.orig), c.at<int>(c.L.cnt), c.at<int>(c.L.bad));
+  FLCE_TRY(launch_ok());
+  prep_total_kernel<<<1, 256, 0, c.st>>>(c.at<int>(c.L.cnt), c.at<int>(c.L.bad), c.L.n_chunks,
+                                         c.hdr);
   return launch_ok();
 }
 
@@ -558,15 +649,18 @@ int noalloc_scratch_address(void** out) {
 // Forward (and, with want_grads, the gradients of the mean loss) from bf16 X/W, or from e4m3
 // operands for the logits when fp8.X8 is set (X/W then only feed the gradient contractions).
 int forward_impl(const flce_shape* s, const void* X, const void* W, const Fp8Logits& fp8,
-                 const int64_t* targets, float* loss, float* lse, int want_grads, void* dX,
-                 float* dW, int accumulate_dW, void* workspace, size_t workspace_bytes,
-                 void* stream, const int64_t* nv_total = nullptr) {
+                 const int64_t* targets, float* loss, float* lse, int want_grads,
+                 const float* grad_scale, void* dX, void* dW, int dW_dtype, int accumulate_dW,
+                 void* workspace, size_t workspace_bytes, void* stream,
+                 const int64_t* nv_total = nullptr, const Buckets* buckets = nullptr) {
   want_grads = want_grads ? 1 : 0;
   if (loss == nullptr || (s->N > 0 && lse == nullptr)) return FLCE_ERR_ARG;
   if (!aligned4(loss) || !aligned4(lse)) return FLCE_ERR_ALIGN;
   if (want_grads) {
     if ((s->N > 0 && dX == nullptr) || dW == nullptr) return FLCE_ERR_ARG;
+    if (dW_dtype != FLCE_DTYPE_F32 && dW_dtype != FLCE_DTYPE_BF16) return FLCE_ERR_ARG;
     if (!aligned16(dX) || !aligned16(dW)) return FLCE_ERR_ALIGN;
+    if (grad_scale != nullptr && !aligned4(grad_scale)) return FLCE_ERR_ALIGN;
   }
   DeviceInfo* di = nullptr;
   FLCE_TRY(device_info(&di));
@@ -574,6 +668,7 @@ int forward_impl(const flce_shape* s, const void* X, const void* W, const Fp8Log
   c.s = s;
   c.fp8 = fp8;
   c.nv_total = reinterpret_cast<const long long*>(nv_total);
+  c.dW_bf16 = want_grads && dW_dtype == FLCE_DTYPE_BF16 ? 1 : 0;
   c.L = make_layout(s, want_grads);
   c.ws = static_cast<uint8_t*>(workspace);
   c.di = di;
@@ -582,21 +677,36 @@ int forward_impl(const flce_shape* s, const void* X, const void* W, const Fp8Log
   const auto* Xb = static_cast<const __nv_bfloat16*>(X);
   const auto* Wb = static_cast<const __nv_bfloat16*>(W);
 
-  prep_targets_kernel<<<1, 1024, 0, c.st>>>(reinterpret_cast<const long long*>(targets), s->N,
-                                            s->Vreal, s->ignore_index, c.at<int>(c.L.tgt), c.hdr);
-  FLCE_TRY(launch_ok());
+  FLCE_TRY(prep(c, targets));
   if (s->N == 0) {
     zero_loss_kernel<<<1, 1, 0, c.st>>>(loss);
     FLCE_TRY(launch_ok());
     if (want_grads && !accumulate_dW) FLCE_TRY(zero_dW(c, dW));
+    if (buckets != nullptr) {
+      // nothing to wait for: every bucket is final now
+      for (int b = 0; b < buckets->n; ++b) {
+        if (buckets->events[b] != nullptr &&
+            cudaEventRecord(static_cast<cudaEvent_t>(buckets->events[b]), c.st) != cudaSuccess)
+          return FLCE_ERR_CUDA;
+        if (buckets->bounds != nullptr) {
+          const int vtiles = static_cast<int>((s->Vpad + Cfg::BM - 1) / Cfg::BM);
+          buckets->bounds[b] = static_cast<int64_t>(b) * vtiles / buckets->n * Cfg::BM;
+          buckets->bounds[b + 1] =
+              b + 1 == buckets->n ? s->Vpad
+                                  : static_cast<int64_t>(b + 1) * vtiles / buckets->n * Cfg::BM;
+        }
+      }
+    }
     return FLCE_OK;
   }
   if (want_grads && c.L.fixed_ref) {
     for (int64_t row0 = 0; row0 < s->N; row0 += c.L.chunk) {
       const int rows = static_cast<int>(s->N - row0 < c.L.chunk ? s->N - row0 : c.L.chunk);
-      FLCE_TRY(grad_chunk(c, row0, rows, Xb, Wb, nullptr, lse, nullptr,
+      const bool last = row0 + rows >= s->N;
+      FLCE_TRY(grad_chunk(c, row0, rows, Xb, Wb, nullptr, lse, grad_scale,
                           static_cast<__nv_bfloat16*>(dX), dW,
-                          (row0 > 0 || accumulate_dW) ? 1 : 0, LOGITS_FUSED));
+                          (row0 > 0 || accumulate_dW) ? 1 : 0, LOGITS_FUSED,
+                          last ? buckets : nullptr));
     }
   } else {
     FLCE_TRY(stats_pass(c, Xb, Wb, lse));
@@ -607,9 +717,11 @@ int forward_impl(const flce_shape* s, const void* X, const void* W, const Fp8Log
     // Without a fixed exp reference the gradient needs lse first: recompute with it.
     for (int64_t row0 = 0; row0 < s->N; row0 += c.L.chunk) {
       const int rows = static_cast<int>(s->N - row0 < c.L.chunk ? s->N - row0 : c.L.chunk);
-      FLCE_TRY(grad_chunk(c, row0, rows, Xb, Wb, lse, nullptr, nullptr,
+      const bool last = row0 + rows >= s->N;
+      FLCE_TRY(grad_chunk(c, row0, rows, Xb, Wb, lse, nullptr, grad_scale,
                           static_cast<__nv_bfloat16*>(dX), dW,
-                          (row0 > 0 || accumulate_dW) ? 1 : 0, LOGITS_RECOMPUTE));
+                          (row0 > 0 || accumulate_dW) ? 1 : 0, LOGITS_RECOMPUTE,
+                          last ? buckets : nullptr));
     }
   }
   return FLCE_OK;
@@ -625,11 +737,12 @@ size_t flce_workspace_bytes(const flce_shape* shape, int want_grads) {
 }
 
 int flce_forward(const flce_shape* s, const void* X, const void* W, const int64_t* targets,
-                 float* loss, float* lse, int want_grads, void* dX, float* dW, int accumulate_dW,
-                 void* workspace, size_t workspace_bytes, void* stream) {
+                 float* loss, float* lse, int want_grads, const float* grad_scale, void* dX,
+                 void* dW, int dW_dtype, int accumulate_dW, void* workspace,
+                 size_t workspace_bytes, void* stream) {
   FLCE_TRY(common_checks(s, X, W, targets, workspace, workspace_bytes, want_grads ? 1 : 0));
-  return forward_impl(s, X, W, Fp8Logits{}, targets, loss, lse, want_grads, dX, dW,
-                      accumulate_dW, workspace, workspace_bytes, stream);
+  return forward_impl(s, X, W, Fp8Logits{}, targets, loss, lse, want_grads, grad_scale, dX, dW,
+                      dW_dtype, accumulate_dW, workspace, workspace_bytes, stream);
 }
 
 int flce_count_valid(const flce_shape* s, const int64_t* targets, int64_t* n_valid_out,
@@ -648,19 +761,41 @@ int flce_count_valid(const flce_shape* s, const int64_t* targets, int64_t* n_val
 
 int flce_forward_dp(const flce_shape* s, const void* X, const void* W, const int64_t* targets,
                     const int64_t* n_valid_total, float* loss, float* lse, int want_grads,
-                    void* dX, float* dW, int accumulate_dW, void* workspace,
-                    size_t workspace_bytes, void* stream) {
+                    const float* grad_scale, void* dX, void* dW, int dW_dtype,
+                    int accumulate_dW, void* workspace, size_t workspace_bytes, void* stream) {
   FLCE_TRY(common_checks(s, X, W, targets, workspace, workspace_bytes, want_grads ? 1 : 0));
   if (n_valid_total == nullptr) return FLCE_ERR_ARG;
   if ((reinterpret_cast<uintptr_t>(n_valid_total) & 7u) != 0) return FLCE_ERR_ALIGN;
-  return forward_impl(s, X, W, Fp8Logits{}, targets, loss, lse, want_grads, dX, dW,
-                      accumulate_dW, workspace, workspace_bytes, stream, n_valid_total);
+  return forward_impl(s, X, W, Fp8Logits{}, targets, loss, lse, want_grads, grad_scale, dX, dW,
+                      dW_dtype, accumulate_dW, workspace, workspace_bytes, stream,
+                      n_valid_total);
+}
+
+int flce_forward_dp_bucketed(const flce_shape* s, const void* X, const void* W,
+                             const int64_t* targets, const int64_t* n_valid_total, float* loss,
+                             float* lse, const float* grad_scale, void* dX, void* dW,
+                             int dW_dtype, int accumulate_dW, int n_buckets,
+                             void* const* bucket_events, int64_t* bucket_bounds,
+                             void* workspace, size_t workspace_bytes, void* stream) {
+  FLCE_TRY(common_checks(s, X, W, targets, workspace, workspace_bytes, 1));
+  if (n_valid_total == nullptr || bucket_events == nullptr || bucket_bounds == nullptr)
+    return FLCE_ERR_ARG;
+  if ((reinterpret_cast<uintptr_t>(n_valid_total) & 7u) != 0) return FLCE_ERR_ALIGN;
+  const int64_t vtiles = (s->Vpad + Cfg::BM - 1) / Cfg::BM;
+  if (n_buckets < 1 || n_buckets > 64 || n_buckets > vtiles) return FLCE_ERR_ARG;
+  for (int b = 0; b < n_buckets; ++b)
+    if (bucket_events[b] == nullptr) return FLCE_ERR_ARG;
+  const Buckets bk{n_buckets, bucket_events, bucket_bounds};
+  return forward_impl(s, X, W, Fp8Logits{}, targets, loss, lse, 1, grad_scale, dX, dW,
+                      dW_dtype, accumulate_dW, workspace, workspace_bytes, stream,
+                      n_valid_total, &bk);
 }
 
 int flce_forward_fp8(const flce_shape* s, const void* X8, const void* W8, const float* scale_x,
                      const float* scale_w, const void* X, const void* W, const int64_t* targets,
-                     float* loss, float* lse, int want_grads, void* dX, float* dW,
-                     int accumulate_dW, void* workspace, size_t workspace_bytes, void* stream) {
+                     float* loss, float* lse, int want_grads, const float* grad_scale, void* dX,
+                     void* dW, int dW_dtype, int accumulate_dW, void* workspace,
+                     size_t workspace_bytes, void* stream) {
   if (!shape_ok(s)) return FLCE_ERR_ARG;
   if ((s->d % 16) != 0 || (s->Vpad % 8) != 0) return FLCE_ERR_ALIGN;  // 16-byte e4m3 rows
   if ((s->N > 0 && (X8 == nullptr || targets == nullptr)) || W8 == nullptr ||
@@ -678,8 +813,8 @@ int flce_forward_fp8(const flce_shape* s, const void* X8, const void* W8, const 
   fp8.W8 = static_cast<const uint8_t*>(W8);
   fp8.scale_x = scale_x;
   fp8.scale_w = scale_w;
-  return forward_impl(s, X, W, fp8, targets, loss, lse, want_grads, dX, dW, accumulate_dW,
-                      workspace, workspace_bytes, stream);
+  return forward_impl(s, X, W, fp8, targets, loss, lse, want_grads, grad_scale, dX, dW,
+                      dW_dtype, accumulate_dW, workspace, workspace_bytes, stream);
 }
 
 int flce_quantize_e4m3(const void* src, int64_t n, void* dst, float* scale_out, void* stream) {
@@ -705,21 +840,28 @@ int flce_quantize_e4m3(const void* src, int64_t n, void* dst, float* scale_out, 
 }
 
 int flce_backward(const flce_shape* s, const void* X, const void* W, const int64_t* targets,
-                  const float* lse, const float* grad_out, void* dX, float* dW, int accumulate_dW,
-                  int grads_precomputed, void* workspace, size_t workspace_bytes, void* stream) {
+                  const float* lse, const float* grad_out, void* dX, void* dW, int dW_dtype,
+                  int accumulate_dW, int grads_precomputed, void* workspace,
+                  size_t workspace_bytes, void* stream) {
   if (!shape_ok(s)) return FLCE_ERR_ARG;
   if ((s->N > 0 && dX == nullptr) || dW == nullptr) return FLCE_ERR_ARG;
+  if (dW_dtype != FLCE_DTYPE_F32 && dW_dtype != FLCE_DTYPE_BF16) return FLCE_ERR_ARG;
   if (!aligned16(dX) || !aligned16(dW)) return FLCE_ERR_ALIGN;
   if (grad_out != nullptr && (reinterpret_cast<uintptr_t>(grad_out) & 3u) != 0)
     return FLCE_ERR_ALIGN;
+  const int dW_bf16 = dW_dtype == FLCE_DTYPE_BF16 ? 1 : 0;
   if (grads_precomputed) {
+    // Scaling after the fact is only right for gradients this call's forward wrote; a dW that
+    // holds earlier micro-batches must get g through the forward's grad_scale instead.
+    if (accumulate_dW) return FLCE_ERR_ARG;
     if ((s->d % 8) != 0) return FLCE_ERR_ALIGN;
     DeviceInfo* di = nullptr;
     FLCE_TRY(device_info(&di));
     if (grad_out == nullptr) return FLCE_OK;
-    const long long nX8 = s->N * s->d / 8, nW4 = s->Vpad * s->d / 4;
+    const long long nX8 = s->N * s->d / 8;
+    const long long nW = s->Vpad * s->d / (dW_bf16 ? 8 : 4);
     scale_grads_kernel<<<4 * di->sms, 256, 0, static_cast<cudaStream_t>(stream)>>>(
-        static_cast<__nv_bfloat16*>(dX), nX8, dW, nW4, grad_out);
+        static_cast<__nv_bfloat16*>(dX), nX8, dW, nW, dW_bf16, grad_out);
     return launch_ok();
   }
   FLCE_TRY(common_checks(s, X, W, targets, workspace, workspace_bytes, 1));
@@ -729,14 +871,13 @@ int flce_backward(const flce_shape* s, const void* X, const void* W, const int64
   FLCE_TRY(device_info(&di));
   Ctx c{};
   c.s = s;
+  c.dW_bf16 = dW_bf16;
   c.L = make_layout(s, 1);
   c.ws = static_cast<uint8_t*>(workspace);
   c.di = di;
   c.st = static_cast<cudaStream_t>(stream);
   c.hdr = c.at<DevHeader>(c.L.hdr);
-  prep_targets_kernel<<<1, 1024, 0, c.st>>>(reinterpret_cast<const long long*>(targets), s->N,
-                                            s->Vreal, s->ignore_index, c.at<int>(c.L.tgt), c.hdr);
-  FLCE_TRY(launch_ok());
+  FLCE_TRY(prep(c, targets));
   if (s->N == 0) {
     if (!accumulate_dW) FLCE_TRY(zero_dW(c, dW));
     return FLCE_OK;
@@ -771,8 +912,8 @@ int flce_forward_noalloc(const flce_shape* shape, const void* X, const void* W,
   FLCE_TRY(device_info(&di));
   void* scratch = nullptr;
   FLCE_TRY(noalloc_scratch_address(&scratch));
-  return flce_forward(&s, X, W, targets, loss, lse, 0, nullptr, nullptr, 0, scratch,
-                      FLCE_NOALLOC_SCRATCH_BYTES, stream);
+  return flce_forward(&s, X, W, targets, loss, lse, 0, nullptr, nullptr, nullptr,
+                      FLCE_DTYPE_F32, 0, scratch, FLCE_NOALLOC_SCRATCH_BYTES, stream);
 }
 
 constexpr int kRmsRowsPerPart = 128;
@@ -886,7 +1027,12 @@ int flce_check_pair_schedule(int pairs, int T0, int c0, int T1, int c1, int64_t*
 
 int flce_read_status(const void* workspace, uint32_t* dev_status_out, int64_t* n_valid_out,
                      void* stream) {
-  if (workspace == nullptr) return FLCE_ERR_ARG;
+  if (workspace == nullptr) {
+    // the fixed scratch of flce_forward_noalloc on the current device
+    void* scratch = nullptr;
+    FLCE_TRY(noalloc_scratch_address(&scratch));
+    workspace = scratch;
+  }
   DevHeader h;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (cudaMemcpyAsync(&h, workspace, sizeof(h), cudaMemcpyDeviceToHost, st) != cudaSuccess)

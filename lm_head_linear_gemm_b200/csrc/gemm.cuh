@@ -23,6 +23,16 @@ namespace flce {
 
 enum class Major : int { K = 0, MN = 1 };
 
+// 32 accumulator columns of this thread's TMEM lane, or zeros (warp-uniform `zero`).
+__device__ __forceinline__ void tmem_ld32_or_zero(uint32_t taddr, float (&v)[32], bool zero) {
+  if (zero) {
+#pragma unroll
+    for (int k = 0; k < 32; ++k) v[k] = 0.f;
+  } else {
+    tmem_ld32(taddr, v);
+  }
+}
+
 // ----------------------------------------------------------------------------------------------
 // Tile loaders: K-major -> one TMA box {64 (K), rows}; MN-major -> rows/64 boxes {64 (MN), 64 (K)}.
 // The copy completes on the pair leader's barrier (shared::cluster address).
@@ -119,13 +129,29 @@ struct PairProblem {
   int m_fastest;        // tile order: 1 = consecutive tiles walk M first
   int wide;             // problem 0 only: 1 = wide tiles (see below)
   int l2_a, l2_b;       // L2 priority of the A / B operand reads (l2_policy: 0, 1 first, 2 last)
+  int dyn;              // DYN_M / DYN_K: that extent is min(extent, *PairArgs::dyn)
 };
+
+enum : int { DYN_M = 1, DYN_K = 2 };
 
 struct PairArgs {
   PairProblem prob[2];
   uint32_t* status;     // device status word (DEV_TIMEOUT is or-ed in)
   uint64_t limit_ns;    // bound on every wait
+  const int* dyn;       // device count bounding the extents flagged in PairProblem::dyn
 };
+
+// Extents of a problem after the device-side bound (a count formed by an earlier kernel of the
+// same stream, e.g. a chunk's number of rows in the loss).
+struct Extents {
+  int M, N, K;
+};
+__device__ __forceinline__ Extents extents_of(const PairProblem& p, int dynv) {
+  Extents e{p.M, p.N, p.K};
+  if (p.dyn & DYN_M) e.M = dynv < e.M ? dynv : e.M;
+  if (p.dyn & DYN_K) e.K = dynv < e.K ? dynv : e.K;
+  return e;
+}
 
 // Pair `pair` of `P` takes n0 tiles of problem 0 (pair, pair + P, ...).  Problem 0 has
 // a = T0 / P tiles per pair plus one more on the first T0 % P pairs ("heavy" pairs).  Problem 1
@@ -201,12 +227,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
   const int pair = static_cast<int>(cluster_id_x());
   const int npairs = static_cast<int>(num_clusters_x());
 
-  const int m_tiles0 = (args.prob[0].M + C::BM - 1) / C::BM;
-  const int n_tiles0 = (args.prob[0].N + C::BN - 1) / C::BN;
-  const int nkb0 = (args.prob[0].K + C::KSLOT - 1) / C::KSLOT;   // ring slots per tile
-  const int m_tiles1 = (args.prob[1].M + C::BM - 1) / C::BM;
-  const int n_tiles1 = (args.prob[1].N + C::BN - 1) / C::BN;
-  const int nkb1 = (args.prob[1].K + C::KSLOT - 1) / C::KSLOT;
+  // extents (the device-side bound was written by an earlier kernel of this stream)
+  const int dynv = args.dyn != nullptr ? *args.dyn : 0x7fffffff;
+  const Extents ex0 = extents_of(args.prob[0], dynv);
+  const Extents ex1 = extents_of(args.prob[1], dynv);
+  const int m_tiles0 = (ex0.M + C::BM - 1) / C::BM;
+  const int n_tiles0 = (ex0.N + C::BN - 1) / C::BN;
+  const int nkb0 = (ex0.K + C::KSLOT - 1) / C::KSLOT;   // ring slots per tile
+  const int m_tiles1 = (ex1.M + C::BM - 1) / C::BM;
+  const int n_tiles1 = (ex1.N + C::BN - 1) / C::BN;
+  const int nkb1 = (ex1.K + C::KSLOT - 1) / C::KSLOT;
   // Wide tiles (problem 0, bf16): two adjacent BN-column blocks share every staged k-block of
   // A, one TMEM accumulator each, so a pair stages 256 + 512 operand rows per k-block instead
   // of 2 x (256 + 256).  The second B block goes into the next ring slot (its A area unused),
@@ -230,7 +260,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
     *abort_flag = 0;
     const PairSchedule mine = pair_schedule(pair, npairs, m_tiles0 * w_tiles0,
                                             wide0 ? 2 * nkb0 : nkb0,
-                                            args.prob[1].M > 0 ? m_tiles1 * n_tiles1 : 0,
+                                            ex1.M > 0 ? m_tiles1 * n_tiles1 : 0,
                                             nkb1 > 0 ? nkb1 : 1);
     sched[0] = mine.n0;
     sched[1] = mine.qa;
@@ -243,7 +273,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA0);
     tma_prefetch_desc(&tmB0);
-    if (args.prob[1].M > 0) {
+    if (ex1.M > 0) {
       tma_prefetch_desc(&tmA1);
       tma_prefetch_desc(&tmB1);
     }
@@ -548,10 +578,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
           const int nbs = nb * NSUB + sub;
           const int row = mb * C::BM + static_cast<int>(rank) * C::BM_CTA + row_in_cta;
           const int col0 = nbs * C::BN + slab * C::COLS_PER_WARP;
+          // a tile with no k-blocks (a device-bounded K of 0) contributes a zero tile
+          const bool zero = kbs == 0;
           if (prob == 0)
-            E0::template apply<C::COLS_PER_WARP>(ep0, row, col0, taddr, nbs * C::COL_SPLIT + slab);
+            E0::template apply<C::COLS_PER_WARP>(ep0, row, col0, taddr, nbs * C::COL_SPLIT + slab,
+                                                 zero);
           else
-            E1::template apply<C::COLS_PER_WARP>(ep1, row, col0, taddr, nbs * C::COL_SPLIT + slab);
+            E1::template apply<C::COLS_PER_WARP>(ep1, row, col0, taddr, nbs * C::COL_SPLIT + slab,
+                                                 zero);
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive_cluster(leader_tempty + 8u * acc);
@@ -636,6 +670,7 @@ struct LogitsParams {
   float* der_t;              // [rows] 1 - tanh^2 at the target
   float* e_t;                // [rows] exp(s_t - reference)
   __nv_bfloat16* A;          // [rows][Vpad] gradient operand (modes FUSED / RECOMPUTE)
+  const int* pos;            // [rows] row of A for each row (-1: not written), or null: same row
 };
 
 struct LogitsEpi {
@@ -644,7 +679,7 @@ struct LogitsEpi {
 
   template <int NCOLS>
   __device__ static __forceinline__ void apply(const Params& p, int row, int col0, uint32_t taddr,
-                                               int slab_index) {
+                                               int slab_index, bool zero) {
     const bool row_ok = row < p.rows;
     const int t = row_ok ? __ldg(p.tgt + row) : -1;
     const bool capped = p.cap > 0.f;
@@ -660,11 +695,15 @@ struct LogitsEpi {
     float run_max = -INFINITY;
     float tv_s = 0.f, tv_der = 0.f, tv_e = 0.f;
     bool has_t = false;
-    __nv_bfloat16* arow = write_a && row_ok ? p.A + static_cast<size_t>(row) * p.Vpad : nullptr;
+    __nv_bfloat16* arow = nullptr;
+    if (write_a && row_ok) {
+      const int at = p.pos != nullptr ? __ldg(p.pos + row) : row;
+      if (at >= 0) arow = p.A + static_cast<size_t>(at) * p.Vpad;
+    }
 #pragma unroll 1
     for (int c = 0; c < NCOLS / 32; ++c) {
       float v[32];
-      tmem_ld32(taddr + c * 32, v);
+      tmem_ld32_or_zero(taddr + c * 32, v, zero);
       const int cbase = col0 + c * 32;
       if (p.fixed_ref) {
         // softcap with the fixed reference: e = exp(s - cap), A = e (1 - tanh^2)
@@ -796,34 +835,50 @@ struct LogitsEpi {
 // Epilogue 2: dX rows = r_i * (A' W)_i, stored as bf16.
 struct DxParams {
   int rows, d;
+  int sector32;              // 1: dX rows and base are 32-byte aligned (full-sector stores)
   const float* r;            // [rows] row scale g/(Nv S_i); 0 for rows not in the loss
   __nv_bfloat16* dX;         // [rows][d]
+  const int* orig;           // compacted rows: dX row of each (null: same row)
+  const int* dyn_rows;       // compacted rows: their device-side count (null: rows)
 };
 
 struct DxEpi {
   using Params = DxParams;
   template <int NCOLS>
   __device__ static __forceinline__ void apply(const Params& p, int row, int col0, uint32_t taddr,
-                                               int) {
-    const bool row_ok = row < p.rows;
+                                               int, bool zero) {
+    const int rows = p.dyn_rows != nullptr ? __ldg(p.dyn_rows) : p.rows;
+    const bool row_ok = row < rows;
     const float sc = row_ok ? __ldg(p.r + row) : 0.f;
-    __nv_bfloat16* out = row_ok ? p.dX + static_cast<size_t>(row) * p.d : nullptr;
+    const int out_row = row_ok && p.orig != nullptr ? __ldg(p.orig + row) : row;
+    __nv_bfloat16* out = row_ok ? p.dX + static_cast<size_t>(out_row) * p.d : nullptr;
 #pragma unroll 1
     for (int c = 0; c < NCOLS / 32; ++c) {
       float v[32];
-      tmem_ld32(taddr + c * 32, v);
+      tmem_ld32_or_zero(taddr + c * 32, v, zero);
       if (out == nullptr) continue;
       const int cbase = col0 + c * 32;
+      uint32_t w[16];
 #pragma unroll
-      for (int g = 0; g < 4; ++g) {
-        const int col = cbase + 8 * g;
-        if (col < p.d) {
-          uint4 w;
-          w.x = pack_bf16x2(v[8 * g + 0] * sc, v[8 * g + 1] * sc);
-          w.y = pack_bf16x2(v[8 * g + 2] * sc, v[8 * g + 3] * sc);
-          w.z = pack_bf16x2(v[8 * g + 4] * sc, v[8 * g + 5] * sc);
-          w.w = pack_bf16x2(v[8 * g + 6] * sc, v[8 * g + 7] * sc);
-          *reinterpret_cast<uint4*>(out + col) = w;
+      for (int k = 0; k < 16; ++k) w[k] = pack_bf16x2(v[2 * k] * sc, v[2 * k + 1] * sc);
+      if (p.sector32) {
+        // two full 32-byte sectors per 32 columns
+#pragma unroll
+        for (int g = 0; g < 2; ++g) {
+          const int col = cbase + 16 * g;
+          if (col < p.d) {
+            const uint32_t q[8] = {w[8 * g],     w[8 * g + 1], w[8 * g + 2], w[8 * g + 3],
+                                   w[8 * g + 4], w[8 * g + 5], w[8 * g + 6], w[8 * g + 7]};
+            st_global_v8(out + col, q);
+          }
+        }
+      } else {
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          const int col = cbase + 8 * g;
+          if (col < p.d)
+            *reinterpret_cast<uint4*>(out + col) =
+                make_uint4(w[4 * g], w[4 * g + 1], w[4 * g + 2], w[4 * g + 3]);
         }
       }
     }
@@ -831,40 +886,124 @@ struct DxEpi {
 };
 
 // ==============================================================================================
-// Epilogue 3: dW rows (vocabulary rows) = (A'^T (r . X))_j, written or accumulated in fp32.
+// Epilogue 3: dW rows (vocabulary rows) = (A'^T (r . X))_j, written or accumulated, in fp32 or in
+// bf16 (bf16: the tile is added to the stored values in fp32 and rounded once).
 struct DwParams {
   int Vpad, d;
   int accumulate;            // 1: dW += tile, 0: dW = tile
-  float* dW;                 // [Vpad][d]
+  int sector32;              // 1: dW rows and base are 32-byte aligned (full-sector accesses)
+  int bf16;                  // 1: dW is bf16, 0: fp32
+  void* dW;                  // [Vpad][d]
 };
 
 struct DwEpi {
   using Params = DwParams;
+
+  // 16 bf16 values <-> 8 packed words
+  __device__ static __forceinline__ void add_bf16x16(float* v, const uint32_t (&o)[8]) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&o[k]));
+      v[2 * k] += f.x;
+      v[2 * k + 1] += f.y;
+    }
+  }
+
   template <int NCOLS>
   __device__ static __forceinline__ void apply(const Params& p, int row, int col0, uint32_t taddr,
-                                               int) {
+                                               int, bool zero) {
     const bool row_ok = row < p.Vpad;
-    float* out = row_ok ? p.dW + static_cast<size_t>(row) * p.d : nullptr;
+    float* out = row_ok ? static_cast<float*>(p.dW) + static_cast<size_t>(row) * p.d : nullptr;
+    __nv_bfloat16* out16 =
+        row_ok ? static_cast<__nv_bfloat16*>(p.dW) + static_cast<size_t>(row) * p.d : nullptr;
 #pragma unroll 1
     for (int c = 0; c < NCOLS / 32; ++c) {
       float v[32];
-      tmem_ld32(taddr + c * 32, v);
-      if (out == nullptr) continue;
+      tmem_ld32_or_zero(taddr + c * 32, v, zero);
+      if (!row_ok) continue;
       const int cbase = col0 + c * 32;
+      if (p.bf16) {
+        if (p.sector32) {
+          // two full 32-byte sectors (16 bf16 each) per 32 columns; d % 16 == 0
 #pragma unroll
-      for (int g = 0; g < 8; ++g) {
-        const int col = cbase + 4 * g;
-        if (col < p.d) {
-          float4* dst = reinterpret_cast<float4*>(out + col);
-          float4 w = make_float4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
-          if (p.accumulate) {
-            const float4 o = *dst;
-            w.x += o.x;
-            w.y += o.y;
-            w.z += o.z;
-            w.w += o.w;
+          for (int g = 0; g < 2; ++g) {
+            const int col = cbase + 16 * g;
+            if (col < p.d) {
+              __nv_bfloat16* dst = out16 + col;
+              if (p.accumulate) {
+                float f[8];
+                ld_global_v8f(reinterpret_cast<const float*>(dst), f);
+                uint32_t o[8];
+#pragma unroll
+                for (int k = 0; k < 8; ++k) o[k] = __float_as_uint(f[k]);
+                add_bf16x16(v + 16 * g, o);
+              }
+              uint32_t q[8];
+#pragma unroll
+              for (int k = 0; k < 8; ++k) q[k] = pack_bf16x2(v[16 * g + 2 * k], v[16 * g + 2 * k + 1]);
+              st_global_v8(dst, q);
+            }
           }
-          *dst = w;
+        } else {
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            const int col = cbase + 8 * g;
+            if (col < p.d) {
+              uint4* dst = reinterpret_cast<uint4*>(out16 + col);
+              if (p.accumulate) {
+                const uint4 raw = *dst;
+                const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                  const float2 f = __bfloat1622float2(h[k]);
+                  v[8 * g + 2 * k] += f.x;
+                  v[8 * g + 2 * k + 1] += f.y;
+                }
+              }
+              *dst = make_uint4(pack_bf16x2(v[8 * g], v[8 * g + 1]),
+                                pack_bf16x2(v[8 * g + 2], v[8 * g + 3]),
+                                pack_bf16x2(v[8 * g + 4], v[8 * g + 5]),
+                                pack_bf16x2(v[8 * g + 6], v[8 * g + 7]));
+            }
+          }
+        }
+      } else if (p.sector32) {
+        // whole 32-byte sectors: a partly written sector never reaches the L2 on its own
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          const int col = cbase + 8 * g;
+          if (col < p.d) {
+            float* dst = out + col;
+            if (p.accumulate) {
+              float o[8];
+              ld_global_v8f(dst, o);
+#pragma unroll
+              for (int k = 0; k < 8; ++k) v[8 * g + k] += o[k];
+            }
+            const uint32_t q[8] = {
+                __float_as_uint(v[8 * g]),     __float_as_uint(v[8 * g + 1]),
+                __float_as_uint(v[8 * g + 2]), __float_as_uint(v[8 * g + 3]),
+                __float_as_uint(v[8 * g + 4]), __float_as_uint(v[8 * g + 5]),
+                __float_as_uint(v[8 * g + 6]), __float_as_uint(v[8 * g + 7])};
+            st_global_v8(dst, q);
+          }
+        }
+      } else {
+#pragma unroll
+        for (int g = 0; g < 8; ++g) {
+          const int col = cbase + 4 * g;
+          if (col < p.d) {
+            float4* dst = reinterpret_cast<float4*>(out + col);
+            float4 w = make_float4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
+            if (p.accumulate) {
+              const float4 o = *dst;
+              w.x += o.x;
+              w.y += o.y;
+              w.z += o.z;
+              w.w += o.w;
+            }
+            *dst = w;
+          }
         }
       }
     }

@@ -51,6 +51,99 @@ __global__ void __launch_bounds__(1024) prep_targets_kernel(const long long* __r
   }
 }
 
+// Per chunk of Nc rows (one block each): effective targets, and the compaction of the rows in the
+// loss that the gradient contractions run over.  pos[i] is row i's position among its chunk's
+// rows in the loss (-1 when ignored or invalid), orig[c*Nc + q] the chunk-local index of the
+// chunk's q-th row in the loss, cnt[c] their number and bad[c] whether the chunk holds a target
+// outside [0, Vreal) that is not ignore_index.  Rows keep their order (a stable partition).
+__global__ void __launch_bounds__(1024) prep_chunks_kernel(const long long* __restrict__ targets,
+                                                           long long N, long long Nc,
+                                                           long long Vreal, long long ignore_index,
+                                                           int* __restrict__ tgt,
+                                                           int* __restrict__ pos,
+                                                           int* __restrict__ orig,
+                                                           int* __restrict__ cnt,
+                                                           int* __restrict__ bad) {
+  __shared__ int s_scan[32];
+  __shared__ int s_base;
+  __shared__ int s_bad;
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  const long long c0 = static_cast<long long>(blockIdx.x) * Nc;
+  const long long c1 = c0 + Nc < N ? c0 + Nc : N;
+  if (threadIdx.x == 0) {
+    s_base = 0;
+    s_bad = 0;
+  }
+  __syncthreads();
+  for (long long b = c0; b < c1; b += blockDim.x) {
+    const long long i = b + threadIdx.x;
+    int ok = 0;
+    if (i < c1) {
+      const long long t = targets[i];
+      const bool ignored = t == ignore_index;
+      ok = (t >= 0 && t < Vreal && !ignored) ? 1 : 0;
+      if (!ok && !ignored) s_bad = 1;
+      tgt[i] = ok ? static_cast<int>(t) : -1;
+    }
+    const unsigned m = __ballot_sync(0xffffffffu, ok);
+    if (lane == 0) s_scan[w] = __popc(m);
+    __syncthreads();
+    if (w == 0) {
+      int v = lane < nw ? s_scan[lane] : 0;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += u;
+      }
+      s_scan[lane] = v;                                  // inclusive over warps
+    }
+    __syncthreads();
+    const int base = s_base;
+    const int total = s_scan[nw - 1];
+    const int p = base + (w > 0 ? s_scan[w - 1] : 0) + __popc(m & ((1u << lane) - 1u));
+    if (i < c1) {
+      pos[i] = ok ? p : -1;
+      if (ok) orig[c0 + p] = static_cast<int>(i - c0);
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) s_base = base + total;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    cnt[blockIdx.x] = s_base;
+    bad[blockIdx.x] = s_bad;
+  }
+}
+
+// One block: rows in the loss and the bad-target bit over all chunks (fixed order).  Resets the
+// status word for this call.
+__global__ void __launch_bounds__(256) prep_total_kernel(const int* __restrict__ cnt,
+                                                         const int* __restrict__ bad, int n_chunks,
+                                                         DevHeader* __restrict__ hdr) {
+  __shared__ long long s_n[256];
+  __shared__ int s_b[256];
+  long long n = 0;
+  int b = 0;
+  for (int c = threadIdx.x; c < n_chunks; c += blockDim.x) {
+    n += cnt[c];
+    b |= bad[c];
+  }
+  s_n[threadIdx.x] = n;
+  s_b[threadIdx.x] = b;
+  __syncthreads();
+  for (int k = blockDim.x >> 1; k > 0; k >>= 1) {
+    if (static_cast<int>(threadIdx.x) < k) {
+      s_n[threadIdx.x] += s_n[threadIdx.x + k];
+      s_b[threadIdx.x] |= s_b[threadIdx.x + k];
+    }
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    hdr->n_valid = s_n[0];
+    hdr->status = s_b[0] ? DEV_BAD_TARGET : 0u;
+  }
+}
+
 struct RowFinishParams {
   int rows;                     // rows of this pass
   int d, Vpad;
@@ -74,13 +167,34 @@ struct RowFinishParams {
   __nv_bfloat16* A;             // [rows][Vpad]
   const __nv_bfloat16* X;       // [rows][d]
   __nv_bfloat16* Xs;            // [rows][d]
+  // Compaction (want_grads with pos != null): r, Xs and the rows of A are indexed by the row's
+  // position among the chunk's rows in the loss; rows not in the loss get a zero dX row here
+  // (the dX contraction skips them), and 64 extra warps zero the rows [cnt, cnt rounded up to
+  // 64) of A and Xs so that the dW contraction's last k-block adds nothing.
+  const int* pos;               // [rows] position or -1
+  const int* cnt;               // this chunk's number of rows in the loss
+  __nv_bfloat16* dX;            // [rows][d] this chunk's dX rows
 };
 
-// One warp per row.
+__device__ __forceinline__ void zero_row_bf16(__nv_bfloat16* row, int n, int lane) {
+  for (int k = lane * 8; k < n; k += 256) *reinterpret_cast<uint4*>(row + k) = make_uint4(0, 0, 0, 0);
+}
+
+// One warp per row (plus, when compacting, 64 warps that clear the tail rows).
 __global__ void __launch_bounds__(256) row_finish_kernel(const RowFinishParams p) {
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
-  if (warp >= p.rows) return;
+  if (warp >= p.rows) {
+    if (p.want_grads && p.pos != nullptr && warp < p.rows + 64) {
+      const int m = *p.cnt;
+      const int q = m + (warp - p.rows);
+      if (q < ((m + 63) & ~63) && q < p.rows) {
+        zero_row_bf16(p.A + static_cast<size_t>(q) * p.Vpad, p.Vpad, lane);
+        zero_row_bf16(p.Xs + static_cast<size_t>(q) * p.d, p.d, lane);
+      }
+    }
+    return;
+  }
   const int row = warp;
   float lse, S = 1.f, ref;
   if (p.from_partials) {
@@ -125,15 +239,23 @@ __global__ void __launch_bounds__(256) row_finish_kernel(const RowFinishParams p
   const long long nv = p.nv_total != nullptr ? *p.nv_total : p.hdr->n_valid;
   const float g = p.grad_out ? *p.grad_out : 1.f;
   const float r = (valid && nv > 0) ? g / (static_cast<float>(nv) * S) : 0.f;
+  int at = row;                                   // row of r, A and Xs
+  if (p.pos != nullptr) {
+    if (!valid) {                                 // not in the loss: dX row is zero
+      zero_row_bf16(p.dX + static_cast<size_t>(row) * p.d, p.d, lane);
+      return;
+    }
+    at = p.pos[row];
+  }
   if (lane == 0) {
-    p.r[row] = r;
+    p.r[at] = r;
     if (valid) {
       const float patched = p.der_t[row] * (p.e_t[row] - S);
-      p.A[static_cast<size_t>(row) * p.Vpad + t] = __float2bfloat16_rn(patched);
+      p.A[static_cast<size_t>(at) * p.Vpad + t] = __float2bfloat16_rn(patched);
     }
   }
   const __nv_bfloat16* xr = p.X + static_cast<size_t>(row) * p.d;
-  __nv_bfloat16* xs = p.Xs + static_cast<size_t>(row) * p.d;
+  __nv_bfloat16* xs = p.Xs + static_cast<size_t>(at) * p.d;
   for (int k = lane * 8; k < p.d; k += 256) {
     const uint4 raw = *reinterpret_cast<const uint4*>(xr + k);
     const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
@@ -169,33 +291,40 @@ __global__ void __launch_bounds__(1024) loss_kernel(const float* __restrict__ ro
   }
 }
 
-// dX *= g, dW *= g for gradients formed with g = 1; returns at once when g == 1.
+// dX *= g, dW *= g for gradients formed with g = 1; returns at once when g == 1.  dW is fp32
+// (nW = elements / 4, float4 groups) or bf16 (dW_bf16 = 1, nW = elements / 8, groups of 8).
 __global__ void scale_grads_kernel(__nv_bfloat16* __restrict__ dX, long long nX8,
-                                   float* __restrict__ dW, long long nW4,
+                                   void* __restrict__ dW, long long nW, int dW_bf16,
                                    const float* __restrict__ grad_out) {
   const float g = *grad_out;
   if (g == 1.f) return;
   const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
-  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < nX8;
-       i += stride) {
-    uint4 raw = reinterpret_cast<uint4*>(dX)[i];
+  auto scale_bf16x8 = [g](uint4* p) {
+    uint4 raw = *p;
     __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&raw);
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       const float2 f = __bfloat1622float2(h[q]);
       h[q] = __floats2bfloat162_rn(f.x * g, f.y * g);
     }
-    reinterpret_cast<uint4*>(dX)[i] = raw;
-  }
+    *p = raw;
+  };
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < nX8;
+       i += stride)
+    scale_bf16x8(reinterpret_cast<uint4*>(dX) + i);
   if (dW != nullptr) {
-    for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < nW4;
+    for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < nW;
          i += stride) {
-      float4 v = reinterpret_cast<float4*>(dW)[i];
-      v.x *= g;
-      v.y *= g;
-      v.z *= g;
-      v.w *= g;
-      reinterpret_cast<float4*>(dW)[i] = v;
+      if (dW_bf16) {
+        scale_bf16x8(reinterpret_cast<uint4*>(dW) + i);
+      } else {
+        float4 v = reinterpret_cast<float4*>(dW)[i];
+        v.x *= g;
+        v.y *= g;
+        v.z *= g;
+        v.w *= g;
+        reinterpret_cast<float4*>(dW)[i] = v;
+      }
     }
   }
 }

@@ -259,6 +259,15 @@ __device__ __forceinline__ void st_global_v8(void* dst, const uint32_t (&w)[8]) 
                : "memory");
 }
 
+// 32-byte global load of eight fp32 values (one full sector); src must be 32-byte aligned.
+__device__ __forceinline__ void ld_global_v8f(const float* src, float (&v)[8]) {
+  asm volatile("ld.global.v8.f32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+               : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]), "=f"(v[4]), "=f"(v[5]),
+                 "=f"(v[6]), "=f"(v[7])
+               : "l"(src)
+               : "memory");
+}
+
 // The same copy with an L2 cache policy (createpolicy) for the bytes it reads.
 __device__ __forceinline__ void tma_load_2d_pair_hint(void* smem_dst, const CUtensorMap* map,
                                                       uint32_t leader_bar, int32_t x, int32_t y,

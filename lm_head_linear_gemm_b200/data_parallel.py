@@ -11,9 +11,16 @@ rows:
      share of the mean loss, dX for its rows, its contribution to dW;
   4. all-reduce (sum) of the loss shares and of dW.
 
-With gradient accumulation over micro-batches (``accumulate_dW``) the dW all-reduce is needed
-only once per optimizer step; ``allreduce_dW=False`` skips it for the intermediate
-micro-batches (as DDP's no_sync does).
+With ``buckets > 1`` step 4's dW all-reduce overlaps step 3: the library completes dW in
+vocabulary buckets (``flce_forward_dp_bucketed``, the last chunk's gradient contractions run
+bucket by bucket, dX with the last one) and records a CUDA event per bucket; each bucket is
+all-reduced on a communication stream as soon as its event fires, while the remaining buckets
+and dX are still being computed.  DDP overlaps its bucketed gradient all-reduce with the
+backward pass in the same way.
+
+With gradient accumulation over micro-batches (``accumulate_dW``, ``grad_scale`` = 1/m for m
+micro-batches) the dW all-reduce is needed only once per optimizer step; ``allreduce_dW=False``
+skips it for the intermediate micro-batches (as DDP's no_sync does).
 """
 from __future__ import annotations
 
@@ -22,6 +29,9 @@ from . import _abi
 
 class LibraryOps:
     """Device work of a step, all in libflce kernels."""
+
+    def __init__(self):
+        self._comm = {}
 
     def count_valid(self, targets, Vreal, ignore_index):
         import torch
@@ -36,26 +46,62 @@ class LibraryOps:
         return out
 
     def forward(self, X, W, targets, n_valid_total, Vreal, cap, ignore_index, dW,
-                accumulate_dW, workspace, chunk_rows):
+                accumulate_dW, workspace, chunk_rows, grad_scale=None):
         return _abi.forward_dp(X, W, targets, n_valid_total, Vreal, cap, ignore_index, True,
                                dW=dW, accumulate_dW=accumulate_dW, workspace=workspace,
-                               chunk_rows=chunk_rows)
+                               chunk_rows=chunk_rows, grad_scale=grad_scale)
+
+    def forward_buckets(self, X, W, targets, n_valid_total, Vreal, cap, ignore_index, dW,
+                        accumulate_dW, workspace, chunk_rows, n_buckets, grad_scale=None):
+        """The forward with dW completed in vocabulary buckets.  Returns (loss, lse, dX, dW,
+        [(row slice of dW, CUDA event that marks it final), ...])."""
+        import torch
+        events = [torch.cuda.Event() for _ in range(n_buckets)]
+        loss, lse, dX, dW, bounds, _ = _abi.forward_dp_bucketed(
+            X, W, targets, n_valid_total, Vreal, cap, ignore_index, events, dW=dW,
+            accumulate_dW=accumulate_dW, workspace=workspace, chunk_rows=chunk_rows,
+            grad_scale=grad_scale)
+        return loss, lse, dX, dW, [(slice(bounds[b], bounds[b + 1]), events[b])
+                                   for b in range(n_buckets)]
+
+    def allreduce_async(self, t, ready, group):
+        """All-reduce ``t`` on this device's communication stream once ``ready`` has fired."""
+        import torch
+        import torch.distributed as dist
+        comm = self._comm.get(t.device)
+        if comm is None:
+            comm = self._comm[t.device] = torch.cuda.Stream(device=t.device)
+        comm.wait_event(ready)
+        with torch.cuda.stream(comm):
+            return dist.all_reduce(t, group=group, async_op=True)
 
 
 def dp_step(X, W, targets, Vreal: int, cap: float = 15.0, ignore_index: int = -1, *,
             group=None, dW=None, accumulate_dW: bool = False, allreduce_dW: bool = True,
-            workspace=None, chunk_rows: int = 0, ops=None):
+            workspace=None, chunk_rows: int = 0, ops=None, grad_scale=None, buckets: int = 1):
     """One data-parallel fused step.  Returns ``(loss, lse, dX, dW, n_valid_total)`` where loss
     is the mean over all ranks' rows in the loss and dW is summed over ranks (when
-    ``allreduce_dW``)."""
+    ``allreduce_dW``).  ``buckets > 1`` overlaps the dW all-reduce with the step's last
+    gradient contractions (same result)."""
     import torch.distributed as dist
     ops = ops or LibraryOps()
+    distributed = dist.is_initialized()
     nv = ops.count_valid(targets, Vreal, ignore_index)
-    if dist.is_initialized():
+    if distributed:
         dist.all_reduce(nv, group=group)
+    if distributed and allreduce_dW and buckets > 1:
+        loss, lse, dX, dW, pieces = ops.forward_buckets(X, W, targets, nv, Vreal, cap,
+                                                        ignore_index, dW, accumulate_dW,
+                                                        workspace, chunk_rows, buckets,
+                                                        grad_scale)
+        works = [ops.allreduce_async(dW[sl], ready, group) for sl, ready in pieces]
+        dist.all_reduce(loss, group=group)
+        for w in works:
+            w.wait()
+        return loss, lse, dX, dW, nv
     loss, lse, dX, dW, _ = ops.forward(X, W, targets, nv, Vreal, cap, ignore_index, dW,
-                                      accumulate_dW, workspace, chunk_rows)
-    if dist.is_initialized():
+                                       accumulate_dW, workspace, chunk_rows, grad_scale)
+    if distributed:
         dist.all_reduce(loss, group=group)
         if allreduce_dW:
             dist.all_reduce(dW, group=group)

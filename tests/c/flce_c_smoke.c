@@ -79,8 +79,10 @@ int main(void) {
   CHECK_CUDA(cudaMemcpy(W, hW, sizeof(uint16_t) * Vpad * d, cudaMemcpyHostToDevice));
   CHECK_CUDA(cudaMemcpy(t, ht, sizeof(int64_t) * N, cudaMemcpyHostToDevice));
 
-  CHECK_FLCE(flce_forward(&s, X, W, t, loss, lse, 1, dX, dW, 0, ws, ws_bytes, NULL));
-  CHECK_FLCE(flce_forward(&s, X, W, t, loss + 1, lse, 0, NULL, NULL, 0, ws, ws_bytes, NULL));
+  CHECK_FLCE(flce_forward(&s, X, W, t, loss, lse, 1, NULL, dX, dW, FLCE_DTYPE_F32, 0, ws,
+                          ws_bytes, NULL));
+  CHECK_FLCE(flce_forward(&s, X, W, t, loss + 1, lse, 0, NULL, NULL, NULL, FLCE_DTYPE_F32, 0, ws,
+                          ws_bytes, NULL));
   uint32_t status = 0;
   int64_t n_valid = 0;
   CHECK_FLCE(flce_read_status(ws, &status, &n_valid, NULL));

@@ -26,7 +26,8 @@ def test_exports_every_declared_symbol(L):
                           "flce_read_status", "flce_status_string", "flce_instrument",
                           "flce_instrument_read", "flce_forward_noalloc", "flce_forward_fp8",
                           "flce_quantize_e4m3", "flce_selftest_wait_timeout",
-                          "flce_count_valid", "flce_forward_dp", "flce_rmsnorm_forward",
+                          "flce_count_valid", "flce_forward_dp", "flce_forward_dp_bucketed",
+                          "flce_rmsnorm_forward",
                           "flce_rmsnorm_workspace_bytes", "flce_rmsnorm_backward",
                           "flce_check_pair_schedule"}
     for n in names:
@@ -82,8 +83,9 @@ def test_host_rejects_bad_arguments_before_launch(L):
     def fwd(**over):
         a = dict(args)
         a.update(over)
-        return flce.raw_forward(s, a["X"], a["W"], a["t"], a["loss"], a["lse"], 1, a["dX"],
-                                a["dW"], 0, a["ws"], over.get("ws_bytes", ws), None)
+        return flce.raw_forward(s, a["X"], a["W"], a["t"], a["loss"], a["lse"], 1,
+                                over.get("g"), a["dX"], a["dW"], over.get("dtype", 0), 0,
+                                a["ws"], over.get("ws_bytes", ws), None)
 
     assert fwd(X=None) == -1
     assert fwd(t=None) == -1
@@ -92,12 +94,19 @@ def test_host_rejects_bad_arguments_before_launch(L):
     assert fwd(X=good + 2) == -2
     assert fwd(ws=good + 16) == -2                 # workspace must be 256-byte aligned
     assert fwd(ws_bytes=ws - 1) == -3
+    assert fwd(dtype=2) == -1                      # dW element type other than fp32 / bf16
+    assert fwd(g=good + 2) == -2                   # grad_scale not 4-byte aligned
     bad_d = flce.make_shape(8, 60, 128, 100)
-    assert flce.raw_forward(bad_d, good, good, good, good, good, 0, None, None, 0, good, 1 << 30,
-                            None) == -2
-    assert flce.raw_backward(s, good, good, good, None, None, good, good, 0, 0, good, ws,
+    assert flce.raw_forward(bad_d, good, good, good, good, good, 0, None, None, None, 0, 0, good,
+                            1 << 30, None) == -2
+    assert flce.raw_backward(s, good, good, good, None, None, good, good, 0, 0, 0, good, ws,
                              None) == -1       # lse missing on the recompute path
-    assert flce.raw_backward(s, good, good, good, good, None, None, good, 0, 0, good, ws,
+    assert flce.raw_backward(s, good, good, good, good, None, None, good, 0, 0, 0, good, ws,
+                             None) == -1
+    assert flce.raw_backward(s, good, good, good, good, None, good, good, 3, 0, 0, good, ws,
+                             None) == -1       # bad dW element type
+    # an accumulated dW cannot be scaled after the fact: g belongs in the forward's grad_scale
+    assert flce.raw_backward(s, good, good, good, good, good, good, good, 0, 1, 1, None, 0,
                              None) == -1
 
 
@@ -151,21 +160,46 @@ def test_fp8_dp_and_count_entry_points_reject_bad_arguments_before_launch(L):
     ws = flce.workspace_bytes(s, True)
     sp = ctypes.byref(s)
     f8 = L.flce_forward_fp8
-    # X8, W8, sx, sw, X, W, t, loss, lse, want_grads, dX, dW, acc, ws, ws_bytes, stream
-    assert f8(sp, p, p, None, p, p, p, p, p, p, 1, p, p, 0, p, ws, None) == -1    # scale_x
-    assert f8(sp, p, p, p, p, None, p, p, p, p, 1, p, p, 0, p, ws, None) == -1    # X for grads
-    assert f8(sp, p, p, p + 2, p, p, p, p, p, p, 1, p, p, 0, p, ws, None) == -2   # scale align
-    assert f8(sp, p + 8, p, p, p, p, p, p, p, p, 1, p, p, 0, p, ws, None) == -2   # X8 align
-    assert f8(sp, p, p, p, p, p, p, p, p, p, 1, p, p, 0, p, ws - 1, None) == -3
+    # X8, W8, sx, sw, X, W, t, loss, lse, want_grads, g, dX, dW, dW_dtype, acc, ws, ws_bytes,
+    # stream
+    assert f8(sp, p, p, None, p, p, p, p, p, p, 1, None, p, p, 0, 0, p, ws, None) == -1  # sx
+    assert f8(sp, p, p, p, p, None, p, p, p, p, 1, None, p, p, 0, 0, p, ws, None) == -1  # X
+    assert f8(sp, p, p, p + 2, p, p, p, p, p, p, 1, None, p, p, 0, 0, p, ws, None) == -2
+    assert f8(sp, p + 8, p, p, p, p, p, p, p, p, 1, None, p, p, 0, 0, p, ws, None) == -2
+    assert f8(sp, p, p, p, p, p, p, p, p, p, 1, None, p, p, 0, 0, p, ws - 1, None) == -3
     s48 = flce.make_shape(8, 72, 128, 100)          # d % 16 != 0: e4m3 rows not 16-byte
-    assert f8(ctypes.byref(s48), p, p, p, p, p, p, p, p, p, 0, None, None, 0, p, 1 << 30,
-              None) == -2
+    assert f8(ctypes.byref(s48), p, p, p, p, p, p, p, p, p, 0, None, None, None, 0, 0, p,
+              1 << 30, None) == -2
     dp = L.flce_forward_dp
-    # X, W, t, nv_total, loss, lse, want_grads, dX, dW, acc, ws, ws_bytes, stream
-    assert dp(sp, p, p, p, None, p, p, 1, p, p, 0, p, ws, None) == -1             # count
-    assert dp(sp, p, p, p, p + 4, p, p, 1, p, p, 0, p, ws, None) == -2            # 8-byte
+    # X, W, t, nv_total, loss, lse, want_grads, g, dX, dW, dW_dtype, acc, ws, ws_bytes, stream
+    assert dp(sp, p, p, p, None, p, p, 1, None, p, p, 0, 0, p, ws, None) == -1    # count
+    assert dp(sp, p, p, p, p + 4, p, p, 1, None, p, p, 0, 0, p, ws, None) == -2   # 8-byte
     cv = L.flce_count_valid
     assert cv(sp, p, None, None) == -1
     assert cv(sp, p, p + 4, None) == -2
     bad = flce.make_shape(8, 64, 128, 200)          # Vreal > Vpad
     assert cv(ctypes.byref(bad), p, p, None) == -1
+
+
+def test_bucketed_entry_point_rejects_bad_arguments_before_launch(L):
+    p = 0x10000000      # never dereferenced: argument checks come first
+    s = flce.make_shape(8, 64, 1024, 1000)          # 4 vocabulary tiles of 256 rows
+    ws = flce.workspace_bytes(s, True)
+    f = L.flce_forward_dp_bucketed
+    P = ctypes.c_void_p
+
+    def call(n, events, bounds=True, nv=p):
+        ev = (P * max(n, 1))(*([p] * max(n, 1))) if events else None
+        bd = (ctypes.c_int64 * (max(n, 1) + 1))() if bounds else None
+        return f(ctypes.byref(s), p, p, p, nv, p, p, None, p, p, 0, 0, n, ev, bd, p, ws, None)
+
+    assert call(0, True) == -1                       # at least one bucket
+    assert call(5, True) == -1                       # more buckets than vocabulary tiles
+    assert call(2, False) == -1                      # events missing
+    assert call(2, True, bounds=False) == -1         # bounds missing
+    assert call(2, True, nv=None) == -1              # global count missing
+    assert call(2, True, nv=p + 4) == -2             # count not 8-byte aligned
+    null_event = (P * 2)(p, None)
+    bd = (ctypes.c_int64 * 3)()
+    assert f(ctypes.byref(s), p, p, p, p, p, p, None, p, p, 0, 0, 2, null_event, bd, p, ws,
+             None) == -1

@@ -46,7 +46,7 @@ def inputs():
 
 @pytest.mark.parametrize("dX,dW,err", [
     (Buf((N, D), torch.float32), None, TypeError),            # dX must be bf16
-    (None, Buf((V, D), torch.bfloat16), TypeError),           # dW must be fp32
+    (None, Buf((V, D), torch.float16), TypeError),            # dW must be fp32 or bf16
     (None, Buf((V - 8, D), torch.float32), ValueError),       # dW rows must be Vpad
     (Buf((N, D + 8), torch.bfloat16), None, ValueError),      # dX shape
     (None, Buf((V, D), torch.float32, contiguous=False), ValueError),

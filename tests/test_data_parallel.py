@@ -1,10 +1,12 @@
 """The data-parallel exchange (dp_step) on world_size-2 gloo ranks on the CPU.
 
 The device work is stood in for by the fp64 oracle (test-side only: ``OracleOps`` implements
-the contract of flce_count_valid / flce_forward_dp); what is under test is the exchange:
-counts all-reduced before the forward, loss shares and dW all-reduced after it.  The two-rank
-result must equal a single oracle call on the union of both ranks' rows, also when the split
-is uneven and when one rank has no row in the loss.
+the contract of flce_count_valid / flce_forward_dp / flce_forward_dp_bucketed); what is under
+test is the exchange: counts all-reduced before the forward, loss shares and dW all-reduced
+after it, in one piece or in vocabulary buckets issued as asynchronous all-reduces.  The
+two-rank result must equal a single oracle call on the union of both ranks' rows, also when the
+split is uneven, when one rank has no row in the loss, and over two accumulated micro-batches
+with the upstream gradient 1/2 passed to the forward.
 """
 import os
 import socket
@@ -26,18 +28,32 @@ class OracleOps:
         return torch.tensor([int(valid.sum())], dtype=torch.int64)
 
     def forward(self, X, W, targets, n_valid_total, Vreal, cap, ignore_index, dW, accumulate_dW,
-                workspace, chunk_rows):
+                workspace, chunk_rows, grad_scale=None):
         Xn, Wn, t = X.numpy(), W.numpy(), targets.numpy()
         nt = int(n_valid_total.item())
         f = oracle.forward(Xn, Wn, t, Vreal, cap, ignore_index)
         nl = f["n_valid"]
-        g = nl / nt if nt else 0.0
-        dX, dWl = oracle.backward(Xn, Wn, t, Vreal, cap, ignore_index, g=g, lse=f["lse"])
-        loss = torch.tensor(f["loss"] * g, dtype=torch.float64)
+        share = nl / nt if nt else 0.0
+        gs = 1.0 if grad_scale is None else float(grad_scale)
+        dX, dWl = oracle.backward(Xn, Wn, t, Vreal, cap, ignore_index, g=share * gs,
+                                  lse=f["lse"])
+        loss = torch.tensor(f["loss"] * share, dtype=torch.float64)
         dWt = torch.from_numpy(dWl)
         if dW is not None and accumulate_dW:
             dWt = dW + dWt
         return loss, torch.from_numpy(f["lse"]), torch.from_numpy(dX), dWt, None
+
+    def forward_buckets(self, X, W, targets, n_valid_total, Vreal, cap, ignore_index, dW,
+                        accumulate_dW, workspace, chunk_rows, n_buckets, grad_scale=None):
+        loss, lse, dX, dWt, _ = self.forward(X, W, targets, n_valid_total, Vreal, cap,
+                                             ignore_index, dW, accumulate_dW, workspace,
+                                             chunk_rows, grad_scale)
+        edges = np.linspace(0, dWt.shape[0], n_buckets + 1).astype(int)
+        return loss, lse, dX, dWt, [(slice(edges[b], edges[b + 1]), None)
+                                    for b in range(n_buckets)]
+
+    def allreduce_async(self, t, ready, group):
+        return dist.all_reduce(t, group=group, async_op=True)
 
 
 def _data(seed=0, N=30):
@@ -49,7 +65,7 @@ def _data(seed=0, N=30):
     return X, W, t
 
 
-def _worker(rank, world, port, split, all_ignored_rank, q):
+def _worker(rank, world, port, split, all_ignored_rank, buckets, micro, q):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
@@ -61,8 +77,26 @@ def _worker(rank, world, port, split, all_ignored_rank, q):
             t[lo:hi] = -1
         Xr = torch.from_numpy(X[lo:hi].copy())
         tr = torch.from_numpy(t[lo:hi].copy())
-        loss, lse, dX, dW, nv = dp_step(Xr, torch.from_numpy(W), tr, VR, CAP, -1, ops=OracleOps())
-        q.put((rank, float(loss), dX.numpy(), dW.numpy(), int(nv.item()), t))
+        Wt = torch.from_numpy(W)
+        if micro == 1:
+            loss, lse, dX, dW, nv = dp_step(Xr, Wt, tr, VR, CAP, -1, ops=OracleOps(),
+                                            buckets=buckets)
+        else:
+            # the same rows as `micro` micro-batches (halves of this rank's rows), dW
+            # accumulated with grad_scale 1/micro and all-reduced after the last one
+            cut = [lo + (hi - lo) * k // micro for k in range(micro + 1)]
+            dW, dXs, losses = None, [], []
+            for k in range(micro):
+                a, b = cut[k] - lo, cut[k + 1] - lo
+                loss, lse, dXk, dW, nv = dp_step(Xr[a:b], Wt, tr[a:b], VR, CAP, -1,
+                                                 ops=OracleOps(), dW=dW, accumulate_dW=k > 0,
+                                                 allreduce_dW=k == micro - 1,
+                                                 grad_scale=1.0 / micro, buckets=buckets)
+                dXs.append(dXk)
+                losses.append(float(loss))
+            dX = torch.cat(dXs)
+            loss = losses
+        q.put((rank, loss, dX.numpy(), dW.numpy(), int(nv.item()), t))
     finally:
         dist.destroy_process_group()
 
@@ -75,12 +109,12 @@ def _free_port():
     return p
 
 
-@pytest.mark.parametrize("split,all_ignored_rank", [(15, -1), (7, -1), (20, 1)])
-def test_two_rank_exchange_equals_union_batch(split, all_ignored_rank):
+def _run(split, all_ignored_rank, buckets, micro):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_worker, args=(r, 2, port, split, all_ignored_rank, q))
+    procs = [ctx.Process(target=_worker,
+                         args=(r, 2, port, split, all_ignored_rank, buckets, micro, q))
              for r in range(2)]
     for p in procs:
         p.start()
@@ -91,6 +125,14 @@ def test_two_rank_exchange_equals_union_batch(split, all_ignored_rank):
     for p in procs:
         p.join(timeout=60)
         assert p.exitcode == 0
+    return res
+
+
+@pytest.mark.parametrize("split,all_ignored_rank,buckets", [(15, -1, 1), (7, -1, 1),
+                                                            (20, 1, 1), (15, -1, 4),
+                                                            (20, 1, 3)])
+def test_two_rank_exchange_equals_union_batch(split, all_ignored_rank, buckets):
+    res = _run(split, all_ignored_rank, buckets, 1)
     X, W, t = _data()
     t = t.copy()
     if all_ignored_rank == 0:
@@ -104,3 +146,25 @@ def test_two_rank_exchange_equals_union_batch(split, all_ignored_rank):
         assert res[r][4] == ref["n_valid"]
     dX = np.concatenate([res[0][2], res[1][2]])
     np.testing.assert_allclose(dX, ref["dX"], atol=1e-14)
+
+
+@pytest.mark.parametrize("buckets", [1, 4])
+def test_two_rank_accumulation_over_micro_batches(buckets):
+    """Each rank's rows as two micro-batches with grad_scale 1/2 and dW accumulated; dW is
+    all-reduced after the second.  The micro-batch means are over the global count of each
+    micro-batch, so the accumulated dW equals the mean of the two micro-batch oracle gradients
+    on the union of the ranks' rows of that micro-batch."""
+    split = 14
+    res = _run(split, -1, buckets, 2)
+    X, W, t = _data()
+    N = X.shape[0]
+    halves = [np.r_[0:7, split:split + (N - split) // 2],
+              np.r_[7:split, split + (N - split) // 2:N]]
+    ref_dW = np.zeros_like(W)
+    for k, rows in enumerate(halves):
+        f = oracle.forward_backward(X[rows], W, t[rows], VR, CAP, -1, g=0.5)
+        ref_dW += f["dW"]
+        for r in (0, 1):
+            assert abs(res[r][1][k] - f["loss"]) < 1e-12
+    for r in (0, 1):
+        np.testing.assert_allclose(res[r][3], ref_dW, atol=1e-14)

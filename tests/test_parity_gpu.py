@@ -172,8 +172,8 @@ def test_softcap_variants(cuda_device, cap, w_std):
 
 @pytest.mark.parametrize("w_std,cap", [(2.0, 15.0), (0.05, 15.0), (1.0, 2.0)])
 def test_softcap_math_tight(cuda_device, w_std, cap):
-    """The epilogue's tanh / exp evaluation (one special-function exp2, a Newton reciprocal and
-    a polynomial exp2) against fp64 with a tolerance 10x tighter than the parity bar: with
+    """The epilogue's tanh / exp evaluation (two special-function exp2 and one special-function
+    reciprocal per logit) against fp64 with a tolerance 10x tighter than the parity bar: with
     w_std = 2 the logits reach |z| ~ 80, far into the softcap's saturation; w_std = 0.05 keeps
     them near 0 where tanh is almost linear."""
     c = synth.custom_config("tight", N=256, d=128, Vreal=1000, Vpad=1024, x_dist="normal",
@@ -258,6 +258,27 @@ def test_accumulate_and_upstream_gradient(cuda_device):
                              accumulate_dW=True, chunk_rows=128)
     check_tensor("dX g=2", dX3.double().cpu().numpy(), 2 * ref["dX"])
     check_tensor("dW g=2 acc", (dW3 - R).double().cpu().numpy(), 2 * ref["dW"])
+
+
+def test_compaction_across_chunks(cuda_device):
+    """The gradient contractions run over each chunk's rows in the loss only.  Chunks of 256
+    rows: the first keeps 192 rows (a whole number of 64-row k-blocks), the second none (its dW
+    contribution is a zero tile added to the first chunk's), the last 88 of 88 (ragged).  Every
+    element against the oracle, fused and recomputing; ignored rows have zero dX."""
+    inp = synth.make_inputs(synth.custom_config("compact", N=600, d=200, Vreal=1500, Vpad=1544,
+                                                x_dist="normal", w_std=0.05,
+                                                target_dist="uniform", ignore_count=0))
+    t = inp["targets"].copy()
+    rng = np.random.default_rng(5)
+    t[rng.permutation(256)[:64]] = -1
+    t[256:512] = -1
+    inp = dict(inp, targets=t)
+    ref = oracle_full(inp)
+    assert ref["n_valid"] == 192 + 88
+    for recompute in (False, True):
+        got = run_gpu(inp, chunk_rows=256, recompute=recompute)
+        compare_full(got, ref)
+        assert np.abs(got["dX"][t == -1]).max() == 0.0
 
 
 def test_deterministic(cuda_device):
