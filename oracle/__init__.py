@@ -24,7 +24,10 @@ inputs (the GPU path reads the same bf16 values):
   ``dz = g/Nv * (softmax(s) - onehot(t)) * (1 - tanh^2(z/cap))``.
 * FP8 variant (the write-ups train with FP8 GEMMs under dynamic tensorwise scaling,
   "Increasing throughput"): the logits come from the e4m3 operands times their scales while
-  the two gradient products use the bf16 copies -- ``backward(..., Xg=, Wg=)``.
+  the two gradient products use the bf16 copies -- ``backward(..., Xg=, Wg=)``; or, with FP8
+  gradient products too (the write-ups' "three GEMMs in FP8": one forward, two backward),
+  ``backward_fp8`` -- the softmax gradient is encoded in e5m2 and multiplied with the e4m3
+  operands.
 
 The fused method (the lm_head matmul computed chunk by chunk inside the loss so
 the ``(B*T, vocab)`` logits are never materialised -- "Increasing throughput",
@@ -48,7 +51,8 @@ import numpy as np
 __all__ = [
     "logits", "softcap", "softcap_derivative", "valid_rows", "row_forward", "forward",
     "row_dlogits", "backward", "forward_backward", "dW_rows", "rmsnorm_forward",
-    "rmsnorm_backward",
+    "rmsnorm_backward", "round_bf16", "encode_e5m2", "E5M2_SCALE", "dlogits_e5m2",
+    "backward_fp8",
 ]
 
 
@@ -226,3 +230,87 @@ def rmsnorm_backward(H, gamma, dX, eps: float = 1e-6):
     g = dX * gamma[None, :]
     dH = rstd[:, None] * (g - xh * np.mean(g * xh, axis=1, keepdims=True))
     return dH, np.sum(dX * xh, axis=0)
+
+
+# ------------------------------------------------------------------------ FP8 gradient products
+# The write-ups run all three GEMMs of a linear layer in FP8 with dynamic tensorwise scaling
+# ("Increasing throughput": one forward and two backward GEMMs).  Reading adopted for the head
+# (the pages give no format for the gradient): the logits operands are e4m3 (as above), the
+# softmax gradient is e5m2 -- the format with the wider exponent range, needed because the
+# softmax probabilities of one row span many binades -- and the two gradient products multiply
+# it with the same e4m3 operands.  The gradient is normalised before it is encoded:
+#   dz_ij = g/Nv * dzn_ij,   dzn_ij = (softmax(s_i)_j - [j = t_i]) (1 - tanh^2(z_ij / cap)),
+# and |dzn| <= 1, so a fixed power-of-two scale 2^15 (below the e5m2 maximum 57344) covers its
+# range without an amax pass; the factor g/(Nv 2^15) and the operands' tensorwise scales are
+# applied to the products' fp32 results.  dzn is formed as A_ij / S_i from the unnormalised
+# operand A_ij = exp(s_ij - cap)(1 - tanh^2) -- rounded to bf16 -- with S_i = sum_j exp(s_ij -
+# cap) and the target element A_{i,t_i} = (1 - tanh^2)(exp(s_{i,t_i} - cap) - S_i), rounded to
+# bf16 as well (the reference cap is what keeps exp(s - cap) <= 1 before the row sum is known).
+
+E5M2_SCALE = float(2 ** 15)
+
+
+def round_bf16(a):
+    """Round float64 values to the nearest bfloat16 (ties to even), returned as float64."""
+    import torch
+    return torch.from_numpy(np.asarray(a, np.float64)).to(torch.bfloat16).to(torch.float64).numpy()
+
+
+def encode_e5m2(a):
+    """Round float64 values to the nearest e5m2 value (ties to even); |a| <= 57344 here."""
+    import torch
+    return (torch.from_numpy(np.asarray(a, np.float64)).to(torch.float32)
+            .to(torch.float8_e5m2).to(torch.float64).numpy())
+
+
+def dlogits_e5m2(X, W, t, Vreal: int, cap: float, ignore_index: int, round_operand: bool = True,
+                 encode: bool = True):
+    """The e5m2 codes (as values, times 2^15) of the normalised softmax gradient dzn of a
+    block of rows; rows not in the loss and padded columns are 0.  ``round_operand`` /
+    ``encode`` switch the bf16 rounding of A and the e5m2 encoding off (exact dzn * 2^15)."""
+    if not cap > 0:
+        raise ValueError("the FP8 gradient path takes the reference exp(s - cap): cap > 0")
+    z = logits(X, W)
+    Vpad = z.shape[1]
+    s = softcap(z, cap)
+    der = softcap_derivative(z, cap)
+    e = np.exp(s - cap)
+    e[:, Vreal:] = 0.0
+    S = e.sum(axis=1)
+    A = e * der
+    valid, _ = valid_rows(t, Vreal, ignore_index)
+    rows = np.nonzero(valid)[0]
+    tt = np.asarray(t, np.int64)[rows]
+    A[rows, tt] = der[rows, tt] * (e[rows, tt] - S[rows])
+    if round_operand:
+        A = round_bf16(A)
+    q = A / S[:, None] * E5M2_SCALE
+    if encode:
+        q = encode_e5m2(q)
+    q[~valid] = 0.0
+    assert q.shape[1] == Vpad
+    return q
+
+
+def backward_fp8(Xq, Wq, t, Vreal: int, cap: float, ignore_index: int, g: float = 1.0,
+                 block_rows: int = 1024, round_operand: bool = True, encode: bool = True):
+    """Gradients of ``g * loss`` with FP8 gradient products: dX = g/(Nv 2^15) q Wq and
+    dW = g/(Nv 2^15) q^T Xq, q = dlogits_e5m2(...), with Xq / Wq the (dequantised) e4m3
+    operands of the logits.  With round_operand = encode = False this is ``backward`` on
+    (Xq, Wq)."""
+    Xq = np.asarray(Xq, np.float64)
+    Wq = np.asarray(Wq, np.float64)
+    valid, _ = valid_rows(t, Vreal, ignore_index)
+    nv = int(np.count_nonzero(valid))
+    dX = np.zeros_like(Xq)
+    dW = np.zeros_like(Wq)
+    if nv == 0:
+        return dX, dW
+    f = g / (nv * E5M2_SCALE)
+    for r0 in range(0, Xq.shape[0], block_rows):
+        r1 = min(Xq.shape[0], r0 + block_rows)
+        q = dlogits_e5m2(Xq[r0:r1], Wq, t[r0:r1], Vreal, cap, ignore_index, round_operand,
+                         encode)
+        dX[r0:r1] = f * (q @ Wq)
+        dW += f * (q.T @ Xq[r0:r1])
+    return dX, dW

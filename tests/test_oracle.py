@@ -456,3 +456,74 @@ def test_against_torch_on_random_shapes():
         assert not f["dW"][Vr:].any()
 
     check()
+
+
+# ------------------------------------------------------------------------ FP8 gradient products
+def test_e5m2_and_bf16_rounding_of_known_values():
+    """e5m2: 1 sign, 5 exponent, 2 mantissa bits (bias 15): 1, 1.25, 1.5, 1.75 times powers of
+    two are exact; midpoints go to the even mantissa; 2^-16 is the smallest subnormal; 57344 is
+    the largest finite value.  bf16 keeps 8 significant bits, ties to even."""
+    exact = np.array([1.0, 1.25, 1.5, 1.75, 2.0 ** -14, 2.0 ** -16, 3 * 2.0 ** -16, 2.0 ** 15,
+                      57344.0, -1.75 * 2.0 ** -3])
+    np.testing.assert_array_equal(oracle.encode_e5m2(exact), exact)
+    ties = np.array([1.125, 1.375, 1.625, 1.875, 2.5 * 2.0 ** -16])
+    np.testing.assert_array_equal(oracle.encode_e5m2(ties), [1.0, 1.5, 1.5, 2.0, 2.0 ** -15])
+    near = np.array([1.126, 1.374, 0.3])
+    np.testing.assert_array_equal(oracle.encode_e5m2(near), [1.25, 1.25, 0.3125])
+    b = np.array([1.0, 1 + 2.0 ** -8, 1 + 2.0 ** -9, 1 + 3 * 2.0 ** -9, 1 + 2.0 ** -7])
+    np.testing.assert_array_equal(oracle.round_bf16(b), [1.0, 1.0, 1.0, 1 + 2.0 ** -7,
+                                                         1 + 2.0 ** -7])
+    # 1 + 2^-8 is the tie between 1 and 1 + 2^-7: even (1); 1 + 3*2^-9 rounds up
+
+
+def _fp8_case(seed=0, N=40, d=24, Vr=60, Vp=64, w_std=0.6, cap=15.0):
+    rng = np.random.default_rng(seed)
+    X = rng.standard_normal((N, d))
+    W = rng.standard_normal((Vp, d)) * w_std
+    t = rng.integers(0, Vr, N)
+    t[[3, 17]] = -1
+    t[9] = Vr + 2                                # invalid: treated as ignored
+    return X, W, t, Vr, cap
+
+
+@pytest.mark.parametrize("cap,g", [(15.0, 1.0), (2.0, 0.25), (30.0, 3.0)])
+def test_fp8_gradients_without_rounding_are_the_exact_gradients(cap, g):
+    """With the bf16 rounding of A and the e5m2 encoding switched off, the FP8 path's algebra
+    (A / S * 2^15 with the target patch, scaled by g/(Nv 2^15)) must give ``backward``."""
+    X, W, t, Vr, _ = _fp8_case(cap=cap)
+    dX, dW = oracle.backward_fp8(X, W, t, Vr, cap, -1, g=g, round_operand=False, encode=False)
+    rX, rW = oracle.backward(X, W, t, Vr, cap, -1, g=g)
+    np.testing.assert_allclose(dX, rX, rtol=0, atol=1e-12 * np.abs(rX).max())
+    np.testing.assert_allclose(dW, rW, rtol=0, atol=1e-12 * np.abs(rW).max())
+    assert np.abs(dW[Vr:]).max() == 0.0
+
+
+def test_fp8_gradient_codes_are_e5m2_of_the_normalised_gradient():
+    """Each code is the nearest e5m2 value of dzn * 2^15 (|dzn| <= 1): relative error at most
+    2^-3 for normals (two mantissa bits), and some codes do come close to that bound (e4m3, with
+    three mantissa bits, would stay within 2^-4).  Rows not in the loss are zero."""
+    X, W, t, Vr, cap = _fp8_case(N=200, seed=3)
+    exact = oracle.dlogits_e5m2(X, W, t, Vr, cap, -1, round_operand=False, encode=False)
+    q = oracle.dlogits_e5m2(X, W, t, Vr, cap, -1, round_operand=False, encode=True)
+    assert np.abs(exact).max() <= oracle.E5M2_SCALE * (1 + 1e-12)
+    normal = np.abs(exact) >= 2.0 ** -14
+    rel = np.abs(q - exact)[normal] / np.abs(exact)[normal]
+    assert rel.max() <= 2.0 ** -3 * (1 + 1e-12)
+    assert rel.max() > 2.0 ** -4
+    assert np.abs(q - exact)[~normal].max() <= 2.0 ** -17
+    valid, _ = oracle.valid_rows(t, Vr, -1)
+    assert np.abs(q[~valid]).max() == 0.0
+    # rows of dzn (before encoding) sum to zero once the tanh factor is divided out
+    z = oracle.logits(X, W)
+    gs = exact[:, :Vr] / oracle.softcap_derivative(z, cap)[:, :Vr]
+    assert np.abs(gs[valid].sum(axis=1)).max() <= 1e-9 * oracle.E5M2_SCALE
+
+
+def test_fp8_gradients_close_to_exact():
+    """With both roundings the gradients stay within the e5m2 error: relL2 a few percent."""
+    X, W, t, Vr, cap = _fp8_case(N=200, seed=4)
+    dX, dW = oracle.backward_fp8(X, W, t, Vr, cap, -1)
+    rX, rW = oracle.backward(X, W, t, Vr, cap, -1)
+    for got, ref in ((dX, rX), (dW, rW)):
+        r = np.linalg.norm(got - ref) / np.linalg.norm(ref)
+        assert 1e-4 < r < 0.1
