@@ -59,6 +59,9 @@ def parse_args():
                          "all-reduced after the last (the write-ups: 7)")
     ap.add_argument("--no-allreduce", action="store_true",
                     help="N>1: independent replicas with no collective (weak-scaling floor)")
+    ap.add_argument("--grad-fp8", action="store_true",
+                    help="fp8 workload: the gradient contractions in FP8 too (e5m2 gradient x "
+                         "e4m3 operands) instead of bf16")
     ap.add_argument("--buckets", type=int, default=4,
                     help="N>1: vocabulary buckets of the dW all-reduce, each exchanged as soon "
                          "as the last chunk's gradient launch for it is done (1: one all-reduce "
@@ -324,7 +327,8 @@ def main_gpu(args):
         if fp8:
             loss, lse, _, _, _ = flce.forward_fp8(X8, W8, sX, sW, Xd, W, td, Vr, c.cap,
                                                   c.ignore_index, True, dX=dX, dW=dW,
-                                                  workspace=ws, chunk_rows=args.chunk_rows)
+                                                  workspace=ws, chunk_rows=args.chunk_rows,
+                                                  grad_fp8=args.grad_fp8)
         else:
             loss, lse, _, _, _ = flce.forward(Xd, W, td, Vr, c.cap, c.ignore_index, True, dX=dX,
                                               dW=dW, workspace=ws, chunk_rows=args.chunk_rows)
@@ -501,7 +505,8 @@ def main_gpu(args):
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None,
-            "dtype": "e4m3 logits + bf16 gradients" if fp8 else "bf16", "data": "synthetic",
+            "dtype": ("e4m3 logits + e5m2 x e4m3 gradients" if fp8 and args.grad_fp8 else
+                      "e4m3 logits + bf16 gradients" if fp8 else "bf16"), "data": "synthetic",
             "config": arm_config(c, shape.chunk_rows or min(N, AUTO_CHUNK_ROWS), world, dp,
                                  args.accum_steps, args.buckets),
             "tflops": tflops,

@@ -195,16 +195,22 @@ int flce_forward_dp_bucketed(const flce_shape* shape, const void* X, const void*
  * tensorwise scales (x ~ X8 * *scale_x, w ~ W8 * *scale_w; the scales are device scalars) on the
  * tensor cores' fp8 path, with both scales applied to z before the softcap.  This follows the
  * write-ups' FP8 training ("Increasing throughput": GEMMs in FP8 with dynamic tensorwise scaling
- * through torch._scaled_mm, +25%); here only the logits contraction reads fp8.  With
- * want_grads = 1 the softmax gradient is formed from those logits and the two gradient
- * contractions use the bf16 copies X [N, d] and W [Vpad, d] (dX = dz W, dW = dz^T X), which may
- * be NULL when want_grads = 0.
+ * through torch._scaled_mm, one forward and two backward GEMMs per layer).
+ * With want_grads = 1 the softmax gradient is formed from those logits and the two gradient
+ * contractions run
+ *   grad_fp8 = 0: in bf16, on the bf16 copies X [N, d] and W [Vpad, d] (dX = dz W, dW = dz^T X);
+ *   grad_fp8 = 1: in FP8 as well: the normalised gradient dz * Nv/g (|.| <= 1) times 2^15 is
+ *     encoded in e5m2 (a fixed power-of-two scale suffices: no amax pass) and multiplied with the
+ *     e4m3 operands, dX = g/(Nv 2^15) * scale_w * (q W8) and dW = g/(Nv 2^15) * scale_x *
+ *     (q^T X8), on the tensor cores' 8-bit path.  Needs 0 < cap <= 32; X and W may be NULL.
+ * With want_grads = 0 (or grad_fp8 = 1) X and W may be NULL.
  *   X8 [N, d], W8 [Vpad, d]: e4m3 bytes, row-major; d must be a multiple of 16.
- * Outputs, workspace (flce_workspace_bytes of the same shape) and errors as flce_forward.
+ * Outputs, grad_scale, dW_dtype, workspace (flce_workspace_bytes of the same shape) and errors as
+ * flce_forward.
  */
 int flce_forward_fp8(const flce_shape* shape, const void* X8, const void* W8,
                      const float* scale_x, const float* scale_w, const void* X, const void* W,
-                     const int64_t* targets, float* loss, float* lse, int want_grads,
+                     const int64_t* targets, float* loss, float* lse, int want_grads, int grad_fp8,
                      const float* grad_scale, void* dX, void* dW, int dW_dtype,
                      int accumulate_dW, void* workspace, size_t workspace_bytes, void* stream);
 

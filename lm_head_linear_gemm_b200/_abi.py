@@ -82,7 +82,7 @@ def lib() -> ctypes.CDLL:
     L.flce_read_status.argtypes = [P, ctypes.POINTER(ctypes.c_uint32),
                                    ctypes.POINTER(ctypes.c_int64), P]
     L.flce_read_status.restype = ctypes.c_int
-    L.flce_forward_fp8.argtypes = [shp, P, P, P, P, P, P, P, P, P, I, P, P, P, I, I, P,
+    L.flce_forward_fp8.argtypes = [shp, P, P, P, P, P, P, P, P, P, I, I, P, P, P, I, I, P,
                                    ctypes.c_size_t, P]
     L.flce_forward_fp8.restype = ctypes.c_int
     L.flce_quantize_e4m3.argtypes = [P, ctypes.c_int64, P, P, P]
@@ -501,9 +501,10 @@ def quantize_e4m3(x, out=None, scale=None, stream=None):
 def forward_fp8(X8, W8, scale_x, scale_w, X, W, targets, Vreal: int, cap: float = 15.0,
                 ignore_index: int = -1, want_grads: bool = False, dX=None, dW=None,
                 accumulate_dW: bool = False, workspace=None, chunk_rows: int = 0, stream=None,
-                grad_scale=None, dW_dtype=None):
-    """Fused forward with e4m3 logits operands (uint8 codes + fp32 device scales) and bf16
-    copies X/W for the gradient contractions.  Returns (loss, lse, dX, dW, workspace)."""
+                grad_scale=None, dW_dtype=None, grad_fp8: bool = False):
+    """Fused forward with e4m3 logits operands (uint8 codes + fp32 device scales).  The
+    gradient contractions use the bf16 copies X/W, or, with ``grad_fp8``, an e5m2 gradient and
+    the e4m3 operands (X/W may then be None).  Returns (loss, lse, dX, dW, workspace)."""
     import torch
     for name, t in (("X8", X8), ("W8", W8)):
         if not t.is_cuda or t.dtype not in (torch.uint8, getattr(torch, "float8_e4m3fn", None)):
@@ -524,7 +525,8 @@ def forward_fp8(X8, W8, scale_x, scale_w, X, W, targets, Vreal: int, cap: float 
     _check_buffer(targets, "targets", torch.int64, (N,), dev)
     dw_t, dw_code = _dW_type(dW, dW_dtype)
     if want_grads:
-        _check(X, W, targets)
+        if not grad_fp8:
+            _check(X, W, targets)
         _check_buffer(X, "X", torch.bfloat16, (N, d), dev)
         _check_buffer(W, "W", torch.bfloat16, tuple(W8.shape), dev)
         _check_buffer(dX, "dX", torch.bfloat16, (N, d), dev)
@@ -536,14 +538,14 @@ def forward_fp8(X8, W8, scale_x, scale_w, X, W, targets, Vreal: int, cap: float 
     lse = torch.empty(max(N, 1), dtype=torch.float32, device=dev)[:N]
     if want_grads:
         if dX is None:
-            dX = torch.empty_like(X)
+            dX = torch.empty((N, d), dtype=torch.bfloat16, device=dev)
         if dW is None:
-            dW = torch.empty(W.shape, dtype=dw_t, device=dev)
+            dW = torch.empty(tuple(W8.shape), dtype=dw_t, device=dev)
     if workspace is None:
         workspace = alloc_workspace(shape, want_grads, dev)
     rc = lib().flce_forward_fp8(ctypes.byref(shape), _ptr(X8), _ptr(W8), _ptr(scale_x),
                                 _ptr(scale_w), _ptr(X), _ptr(W), _ptr(targets), _ptr(loss),
-                                _ptr(lse), 1 if want_grads else 0,
+                                _ptr(lse), 1 if want_grads else 0, 1 if grad_fp8 else 0,
                                 _ptr(grad_scale) if want_grads else None,
                                 _ptr(dX) if want_grads else None,
                                 _ptr(dW) if want_grads else None, dw_code, int(accumulate_dW),

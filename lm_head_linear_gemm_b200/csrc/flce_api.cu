@@ -101,6 +101,12 @@ static_assert(CfgL::BN == Cfg8::BN && CfgL::COL_SPLIT == Cfg8::COL_SPLIT,
 // gradients in one launch: dX = A' W (A' K-major, W MN-major), dW = A'^T Xs (both MN-major)
 constexpr auto kGradKernel = gemm_pair_kernel<Cfg, DxEpi, DwEpi, Major::K, Major::MN, Major::MN,
                                              Major::MN, FLCE_DX_WIDE != 0>;
+// gradients from 8-bit operands: dX = dz8 W8 (dz8 e5m2 K-major, W8 e4m3 MN-major) and
+// dW = dz8^T Xs8 (dz8 e5m2 MN-major, Xs8 e4m3 MN-major), kind::f8f6f4
+using CfgG8 = PairCfg<256, FLCE_GRAD_STAGES, FLCE_EPI_WARPS, 1, 1>;
+constexpr auto kGradKernel8 =
+    gemm_pair_kernel<CfgG8, DxEpi, DwEpi, Major::K, Major::MN, Major::MN, Major::MN,
+                     FLCE_DX_WIDE != 0, 1, F8_A0 | F8_A1>;
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s bound on every in-kernel wait
 constexpr float kFixedRefMaxCap = 32.f;           // exp(s - cap) >= e^{-64}: no underflow in fp32
@@ -116,7 +122,7 @@ struct Layout {
   int n_slabs;        // per-row partial slots of the logits pass
   bool fixed_ref;
   bool compact;       // gradients over each chunk's rows in the loss only
-  size_t hdr, tgt, s_t, der_t, e_t, row_loss, partial, r, A, Xs, pos, orig, cnt, bad, total;
+  size_t hdr, tgt, s_t, der_t, e_t, row_loss, partial, r, A, Xs, pos, orig, cnt, bad, gsc, total;
 };
 
 bool shape_ok(const flce_shape* s) {
@@ -165,6 +171,7 @@ Layout make_layout(const flce_shape* s, int want_grads) {
       L.orig = take(n * sizeof(int));
       L.cnt = take(static_cast<size_t>(L.n_chunks) * sizeof(int));
       L.bad = take(static_cast<size_t>(L.n_chunks) * sizeof(int));
+      L.gsc = take(2 * sizeof(float));
     }
   }
   L.total = off;
@@ -204,7 +211,9 @@ int device_info(DeviceInfo** out) {
         cudaFuncSetAttribute(kGradKernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              Cfg::SMEM_BYTES) != cudaSuccess ||
         cudaFuncSetAttribute(kLogitsKernel8, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             Cfg8::SMEM_BYTES) != cudaSuccess)
+                             Cfg8::SMEM_BYTES) != cudaSuccess ||
+        cudaFuncSetAttribute(kGradKernel8, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             CfgG8::SMEM_BYTES) != cudaSuccess)
       return FLCE_ERR_CUDA;
     di.attrs_set = true;
   }
@@ -351,6 +360,7 @@ struct Ctx {
   Fp8Logits fp8;
   const long long* nv_total = nullptr;   // data-parallel normaliser (null: this call's rows)
   int dW_bf16 = 0;                       // dW element type: 0 fp32, 1 bf16
+  int grad_fp8 = 0;                      // gradient contractions from e5m2 / e4m3 operands
   Layout L;
   uint8_t* ws;
   DevHeader* hdr;
@@ -433,10 +443,20 @@ int grad_chunk(const Ctx& c, int64_t row0, int rows, const __nv_bfloat16* X,
   float* r = c.at<float>(c.L.r);
 
   CUtensorMap mA_k, mW_mn, mA_mn, mXs_mn;
-  FLCE_TRY(make_map(&mA_k, Abuf, Vpad, rows, Vpad, Cfg::BM_CTA));
-  FLCE_TRY(make_map(&mW_mn, W, d, Vpad, d, 64));
-  FLCE_TRY(make_map(&mA_mn, Abuf, Vpad, rows, Vpad, 64));
-  FLCE_TRY(make_map(&mXs_mn, Xs, d, rows, d, 64));
+  uint8_t* Xs8 = reinterpret_cast<uint8_t*>(Xs);
+  if (c.grad_fp8) {
+    // e5m2 gradient rows in place of the bf16 rows of A (row stride 2 Vpad bytes), e4m3 W8 and
+    // compacted X8 rows; boxes of 128 bytes x 128 rows
+    FLCE_TRY(make_map(&mA_k, Abuf, Vpad, rows, 2 * static_cast<uint64_t>(Vpad), CfgG8::BM_CTA, 1));
+    FLCE_TRY(make_map(&mW_mn, c.fp8.W8, d, Vpad, d, CfgG8::BK, 1));
+    FLCE_TRY(make_map(&mA_mn, Abuf, Vpad, rows, 2 * static_cast<uint64_t>(Vpad), CfgG8::BK, 1));
+    FLCE_TRY(make_map(&mXs_mn, Xs8, d, rows, d, CfgG8::BK, 1));
+  } else {
+    FLCE_TRY(make_map(&mA_k, Abuf, Vpad, rows, Vpad, Cfg::BM_CTA));
+    FLCE_TRY(make_map(&mW_mn, W, d, Vpad, d, 64));
+    FLCE_TRY(make_map(&mA_mn, Abuf, Vpad, rows, Vpad, 64));
+    FLCE_TRY(make_map(&mXs_mn, Xs, d, rows, d, 64));
+  }
 
   LogitsParams lp{};
   lp.rows = rows;
@@ -488,6 +508,9 @@ int grad_chunk(const Ctx& c, int64_t row0, int rows, const __nv_bfloat16* X,
   rp.pos = lp.pos;
   rp.cnt = cnt;
   rp.dX = dXc;
+  rp.fp8 = c.grad_fp8;
+  rp.X8 = c.grad_fp8 ? c.fp8.X8 + row0 * s->d : nullptr;
+  rp.Xs8 = Xs8;
   const int finish_warps = rows + (c.L.compact ? 64 : 0);
   row_finish_kernel<<<(finish_warps + 7) / 8, 256, 0, c.st>>>(rp);
   FLCE_TRY(launch_ok());
@@ -496,7 +519,9 @@ int grad_chunk(const Ctx& c, int64_t row0, int rows, const __nv_bfloat16* X,
   // compaction both run over the chunk's rows in the loss only (a device-side count: dX's M
   // and dW's K), dX rows scattered back to their places
   const int dx32 = FLCE_EPI_SECTOR32 && (d % 16) == 0 && aligned32(dXc);
-  DxParams xp{rows, d, dx32, r, dXc, c.L.compact ? c.at<int>(c.L.orig) + row0 : nullptr, cnt};
+  const float* gsc = c.grad_fp8 ? c.at<float>(c.L.gsc) : nullptr;
+  DxParams xp{rows, d, dx32, r, dXc, c.L.compact ? c.at<int>(c.L.orig) + row0 : nullptr, cnt,
+              gsc};
   const int dyn_x = c.L.compact ? DYN_M : 0, dyn_w = c.L.compact ? DYN_K : 0;
   const PairProblem pdx{rows, d, Vpad, 0, FLCE_DX_WIDE, FLCE_L2_DX_A, FLCE_L2_DX_W, dyn_x};
   const PairProblem none{0, 0, 0, 0, 0, 0, 0, 0};
@@ -512,14 +537,27 @@ int grad_chunk(const Ctx& c, int64_t row0, int rows, const __nv_bfloat16* X,
     void* dWb = static_cast<uint8_t*>(dW) +
                 static_cast<size_t>(v0) * s->d * (c.dW_bf16 ? 2 : 4);
     const int dw32 = FLCE_EPI_SECTOR32 && aligned32(dWb) && (!c.dW_bf16 || (d % 16) == 0);
-    DwParams wp{v1 - v0, d, accumulate, dw32, c.dW_bf16, dWb};
+    DwParams wp{v1 - v0, d, accumulate, dw32, c.dW_bf16, dWb, gsc != nullptr ? gsc + 1 : nullptr};
     const PairProblem pdw{v1 - v0, d, rows, 0, 0, FLCE_L2_DW_A, FLCE_L2_DW_XS, dyn_w};
     CUtensorMap mA_mn_b = mA_mn;
-    if (v0 > 0) FLCE_TRY(make_map(&mA_mn_b, Abuf + v0, Vpad - v0, rows, Vpad, 64));
-    if (v1 > v0 || b + 1 == nb)
-      FLCE_TRY((launch_pair<DxEpi, DwEpi>(kGradKernel, c.di, mA_k, mW_mn, mA_mn_b, mXs_mn,
-                                           b + 1 == nb ? pdx : none, v1 > v0 ? pdw : none,
-                                           &c.hdr->status, xp, wp, c.st, 1, cnt)));
+    if (v0 > 0) {
+      if (c.grad_fp8)
+        FLCE_TRY(make_map(&mA_mn_b, reinterpret_cast<uint8_t*>(Abuf) + v0, Vpad - v0, rows,
+                          2 * static_cast<uint64_t>(Vpad), CfgG8::BK, 1));
+      else
+        FLCE_TRY(make_map(&mA_mn_b, Abuf + v0, Vpad - v0, rows, Vpad, 64));
+    }
+    if (v1 > v0 || b + 1 == nb) {
+      if (c.grad_fp8)
+        FLCE_TRY((launch_pair<DxEpi, DwEpi, CfgG8>(kGradKernel8, c.di, mA_k, mW_mn, mA_mn_b,
+                                                   mXs_mn, b + 1 == nb ? pdx : none,
+                                                   v1 > v0 ? pdw : none, &c.hdr->status, xp, wp,
+                                                   c.st, 1, cnt)));
+      else
+        FLCE_TRY((launch_pair<DxEpi, DwEpi>(kGradKernel, c.di, mA_k, mW_mn, mA_mn_b, mXs_mn,
+                                             b + 1 == nb ? pdx : none, v1 > v0 ? pdw : none,
+                                             &c.hdr->status, xp, wp, c.st, 1, cnt)));
+    }
     if (buckets != nullptr && buckets->events[b] != nullptr) {
       if (cudaEventRecord(static_cast<cudaEvent_t>(buckets->events[b]), c.st) != cudaSuccess)
         return FLCE_ERR_CUDA;
@@ -652,7 +690,8 @@ int forward_impl(const flce_shape* s, const void* X, const void* W, const Fp8Log
                  const int64_t* targets, float* loss, float* lse, int want_grads,
                  const float* grad_scale, void* dX, void* dW, int dW_dtype, int accumulate_dW,
                  void* workspace, size_t workspace_bytes, void* stream,
-                 const int64_t* nv_total = nullptr, const Buckets* buckets = nullptr) {
+                 const int64_t* nv_total = nullptr, const Buckets* buckets = nullptr,
+                 int grad_fp8 = 0) {
   want_grads = want_grads ? 1 : 0;
   if (loss == nullptr || (s->N > 0 && lse == nullptr)) return FLCE_ERR_ARG;
   if (!aligned4(loss) || !aligned4(lse)) return FLCE_ERR_ALIGN;
@@ -669,7 +708,11 @@ int forward_impl(const flce_shape* s, const void* X, const void* W, const Fp8Log
   c.fp8 = fp8;
   c.nv_total = reinterpret_cast<const long long*>(nv_total);
   c.dW_bf16 = want_grads && dW_dtype == FLCE_DTYPE_BF16 ? 1 : 0;
+  c.grad_fp8 = want_grads && grad_fp8 ? 1 : 0;
   c.L = make_layout(s, want_grads);
+  // 8-bit gradients need the fixed exp reference and the compacted rows (rows not in the loss
+  // must not enter the e5m2 operand)
+  if (c.grad_fp8 && (!c.L.fixed_ref || !c.L.compact || fp8.X8 == nullptr)) return FLCE_ERR_ARG;
   c.ws = static_cast<uint8_t*>(workspace);
   c.di = di;
   c.st = static_cast<cudaStream_t>(stream);
@@ -678,6 +721,11 @@ int forward_impl(const flce_shape* s, const void* X, const void* W, const Fp8Log
   const auto* Wb = static_cast<const __nv_bfloat16*>(W);
 
   FLCE_TRY(prep(c, targets));
+  if (c.grad_fp8) {
+    fp8_grad_scales_kernel<<<1, 1, 0, c.st>>>(c.hdr, c.nv_total, grad_scale, fp8.scale_w,
+                                              fp8.scale_x, c.at<float>(c.L.gsc));
+    FLCE_TRY(launch_ok());
+  }
   if (s->N == 0) {
     zero_loss_kernel<<<1, 1, 0, c.st>>>(loss);
     FLCE_TRY(launch_ok());
@@ -793,15 +841,20 @@ int flce_forward_dp_bucketed(const flce_shape* s, const void* X, const void* W,
 
 int flce_forward_fp8(const flce_shape* s, const void* X8, const void* W8, const float* scale_x,
                      const float* scale_w, const void* X, const void* W, const int64_t* targets,
-                     float* loss, float* lse, int want_grads, const float* grad_scale, void* dX,
-                     void* dW, int dW_dtype, int accumulate_dW, void* workspace,
-                     size_t workspace_bytes, void* stream) {
+                     float* loss, float* lse, int want_grads, int grad_fp8,
+                     const float* grad_scale, void* dX, void* dW, int dW_dtype,
+                     int accumulate_dW, void* workspace, size_t workspace_bytes, void* stream) {
   if (!shape_ok(s)) return FLCE_ERR_ARG;
   if ((s->d % 16) != 0 || (s->Vpad % 8) != 0) return FLCE_ERR_ALIGN;  // 16-byte e4m3 rows
   if ((s->N > 0 && (X8 == nullptr || targets == nullptr)) || W8 == nullptr ||
       scale_x == nullptr || scale_w == nullptr || workspace == nullptr)
     return FLCE_ERR_ARG;
-  if (want_grads && ((s->N > 0 && X == nullptr) || W == nullptr)) return FLCE_ERR_ARG;
+  // the bf16 copies feed the gradient contractions unless those read the 8-bit operands
+  if (want_grads && !grad_fp8 && ((s->N > 0 && X == nullptr) || W == nullptr))
+    return FLCE_ERR_ARG;
+  // 8-bit gradients: the exp reference is the cap (0 < cap <= 32), the rows are compacted
+  if (want_grads && grad_fp8 && (!(s->cap > 0.f && s->cap <= kFixedRefMaxCap) || !FLCE_COMPACT))
+    return FLCE_ERR_ARG;
   if (!aligned16(X8) || !aligned16(W8) || !aligned16(X) || !aligned16(W) || !aligned16(targets) ||
       (reinterpret_cast<uintptr_t>(scale_x) & 3u) != 0 ||
       (reinterpret_cast<uintptr_t>(scale_w) & 3u) != 0 ||
@@ -814,7 +867,8 @@ int flce_forward_fp8(const flce_shape* s, const void* X8, const void* W8, const 
   fp8.scale_x = scale_x;
   fp8.scale_w = scale_w;
   return forward_impl(s, X, W, fp8, targets, loss, lse, want_grads, grad_scale, dX, dW,
-                      dW_dtype, accumulate_dW, workspace, workspace_bytes, stream);
+                      dW_dtype, accumulate_dW, workspace, workspace_bytes, stream, nullptr,
+                      nullptr, grad_fp8);
 }
 
 int flce_quantize_e4m3(const void* src, int64_t n, void* dst, float* scale_out, void* stream) {

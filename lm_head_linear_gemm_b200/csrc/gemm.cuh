@@ -34,37 +34,55 @@ __device__ __forceinline__ void tmem_ld32_or_zero(uint32_t taddr, float (&v)[32]
 }
 
 // ----------------------------------------------------------------------------------------------
-// Tile loaders: K-major -> one TMA box {64 (K), rows}; MN-major -> rows/64 boxes {64 (MN), 64 (K)}.
+// Staged operand tiles, all in 128-byte swizzled rows (EB = bytes per element: 2 bf16, 1 fp8).
+//   K-major : one TMA box {128 bytes of K, rows}.
+//   MN-major: rows / (128/EB) boxes {128/EB (MN), 128/EB (K)}: each box is one 128-byte-wide
+//             block of M/N elements over the k-block's K rows, boxes laid out one after the
+//             other (the descriptor's leading byte offset is the box size).
 // The copy completes on the pair leader's barrier (shared::cluster address).
-template <Major MAJ, int ROWS>
+template <Major MAJ, int ROWS, int EB = 2>
 __device__ __forceinline__ void load_operand_pair(uint8_t* dst, const CUtensorMap* map,
                                                   uint32_t leader_bar, int row0, int k0,
                                                   uint64_t policy) {
   if constexpr (MAJ == Major::K) {
     tma_load_2d_pair_hint(dst, map, leader_bar, k0, row0, policy);
   } else {
+    constexpr int MNB = 128 / EB;               // elements of one 128-byte block
+    constexpr int BOX = 128 * (128 / EB);       // bytes of one box (k-block rows x 128 bytes)
+    static_assert(ROWS % MNB == 0, "MN-major tiles are whole 128-byte blocks");
 #pragma unroll
-    for (int q = 0; q < ROWS / 64; ++q)
-      tma_load_2d_pair_hint(dst + q * 8192, map, leader_bar, row0 + 64 * q, k0, policy);
+    for (int q = 0; q < ROWS / MNB; ++q)
+      tma_load_2d_pair_hint(dst + q * BOX, map, leader_bar, row0 + MNB * q, k0, policy);
   }
 }
 
 // Descriptor increment between consecutive MMA slices (start address field, 16-byte units);
-// staged tiles sit below 256 KB, so adding to the 14-bit field never carries out of it.
-template <Major MAJ>
+// one slice is 32 bytes of K: 32 bytes along a K-major row, or 32/EB K rows of 128 bytes of an
+// MN-major tile.  Staged tiles sit below 256 KB, so adding to the 14-bit field never carries
+// out of it.
+template <Major MAJ, int EB = 2>
 __device__ __forceinline__ constexpr uint64_t desc_step() {
-  return MAJ == Major::K ? 2u : 128u;
+  return MAJ == Major::K ? 2u : static_cast<uint64_t>(256 / EB);
 }
 
-// Descriptor of the k-th MMA slice of a staged operand tile (32 bytes of K: 16 bf16 or 32 e4m3
-// elements; MN-major slices are bf16 only: 16 K rows = two 1 KB swizzle atoms).
-template <Major MAJ>
+// Descriptor of the k-th MMA slice of a staged operand tile.
+template <Major MAJ, int EB = 2>
 __device__ __forceinline__ uint64_t operand_desc(uint32_t base, int k) {
   if constexpr (MAJ == Major::K) {
     return smem_desc_sw128(base + 32u * k, 16u, 1024u);
   } else {
-    return smem_desc_sw128(base + 2048u * k, 8192u, 1024u);
+    return smem_desc_sw128(base + (4096u / EB) * k, 128u * (128u / EB), 1024u);
   }
+}
+
+// One tcgen05.mma on an SM pair: kind::f16 (bf16) or kind::f8f6f4 (8-bit formats).
+template <int EB>
+__device__ __forceinline__ void mma_pair(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
+                                         uint32_t acc) {
+  if constexpr (EB == 2)
+    mma_bf16_ss_pair(d, a, b, idesc, acc);
+  else
+    mma_e4m3_ss_pair(d, a, b, idesc, acc);
 }
 
 // ==============================================================================================
@@ -199,9 +217,11 @@ __host__ __device__ inline PairTile pair_tile(const PairSchedule& s, int pair, i
 }
 
 // WIDE0: problem 0 may run in wide tiles (below).  ROUND: ring slots per MMA-issue round of
-// the other tiles (1 or 2).
+// the other tiles (1 or 2).  FMT: with 8-bit operands, which of them are e5m2 (F8_A0, F8_B0,
+// F8_A1, F8_B1 bits; the others are e4m3).
+enum : int { F8_A0 = 1, F8_B0 = 2, F8_A1 = 4, F8_B1 = 8 };
 template <class C, class E0, class E1, Major A0, Major B0, Major A1, Major B1, bool WIDE0 = false,
-          int ROUND = 1>
+          int ROUND = 1, int FMT = 0>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
                      const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
@@ -243,7 +263,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
   // so a wide k-block takes two slots and the ring stays in step as long as the slot count and
   // the number of N blocks are even.  Meant for long-K problems: while a wide tile runs, no
   // accumulator is free for the epilogue of the previous tile to overlap with.
-  const bool wide0 = WIDE0 && args.prob[0].wide != 0 && C::ELEM_BYTES == 2 && C::KSUB == 1 &&
+  const bool wide0 = WIDE0 && args.prob[0].wide != 0 && C::KSUB == 1 &&
                      (C::STAGES % 2) == 0 && (n_tiles0 % 2) == 0;
   const int w_tiles0 = wide0 ? n_tiles0 / 2 : n_tiles0;
 
@@ -372,14 +392,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
             for (int j = 0; j < C::KSUB; ++j) {
               const int k0 = kb * C::KSLOT + j * C::BK;
               if (prob == 0) {
-                load_operand_pair<A0, C::BM_CTA>(sA + j * C::A_SUB, &tmA0, bar, a_row, k0, pol_a0);
-                load_operand_pair<B0, C::BN_CTA>(sB + j * C::B_SUB, &tmB0, bar, b_row, k0, pol_b0);
+                load_operand_pair<A0, C::BM_CTA, C::ELEM_BYTES>(sA + j * C::A_SUB, &tmA0, bar,
+                                                                a_row, k0, pol_a0);
+                load_operand_pair<B0, C::BN_CTA, C::ELEM_BYTES>(sB + j * C::B_SUB, &tmB0, bar,
+                                                                b_row, k0, pol_b0);
                 if constexpr (NSUB == 2)
-                  load_operand_pair<B0, C::BN_CTA>(sB + C::STAGE_BYTES, &tmB0, bar + 8u,
-                                                   b_row + C::BN, k0, pol_b0);
+                  load_operand_pair<B0, C::BN_CTA, C::ELEM_BYTES>(sB + C::STAGE_BYTES, &tmB0,
+                                                                  bar + 8u, b_row + C::BN, k0,
+                                                                  pol_b0);
               } else {
-                load_operand_pair<A1, C::BM_CTA>(sA + j * C::A_SUB, &tmA1, bar, a_row, k0, pol_a1);
-                load_operand_pair<B1, C::BN_CTA>(sB + j * C::B_SUB, &tmB1, bar, b_row, k0, pol_b1);
+                load_operand_pair<A1, C::BM_CTA, C::ELEM_BYTES>(sA + j * C::A_SUB, &tmA1, bar,
+                                                                a_row, k0, pol_a1);
+                load_operand_pair<B1, C::BN_CTA, C::ELEM_BYTES>(sB + j * C::B_SUB, &tmB1, bar,
+                                                                b_row, k0, pol_b1);
               }
             }
             arms += NSUB;
@@ -408,17 +433,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
   } else if (warp == 1) {
     if (lane == 0 && leader) {
       // ------------------------------------------------------------ MMA issuer (leader only)
-      static_assert((B0 == Major::K || C::BN_CTA % 64 == 0) && (B1 == Major::K || C::BN_CTA % 64 == 0),
-                    "MN-major B halves are whole 64-wide blocks");
-      static_assert(C::ELEM_BYTES == 2 || (A0 == Major::K && B0 == Major::K && A1 == Major::K &&
-                                           B1 == Major::K),
-                    "e4m3 operands are staged K-major");
+      constexpr int EB = C::ELEM_BYTES;
+      static_assert((B0 == Major::K || C::BN_CTA % (128 / EB) == 0) &&
+                        (B1 == Major::K || C::BN_CTA % (128 / EB) == 0),
+                    "MN-major B halves are whole 128-byte blocks");
+      static_assert(EB == 1 || FMT == 0, "operand formats are for 8-bit operands");
       constexpr uint32_t idesc0 =
-          C::ELEM_BYTES == 1 ? instr_desc_e4m3_f32(C::BM, C::BN)
-                             : instr_desc_bf16_f32(C::BM, C::BN, A0 == Major::MN, B0 == Major::MN);
+          EB == 1 ? instr_desc_f8_f32(C::BM, C::BN, (FMT & F8_A0) ? F8_E5M2 : F8_E4M3,
+                                      (FMT & F8_B0) ? F8_E5M2 : F8_E4M3, A0 == Major::MN,
+                                      B0 == Major::MN)
+                  : instr_desc_bf16_f32(C::BM, C::BN, A0 == Major::MN, B0 == Major::MN);
       constexpr uint32_t idesc1 =
-          C::ELEM_BYTES == 1 ? instr_desc_e4m3_f32(C::BM, C::BN)
-                             : instr_desc_bf16_f32(C::BM, C::BN, A1 == Major::MN, B1 == Major::MN);
+          EB == 1 ? instr_desc_f8_f32(C::BM, C::BN, (FMT & F8_A1) ? F8_E5M2 : F8_E4M3,
+                                      (FMT & F8_B1) ? F8_E5M2 : F8_E4M3, A1 == Major::MN,
+                                      B1 == Major::MN)
+                  : instr_desc_bf16_f32(C::BM, C::BN, A1 == Major::MN, B1 == Major::MN);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
@@ -459,14 +488,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
               // both N blocks from one staged A k-block; the second B block is in the next slot
               const uint32_t d_tmem2 = tmem_base + static_cast<uint32_t>(acc2 * C::BN);
               const uint32_t b_base2 = b_base + C::STAGE_BYTES;
-              const uint64_t da = operand_desc<A0>(a_base, 0), db = operand_desc<B0>(b_base, 0);
-              const uint64_t db2 = operand_desc<B0>(b_base2, 0);
+              const uint64_t da = operand_desc<A0, EB>(a_base, 0);
+              const uint64_t db = operand_desc<B0, EB>(b_base, 0);
+              const uint64_t db2 = operand_desc<B0, EB>(b_base2, 0);
 #pragma unroll
               for (int k = 0; k < C::BK / C::MMA_K; ++k) {
-                mma_bf16_ss_pair(d_tmem, da + desc_step<A0>() * k, db + desc_step<B0>() * k,
-                                 idesc0, (kb | k) != 0 ? 1u : 0u);
-                mma_bf16_ss_pair(d_tmem2, da + desc_step<A0>() * k, db2 + desc_step<B0>() * k,
-                                 idesc0, (kb | k) != 0 ? 1u : 0u);
+                mma_pair<EB>(d_tmem, da + desc_step<A0, EB>() * k, db + desc_step<B0, EB>() * k,
+                             idesc0, (kb | k) != 0 ? 1u : 0u);
+                mma_pair<EB>(d_tmem2, da + desc_step<A0, EB>() * k,
+                             db2 + desc_step<B0, EB>() * k, idesc0, (kb | k) != 0 ? 1u : 0u);
               }
               issued = true;
               mma_commit_pair_both(&empty[stage]);
@@ -486,25 +516,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
                 const uint32_t a_base = smem_u32(smem + st * C::STAGE_BYTES + j * C::A_SUB);
                 const uint32_t b_base = smem_u32(smem + st * C::STAGE_BYTES + C::A_BYTES +
                                                  j * C::B_SUB);
-                const uint64_t da = operand_desc<A0>(a_base, 0), db = operand_desc<B0>(b_base, 0);
-                const uint64_t da1 = operand_desc<A1>(a_base, 0), db1 = operand_desc<B1>(b_base, 0);
                 const int first = kb | j;   // 0 only for the first k-block of the tile
-                if constexpr (C::ELEM_BYTES == 1) {
+                if (prob == 0) {
+                  const uint64_t da = operand_desc<A0, EB>(a_base, 0);
+                  const uint64_t db = operand_desc<B0, EB>(b_base, 0);
 #pragma unroll
                   for (int k = 0; k < C::BK / C::MMA_K; ++k)
-                    mma_e4m3_ss_pair(d_tmem, operand_desc<Major::K>(a_base, k),
-                                     operand_desc<Major::K>(b_base, k), prob == 0 ? idesc0 : idesc1,
-                                     (first | k) != 0 ? 1u : 0u);
-                } else if (prob == 0) {
-#pragma unroll
-                  for (int k = 0; k < C::BK / C::MMA_K; ++k)
-                    mma_bf16_ss_pair(d_tmem, da + desc_step<A0>() * k, db + desc_step<B0>() * k,
-                                     idesc0, (first | k) != 0 ? 1u : 0u);
+                    mma_pair<EB>(d_tmem, da + desc_step<A0, EB>() * k,
+                                 db + desc_step<B0, EB>() * k, idesc0, (first | k) != 0 ? 1u : 0u);
                 } else {
+                  const uint64_t da1 = operand_desc<A1, EB>(a_base, 0);
+                  const uint64_t db1 = operand_desc<B1, EB>(b_base, 0);
 #pragma unroll
                   for (int k = 0; k < C::BK / C::MMA_K; ++k)
-                    mma_bf16_ss_pair(d_tmem, da1 + desc_step<A1>() * k, db1 + desc_step<B1>() * k,
-                                     idesc1, (first | k) != 0 ? 1u : 0u);
+                    mma_pair<EB>(d_tmem, da1 + desc_step<A1, EB>() * k,
+                                 db1 + desc_step<B1, EB>() * k, idesc1,
+                                 (first | k) != 0 ? 1u : 0u);
                 }
               }
             };
@@ -840,6 +867,7 @@ struct DxParams {
   __nv_bfloat16* dX;         // [rows][d]
   const int* orig;           // compacted rows: dX row of each (null: same row)
   const int* dyn_rows;       // compacted rows: their device-side count (null: rows)
+  const float* uscale;       // one scale for every row instead of r (8-bit operands), or null
 };
 
 struct DxEpi {
@@ -849,7 +877,7 @@ struct DxEpi {
                                                int, bool zero) {
     const int rows = p.dyn_rows != nullptr ? __ldg(p.dyn_rows) : p.rows;
     const bool row_ok = row < rows;
-    const float sc = row_ok ? __ldg(p.r + row) : 0.f;
+    const float sc = !row_ok ? 0.f : (p.uscale != nullptr ? __ldg(p.uscale) : __ldg(p.r + row));
     const int out_row = row_ok && p.orig != nullptr ? __ldg(p.orig + row) : row;
     __nv_bfloat16* out = row_ok ? p.dX + static_cast<size_t>(out_row) * p.d : nullptr;
 #pragma unroll 1
@@ -894,6 +922,7 @@ struct DwParams {
   int sector32;              // 1: dW rows and base are 32-byte aligned (full-sector accesses)
   int bf16;                  // 1: dW is bf16, 0: fp32
   void* dW;                  // [Vpad][d]
+  const float* scale;        // factor applied to the tile (8-bit operands), or null
 };
 
 struct DwEpi {
@@ -921,6 +950,11 @@ struct DwEpi {
       float v[32];
       tmem_ld32_or_zero(taddr + c * 32, v, zero);
       if (!row_ok) continue;
+      if (p.scale != nullptr) {
+        const float f = __ldg(p.scale);
+#pragma unroll
+        for (int k = 0; k < 32; ++k) v[k] *= f;
+      }
       const int cbase = col0 + c * 32;
       if (p.bf16) {
         if (p.sector32) {

@@ -174,10 +174,75 @@ struct RowFinishParams {
   const int* pos;               // [rows] position or -1
   const int* cnt;               // this chunk's number of rows in the loss
   __nv_bfloat16* dX;            // [rows][d] this chunk's dX rows
+  // 8-bit gradient operands (fp8 = 1, with compaction and the fixed reference): the row's
+  // softmax gradient normalised by S and scaled by 2^15, q_j = e5m2(A'_j / S * 2^15), replaces
+  // the bf16 row of A in place (its first Vpad bytes; rows keep their 2 Vpad-byte stride), and
+  // the row's e4m3 X8 bytes are copied to Xs8 at its compacted position.
+  int fp8;
+  const uint8_t* X8;            // [rows][d] this chunk's e4m3 rows
+  uint8_t* Xs8;                 // [rows][d]
 };
 
 __device__ __forceinline__ void zero_row_bf16(__nv_bfloat16* row, int n, int lane) {
   for (int k = lane * 8; k < n; k += 256) *reinterpret_cast<uint4*>(row + k) = make_uint4(0, 0, 0, 0);
+}
+
+// One warp: the e5m2 gradient row of a row in the loss (see RowFinishParams::fp8), written over
+// the first half of the bf16 row it is formed from.  The row is converted in batches: each batch
+// reads its bf16 elements into registers, the warp synchronises, then writes their codes, which
+// land on bytes whose bf16 values this or an earlier batch has already read.
+template <class P>
+__device__ __forceinline__ void encode_row_e5m2(const P& p, int row, int at, int t, float S) {
+  const int lane = threadIdx.x & 31;
+  const __nv_bfloat16* arow = p.A + static_cast<size_t>(at) * p.Vpad;
+  uint8_t* qrow = reinterpret_cast<uint8_t*>(p.A + static_cast<size_t>(at) * p.Vpad);
+  // the target element as the bf16 path stores it, (1 - tanh^2)(e_t - S) rounded to bf16
+  const float pv = __bfloat162float(__float2bfloat16_rn(p.der_t[row] * (p.e_t[row] - S)));
+  const float f = 32768.0f / S;
+  constexpr int B = 4;                                 // groups of 8 elements per lane per batch
+  for (int base = 0; base < p.Vpad; base += 32 * 8 * B) {
+    uint4 v[B];
+#pragma unroll
+    for (int b = 0; b < B; ++b) {
+      const int k = base + (b * 32 + lane) * 8;
+      if (k < p.Vpad) v[b] = *reinterpret_cast<const uint4*>(arow + k);
+    }
+    __syncwarp();
+#pragma unroll
+    for (int b = 0; b < B; ++b) {
+      const int k = base + (b * 32 + lane) * 8;
+      if (k < p.Vpad) {
+        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v[b]);
+        float x[8];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float2 f2 = __bfloat1622float2(h[q]);
+          x[2 * q] = f2.x;
+          x[2 * q + 1] = f2.y;
+        }
+        if (static_cast<unsigned>(t - k) < 8u) {
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            if (q == t - k) x[q] = pv;
+        }
+        uint32_t w[2];
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(x[4 * q] * f, x[4 * q + 1] * f),
+                                                       __NV_SATFINITE, __NV_E5M2);
+          const uint32_t hi = __nv_cvt_float2_to_fp8x2(
+              make_float2(x[4 * q + 2] * f, x[4 * q + 3] * f), __NV_SATFINITE, __NV_E5M2);
+          w[q] = lo | (hi << 16);
+        }
+        *reinterpret_cast<uint2*>(qrow + k) = make_uint2(w[0], w[1]);
+      }
+    }
+    __syncwarp();
+  }
+  const uint8_t* xr = p.X8 + static_cast<size_t>(row) * p.d;
+  uint8_t* xs = p.Xs8 + static_cast<size_t>(at) * p.d;
+  for (int k = lane * 16; k < p.d; k += 512)
+    *reinterpret_cast<uint4*>(xs + k) = *reinterpret_cast<const uint4*>(xr + k);
 }
 
 // One warp per row (plus, when compacting, 64 warps that clear the tail rows).
@@ -190,7 +255,11 @@ __global__ void __launch_bounds__(256) row_finish_kernel(const RowFinishParams p
       const int q = m + (warp - p.rows);
       if (q < ((m + 63) & ~63) && q < p.rows) {
         zero_row_bf16(p.A + static_cast<size_t>(q) * p.Vpad, p.Vpad, lane);
-        zero_row_bf16(p.Xs + static_cast<size_t>(q) * p.d, p.d, lane);
+        if (p.fp8)
+          zero_row_bf16(reinterpret_cast<__nv_bfloat16*>(p.Xs8 + static_cast<size_t>(q) * p.d),
+                        p.d / 2, lane);
+        else
+          zero_row_bf16(p.Xs + static_cast<size_t>(q) * p.d, p.d, lane);
       }
     }
     return;
@@ -246,6 +315,10 @@ __global__ void __launch_bounds__(256) row_finish_kernel(const RowFinishParams p
       return;
     }
     at = p.pos[row];
+  }
+  if (p.fp8) {
+    encode_row_e5m2(p, row, at, t, S);
+    return;
   }
   if (lane == 0) {
     p.r[at] = r;
@@ -524,6 +597,21 @@ __global__ void wait_timeout_selftest_kernel(uint32_t* status, unsigned long lon
   mbar_init(&bar, 1);
   fence_barrier_init();
   mbar_wait_bounded(&bar, 0, status, limit_ns);
+}
+
+// Factors of the 8-bit gradient contractions: the e5m2 codes carry dz * Nv/g * 2^15, the e4m3
+// operands W8 and X8 their tensorwise scales, so dX = [g/(Nv 2^15) sW] (q W8) and
+// dW = [g/(Nv 2^15) sX] (q^T Xs8).  out = {dX factor, dW factor}; 0 when no row is in the loss.
+__global__ void fp8_grad_scales_kernel(const DevHeader* __restrict__ hdr,
+                                       const long long* __restrict__ nv_total,
+                                       const float* __restrict__ grad_scale,
+                                       const float* __restrict__ scale_w,
+                                       const float* __restrict__ scale_x, float* __restrict__ out) {
+  const long long nv = nv_total != nullptr ? *nv_total : hdr->n_valid;
+  const float g = grad_scale != nullptr ? *grad_scale : 1.f;
+  const float base = nv > 0 ? g / (static_cast<float>(nv) * 32768.0f) : 0.f;
+  out[0] = base * *scale_w;
+  out[1] = base * *scale_x;
 }
 
 // Writes loss = 0 (used for N = 0, where nothing else runs).

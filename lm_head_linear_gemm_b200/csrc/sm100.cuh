@@ -293,11 +293,20 @@ __device__ __forceinline__ uint64_t l2_policy(int kind) {
   return p;
 }
 
-// Instruction descriptor for kind::f8f6f4 with e4m3 A/B (format 0) and fp32 accumulation.
-__host__ __device__ constexpr uint32_t instr_desc_e4m3_f32(int M, int N) {
-  return (1u << 4) | ((static_cast<uint32_t>(N) >> 3) << 17) |
+// Instruction descriptor for kind::f8f6f4 with fp32 accumulation: A format bits 7-9 and B
+// format bits 10-12 (0 = e4m3, 1 = e5m2), bit 15 / 16 A / B MN-major, N >> 3 at bit 17,
+// M >> 4 at bit 24 (the same layout as kind::f16).
+enum : uint32_t { F8_E4M3 = 0u, F8_E5M2 = 1u };
+__host__ __device__ constexpr uint32_t instr_desc_f8_f32(int M, int N, uint32_t a_fmt,
+                                                         uint32_t b_fmt, bool a_mn, bool b_mn) {
+  return (1u << 4) | (a_fmt << 7) | (b_fmt << 10) | ((a_mn ? 1u : 0u) << 15) |
+         ((b_mn ? 1u : 0u) << 16) | ((static_cast<uint32_t>(N) >> 3) << 17) |
          ((static_cast<uint32_t>(M) >> 4) << 24);
 }
+__host__ __device__ constexpr uint32_t instr_desc_e4m3_f32(int M, int N) {
+  return instr_desc_f8_f32(M, N, F8_E4M3, F8_E4M3, false, false);
+}
+// tcgen05.mma kind::f8f6f4 on an SM pair (the operand formats come from the descriptor).
 __device__ __forceinline__ void mma_e4m3_ss_pair(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
                                                  uint32_t idesc, uint32_t accumulate) {
   asm volatile(

@@ -52,7 +52,7 @@ __all__ = [
     "logits", "softcap", "softcap_derivative", "valid_rows", "row_forward", "forward",
     "row_dlogits", "backward", "forward_backward", "dW_rows", "rmsnorm_forward",
     "rmsnorm_backward", "round_bf16", "encode_e5m2", "E5M2_SCALE", "dlogits_e5m2",
-    "backward_fp8",
+    "backward_fp8", "dW_rows_fp8",
 ]
 
 
@@ -314,3 +314,35 @@ def backward_fp8(Xq, Wq, t, Vreal: int, cap: float, ignore_index: int, g: float 
         dX[r0:r1] = f * (q @ Wq)
         dW += f * (q.T @ Xq[r0:r1])
     return dX, dW
+
+
+def dW_rows_fp8(Xq, Wq, t, lse, vocab_rows, Vreal: int, cap: float, ignore_index: int,
+                g: float = 1.0, block_rows: int = 4096):
+    """Selected rows ``j`` of the FP8-path dW (``backward_fp8``), given the lse of every row:
+    S_i = exp(lse_i - cap) is the row sum the codes are normalised by, so only the columns in
+    ``vocab_rows`` have to be formed."""
+    Xq = np.asarray(Xq, np.float64)
+    Wj = np.asarray(Wq, np.float64)[np.asarray(vocab_rows)]
+    vocab_rows = np.asarray(vocab_rows, np.int64)
+    valid, _ = valid_rows(t, Vreal, ignore_index)
+    nv = int(np.count_nonzero(valid))
+    out = np.zeros((len(vocab_rows), Xq.shape[1]), np.float64)
+    if nv == 0:
+        return out
+    t = np.asarray(t, np.int64)
+    real = vocab_rows < Vreal
+    for r0 in range(0, Xq.shape[0], block_rows):
+        r1 = min(Xq.shape[0], r0 + block_rows)
+        z = Xq[r0:r1] @ Wj.T
+        s = softcap(z, cap)
+        der = softcap_derivative(z, cap)
+        e = np.exp(s - cap)
+        e[:, ~real] = 0.0
+        S = np.exp(np.asarray(lse[r0:r1], np.float64) - cap)
+        A = e * der
+        hit = t[r0:r1, None] == vocab_rows[None, :]
+        A = np.where(hit, der * (e - S[:, None]), A)
+        q = encode_e5m2(round_bf16(A) / S[:, None] * E5M2_SCALE)
+        q[~valid[r0:r1]] = 0.0
+        out += q.T @ Xq[r0:r1]
+    return out * (g / (nv * E5M2_SCALE))

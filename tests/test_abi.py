@@ -160,15 +160,20 @@ def test_fp8_dp_and_count_entry_points_reject_bad_arguments_before_launch(L):
     ws = flce.workspace_bytes(s, True)
     sp = ctypes.byref(s)
     f8 = L.flce_forward_fp8
-    # X8, W8, sx, sw, X, W, t, loss, lse, want_grads, g, dX, dW, dW_dtype, acc, ws, ws_bytes,
-    # stream
-    assert f8(sp, p, p, None, p, p, p, p, p, p, 1, None, p, p, 0, 0, p, ws, None) == -1  # sx
-    assert f8(sp, p, p, p, p, None, p, p, p, p, 1, None, p, p, 0, 0, p, ws, None) == -1  # X
-    assert f8(sp, p, p, p + 2, p, p, p, p, p, p, 1, None, p, p, 0, 0, p, ws, None) == -2
-    assert f8(sp, p + 8, p, p, p, p, p, p, p, p, 1, None, p, p, 0, 0, p, ws, None) == -2
-    assert f8(sp, p, p, p, p, p, p, p, p, p, 1, None, p, p, 0, 0, p, ws - 1, None) == -3
+    # X8, W8, sx, sw, X, W, t, loss, lse, want_grads, grad_fp8, g, dX, dW, dW_dtype, acc, ws,
+    # ws_bytes, stream
+    assert f8(sp, p, p, None, p, p, p, p, p, p, 1, 0, None, p, p, 0, 0, p, ws, None) == -1  # sx
+    assert f8(sp, p, p, p, p, None, p, p, p, p, 1, 0, None, p, p, 0, 0, p, ws, None) == -1  # X
+    assert f8(sp, p, p, p + 2, p, p, p, p, p, p, 1, 0, None, p, p, 0, 0, p, ws, None) == -2
+    assert f8(sp, p + 8, p, p, p, p, p, p, p, p, 1, 0, None, p, p, 0, 0, p, ws, None) == -2
+    assert f8(sp, p, p, p, p, p, p, p, p, p, 1, 0, None, p, p, 0, 0, p, ws - 1, None) == -3
+    # 8-bit gradients need the cap as exp reference: no softcap (cap 0) or cap > 32 is refused
+    for cap in (0.0, 40.0):
+        sc = flce.make_shape(8, 64, 128, 100, cap)
+        assert f8(ctypes.byref(sc), p, p, p, p, None, None, p, p, p, 1, 1, None, p, p, 0, 0, p,
+                  flce.workspace_bytes(sc, True), None) == -1
     s48 = flce.make_shape(8, 72, 128, 100)          # d % 16 != 0: e4m3 rows not 16-byte
-    assert f8(ctypes.byref(s48), p, p, p, p, p, p, p, p, p, 0, None, None, None, 0, 0, p,
+    assert f8(ctypes.byref(s48), p, p, p, p, p, p, p, p, p, 0, 0, None, None, None, 0, 0, p,
               1 << 30, None) == -2
     dp = L.flce_forward_dp
     # X, W, t, nv_total, loss, lse, want_grads, g, dX, dW, dW_dtype, acc, ws, ws_bytes, stream

@@ -1,11 +1,13 @@
 """GPU parity of the FP8 path: logits from e4m3 operands with tensorwise scales
-(tcgen05 kind::f8f6f4), gradient contractions with the bf16 copies.
+(tcgen05 kind::f8f6f4); gradient contractions with the bf16 copies, or (grad_fp8) from an e5m2
+gradient and the e4m3 operands.
 
 * The device quantiser matches the reference encoder bit for bit (codes and scale).
 * Kernel error: against the fp64 oracle evaluated on the dequantised e4m3 values for the
-  logits and on the bf16 copies for the gradient products, with the ordinary parity bar.
+  logits and on the bf16 copies for the gradient products (or, with grad_fp8, the oracle's
+  e5m2 gradient codes times the dequantised operands), with the ordinary parity bar.
 * Quantisation error: against the all-bf16 oracle, reported and bounded loosely (three
-  mantissa bits per operand).
+  mantissa bits per logits operand, two per gradient code).
 """
 import numpy as np
 import pytest
@@ -32,16 +34,18 @@ def _rel(got, ref):
     return float(np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-300))
 
 
-def _run_fp8(inp, chunk_rows=0, want_grads=True):
+def _run_fp8(inp, chunk_rows=0, want_grads=True, grad_fp8=False, **kw):
     import torch
     import lm_head_linear_gemm_b200 as flce
     c = inp["cfg"]
     sx = torch.tensor(float(inp["sX"]), dtype=torch.float32, device="cuda")
     sw = torch.tensor(float(inp["sW"]), dtype=torch.float32, device="cuda")
-    loss, lse, dX, dW, ws = flce.forward_fp8(_dev(inp["X8"]), _dev(inp["W8"]), sx, sw,
-                                             _dev(inp["X"]), _dev(inp["W"]), _dev(inp["targets"]),
-                                             c.Vreal, c.cap, c.ignore_index, want_grads,
-                                             chunk_rows=chunk_rows)
+    X = None if grad_fp8 else _dev(inp["X"])
+    W = None if grad_fp8 else _dev(inp["W"])
+    loss, lse, dX, dW, ws = flce.forward_fp8(_dev(inp["X8"]), _dev(inp["W8"]), sx, sw, X, W,
+                                             _dev(inp["targets"]), c.Vreal, c.cap,
+                                             c.ignore_index, want_grads, chunk_rows=chunk_rows,
+                                             grad_fp8=grad_fp8, **kw)
     torch.cuda.synchronize()
     status, nv = flce.read_status(ws)
     out = dict(loss=float(loss.item()), lse=lse.double().cpu().numpy(), status=status, n_valid=nv)
@@ -84,6 +88,45 @@ def test_fp8_against_dequantised_oracle(cuda_device):
         assert np.abs(got["dW"][c.Vreal:]).max() == 0.0
     stats = _run_fp8(inp, want_grads=False)
     assert abs(stats["loss"] - ref["loss"]) <= LOSS_TOL
+
+
+def _check(name, got, ref, tol=REL_L2):
+    r = _rel(got, ref)
+    assert r <= tol, f"{name}: relL2 {r:.3e}"
+    worst = np.abs(got - ref).max()
+    assert worst <= 0.05 * np.abs(ref).max(), f"{name}: max err {worst:.3e}"
+    return r
+
+
+def test_fp8_gradients_against_quantisation_aware_oracle(cuda_device):
+    """grad_fp8: e5m2 gradient codes times the e4m3 operands (kind::f8f6f4, e5m2 x e4m3), in one
+    chunk and in 256-row chunks, against the oracle's FP8 gradient products; the loss and lse
+    against the oracle on the dequantised operands.  Also accumulating with g = 0.5."""
+    import torch
+    inp = synth.make_fp8_inputs("small", N=640)        # pages' vocabulary, d = 1536
+    c = inp["cfg"]
+    Xq, Wq = _dequantised(inp)
+    t = inp["targets"]
+    f = oracle.forward(Xq, Wq, t, c.Vreal, c.cap, c.ignore_index)
+    rX, rW = oracle.backward_fp8(Xq, Wq, t, c.Vreal, c.cap, c.ignore_index)
+    for chunk in (0, 256):
+        got = _run_fp8(inp, chunk_rows=chunk, grad_fp8=True)
+        assert got["status"] == 0 and got["n_valid"] == f["n_valid"]
+        assert abs(got["loss"] - f["loss"]) <= LOSS_TOL
+        assert np.abs(got["lse"] - f["lse"]).max() <= LSE_TOL
+        _check("dX", got["dX"], rX)
+        _check("dW", got["dW"], rW)
+        assert np.abs(got["dW"][c.Vreal:]).max() == 0.0
+        assert np.abs(got["dX"][t == c.ignore_index]).max() == 0.0
+    R = torch.randn((c.Vpad, c.d), device="cuda", generator=torch.Generator("cuda").manual_seed(2))
+    acc = _run_fp8(inp, chunk_rows=256, grad_fp8=True, dW=R.clone(), accumulate_dW=True,
+                   grad_scale=0.5)
+    _check("dW accumulated, g = 0.5", acc["dW"] - R.double().cpu().numpy(), 0.5 * rW)
+    _check("dX g = 0.5", acc["dX"], 0.5 * rX)
+    bx, bw = oracle.backward(Xq, Wq, t, c.Vreal, c.cap, c.ignore_index,
+                             Xg=synth.bf16_to_f64(inp["X"]), Wg=synth.bf16_to_f64(inp["W"]))
+    print(f"fp8 gradients vs bf16-operand gradients: relL2 dX {_rel(got['dX'], bx):.2e}, "
+          f"dW {_rel(got['dW'], bw):.2e}")
 
 
 def test_fp8_quantisation_error_against_bf16_oracle(cuda_device):
@@ -138,3 +181,13 @@ def test_fp8_full_size_sampled(cuda_device):
           f"{np.abs(got['lse'][rows] - f['lse'][rows]).max():.2e}, relL2 dX "
           f"{_rel(got['dX'][rows], dz @ Wb):.2e}")
     assert e_lse <= 5e-2 and e_dx <= 0.2
+    # the same workload with the gradient contractions in FP8 (e5m2 x e4m3)
+    g8 = _run_fp8(inp, grad_fp8=True)
+    assert g8["status"] == 0 and g8["loss"] == got["loss"]
+    scale = 1.0 / (f["n_valid"] * oracle.E5M2_SCALE)
+    q = oracle.dlogits_e5m2(Xq[rows], Wq, t[rows], c.Vreal, c.cap, c.ignore_index)
+    _check("fp8 dX rows", g8["dX"][rows], scale * (q @ Wq))
+    ref_dW8 = oracle.dW_rows_fp8(Xq, Wq, t, f["lse"], vrows, c.Vreal, c.cap, c.ignore_index)
+    _check("fp8 dW rows", g8["dW"][vrows], ref_dW8)
+    print(f"fp8 gradients N=65536 vs bf16 oracle on {len(rows)} rows: relL2 dX "
+          f"{_rel(g8['dX'][rows], dz_b @ Wb):.2e}")

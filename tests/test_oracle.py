@@ -527,3 +527,12 @@ def test_fp8_gradients_close_to_exact():
     for got, ref in ((dX, rX), (dW, rW)):
         r = np.linalg.norm(got - ref) / np.linalg.norm(ref)
         assert 1e-4 < r < 0.1
+
+
+def test_fp8_dW_rows_match_the_full_fp8_backward():
+    X, W, t, Vr, cap = _fp8_case(N=120, seed=6)
+    _, dW = oracle.backward_fp8(X, W, t, Vr, cap, -1, g=0.5)
+    lse = oracle.forward(X, W, t, Vr, cap, -1)["lse"]
+    rows = np.array([0, 5, int(t[0]), Vr - 1, Vr, 63])
+    got = oracle.dW_rows_fp8(X, W, t, lse, rows, Vr, cap, -1, g=0.5)
+    np.testing.assert_allclose(got, dW[rows], rtol=1e-9, atol=1e-14)
