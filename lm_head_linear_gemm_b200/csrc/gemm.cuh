@@ -148,6 +148,8 @@ struct PairProblem {
   int wide;             // problem 0 only: 1 = wide tiles (see below)
   int l2_a, l2_b;       // L2 priority of the A / B operand reads (l2_policy: 0, 1 first, 2 last)
   int dyn;              // DYN_M / DYN_K: that extent is min(extent, *PairArgs::dyn)
+  int serpentine;       // 1: a pair's odd-numbered tiles walk K backwards, so the operand
+                        //    rows the previous wave read last (still in L2) are read first
 };
 
 enum : int { DYN_M = 1, DYN_K = 2 };
@@ -369,6 +371,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
           tile_of(i, prob, mb, nb, kbs);
           const int a_row = mb * C::BM + static_cast<int>(rank) * C::BM_CTA;
           const int b_row = nb * NSUB * C::BN + static_cast<int>(rank) * C::BN_CTA;
+          const bool rev = args.prob[prob].serpentine && (i & 1);
           for (int kb = 0; kb < kbs; ++kb) {
             // a wide k-block starts on an even slot, so stage + 1 is in the same ring phase
             if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, args.status, args.limit_ns)) {
@@ -390,7 +393,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
             const uint32_t bar = leader_full + 8u * stage;
 #pragma unroll
             for (int j = 0; j < C::KSUB; ++j) {
-              const int k0 = kb * C::KSLOT + j * C::BK;
+              const int k0 = (rev ? kbs - 1 - kb : kb) * C::KSLOT + j * C::BK;
               if (prob == 0) {
                 load_operand_pair<A0, C::BM_CTA, C::ELEM_BYTES>(sA + j * C::A_SUB, &tmA0, bar,
                                                                 a_row, k0, pol_a0);
