@@ -81,6 +81,11 @@ namespace {
 #ifndef FLCE_SERPENTINE
 #define FLCE_SERPENTINE 0
 #endif
+// dW tiles in groups of d-columns (all vocabulary tiles of one group before the next), so the
+// dW tiles running at one time read only that group's columns of Xs
+#ifndef FLCE_DW_GROUPS
+#define FLCE_DW_GROUPS 1
+#endif
 // dX in wide tiles (256 x 512 per SM pair, two accumulators sharing each staged A' k-block)
 #ifndef FLCE_DX_WIDE
 #define FLCE_DX_WIDE 1
@@ -515,7 +520,8 @@ int grad_chunk(const Ctx& c, int64_t row0, int rows, const __nv_bfloat16* X,
   rp.fp8 = c.grad_fp8;
   rp.X8 = c.grad_fp8 ? c.fp8.X8 + row0 * s->d : nullptr;
   rp.Xs8 = Xs8;
-  const int finish_warps = rows + (c.L.compact ? 64 : 0);
+  rp.ktail = c.grad_fp8 ? CfgG8::KSLOT : Cfg::KSLOT;
+  const int finish_warps = rows + (c.L.compact ? rp.ktail : 0);
   row_finish_kernel<<<(finish_warps + 7) / 8, 256, 0, c.st>>>(rp);
   FLCE_TRY(launch_ok());
 
@@ -544,7 +550,7 @@ int grad_chunk(const Ctx& c, int64_t row0, int rows, const __nv_bfloat16* X,
     const int dw32 = FLCE_EPI_SECTOR32 && aligned32(dWb) && (!c.dW_bf16 || (d % 16) == 0);
     DwParams wp{v1 - v0, d, accumulate, dw32, c.dW_bf16, dWb, gsc != nullptr ? gsc + 1 : nullptr};
     const PairProblem pdw{v1 - v0, d, rows, 0, 0, FLCE_L2_DW_A, FLCE_L2_DW_XS, dyn_w,
-                          FLCE_SERPENTINE};
+                          FLCE_SERPENTINE, FLCE_DW_GROUPS};
     CUtensorMap mA_mn_b = mA_mn;
     if (v0 > 0) {
       if (c.grad_fp8)

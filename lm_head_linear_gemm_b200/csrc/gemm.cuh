@@ -150,6 +150,9 @@ struct PairProblem {
   int dyn;              // DYN_M / DYN_K: that extent is min(extent, *PairArgs::dyn)
   int serpentine;       // 1: a pair's odd-numbered tiles walk K backwards, so the operand
                         //    rows the previous wave read last (still in L2) are read first
+  int n_groups;         // > 1 (tiles walking N fastest): the N blocks are taken in n_groups
+                        //    consecutive groups, all M blocks of one group before the next, so
+                        //    the tiles running at one time touch 1/n_groups of the B operand
 };
 
 enum : int { DYN_M = 1, DYN_K = 2 };
@@ -339,8 +342,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
       mb = t % mt;
       nb = t / mt;
     } else {
-      nb = t % nt;
-      mb = t / nt;
+      const int ng = args.prob[prob].n_groups;
+      if (ng > 1 && nt % ng == 0) {
+        const int ntg = nt / ng, per = mt * ntg;
+        const int grp = t / per, u = t - grp * per;
+        nb = grp * ntg + u % ntg;
+        mb = u / ntg;
+      } else {
+        nb = t % nt;
+        mb = t / nt;
+      }
     }
   };
   // Every role walks this pair's tiles in order; the wide tiles (all of problem 0, when wide0)

@@ -169,10 +169,12 @@ struct RowFinishParams {
   __nv_bfloat16* Xs;            // [rows][d]
   // Compaction (want_grads with pos != null): r, Xs and the rows of A are indexed by the row's
   // position among the chunk's rows in the loss; rows not in the loss get a zero dX row here
-  // (the dX contraction skips them), and 64 extra warps zero the rows [cnt, cnt rounded up to
-  // 64) of A and Xs so that the dW contraction's last k-block adds nothing.
+  // (the dX contraction skips them), and `ktail` extra warps zero the rows [cnt, cnt rounded up
+  // to ktail) of A and Xs, ktail being the dW contraction's k-block (64 rows for bf16, 128 for
+  // 8-bit operands), so that its last k-block adds nothing.
   const int* pos;               // [rows] position or -1
   const int* cnt;               // this chunk's number of rows in the loss
+  int ktail;                    // rows per k-block of the dW contraction (64 or 128)
   __nv_bfloat16* dX;            // [rows][d] this chunk's dX rows
   // 8-bit gradient operands (fp8 = 1, with compaction and the fixed reference): the row's
   // softmax gradient normalised by S and scaled by 2^15, q_j = e5m2(A'_j / S * 2^15), replaces
@@ -250,10 +252,10 @@ __global__ void __launch_bounds__(256) row_finish_kernel(const RowFinishParams p
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (warp >= p.rows) {
-    if (p.want_grads && p.pos != nullptr && warp < p.rows + 64) {
+    if (p.want_grads && p.pos != nullptr && warp < p.rows + p.ktail) {
       const int m = *p.cnt;
       const int q = m + (warp - p.rows);
-      if (q < ((m + 63) & ~63) && q < p.rows) {
+      if (q < (m + p.ktail - 1) / p.ktail * p.ktail && q < p.rows) {
         zero_row_bf16(p.A + static_cast<size_t>(q) * p.Vpad, p.Vpad, lane);
         if (p.fp8)
           zero_row_bf16(reinterpret_cast<__nv_bfloat16*>(p.Xs8 + static_cast<size_t>(q) * p.d),
