@@ -1,6 +1,7 @@
 """Build the in-tree C-ABI library ``libflce.so`` for sm_100a with nvcc.
 
     python -m lm_head_linear_gemm_b200.build [--verbose-ptxas]
+    FLCE_BUILD_DEFINES="-DFLCE_DW_GROUPS=2" python -m lm_head_linear_gemm_b200.build --force
 
 The library is written next to this file so that it travels with the source tree;
 nothing is installed into site-packages.
@@ -39,6 +40,8 @@ def nvcc_flags(verbose_ptxas: bool = False) -> list[str]:
     ]
     if verbose_ptxas:
         flags += ["-Xptxas", "-v"]
+    # build-time tuning constants of flce_api.cu (e.g. "-DFLCE_DW_GROUPS=2"), for measurements
+    flags += os.environ.get("FLCE_BUILD_DEFINES", "").split()
     return flags
 
 

@@ -77,6 +77,10 @@ namespace {
 #ifndef FLCE_COMPACT
 #define FLCE_COMPACT 1
 #endif
+// padding of the gradient operand's rows (elements; a multiple of 16): the row stride of A'
+#ifndef FLCE_A_PAD
+#define FLCE_A_PAD 0
+#endif
 // gradient tiles alternate their K direction from one tile of a pair to the next
 #ifndef FLCE_SERPENTINE
 #define FLCE_SERPENTINE 0
@@ -127,6 +131,7 @@ size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 struct Layout {
   int64_t chunk;      // rows per pass
+  int64_t a_ld;       // row stride of A' (elements)
   int n_chunks;
   int n_slabs;        // per-row partial slots of the logits pass
   bool fixed_ref;
@@ -152,6 +157,7 @@ Layout make_layout(const flce_shape* s, int want_grads) {
   if (nc > N) nc = N;
   if (nc < 1) nc = 1;
   L.chunk = nc;
+  L.a_ld = s->Vpad + FLCE_A_PAD;
   L.n_chunks = static_cast<int>(N > 0 ? (N + nc - 1) / nc : 1);
   L.fixed_ref = s->cap > 0.f && s->cap <= kFixedRefMaxCap;
   L.compact = want_grads && FLCE_COMPACT;
@@ -173,7 +179,7 @@ Layout make_layout(const flce_shape* s, int want_grads) {
   L.partial = take(static_cast<size_t>(nc) * L.n_slabs * 2 * sizeof(float));
   if (want_grads) {
     L.r = take(static_cast<size_t>(nc) * sizeof(float));
-    L.A = take(static_cast<size_t>(nc) * s->Vpad * sizeof(__nv_bfloat16));
+    L.A = take(static_cast<size_t>(nc) * L.a_ld * sizeof(__nv_bfloat16));
     L.Xs = take(static_cast<size_t>(nc) * s->d * sizeof(__nv_bfloat16));
     if (L.compact) {
       L.pos = take(n * sizeof(int));
@@ -423,7 +429,7 @@ int launch_logits(const Ctx& c, int64_t row0, int rows, const __nv_bfloat16* X,
     q.e_t = lp.e_t + r0;
     // compacted rows index A from the chunk's first row: only pos moves with the launch
     q.pos = lp.pos != nullptr ? lp.pos + r0 : nullptr;
-    q.A = lp.A != nullptr && lp.pos == nullptr ? lp.A + static_cast<size_t>(r0) * lp.Vpad : lp.A;
+    q.A = lp.A != nullptr && lp.pos == nullptr ? lp.A + static_cast<size_t>(r0) * lp.a_ld : lp.A;
     FLCE_TRY(launch_logits_rows(c, row0 + r0, rr, X, W, q));
   }
   return FLCE_OK;
@@ -456,14 +462,16 @@ int grad_chunk(const Ctx& c, int64_t row0, int rows, const __nv_bfloat16* X,
   if (c.grad_fp8) {
     // e5m2 gradient rows in place of the bf16 rows of A (row stride 2 Vpad bytes), e4m3 W8 and
     // compacted X8 rows; boxes of 128 bytes x 128 rows
-    FLCE_TRY(make_map(&mA_k, Abuf, Vpad, rows, 2 * static_cast<uint64_t>(Vpad), CfgG8::BM_CTA, 1));
+    FLCE_TRY(make_map(&mA_k, Abuf, Vpad, rows, 2 * static_cast<uint64_t>(c.L.a_ld),
+                      CfgG8::BM_CTA, 1));
     FLCE_TRY(make_map(&mW_mn, c.fp8.W8, d, Vpad, d, CfgG8::BK, 1));
-    FLCE_TRY(make_map(&mA_mn, Abuf, Vpad, rows, 2 * static_cast<uint64_t>(Vpad), CfgG8::BK, 1));
+    FLCE_TRY(make_map(&mA_mn, Abuf, Vpad, rows, 2 * static_cast<uint64_t>(c.L.a_ld), CfgG8::BK,
+                      1));
     FLCE_TRY(make_map(&mXs_mn, Xs8, d, rows, d, CfgG8::BK, 1));
   } else {
-    FLCE_TRY(make_map(&mA_k, Abuf, Vpad, rows, Vpad, Cfg::BM_CTA));
+    FLCE_TRY(make_map(&mA_k, Abuf, Vpad, rows, c.L.a_ld, Cfg::BM_CTA));
     FLCE_TRY(make_map(&mW_mn, W, d, Vpad, d, 64));
-    FLCE_TRY(make_map(&mA_mn, Abuf, Vpad, rows, Vpad, 64));
+    FLCE_TRY(make_map(&mA_mn, Abuf, Vpad, rows, c.L.a_ld, 64));
     FLCE_TRY(make_map(&mXs_mn, Xs, d, rows, d, 64));
   }
 
@@ -471,6 +479,7 @@ int grad_chunk(const Ctx& c, int64_t row0, int rows, const __nv_bfloat16* X,
   lp.rows = rows;
   lp.Vreal = static_cast<int>(s->Vreal);
   lp.Vpad = Vpad;
+  lp.a_ld = static_cast<int>(c.L.a_ld);
   lp.mode = mode;
   lp.fixed_ref = c.L.fixed_ref ? 1 : 0;
   lp.cap = s->cap;
@@ -493,6 +502,7 @@ int grad_chunk(const Ctx& c, int64_t row0, int rows, const __nv_bfloat16* X,
   rp.rows = rows;
   rp.d = d;
   rp.Vpad = Vpad;
+  rp.a_ld = lp.a_ld;
   rp.n_slabs = c.L.n_slabs;
   rp.cap = s->cap;
   rp.fixed_ref = lp.fixed_ref;
@@ -555,9 +565,9 @@ int grad_chunk(const Ctx& c, int64_t row0, int rows, const __nv_bfloat16* X,
     if (v0 > 0) {
       if (c.grad_fp8)
         FLCE_TRY(make_map(&mA_mn_b, reinterpret_cast<uint8_t*>(Abuf) + v0, Vpad - v0, rows,
-                          2 * static_cast<uint64_t>(Vpad), CfgG8::BK, 1));
+                          2 * static_cast<uint64_t>(c.L.a_ld), CfgG8::BK, 1));
       else
-        FLCE_TRY(make_map(&mA_mn_b, Abuf + v0, Vpad - v0, rows, Vpad, 64));
+        FLCE_TRY(make_map(&mA_mn_b, Abuf + v0, Vpad - v0, rows, c.L.a_ld, 64));
     }
     if (v1 > v0 || b + 1 == nb) {
       if (c.grad_fp8)
@@ -592,6 +602,7 @@ int stats_pass(const Ctx& c, const __nv_bfloat16* X, const __nv_bfloat16* W, flo
     lp.rows = rows;
     lp.Vreal = static_cast<int>(s->Vreal);
     lp.Vpad = Vpad;
+    lp.a_ld = Vpad;
     lp.mode = LOGITS_STATS;
     lp.fixed_ref = c.L.fixed_ref ? 1 : 0;
     lp.cap = s->cap;
@@ -608,6 +619,7 @@ int stats_pass(const Ctx& c, const __nv_bfloat16* X, const __nv_bfloat16* W, flo
     rp.rows = rows;
     rp.d = d;
     rp.Vpad = Vpad;
+    rp.a_ld = Vpad;
     rp.n_slabs = c.L.n_slabs;
     rp.cap = s->cap;
     rp.fixed_ref = lp.fixed_ref;

@@ -696,6 +696,7 @@ enum LogitsMode : int { LOGITS_STATS = 0, LOGITS_FUSED = 1, LOGITS_RECOMPUTE = 2
 struct LogitsParams {
   int rows;                  // rows of this pass; rows >= rows are padding of the last tile
   int Vreal, Vpad;
+  int a_ld;                  // row stride of A (elements, >= Vpad)
   int mode;                  // LogitsMode
   int fixed_ref;             // 1: exp reference is cap (requires cap > 0); 0: online / lse
   float cap;                 // > 0: softcap value; <= 0: no softcap
@@ -739,7 +740,7 @@ struct LogitsEpi {
     __nv_bfloat16* arow = nullptr;
     if (write_a && row_ok) {
       const int at = p.pos != nullptr ? __ldg(p.pos + row) : row;
-      if (at >= 0) arow = p.A + static_cast<size_t>(at) * p.Vpad;
+      if (at >= 0) arow = p.A + static_cast<size_t>(at) * p.a_ld;
     }
 #pragma unroll 1
     for (int c = 0; c < NCOLS / 32; ++c) {
@@ -830,7 +831,7 @@ struct LogitsEpi {
         uint32_t packed[16];
 #pragma unroll
         for (int k = 0; k < 16; ++k) packed[k] = pack_bf16x2(v[2 * k], v[2 * k + 1]);
-        if ((p.Vpad & 15) == 0) {
+        if ((p.a_ld & 15) == 0) {
           // rows start on 32-byte boundaries: two full-sector stores per 32 columns
 #pragma unroll
           for (int g = 0; g < 2; ++g) {

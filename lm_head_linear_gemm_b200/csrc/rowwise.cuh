@@ -147,6 +147,7 @@ __global__ void __launch_bounds__(256) prep_total_kernel(const int* __restrict__
 struct RowFinishParams {
   int rows;                     // rows of this pass
   int d, Vpad;
+  int a_ld;                     // row stride of A (elements, >= Vpad)
   int n_slabs;
   float cap;                    // softcap value (the exp reference when fixed_ref)
   int fixed_ref;                // 1: partials are sum-exp against cap; 0: (max, sum-exp) pairs
@@ -196,8 +197,8 @@ __device__ __forceinline__ void zero_row_bf16(__nv_bfloat16* row, int n, int lan
 template <class P>
 __device__ __forceinline__ void encode_row_e5m2(const P& p, int row, int at, int t, float S) {
   const int lane = threadIdx.x & 31;
-  const __nv_bfloat16* arow = p.A + static_cast<size_t>(at) * p.Vpad;
-  uint8_t* qrow = reinterpret_cast<uint8_t*>(p.A + static_cast<size_t>(at) * p.Vpad);
+  const __nv_bfloat16* arow = p.A + static_cast<size_t>(at) * p.a_ld;
+  uint8_t* qrow = reinterpret_cast<uint8_t*>(p.A + static_cast<size_t>(at) * p.a_ld);
   // the target element as the bf16 path stores it, (1 - tanh^2)(e_t - S) rounded to bf16
   const float pv = __bfloat162float(__float2bfloat16_rn(p.der_t[row] * (p.e_t[row] - S)));
   const float f = 32768.0f / S;
@@ -256,7 +257,7 @@ __global__ void __launch_bounds__(256) row_finish_kernel(const RowFinishParams p
       const int m = *p.cnt;
       const int q = m + (warp - p.rows);
       if (q < (m + p.ktail - 1) / p.ktail * p.ktail && q < p.rows) {
-        zero_row_bf16(p.A + static_cast<size_t>(q) * p.Vpad, p.Vpad, lane);
+        zero_row_bf16(p.A + static_cast<size_t>(q) * p.a_ld, p.Vpad, lane);
         if (p.fp8)
           zero_row_bf16(reinterpret_cast<__nv_bfloat16*>(p.Xs8 + static_cast<size_t>(q) * p.d),
                         p.d / 2, lane);
@@ -326,7 +327,7 @@ __global__ void __launch_bounds__(256) row_finish_kernel(const RowFinishParams p
     p.r[at] = r;
     if (valid) {
       const float patched = p.der_t[row] * (p.e_t[row] - S);
-      p.A[static_cast<size_t>(at) * p.Vpad + t] = __float2bfloat16_rn(patched);
+      p.A[static_cast<size_t>(at) * p.a_ld + t] = __float2bfloat16_rn(patched);
     }
   }
   const __nv_bfloat16* xr = p.X + static_cast<size_t>(row) * p.d;
