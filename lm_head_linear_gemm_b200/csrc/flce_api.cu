@@ -81,7 +81,9 @@ namespace {
 #ifndef FLCE_A_PAD
 #define FLCE_A_PAD 0
 #endif
-// gradient tiles alternate their K direction from one tile of a pair to the next
+// dW tiles alternate their K direction from one wave to the next (the dX tiles keep theirs, so
+// that a row's dX does not depend on the tile it lands in); measured within box-to-box noise,
+// so off by default
 #ifndef FLCE_SERPENTINE
 #define FLCE_SERPENTINE 0
 #endif
@@ -543,8 +545,7 @@ int grad_chunk(const Ctx& c, int64_t row0, int rows, const __nv_bfloat16* X,
   DxParams xp{rows, d, dx32, r, dXc, c.L.compact ? c.at<int>(c.L.orig) + row0 : nullptr, cnt,
               gsc};
   const int dyn_x = c.L.compact ? DYN_M : 0, dyn_w = c.L.compact ? DYN_K : 0;
-  const PairProblem pdx{rows, d, Vpad, 0, FLCE_DX_WIDE, FLCE_L2_DX_A, FLCE_L2_DX_W, dyn_x,
-                        FLCE_SERPENTINE};
+  const PairProblem pdx{rows, d, Vpad, 0, FLCE_DX_WIDE, FLCE_L2_DX_A, FLCE_L2_DX_W, dyn_x};
   const PairProblem none{0, 0, 0, 0, 0, 0, 0, 0};
   const int nb = buckets != nullptr ? buckets->n : 1;
   const int vtiles = (Vpad + Cfg::BM - 1) / Cfg::BM;
@@ -560,7 +561,7 @@ int grad_chunk(const Ctx& c, int64_t row0, int rows, const __nv_bfloat16* X,
     const int dw32 = FLCE_EPI_SECTOR32 && aligned32(dWb) && (!c.dW_bf16 || (d % 16) == 0);
     DwParams wp{v1 - v0, d, accumulate, dw32, c.dW_bf16, dWb, gsc != nullptr ? gsc + 1 : nullptr};
     const PairProblem pdw{v1 - v0, d, rows, 0, 0, FLCE_L2_DW_A, FLCE_L2_DW_XS, dyn_w,
-                          FLCE_SERPENTINE, FLCE_DW_GROUPS};
+                          FLCE_SERPENTINE, v0 / Cfg::BM, FLCE_DW_GROUPS};
     CUtensorMap mA_mn_b = mA_mn;
     if (v0 > 0) {
       if (c.grad_fp8)

@@ -148,8 +148,12 @@ struct PairProblem {
   int wide;             // problem 0 only: 1 = wide tiles (see below)
   int l2_a, l2_b;       // L2 priority of the A / B operand reads (l2_policy: 0, 1 first, 2 last)
   int dyn;              // DYN_M / DYN_K: that extent is min(extent, *PairArgs::dyn)
-  int serpentine;       // 1: a pair's odd-numbered tiles walk K backwards, so the operand
-                        //    rows the previous wave read last (still in L2) are read first
+  int serpentine;       // 1: tiles of every other wave walk K backwards, so the operand rows
+                        //    the previous wave read last (still in L2) are read first.  The
+                        //    wave is (m_off + m block) * N tiles + n block over the pair count:
+                        //    a property of the tile, so a tile's arithmetic does not depend on
+                        //    the launch it runs in (vocabulary buckets give identical results)
+  int m_off;            // M tiles before this problem's first (a launch over part of M)
   int n_groups;         // > 1 (tiles walking N fastest): the N blocks are taken in n_groups
                         //    consecutive groups, all M blocks of one group before the next, so
                         //    the tiles running at one time touch 1/n_groups of the B operand
@@ -382,7 +386,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(C::THREADS, 1)
           tile_of(i, prob, mb, nb, kbs);
           const int a_row = mb * C::BM + static_cast<int>(rank) * C::BM_CTA;
           const int b_row = nb * NSUB * C::BN + static_cast<int>(rank) * C::BN_CTA;
-          const bool rev = args.prob[prob].serpentine && (i & 1);
+          const int nt_all = prob == 0 ? n_tiles0 : n_tiles1;
+          const bool rev = args.prob[prob].serpentine &&
+                           ((((args.prob[prob].m_off + mb) * nt_all + nb * NSUB) / npairs) & 1);
           for (int kb = 0; kb < kbs; ++kb) {
             // a wide k-block starts on an even slot, so stage + 1 is in the same ring phase
             if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, args.status, args.limit_ns)) {
