@@ -282,7 +282,9 @@ typedef struct {
   int64_t launches_total;      /* all kernels launched while recording */
   int64_t gemm_launches[3];    /* contraction launches by kind */
   double gemm_ms[3];           /* summed event-timed durations by kind, milliseconds */
-  double gemm_flop[3];         /* 2*M*N*K summed over those launches */
+  double gemm_flop[3];         /* 2*M*N*K of the launched extents, summed over those launches;
+                                  the gradient launches run over the rows in the loss only, so
+                                  with ignored rows they compute less than this */
 } flce_kernel_stats;
 
 int flce_instrument(int enable);
