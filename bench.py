@@ -9,8 +9,11 @@ scalar equal to 1, the autograd default for a scalar loss), on one batch of the
 3.8B model's head: N = 16384 tokens (batch 16 x context 1024), d = 3072,
 V = 50257 -> 50304, softcap 15.  Credited work: 6*N*d*Vpad FLOP per step.
 
-Multi-GPU (torchrun): every rank runs an independent replica on its own batch
-(weak scaling, no collective in the data path); the time is the max over ranks.
+Multi-GPU (torchrun): every rank holds W and its own batch (weak scaling) and runs the
+data-parallel step -- loss normalised by the count of rows in the loss over all ranks, dW
+accumulated over --accum-steps micro-batches with each loss divided by their number, and
+all-reduced after the last in --buckets vocabulary buckets that overlap the last gradient
+launches; --no-allreduce gives independent replicas.  The time is the max over ranks.
 ``--impl reference`` times the fp64 CPU oracle on a bounded sample of rows of the
 same workload (rank 0 only).
 """
