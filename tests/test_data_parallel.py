@@ -9,7 +9,8 @@ split is uneven, when one rank has no row in the loss, and over two accumulated 
 with the upstream gradient 1/2 passed to the forward.
 """
 import os
-import socket
+import shutil
+import tempfile
 
 import numpy as np
 import pytest
@@ -65,9 +66,10 @@ def _data(seed=0, N=30):
     return X, W, t
 
 
-def _worker(rank, world, port, split, all_ignored_rank, buckets, micro, q):
-    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
-    dist.init_process_group("gloo", rank=rank, world_size=world)
+def _worker(rank, world, store_path, split, all_ignored_rank, buckets, micro, q):
+    # a file rendezvous: no port that another process could take between its choice and use
+    dist.init_process_group("gloo", init_method=f"file://{store_path}", rank=rank,
+                            world_size=world)
     try:
         from lm_head_linear_gemm_b200.data_parallel import dp_step
         X, W, t = _data()
@@ -101,20 +103,13 @@ def _worker(rank, world, port, split, all_ignored_rank, buckets, micro, q):
         dist.destroy_process_group()
 
 
-def _free_port():
-    s = socket.socket()
-    s.bind(("127.0.0.1", 0))
-    p = s.getsockname()[1]
-    s.close()
-    return p
-
-
 def _run(split, all_ignored_rank, buckets, micro):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
-    port = _free_port()
+    store_dir = tempfile.mkdtemp(prefix="flce_gloo_")
+    store_path = os.path.join(store_dir, "rendezvous")
     procs = [ctx.Process(target=_worker,
-                         args=(r, 2, port, split, all_ignored_rank, buckets, micro, q))
+                         args=(r, 2, store_path, split, all_ignored_rank, buckets, micro, q))
              for r in range(2)]
     for p in procs:
         p.start()
@@ -125,6 +120,7 @@ def _run(split, all_ignored_rank, buckets, micro):
     for p in procs:
         p.join(timeout=60)
         assert p.exitcode == 0
+    shutil.rmtree(store_dir, ignore_errors=True)
     return res
 
 
