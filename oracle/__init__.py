@@ -51,7 +51,7 @@ import numpy as np
 __all__ = [
     "logits", "softcap", "softcap_derivative", "valid_rows", "row_forward", "forward",
     "row_dlogits", "backward", "forward_backward", "dW_rows", "rmsnorm_forward",
-    "rmsnorm_backward", "round_bf16", "encode_e5m2", "E5M2_SCALE", "dlogits_e5m2",
+    "rmsnorm_backward", "rmsnorm_head", "round_bf16", "encode_e5m2", "E5M2_SCALE", "dlogits_e5m2",
     "backward_fp8", "dW_rows_fp8",
 ]
 
@@ -230,6 +230,22 @@ def rmsnorm_backward(H, gamma, dX, eps: float = 1e-6):
     g = dX * gamma[None, :]
     dH = rstd[:, None] * (g - xh * np.mean(g * xh, axis=1, keepdims=True))
     return dH, np.sum(dX * xh, axis=0)
+
+
+def rmsnorm_head(H, gamma, W, t, Vreal: int, cap: float, ignore_index: int, eps: float = 1e-6,
+                 g: float = 1.0, round_x: bool = True, block_rows: int = 1024):
+    """The final RMSNorm and the head as one training step: x = rmsnorm(h) -- rounded to bf16
+    when ``round_x`` (the head reads the normalised hidden in the model's activation type) --,
+    the loss and gradients of the head on x, then the chain rule through the RMSNorm with the
+    exact (unrounded) normalised rows.  Returns the ``forward_backward`` dict with ``X`` (the
+    head's input), ``dH`` and ``dgamma`` added."""
+    x, _ = rmsnorm_forward(H, gamma, eps)
+    if round_x:
+        x = round_bf16(x)
+    f = forward_backward(x, W, t, Vreal, cap, ignore_index, g, block_rows)
+    dH, dgamma = rmsnorm_backward(H, gamma, f["dX"], eps)
+    f.update(X=x, dH=dH, dgamma=dgamma)
+    return f
 
 
 # ------------------------------------------------------------------------ FP8 gradient products

@@ -426,6 +426,104 @@ def test_rmsnorm_then_loss_finite_differences():
     assert np.linalg.norm(num_dg - dg) <= 1e-6 * np.linalg.norm(dg)
 
 
+def _rms_case(seed=9, N=6, d=8, Vr=20, Vp=24):
+    rng = np.random.default_rng(seed)
+    H = rng.standard_normal((N, d)) * 2.0
+    gamma = 1.0 + 0.3 * rng.standard_normal(d)
+    W = rng.standard_normal((Vp, d)) * 1.5
+    t = rng.integers(0, Vr, N)
+    t[2] = -1
+    return H, gamma, W, t, Vr
+
+
+def test_rmsnorm_head_finite_differences():
+    """rmsnorm_head (unrounded x): dH, dgamma and dW of g * loss against central differences of
+    g * loss(rmsnorm(h) W^T) in h, gamma and W; the loss and lse against the plain forward."""
+    H, gamma, W, t, Vr = _rms_case()
+    g = 0.75
+    f = oracle.rmsnorm_head(H, gamma, W, t, Vr, 15.0, -1, g=g, round_x=False)
+
+    def L(H_, g_, W_):
+        x, _ = oracle.rmsnorm_forward(H_, g_)
+        return g * oracle.forward(x, W_, t, Vr, 15.0, -1)["loss"]
+
+    x, _ = oracle.rmsnorm_forward(H, gamma)
+    plain = oracle.forward(x, W, t, Vr, 15.0, -1)
+    assert f["loss"] == plain["loss"]
+    np.testing.assert_array_equal(f["lse"], plain["lse"])
+    h = 1e-6
+
+    def numeric(arr, fn):
+        out = np.zeros_like(arr)
+        for idx in np.ndindex(*arr.shape):
+            ap, am = arr.copy(), arr.copy()
+            ap[idx] += h
+            am[idx] -= h
+            out[idx] = (fn(ap) - fn(am)) / (2 * h)
+        return out
+
+    num_dH = numeric(H, lambda a: L(a, gamma, W))
+    num_dg = numeric(gamma, lambda a: L(H, a, W))
+    num_dW = numeric(W, lambda a: L(H, gamma, a))
+    for got, num in ((f["dH"], num_dH), (f["dgamma"], num_dg), (f["dW"], num_dW)):
+        assert np.linalg.norm(num - got) <= 1e-6 * np.linalg.norm(got)
+
+
+def test_rmsnorm_head_rounds_the_head_input_only():
+    """round_x rounds x to bf16 for the head; the chain rule still uses the exact rows."""
+    H, gamma, W, t, Vr = _rms_case(seed=10)
+    f = oracle.rmsnorm_head(H, gamma, W, t, Vr, 15.0, -1)
+    x, _ = oracle.rmsnorm_forward(H, gamma)
+    xr = oracle.round_bf16(x)
+    np.testing.assert_array_equal(f["X"], xr)
+    assert np.any(xr != x)
+    head = oracle.forward_backward(xr, W, t, Vr, 15.0, -1)
+    np.testing.assert_array_equal(f["dX"], head["dX"])
+    dH, dg = oracle.rmsnorm_backward(H, gamma, head["dX"])
+    np.testing.assert_array_equal(f["dH"], dH)
+    np.testing.assert_array_equal(f["dgamma"], dg)
+
+
+def test_rmsnorm_fold_row_dot_identity():
+    """The RMSNorm backward needs c_i = mean_k x_ik dX_ik per row.  Since dX_i = sum_j dz_ij W_j
+    and z_ij = x_i . W_j, c_i = (1/d) sum_j dz_ij z_ij: a sum over the logits row, formed where
+    dz and z are both at hand.  Checked here on the oracle's own dz and z, and dH rebuilt from it
+    equals the chain rule; and on the fixed-reference pieces the logits pass produces,
+    A_ij = exp(s_ij - cap)(1 - tanh^2) with S_i = sum_j exp(s_ij - cap):
+    sum_j dz_ij z_ij = g/(Nv S_i) (sum_j A_ij z_ij - S_i (1 - tanh^2_t) z_t)."""
+    H, gamma, W, t, Vr = _rms_case(seed=11, N=7, d=16, Vr=40, Vp=48)
+    cap, g = 15.0, 0.5
+    d = H.shape[1]
+    x, rstd = oracle.rmsnorm_forward(H, gamma)
+    f = oracle.forward(x, W, t, Vr, cap, -1)
+    nv = f["n_valid"]
+    dz = oracle.row_dlogits(x, W, t, f["lse"], Vr, cap, -1, nv, g)
+    z = oracle.logits(x, W)
+    dX = dz @ W
+    c_k = np.sum(x * dX, axis=1) / d
+    c_j = np.sum(dz * z, axis=1) / d
+    np.testing.assert_allclose(c_j, c_k, rtol=1e-12, atol=1e-15)
+    xh = H * rstd[:, None]
+    dH = rstd[:, None] * (dX * gamma[None, :] - xh * c_j[:, None])
+    ref_dH, _ = oracle.rmsnorm_backward(H, gamma, dX)
+    np.testing.assert_allclose(dH, ref_dH, rtol=1e-12, atol=1e-15)
+    # the same sum from the fixed-reference pieces
+    s = oracle.softcap(z, cap)
+    der = oracle.softcap_derivative(z, cap)
+    e = np.exp(s - cap)
+    e[:, Vr:] = 0.0
+    S = e.sum(axis=1)
+    A = e * der
+    valid, _ = oracle.valid_rows(t, Vr, -1)
+    for i in range(len(t)):
+        if not valid[i]:
+            assert c_j[i] == 0.0
+            continue
+        ti = t[i]
+        folded = g / (nv * S[i]) * (np.sum(A[i] * z[i]) - S[i] * der[i, ti] * z[i, ti])
+        assert abs(folded - c_j[i] * d) <= 1e-12 * max(1.0, abs(folded))
+
+
 # --------------------------------------------------------------------------- randomised library check
 def test_against_torch_on_random_shapes():
     """The library special case (torch cross_entropy + autograd in fp64, through torch.tanh
