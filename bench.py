@@ -729,44 +729,98 @@ def compare_cublas(args):
 
 
 def norm_bench(args):
-    """RMSNorm forward / backward at N x d of the workload; HBM-bound, so achieved GB/s of the
-    algorithmic bytes against the measured copy bandwidth."""
+    """The model's final RMSNorm on the workload's shape, two ways:
+    * its row kernels alone (forward, backward), HBM-bound: achieved GB/s of the algorithmic
+      bytes against the measured copy bandwidth;
+    * a training step of the norm and the head (loss and the gradients of H, gamma and W, on the
+      workload's W and targets): the head alone (for reference), the norm's row kernels around
+      the head, and one flce_forward_rmsnorm call, whose dX epilogue writes dH directly (the
+      norm's backward folded into the dX contraction).  CUDA-event timed, interleaved."""
     import torch
     import lm_head_linear_gemm_b200 as flce
     import synth
-    c = synth.CONFIGS[args.config]
-    N, d = args.rows or c.N, c.d
+    cfg = synth.CONFIGS[args.config]
+    inp = synth.make_rmsnorm_inputs(cfg, N=args.rows or None)
+    c = inp["cfg"]
+    N, d = c.N, c.d
     dev = torch.device("cuda", 0)
+
+    def D(a):
+        import numpy as np
+        a = np.ascontiguousarray(a)
+        if a.dtype == np.uint16:
+            return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)
+        return torch.from_numpy(a).to(dev)
+
+    H, gamma, W, t = D(inp["H"]), D(inp["gamma"]), D(inp["W"]), D(inp["targets"])
     g = torch.Generator(device=dev).manual_seed(0)
-    H = (torch.randn(N, d, device=dev, generator=g) * 2).to(torch.bfloat16)
-    gamma = (1 + 0.1 * torch.randn(d, device=dev, generator=g)).to(torch.bfloat16)
-    dX = (torch.randn(N, d, device=dev, generator=g) * 1e-3).to(torch.bfloat16)
+    dXr = (torch.randn(N, d, device=dev, generator=g) * 1e-3).to(torch.bfloat16)
     X, rstd = flce.rmsnorm_forward(H, gamma)
-    dH, dgamma = flce.rmsnorm_backward(H, gamma, rstd, dX)
+    dH, dgamma = flce.rmsnorm_backward(H, gamma, rstd, dXr)
     peaks, src = load_peaks()
     hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
-    out = {}
-    for name, fn, nbytes in (
-            ("forward", lambda: flce.rmsnorm_forward(H, gamma, X=X, rstd=rstd), 4 * N * d + 4 * N),
-            ("backward", lambda: flce.rmsnorm_backward(H, gamma, rstd, dX, dH=dH, dgamma=dgamma),
-             10 * N * d + 8 * N)):
-        for _ in range(5):
+
+    def timed(fn, reps):
+        for _ in range(3):
             fn()
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        reps = 50
         e0.record()
         for _ in range(reps):
             fn()
         e1.record()
         torch.cuda.synchronize()
-        ms = e0.elapsed_time(e1) / reps
+        return e0.elapsed_time(e1) / reps
+
+    out = {}
+    for name, fn, nbytes in (
+            ("forward", lambda: flce.rmsnorm_forward(H, gamma, X=X, rstd=rstd), 4 * N * d + 4 * N),
+            ("backward", lambda: flce.rmsnorm_backward(H, gamma, rstd, dXr, dH=dH, dgamma=dgamma),
+             10 * N * d + 8 * N)):
+        ms = timed(fn, 50)
         gbs = nbytes / (ms * 1e-3) / 1e9
         out[name] = {"ms": ms, "algorithmic_bytes": nbytes, "GB/s": gbs, "frac_of_hbm": gbs / hbm}
-    print(json.dumps({"rmsnorm": out, "N": N, "d": d, "hbm_peak_gbs": hbm, "peak_source": src,
+
+    # a training step of the norm and the head
+    g_one = torch.ones((), dtype=torch.float32, device=dev)
+    dX = torch.empty_like(H)
+    dW = torch.empty(W.shape, dtype=torch.float32, device=dev)
+    shape = flce.make_shape(N, d, c.Vpad, c.Vreal, c.cap, c.ignore_index, args.chunk_rows)
+    ws = flce.alloc_workspace(shape, True, dev)
+    import ctypes
+    ws_r = torch.empty(int(flce.lib().flce_workspace_bytes_rmsnorm(ctypes.byref(shape), 1)),
+                       dtype=torch.uint8, device=dev)
+
+    def head():
+        _, lse, _, _, _ = flce.forward(X, W, t, c.Vreal, c.cap, c.ignore_index, True, dX=dX,
+                                       dW=dW, workspace=ws, chunk_rows=args.chunk_rows)
+        flce.backward(X, W, t, lse, c.Vreal, c.cap, c.ignore_index, grad_out=g_one, dX=dX,
+                      dW=dW, grads_precomputed=True)
+
+    def separate():
+        flce.rmsnorm_forward(H, gamma, X=X, rstd=rstd)
+        head()
+        flce.rmsnorm_backward(H, gamma, rstd, dX, dH=dH, dgamma=dgamma)
+
+    def fused():
+        flce.forward_rmsnorm(H, gamma, W, t, c.Vreal, c.cap, c.ignore_index, 1e-6, True, dH=dH,
+                             dgamma=dgamma, dW=dW, workspace=ws_r, chunk_rows=args.chunk_rows)
+        flce.scale_grads_rmsnorm(g_one, dH, dgamma, dW, c.Vreal, c.cap, c.ignore_index)
+
+    steps = {}
+    for _ in range(2):
+        for name, fn in (("head alone", head), ("norm kernels around the head", separate),
+                         ("one call, norm backward folded into dX", fused)):
+            steps.setdefault(name, []).append(timed(fn, args.steps))
+    print(json.dumps({"rmsnorm": out, "N": N, "d": d, "Vpad": c.Vpad, "hbm_peak_gbs": hbm,
+                      "peak_source": src,
                       "bytes": "forward: read h, write x (2+2 B per element) + rstd; backward: "
                                "dH pass reads h, dX, writes dH (6 B), dgamma pass re-reads h, "
-                               "dX (4 B)"}), flush=True)
+                               "dX (4 B)",
+                      "step_ms": steps,
+                      "step": f"{c.name}: loss and the gradients of H, gamma and W; "
+                              f"{args.steps} steps per timing, two interleaved rounds"}),
+          flush=True)
     return 0
 
 

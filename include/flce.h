@@ -242,6 +242,38 @@ int flce_rmsnorm_backward(const void* H, const void* gamma, const float* rstd, c
                           void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * The final RMSNorm and the head as one training step (the write-ups' model: final RMSNorm,
+ * then the untied head and the softcapped loss).  H [N, d] bf16 holds the rows before the norm;
+ * the head reads x = h rstd gamma, rounded to bf16 (written to the workspace), and the call
+ * returns what flce_forward returns for that x, with dH and dgamma in place of dX:
+ *   dH = rstd (gamma . dX - xh c),  c_i = mean_k x_ik dX_ik,  dgamma = sum_i dX_i . xh_i,
+ * dX the gradient of g * loss with respect to x (never stored when 0 < cap <= 32) and
+ * xh = h rstd.  With 0 < cap <= 32 the backward of the norm is folded into the dX contraction:
+ * c_i equals (1/d) sum_j dz_ij z_ij, which the logits pass sums next to the softmax, so the dX
+ * epilogue writes dH rows directly and per 32 rows the column sums that make dgamma (summed in
+ * row-block order: deterministic).  Otherwise dX goes to the workspace and separate row
+ * kernels follow.
+ *   eps >= 0 (the write-ups' config: 1e-6).  H, gamma, W, targets, dH, dW 16-byte aligned;
+ *   dgamma [d] fp32, 4-byte aligned.  want_grads = 0: loss and lse only (dH, dgamma, dW unused).
+ *   grad_scale, dW_dtype: as in flce_forward.  accumulate = 1 adds into both dW and dgamma (the
+ *   parameters), 0 writes them; dH is always written.
+ *   workspace: flce_workspace_bytes_rmsnorm(shape, want_grads) bytes, 256-byte aligned.
+ *   Errors: as flce_forward; FLCE_ERR_ARG also for eps < 0 or a null gamma, or a null dgamma
+ *   with want_grads.
+ * flce_scale_grads_rmsnorm multiplies dH, dgamma and dW in place by the device scalar *grad_out
+ * (nothing when it is 1, or when grad_out is NULL): the upstream gradient applied to gradients
+ * that flce_forward_rmsnorm formed with g = 1 and accumulate = 0.
+ */
+size_t flce_workspace_bytes_rmsnorm(const flce_shape* shape, int want_grads);
+int flce_forward_rmsnorm(const flce_shape* shape, const void* H, const void* gamma, float eps,
+                         const void* W, const int64_t* targets, float* loss, float* lse,
+                         int want_grads, const float* grad_scale, void* dH, float* dgamma,
+                         void* dW, int dW_dtype, int accumulate, void* workspace,
+                         size_t workspace_bytes, void* stream);
+int flce_scale_grads_rmsnorm(const flce_shape* shape, const float* grad_out, void* dH,
+                             float* dgamma, void* dW, int dW_dtype, void* stream);
+
+/*
  * Self-test of failure detection (no counterpart on the pages): runs the library's bounded
  * pipeline wait on a barrier that nothing arrives at, with a limit of limit_ns (1 ns .. 10 s).
  * The wait runs out, FLCE_DEV_TIMEOUT is or-ed into the status word of `workspace` (read it with

@@ -6,17 +6,23 @@ arguments to it.  Entry points raise if the library is missing: there is no
 fallback implementation.
 """
 from ._abi import (DEV_BAD_TARGET, DEV_TIMEOUT, FlceError, alloc_workspace, backward,
-                   declared_functions, forward, forward_dp, forward_dp_bucketed, forward_fp8, instrument, instrument_read, lib, make_shape, raw_backward, raw_forward,
-                   quantize_e4m3, raw_forward_noalloc, read_status, rmsnorm_backward, rmsnorm_forward,
-                   selftest_wait_timeout, status_string, workspace_bytes)
-from .autograd import FusedLinearCrossEntropy, RMSNorm, fused_linear_cross_entropy, rmsnorm
+                   declared_functions, forward, forward_dp, forward_dp_bucketed, forward_fp8,
+                   forward_rmsnorm, instrument, instrument_read, lib, make_shape, raw_backward,
+                   raw_forward, quantize_e4m3, raw_forward_noalloc, read_status, rmsnorm_backward,
+                   rmsnorm_forward, scale_grads_rmsnorm, selftest_wait_timeout, status_string,
+                   workspace_bytes)
+from .autograd import (FusedLinearCrossEntropy, FusedRMSNormLinearCrossEntropy, RMSNorm,
+                       fused_linear_cross_entropy, fused_rmsnorm_linear_cross_entropy, rmsnorm)
 from . import data_parallel
 from .data_parallel import dp_step
 
 __all__ = [
     "DEV_BAD_TARGET", "DEV_TIMEOUT", "FlceError", "alloc_workspace", "backward",
-    "declared_functions", "forward", "forward_dp", "forward_dp_bucketed", "forward_fp8", "instrument", "instrument_read", "lib", "make_shape", "raw_backward", "raw_forward",
-    "quantize_e4m3", "raw_forward_noalloc", "read_status", "rmsnorm_backward",
-    "rmsnorm_forward", "selftest_wait_timeout", "status_string", "workspace_bytes", "FusedLinearCrossEntropy",
-    "fused_linear_cross_entropy", "dp_step", "RMSNorm", "rmsnorm",
+    "declared_functions", "forward", "forward_dp", "forward_dp_bucketed", "forward_fp8",
+    "forward_rmsnorm", "instrument", "instrument_read", "lib", "make_shape", "raw_backward",
+    "raw_forward", "quantize_e4m3", "raw_forward_noalloc", "read_status", "rmsnorm_backward",
+    "rmsnorm_forward", "scale_grads_rmsnorm", "selftest_wait_timeout", "status_string",
+    "workspace_bytes", "FusedLinearCrossEntropy", "FusedRMSNormLinearCrossEntropy",
+    "fused_linear_cross_entropy", "fused_rmsnorm_linear_cross_entropy", "dp_step", "RMSNorm",
+    "rmsnorm",
 ]

@@ -106,6 +106,13 @@ def lib() -> ctypes.CDLL:
     L.flce_rmsnorm_backward.argtypes = [P, P, P, P, ctypes.c_int64, ctypes.c_int64, P, P,
                                         ctypes.c_int, P, ctypes.c_size_t, P]
     L.flce_rmsnorm_backward.restype = ctypes.c_int
+    L.flce_workspace_bytes_rmsnorm.argtypes = [shp, ctypes.c_int]
+    L.flce_workspace_bytes_rmsnorm.restype = ctypes.c_size_t
+    L.flce_forward_rmsnorm.argtypes = [shp, P, P, ctypes.c_float, P, P, P, P, I, P, P, P, P, I,
+                                       I, P, ctypes.c_size_t, P]
+    L.flce_forward_rmsnorm.restype = ctypes.c_int
+    L.flce_scale_grads_rmsnorm.argtypes = [shp, P, P, P, P, I, P]
+    L.flce_scale_grads_rmsnorm.restype = ctypes.c_int
     L.flce_selftest_wait_timeout.argtypes = [P, ctypes.c_uint64, P]
     L.flce_selftest_wait_timeout.restype = ctypes.c_int
     L.flce_check_pair_schedule.argtypes = [ctypes.c_int] * 5 + [
@@ -450,6 +457,75 @@ def rmsnorm_forward(H, gamma, eps: float = 1e-6, X=None, rstd=None, stream=None)
     if rc != FLCE_OK:
         raise FlceError(rc, "flce_rmsnorm_forward")
     return X, rstd
+
+
+def forward_rmsnorm(H, gamma, W, targets, Vreal: int, cap: float = 15.0, ignore_index: int = -1,
+                    eps: float = 1e-6, want_grads: bool = False, dH=None, dgamma=None, dW=None,
+                    accumulate: bool = False, workspace=None, chunk_rows: int = 0, stream=None,
+                    grad_scale=None, dW_dtype=None):
+    """The final RMSNorm and the head in one call (flce_forward_rmsnorm).  Returns
+    ``(loss, lse, dH, dgamma, dW, workspace)``; the gradients (None unless ``want_grads``) are
+    those of ``grad_scale * loss`` with respect to the rows before the norm, its gamma and the
+    head; ``accumulate`` adds into dgamma and dW."""
+    import torch
+    _check(H, W, targets)
+    N, d = H.shape
+    dev = H.device
+    _check_buffer(gamma, "gamma", torch.bfloat16, (d,), dev)
+    if gamma is None:
+        raise TypeError("gamma must be a bfloat16 CUDA tensor [d]")
+    dw_t, dw_code = _dW_type(dW, dW_dtype)
+    if want_grads:
+        _check_buffer(dH, "dH", torch.bfloat16, H.shape, dev)
+        _check_buffer(dgamma, "dgamma", torch.float32, (d,), dev)
+        _check_buffer(dW, "dW", dw_t, W.shape, dev)
+        grad_scale = _grad_scale(grad_scale, dev)
+    _check_workspace(workspace, dev)
+    shape = make_shape(N, d, W.shape[0], Vreal, cap, ignore_index, chunk_rows)
+    loss = torch.empty((), dtype=torch.float32, device=dev)
+    lse = torch.empty(max(N, 1), dtype=torch.float32, device=dev)[:N]
+    if want_grads:
+        if dH is None:
+            dH = torch.empty_like(H)
+        if dgamma is None:
+            dgamma = torch.empty(d, dtype=torch.float32, device=dev)
+        if dW is None:
+            dW = torch.empty(W.shape, dtype=dw_t, device=dev)
+    if workspace is None:
+        nbytes = int(lib().flce_workspace_bytes_rmsnorm(ctypes.byref(shape), int(want_grads)))
+        if nbytes == 0:
+            raise FlceError(-1, "flce_workspace_bytes_rmsnorm")
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    g = want_grads
+    rc = lib().flce_forward_rmsnorm(ctypes.byref(shape), _ptr(H), _ptr(gamma), float(eps),
+                                    _ptr(W), _ptr(targets), _ptr(loss), _ptr(lse), int(g),
+                                    _ptr(grad_scale) if g else None, _ptr(dH) if g else None,
+                                    _ptr(dgamma) if g else None, _ptr(dW) if g else None,
+                                    dw_code, int(accumulate), _ptr(workspace),
+                                    workspace.numel(), _stream(stream))
+    if rc != FLCE_OK:
+        raise FlceError(rc, "flce_forward_rmsnorm")
+    if not g:
+        return loss, lse, None, None, None, workspace
+    return loss, lse, dH, dgamma, dW, workspace
+
+
+def scale_grads_rmsnorm(grad_out, dH, dgamma, dW, Vreal: int, cap: float = 15.0,
+                        ignore_index: int = -1, stream=None):
+    """dH, dgamma, dW *= grad_out (a one-element float32 device tensor) in place."""
+    import torch
+    N, d = dH.shape
+    dev = dH.device
+    _check_scalar(grad_out, "grad_out", torch.float32, dev)
+    _check_buffer(dH, "dH", torch.bfloat16, (N, d), dev)
+    _check_buffer(dgamma, "dgamma", torch.float32, (d,), dev)
+    dw_t, dw_code = _dW_type(dW, None)
+    _check_buffer(dW, "dW", dw_t, (dW.shape[0], d), dev)
+    shape = make_shape(N, d, dW.shape[0], Vreal, cap, ignore_index, 0)
+    rc = lib().flce_scale_grads_rmsnorm(ctypes.byref(shape), _ptr(grad_out), _ptr(dH),
+                                        _ptr(dgamma), _ptr(dW), dw_code, _stream(stream))
+    if rc != FLCE_OK:
+        raise FlceError(rc, "flce_scale_grads_rmsnorm")
 
 
 def rmsnorm_backward(H, gamma, rstd, dX, dH=None, dgamma=None, accumulate_dgamma: bool = False,

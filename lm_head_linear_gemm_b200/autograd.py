@@ -1,4 +1,5 @@
-"""``torch.autograd`` drop-ins for the fused linear cross-entropy and the final RMSNorm.
+"""``torch.autograd`` drop-ins for the fused linear cross-entropy, the final RMSNorm, and the two
+in one call.
 
     loss = fused_linear_cross_entropy(hidden, lm_head_weight, targets, Vreal=50257, cap=15.0)
     loss.backward()
@@ -105,6 +106,53 @@ def fused_linear_cross_entropy(X, W, targets, Vreal: int, cap: float = 15.0,
     caller will back-propagate (the forward then accumulates into main_grad in the same pass)."""
     return FusedLinearCrossEntropy.apply(X, W, targets, Vreal, cap, ignore_index, chunk_rows,
                                          grad_scale)
+
+
+class FusedRMSNormLinearCrossEntropy(torch.autograd.Function):
+    """The model's final RMSNorm and the head in one library call (flce_forward_rmsnorm): the
+    forward forms the loss and, for g = 1, the gradients of the rows before the norm, of gamma
+    and of the head -- the norm's backward folded into the dX contraction, so dX itself is never
+    stored -- and backward multiplies them by the upstream gradient in place."""
+
+    @staticmethod
+    def forward(ctx, H, gamma, W, targets, Vreal, cap, ignore_index, eps, chunk_rows):
+        ctx.meta = (Vreal, cap, ignore_index)
+        ctx.done = False
+        if not any(ctx.needs_input_grad[:3]):
+            loss, _, _, _, _, _ = _abi.forward_rmsnorm(H, gamma, W, targets, Vreal, cap,
+                                                       ignore_index, eps, chunk_rows=chunk_rows)
+            return loss
+        dW_dtype = W.dtype if W.dtype in (torch.float32, torch.bfloat16) else torch.float32
+        loss, _, dH, dgamma, dW, _ = _abi.forward_rmsnorm(
+            H, gamma, W, targets, Vreal, cap, ignore_index, eps, want_grads=True,
+            chunk_rows=chunk_rows, dW_dtype=dW_dtype)
+        ctx.save_for_backward(dH, dgamma, dW)
+        return loss
+
+    @staticmethod
+    @once_differentiable
+    def backward(ctx, g):
+        if ctx.done:
+            raise RuntimeError("fused_rmsnorm_linear_cross_entropy: backward already ran for this "
+                               "graph (its gradients were formed in place)")
+        ctx.done = True
+        Vreal, cap, ignore_index = ctx.meta
+        dH, dgamma, dW = ctx.saved_tensors
+        g = g.detach().to(torch.float32).contiguous()
+        _abi.scale_grads_rmsnorm(g, dH, dgamma, dW, Vreal, cap, ignore_index)
+        wants = ctx.needs_input_grad
+        return (dH if wants[0] else None, dgamma if wants[1] else None, dW if wants[2] else None,
+                None, None, None, None, None, None)
+
+
+def fused_rmsnorm_linear_cross_entropy(H, gamma, W, targets, Vreal: int, cap: float = 15.0,
+                                       ignore_index: int = -1, eps: float = 1e-6,
+                                       chunk_rows: int = 0):
+    """Mean softcapped cross entropy of ``rmsnorm(H, gamma) W^T`` over rows whose target is not
+    ignore_index, with gradients into H, gamma and W (gamma's gradient is formed in float32 and
+    cast to gamma's dtype by autograd)."""
+    return FusedRMSNormLinearCrossEntropy.apply(H, gamma, W, targets, Vreal, cap, ignore_index,
+                                                eps, chunk_rows)
 
 
 class RMSNorm(torch.autograd.Function):

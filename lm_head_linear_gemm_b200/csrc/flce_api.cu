@@ -126,6 +126,7 @@ constexpr auto kGradKernel8 =
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s bound on every in-kernel wait
 constexpr float kFixedRefMaxCap = 32.f;           // exp(s - cap) >= e^{-64}: no underflow in fp32
 constexpr int64_t kAutoChunkRows = 8192;   // rows per chunk when chunk_rows = 0
+constexpr int kRmsRowsPerPart = 128;       // rows per dgamma partial of the RMSNorm backward
 constexpr int kLogitsRows = 4096;          // rows per logits launch (launch_logits)
 constexpr size_t kAlign = 256;
 
@@ -139,6 +140,11 @@ struct Layout {
   bool fixed_ref;
   bool compact;       // gradients over each chunk's rows in the loss only
   size_t hdr, tgt, s_t, der_t, e_t, row_loss, partial, r, A, Xs, pos, orig, cnt, bad, gsc, total;
+  // final RMSNorm in front of the head (flce_forward_rmsnorm): the normalised rows and rstd;
+  // with gradients either the folded backward's pieces (fixed reference) or a dX buffer and
+  // dgamma partials for the separate backward kernels
+  bool rms;
+  size_t Xn, rstd, qpart, zt, cdot, dgpart, dXtmp, rmspart;
 };
 
 bool shape_ok(const flce_shape* s) {
@@ -152,7 +158,7 @@ bool shape_ok(const flce_shape* s) {
   return true;
 }
 
-Layout make_layout(const flce_shape* s, int want_grads) {
+Layout make_layout(const flce_shape* s, int want_grads, int rms = 0) {
   Layout L{};
   const int64_t N = s->N;
   int64_t nc = s->chunk_rows > 0 ? s->chunk_rows : kAutoChunkRows;
@@ -189,6 +195,22 @@ Layout make_layout(const flce_shape* s, int want_grads) {
       L.cnt = take(static_cast<size_t>(L.n_chunks) * sizeof(int));
       L.bad = take(static_cast<size_t>(L.n_chunks) * sizeof(int));
       L.gsc = take(2 * sizeof(float));
+    }
+  }
+  if (rms) {
+    L.rms = true;
+    L.Xn = take(n * static_cast<size_t>(s->d) * sizeof(__nv_bfloat16));
+    L.rstd = take(n * sizeof(float));
+    if (want_grads && L.fixed_ref) {
+      L.qpart = take(static_cast<size_t>(nc) * L.n_slabs * sizeof(float));
+      L.zt = take(n * sizeof(float));
+      L.cdot = take(static_cast<size_t>(nc) * sizeof(float));
+      // one row of partials per 32 rows of the chunk's 256-row tiles
+      L.dgpart = take(static_cast<size_t>((nc + 255) / 256 * 8) * s->d * sizeof(float));
+    } else if (want_grads) {
+      L.dXtmp = take(n * static_cast<size_t>(s->d) * sizeof(__nv_bfloat16));
+      L.rmspart = take(static_cast<size_t>((n + kRmsRowsPerPart - 1) / kRmsRowsPerPart) * s->d *
+                       sizeof(float));
     }
   }
   L.total = off;
@@ -372,9 +394,20 @@ struct Fp8Logits {
   const float* scale_w = nullptr;
 };
 
+// The final RMSNorm x = h rstd gamma in front of the head, and where its gradients go.
+struct RmsFold {
+  const __nv_bfloat16* H;
+  const __nv_bfloat16* gamma;
+  float eps;
+  __nv_bfloat16* dH;
+  float* dgamma;
+  int accumulate;            // dgamma += (else =)
+};
+
 struct Ctx {
   const flce_shape* s;
   Fp8Logits fp8;
+  const RmsFold* rms = nullptr;          // RMSNorm backward folded into the dX epilogue
   const long long* nv_total = nullptr;   // data-parallel normaliser (null: this call's rows)
   int dW_bf16 = 0;                       // dW element type: 0 fp32, 1 bf16
   int grad_fp8 = 0;                      // gradient contractions from e5m2 / e4m3 operands
@@ -429,6 +462,10 @@ int launch_logits(const Ctx& c, int64_t row0, int rows, const __nv_bfloat16* X,
     q.s_t = lp.s_t + r0;
     q.der_t = lp.der_t + r0;
     q.e_t = lp.e_t + r0;
+    if (lp.q_partial != nullptr) {
+      q.q_partial = lp.q_partial + static_cast<size_t>(r0) * lp.n_slabs;
+      q.z_t = lp.z_t + r0;
+    }
     // compacted rows index A from the chunk's first row: only pos moves with the launch
     q.pos = lp.pos != nullptr ? lp.pos + r0 : nullptr;
     q.A = lp.A != nullptr && lp.pos == nullptr ? lp.A + static_cast<size_t>(r0) * lp.a_ld : lp.A;
@@ -498,6 +535,11 @@ int grad_chunk(const Ctx& c, int64_t row0, int rows, const __nv_bfloat16* X,
   const int chunk_index = static_cast<int>(row0 / c.L.chunk);
   const int* cnt = c.L.compact ? c.at<int>(c.L.cnt) + chunk_index : nullptr;
   lp.pos = c.L.compact ? c.at<int>(c.L.pos) + row0 : nullptr;
+  const bool fold = c.rms != nullptr;
+  if (fold) {
+    lp.q_partial = c.at<float>(c.L.qpart);
+    lp.z_t = c.at<float>(c.L.zt) + row0;
+  }
   FLCE_TRY(launch_logits(c, row0, rows, X, W, lp));
 
   RowFinishParams rp{};
@@ -533,6 +575,11 @@ int grad_chunk(const Ctx& c, int64_t row0, int rows, const __nv_bfloat16* X,
   rp.X8 = c.grad_fp8 ? c.fp8.X8 + row0 * s->d : nullptr;
   rp.Xs8 = Xs8;
   rp.ktail = c.grad_fp8 ? CfgG8::KSLOT : Cfg::KSLOT;
+  if (fold) {
+    rp.q_partial = lp.q_partial;
+    rp.z_t = lp.z_t;
+    rp.cdot = c.at<float>(c.L.cdot);
+  }
   const int finish_warps = rows + (c.L.compact ? rp.ktail : 0);
   row_finish_kernel<<<(finish_warps + 7) / 8, 256, 0, c.st>>>(rp);
   FLCE_TRY(launch_ok());
@@ -544,6 +591,13 @@ int grad_chunk(const Ctx& c, int64_t row0, int rows, const __nv_bfloat16* X,
   const float* gsc = c.grad_fp8 ? c.at<float>(c.L.gsc) : nullptr;
   DxParams xp{rows, d, dx32, r, dXc, c.L.compact ? c.at<int>(c.L.orig) + row0 : nullptr, cnt,
               gsc};
+  if (fold) {
+    xp.H = c.rms->H + row0 * s->d;
+    xp.gamma = c.rms->gamma;
+    xp.rstd = c.at<float>(c.L.rstd) + row0;
+    xp.cdot = c.at<float>(c.L.cdot);
+    xp.dg_part = c.at<float>(c.L.dgpart);
+  }
   const int dyn_x = c.L.compact ? DYN_M : 0, dyn_w = c.L.compact ? DYN_K : 0;
   const PairProblem pdx{rows, d, Vpad, 0, FLCE_DX_WIDE, FLCE_L2_DX_A, FLCE_L2_DX_W, dyn_x};
   const PairProblem none{0, 0, 0, 0, 0, 0, 0, 0};
@@ -589,6 +643,11 @@ int grad_chunk(const Ctx& c, int64_t row0, int rows, const __nv_bfloat16* X,
       buckets->bounds[b] = v0;
       buckets->bounds[b + 1] = v1;
     }
+  }
+  if (fold) {
+    rmsnorm_dgamma_chunk_kernel<<<(d + 255) / 256, 256, 0, c.st>>>(
+        xp.dg_part, d, rows, cnt, c.rms->dgamma, (row0 > 0 || c.rms->accumulate) ? 1 : 0);
+    FLCE_TRY(launch_ok());
   }
   return FLCE_OK;
 }
@@ -654,6 +713,27 @@ int zero_dW(const Ctx& c, void* dW) {
   return launch_ok();
 }
 
+// The RMSNorm backward as row kernels, for a dX already formed: dH per row, dgamma in two
+// deterministic stages (partials of kRmsRowsPerPart rows, then summed in order).
+int rmsnorm_backward_kernels(const __nv_bfloat16* H, const __nv_bfloat16* gamma,
+                             const float* rstd, const __nv_bfloat16* dX, int64_t N, int d,
+                             __nv_bfloat16* dH, float* dgamma, int accumulate, float* partial,
+                             cudaStream_t st) {
+  int parts = 0;
+  if (N > 0) {
+    rmsnorm_bwd_rows_kernel<<<static_cast<unsigned>((N + 7) / 8), 256, 0, st>>>(H, gamma, rstd,
+                                                                                dX, N, d, dH);
+    FLCE_TRY(launch_ok());
+    parts = static_cast<int>((N + kRmsRowsPerPart - 1) / kRmsRowsPerPart);
+    rmsnorm_dgamma_partial_kernel<<<dim3((d / 2 + 255) / 256, parts), 256, 0, st>>>(
+        H, rstd, dX, N, d, kRmsRowsPerPart, partial);
+    FLCE_TRY(launch_ok());
+  }
+  rmsnorm_dgamma_final_kernel<<<(d + 255) / 256, 256, 0, st>>>(partial, parts, d, dgamma,
+                                                                accumulate);
+  return launch_ok();
+}
+
 // Targets -> effective ids, the count of rows in the loss and the status word; with compaction
 // also each chunk's positions of its rows in the loss (prep_chunks_kernel).
 int prep(const Ctx& c, const int64_t* targets) {
@@ -716,7 +796,7 @@ int forward_impl(const flce_shape* s, const void* X, const void* W, const Fp8Log
                  const float* grad_scale, void* dX, void* dW, int dW_dtype, int accumulate_dW,
                  void* workspace, size_t workspace_bytes, void* stream,
                  const int64_t* nv_total = nullptr, const Buckets* buckets = nullptr,
-                 int grad_fp8 = 0) {
+                 int grad_fp8 = 0, const RmsFold* rms = nullptr) {
   want_grads = want_grads ? 1 : 0;
   if (loss == nullptr || (s->N > 0 && lse == nullptr)) return FLCE_ERR_ARG;
   if (!aligned4(loss) || !aligned4(lse)) return FLCE_ERR_ALIGN;
@@ -734,7 +814,7 @@ int forward_impl(const flce_shape* s, const void* X, const void* W, const Fp8Log
   c.nv_total = reinterpret_cast<const long long*>(nv_total);
   c.dW_bf16 = want_grads && dW_dtype == FLCE_DTYPE_BF16 ? 1 : 0;
   c.grad_fp8 = want_grads && grad_fp8 ? 1 : 0;
-  c.L = make_layout(s, want_grads);
+  c.L = make_layout(s, want_grads, rms != nullptr ? 1 : 0);
   // 8-bit gradients need the fixed exp reference and the compacted rows (rows not in the loss
   // must not enter the e5m2 operand)
   if (c.grad_fp8 && (!c.L.fixed_ref || !c.L.compact || fp8.X8 == nullptr)) return FLCE_ERR_ARG;
@@ -744,6 +824,28 @@ int forward_impl(const flce_shape* s, const void* X, const void* W, const Fp8Log
   c.hdr = c.at<DevHeader>(c.L.hdr);
   const auto* Xb = static_cast<const __nv_bfloat16*>(X);
   const auto* Wb = static_cast<const __nv_bfloat16*>(W);
+  // With the final RMSNorm in front, the head reads the normalised rows written here.  Its
+  // backward is folded into the dX epilogue on the fixed-reference path (dX is then never
+  // formed: the epilogue writes dH), else dX goes to a buffer and the RMSNorm backward kernels
+  // follow the head.
+  const bool fold = rms != nullptr && want_grads && c.L.fixed_ref;
+  auto* dXout = static_cast<__nv_bfloat16*>(dX);
+  if (rms != nullptr) {
+    if (s->N > 0) {
+      auto* Xn = c.at<__nv_bfloat16>(c.L.Xn);
+      rmsnorm_fwd_kernel<<<static_cast<unsigned>((s->N + 7) / 8), 256, 0, c.st>>>(
+          rms->H, rms->gamma, rms->eps, s->N, static_cast<int>(s->d), Xn,
+          c.at<float>(c.L.rstd));
+      FLCE_TRY(launch_ok());
+      Xb = Xn;
+    }
+    if (fold) {
+      c.rms = rms;
+      dXout = rms->dH;
+    } else if (want_grads) {
+      dXout = c.at<__nv_bfloat16>(c.L.dXtmp);
+    }
+  }
 
   FLCE_TRY(prep(c, targets));
   if (c.grad_fp8) {
@@ -755,6 +857,10 @@ int forward_impl(const flce_shape* s, const void* X, const void* W, const Fp8Log
     zero_loss_kernel<<<1, 1, 0, c.st>>>(loss);
     FLCE_TRY(launch_ok());
     if (want_grads && !accumulate_dW) FLCE_TRY(zero_dW(c, dW));
+    if (want_grads && rms != nullptr && !rms->accumulate) {
+      fill_zero_f32_kernel<<<1, 256, 0, c.st>>>(rms->dgamma, s->d);
+      FLCE_TRY(launch_ok());
+    }
     if (buckets != nullptr) {
       // nothing to wait for: every bucket is final now
       for (int b = 0; b < buckets->n; ++b) {
@@ -776,8 +882,7 @@ int forward_impl(const flce_shape* s, const void* X, const void* W, const Fp8Log
     for (int64_t row0 = 0; row0 < s->N; row0 += c.L.chunk) {
       const int rows = static_cast<int>(s->N - row0 < c.L.chunk ? s->N - row0 : c.L.chunk);
       const bool last = row0 + rows >= s->N;
-      FLCE_TRY(grad_chunk(c, row0, rows, Xb, Wb, nullptr, lse, grad_scale,
-                          static_cast<__nv_bfloat16*>(dX), dW,
+      FLCE_TRY(grad_chunk(c, row0, rows, Xb, Wb, nullptr, lse, grad_scale, dXout, dW,
                           (row0 > 0 || accumulate_dW) ? 1 : 0, LOGITS_FUSED,
                           last ? buckets : nullptr));
     }
@@ -791,12 +896,15 @@ int forward_impl(const flce_shape* s, const void* X, const void* W, const Fp8Log
     for (int64_t row0 = 0; row0 < s->N; row0 += c.L.chunk) {
       const int rows = static_cast<int>(s->N - row0 < c.L.chunk ? s->N - row0 : c.L.chunk);
       const bool last = row0 + rows >= s->N;
-      FLCE_TRY(grad_chunk(c, row0, rows, Xb, Wb, lse, nullptr, grad_scale,
-                          static_cast<__nv_bfloat16*>(dX), dW,
+      FLCE_TRY(grad_chunk(c, row0, rows, Xb, Wb, lse, nullptr, grad_scale, dXout, dW,
                           (row0 > 0 || accumulate_dW) ? 1 : 0, LOGITS_RECOMPUTE,
                           last ? buckets : nullptr));
     }
   }
+  if (rms != nullptr && want_grads && !fold)
+    FLCE_TRY(rmsnorm_backward_kernels(rms->H, rms->gamma, c.at<float>(c.L.rstd), dXout, s->N,
+                                      static_cast<int>(s->d), rms->dH, rms->dgamma,
+                                      rms->accumulate, c.at<float>(c.L.rmspart), c.st));
   return FLCE_OK;
 }
 
@@ -995,9 +1103,8 @@ int flce_forward_noalloc(const flce_shape* shape, const void* X, const void* W,
                       FLCE_DTYPE_F32, 0, scratch, FLCE_NOALLOC_SCRATCH_BYTES, stream);
 }
 
-constexpr int kRmsRowsPerPart = 128;
 
-int rms_args_ok(const void* H, const void* gamma, int64_t N, int64_t d) {
+static int rms_args_ok(const void* H, const void* gamma, int64_t N, int64_t d) {
   if (N < 0 || d <= 0 || d > (int64_t(1) << 24) || gamma == nullptr || (N > 0 && H == nullptr))
     return FLCE_ERR_ARG;
   if ((d % 8) != 0 || !aligned16(H) || !aligned16(gamma)) return FLCE_ERR_ALIGN;
@@ -1040,25 +1147,61 @@ int flce_rmsnorm_backward(const void* H, const void* gamma, const float* rstd, c
   DeviceInfo* di = nullptr;
   FLCE_TRY(device_info(&di));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const auto* Hb = static_cast<const __nv_bfloat16*>(H);
-  const auto* dXb = static_cast<const __nv_bfloat16*>(dX);
-  const int di32 = static_cast<int>(d);
-  float* partial = static_cast<float*>(workspace);
-  int parts = 1;
-  if (N > 0) {
-    rmsnorm_bwd_rows_kernel<<<static_cast<unsigned>((N + 7) / 8), 256, 0, st>>>(
-        Hb, static_cast<const __nv_bfloat16*>(gamma), rstd, dXb, N, di32,
-        static_cast<__nv_bfloat16*>(dH));
-    FLCE_TRY(launch_ok());
-    parts = static_cast<int>((N + kRmsRowsPerPart - 1) / kRmsRowsPerPart);
-    rmsnorm_dgamma_partial_kernel<<<dim3((di32 / 2 + 255) / 256, parts), 256, 0, st>>>(
-        Hb, rstd, dXb, N, di32, kRmsRowsPerPart, partial);
-    FLCE_TRY(launch_ok());
-  } else {
-    parts = 0;
+  return rmsnorm_backward_kernels(
+      static_cast<const __nv_bfloat16*>(H), static_cast<const __nv_bfloat16*>(gamma), rstd,
+      static_cast<const __nv_bfloat16*>(dX), N, static_cast<int>(d),
+      static_cast<__nv_bfloat16*>(dH), dgamma, accumulate_dgamma,
+      static_cast<float*>(workspace), st);
+}
+
+size_t flce_workspace_bytes_rmsnorm(const flce_shape* shape, int want_grads) {
+  if (!shape_ok(shape)) return 0;
+  return make_layout(shape, want_grads ? 1 : 0, 1).total;
+}
+
+int flce_forward_rmsnorm(const flce_shape* s, const void* H, const void* gamma, float eps,
+                         const void* W, const int64_t* targets, float* loss, float* lse,
+                         int want_grads, const float* grad_scale, void* dH, float* dgamma,
+                         void* dW, int dW_dtype, int accumulate, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+  want_grads = want_grads ? 1 : 0;
+  if (!shape_ok(s)) return FLCE_ERR_ARG;
+  FLCE_TRY(rms_args_ok(H, gamma, s->N, s->d));
+  if (!(eps >= 0.f)) return FLCE_ERR_ARG;
+  if ((s->Vpad % 8) != 0) return FLCE_ERR_ALIGN;
+  if ((s->N > 0 && targets == nullptr) || W == nullptr || workspace == nullptr)
+    return FLCE_ERR_ARG;
+  if (!aligned16(W) || !aligned16(targets) ||
+      (reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0)
+    return FLCE_ERR_ALIGN;
+  if (workspace_bytes < make_layout(s, want_grads, 1).total) return FLCE_ERR_WORKSPACE;
+  if (want_grads) {
+    if (dgamma == nullptr) return FLCE_ERR_ARG;
+    if (!aligned4(dgamma)) return FLCE_ERR_ALIGN;
   }
-  rmsnorm_dgamma_final_kernel<<<(di32 + 255) / 256, 256, 0, st>>>(partial, parts, di32, dgamma,
-                                                                    accumulate_dgamma);
+  const RmsFold rf{static_cast<const __nv_bfloat16*>(H), static_cast<const __nv_bfloat16*>(gamma),
+                   eps, static_cast<__nv_bfloat16*>(dH), dgamma, accumulate ? 1 : 0};
+  // the head's input is the normalised rows forward_impl writes; dH takes dX's place
+  return forward_impl(s, nullptr, W, Fp8Logits{}, targets, loss, lse, want_grads, grad_scale, dH,
+                      dW, dW_dtype, accumulate, workspace, workspace_bytes, stream, nullptr,
+                      nullptr, 0, &rf);
+}
+
+int flce_scale_grads_rmsnorm(const flce_shape* s, const float* grad_out, void* dH, float* dgamma,
+                             void* dW, int dW_dtype, void* stream) {
+  if (!shape_ok(s) || dgamma == nullptr || dW == nullptr || (s->N > 0 && dH == nullptr))
+    return FLCE_ERR_ARG;
+  if (dW_dtype != FLCE_DTYPE_F32 && dW_dtype != FLCE_DTYPE_BF16) return FLCE_ERR_ARG;
+  if ((s->d % 8) != 0 || !aligned16(dH) || !aligned16(dW) || !aligned4(dgamma) ||
+      !aligned4(grad_out))
+    return FLCE_ERR_ALIGN;
+  DeviceInfo* di = nullptr;
+  FLCE_TRY(device_info(&di));
+  if (grad_out == nullptr) return FLCE_OK;
+  const int dW_bf16 = dW_dtype == FLCE_DTYPE_BF16 ? 1 : 0;
+  scale_grads_kernel<<<4 * di->sms, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<__nv_bfloat16*>(dH), s->N * s->d / 8, dW, s->Vpad * s->d / (dW_bf16 ? 8 : 4),
+      dW_bf16, grad_out, dgamma, s->d);
   return launch_ok();
 }
 

@@ -719,6 +719,11 @@ struct LogitsParams {
   float* e_t;                // [rows] exp(s_t - reference)
   __nv_bfloat16* A;          // [rows][Vpad] gradient operand (modes FUSED / RECOMPUTE)
   const int* pos;            // [rows] row of A for each row (-1: not written), or null: same row
+  // The final RMSNorm's backward folded into dX (fixed reference only): per slab the sum of
+  // A_ij z_ij over its columns (z the logit before the softcap), and the target's z.  With the
+  // row sum S_i they give sum_j dz_ij z_ij, which is d times the RMSNorm's row term.
+  float* q_partial;          // [rows][n_slabs], or null
+  float* z_t;                // [rows] (with q_partial)
 };
 
 struct LogitsEpi {
@@ -741,8 +746,10 @@ struct LogitsEpi {
                                   : ((p.mode == LOGITS_RECOMPUTE && row_ok) ? __ldg(p.ref + row) : 0.f);
     float sum = 0.f;
     float run_max = -INFINITY;
-    float tv_s = 0.f, tv_der = 0.f, tv_e = 0.f;
+    float tv_s = 0.f, tv_der = 0.f, tv_e = 0.f, tv_z = 0.f;
     bool has_t = false;
+    const bool want_q = p.q_partial != nullptr;
+    float qsum = 0.f;                                  // sum of A_ij z_ij / zs
     __nv_bfloat16* arow = nullptr;
     if (write_a && row_ok) {
       const int at = p.pos != nullptr ? __ldg(p.pos + row) : row;
@@ -764,22 +771,27 @@ struct LogitsEpi {
           tv_s = sc.s;
           tv_der = sc.der;
           tv_e = sc.e;
+          tv_z = zt * zs;
           has_t = true;
         }
         if (cbase + 32 <= p.Vreal) {
 #pragma unroll
           for (int k = 0; k < 32; ++k) {
-            const Softcapped sc = softcap_fixed_ref(v[k], k_u, p.m2c_log2e, p.cap);
+            const float z = v[k];
+            const Softcapped sc = softcap_fixed_ref(z, k_u, p.m2c_log2e, p.cap);
             sum += sc.e;
             v[k] = sc.e * sc.der;
+            if (want_q) qsum = fmaf(v[k], z, qsum);
           }
         } else {                                            // last vocabulary tile: padded columns
 #pragma unroll
           for (int k = 0; k < 32; ++k) {
-            const Softcapped sc = softcap_fixed_ref(v[k], k_u, p.m2c_log2e, p.cap);
+            const float z = v[k];
+            const Softcapped sc = softcap_fixed_ref(z, k_u, p.m2c_log2e, p.cap);
             const float e = cbase + k < p.Vreal ? sc.e : 0.f;
             sum += e;
             v[k] = e * sc.der;
+            if (want_q) qsum = fmaf(v[k], z, qsum);
           }
         }
       } else {
@@ -865,6 +877,7 @@ struct LogitsEpi {
     if (p.mode != LOGITS_RECOMPUTE) {
       if (!online) {
         p.partial[static_cast<size_t>(row) * p.n_slabs + slab_index] = sum;
+        if (want_q) p.q_partial[static_cast<size_t>(row) * p.n_slabs + slab_index] = qsum * zs;
       } else {
         float* pp = p.partial + (static_cast<size_t>(row) * p.n_slabs + slab_index) * 2;
         pp[0] = run_max;
@@ -875,6 +888,7 @@ struct LogitsEpi {
       p.s_t[row] = tv_s;
       p.der_t[row] = tv_der;
       p.e_t[row] = tv_e;
+      if (want_q) p.z_t[row] = tv_z;
     }
   }
 };
@@ -889,13 +903,120 @@ struct DxParams {
   const int* orig;           // compacted rows: dX row of each (null: same row)
   const int* dyn_rows;       // compacted rows: their device-side count (null: rows)
   const float* uscale;       // one scale for every row instead of r (8-bit operands), or null
+  // The final RMSNorm x = h rstd gamma folded in (H != null): the rows are written as
+  //   dH = rstd (gamma . dX - xh c),  xh = h rstd,  c = mean_k x_k dX_k
+  // in place of dX, and for every block of 32 rows the column sums of dX . xh (the terms of
+  // dgamma) go to dg_part.
+  const __nv_bfloat16* H;    // [rows][d] the rows before the norm (indexed like dX)
+  const __nv_bfloat16* gamma;// [d]
+  const float* rstd;         // [rows] (indexed like dX)
+  const float* cdot;         // [rows] c of each row (indexed like r)
+  float* dg_part;            // [row blocks of 32][d] (blocks of the rows indexed like r)
 };
 
 struct DxEpi {
   using Params = DxParams;
+
+  // On return lane L holds in a[0] the sum over the warp's 32 lanes of a[L]: five exchange
+  // rounds, each halving the columns a lane keeps (the lanes with the round's bit set keep the
+  // upper half).
+  __device__ static __forceinline__ void warp_column_sums(float (&a)[32], int lane) {
+#pragma unroll
+    for (int s = 16; s >= 1; s >>= 1) {
+      const bool upper = (lane & s) != 0;
+#pragma unroll
+      for (int k = 0; k < s; ++k) {
+        const float send = upper ? a[k] : a[k + s];
+        const float keep = upper ? a[k + s] : a[k];
+        a[k] = keep + __shfl_xor_sync(0xffffffffu, send, s);
+      }
+    }
+  }
+
+  template <int NCOLS>
+  __device__ static __forceinline__ void apply_rmsnorm(const Params& p, int row, int col0,
+                                                       uint32_t taddr, bool zero) {
+    const int lane = threadIdx.x & 31;
+    const int rows = p.dyn_rows != nullptr ? __ldg(p.dyn_rows) : p.rows;
+    const bool row_ok = row < rows;
+    const float sc = row_ok ? __ldg(p.r + row) : 0.f;
+    const float c = row_ok ? __ldg(p.cdot + row) : 0.f;
+    const int out_row = row_ok && p.orig != nullptr ? __ldg(p.orig + row) : row;
+    const float rs = row_ok ? __ldg(p.rstd + out_row) : 0.f;
+    const __nv_bfloat16* hrow = p.H + static_cast<size_t>(row_ok ? out_row : 0) * p.d;
+    __nv_bfloat16* out = row_ok ? p.dX + static_cast<size_t>(out_row) * p.d : nullptr;
+    float* dgp = p.dg_part + static_cast<size_t>(row >> 5) * p.d;   // the warp's 32-row block
+#pragma unroll 1
+    for (int cc = 0; cc < NCOLS / 32; ++cc) {
+      float v[32];
+      tmem_ld32_or_zero(taddr + cc * 32, v, zero);
+      const int cbase = col0 + cc * 32;
+      if (cbase >= p.d) continue;                      // the same for the whole warp
+      float dg[32];
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        const int col = cbase + 8 * g;
+        uint4 hr = make_uint4(0, 0, 0, 0), gr = make_uint4(0, 0, 0, 0);
+        if (col < p.d) {
+          gr = __ldg(reinterpret_cast<const uint4*>(p.gamma + col));
+          if (row_ok) hr = __ldg(reinterpret_cast<const uint4*>(hrow + col));
+        }
+        const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&hr);
+        const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&gr);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float2 hf = __bfloat1622float2(h2[q]);
+          const float2 gf = __bfloat1622float2(g2[q]);
+          const int k = 8 * g + 2 * q;
+          const float xh0 = hf.x * rs, xh1 = hf.y * rs;
+          const float dx0 = v[k] * sc, dx1 = v[k + 1] * sc;
+          v[k] = rs * (gf.x * dx0 - xh0 * c);
+          v[k + 1] = rs * (gf.y * dx1 - xh1 * c);
+          dg[k] = dx0 * xh0;
+          dg[k + 1] = dx1 * xh1;
+        }
+      }
+      if (out != nullptr) store_row32(p, out, cbase, v);
+      warp_column_sums(dg, lane);
+      if (cbase + lane < p.d) dgp[cbase + lane] = dg[0];
+    }
+  }
+
+  // 32 values of one row as bf16 at columns [cbase, cbase + 32) (those below d).
+  __device__ static __forceinline__ void store_row32(const Params& p, __nv_bfloat16* out,
+                                                     int cbase, const float (&v)[32]) {
+    uint32_t w[16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) w[k] = pack_bf16x2(v[2 * k], v[2 * k + 1]);
+    if (p.sector32) {
+      // two full 32-byte sectors per 32 columns
+#pragma unroll
+      for (int g = 0; g < 2; ++g) {
+        const int col = cbase + 16 * g;
+        if (col < p.d) {
+          const uint32_t q[8] = {w[8 * g],     w[8 * g + 1], w[8 * g + 2], w[8 * g + 3],
+                                 w[8 * g + 4], w[8 * g + 5], w[8 * g + 6], w[8 * g + 7]};
+          st_global_v8(out + col, q);
+        }
+      }
+    } else {
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        const int col = cbase + 8 * g;
+        if (col < p.d)
+          *reinterpret_cast<uint4*>(out + col) =
+              make_uint4(w[4 * g], w[4 * g + 1], w[4 * g + 2], w[4 * g + 3]);
+      }
+    }
+  }
+
   template <int NCOLS>
   __device__ static __forceinline__ void apply(const Params& p, int row, int col0, uint32_t taddr,
                                                int, bool zero) {
+    if (p.H != nullptr) {
+      apply_rmsnorm<NCOLS>(p, row, col0, taddr, zero);
+      return;
+    }
     const int rows = p.dyn_rows != nullptr ? __ldg(p.dyn_rows) : p.rows;
     const bool row_ok = row < rows;
     const float sc = !row_ok ? 0.f : (p.uscale != nullptr ? __ldg(p.uscale) : __ldg(p.r + row));
@@ -906,30 +1027,9 @@ struct DxEpi {
       float v[32];
       tmem_ld32_or_zero(taddr + c * 32, v, zero);
       if (out == nullptr) continue;
-      const int cbase = col0 + c * 32;
-      uint32_t w[16];
 #pragma unroll
-      for (int k = 0; k < 16; ++k) w[k] = pack_bf16x2(v[2 * k] * sc, v[2 * k + 1] * sc);
-      if (p.sector32) {
-        // two full 32-byte sectors per 32 columns
-#pragma unroll
-        for (int g = 0; g < 2; ++g) {
-          const int col = cbase + 16 * g;
-          if (col < p.d) {
-            const uint32_t q[8] = {w[8 * g],     w[8 * g + 1], w[8 * g + 2], w[8 * g + 3],
-                                   w[8 * g + 4], w[8 * g + 5], w[8 * g + 6], w[8 * g + 7]};
-            st_global_v8(out + col, q);
-          }
-        }
-      } else {
-#pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          const int col = cbase + 8 * g;
-          if (col < p.d)
-            *reinterpret_cast<uint4*>(out + col) =
-                make_uint4(w[4 * g], w[4 * g + 1], w[4 * g + 2], w[4 * g + 3]);
-        }
-      }
+      for (int k = 0; k < 32; ++k) v[k] *= sc;
+      store_row32(p, out, col0 + c * 32, v);
     }
   }
 };

@@ -184,6 +184,12 @@ struct RowFinishParams {
   int fp8;
   const uint8_t* X8;            // [rows][d] this chunk's e4m3 rows
   uint8_t* Xs8;                 // [rows][d]
+  // The final RMSNorm's backward folded into dX (fixed reference, from partials): the row term
+  // c_i = mean_k x_ik dX_ik = (1/d) sum_j dz_ij z_ij = r_i (Q_i - S_i der_t z_t) / d, Q_i the
+  // sum of the per-slab partials of A_ij z_ij (A before the target patch); 0 outside the loss.
+  const float* q_partial;       // [rows][n_slabs], or null (no fold)
+  const float* z_t;             // [rows] target logit before the softcap
+  float* cdot;                  // [rows] c_i (indexed like r)
 };
 
 __device__ __forceinline__ void zero_row_bf16(__nv_bfloat16* row, int n, int lane) {
@@ -301,6 +307,13 @@ __global__ void __launch_bounds__(256) row_finish_kernel(const RowFinishParams p
     ref = p.fixed_ref ? p.cap : lse;
     S = p.fixed_ref ? expf(lse - ref) : 1.f;
   }
+  float Q = 0.f;                                  // RMSNorm fold: sum_j A_ij z_ij
+  if (p.q_partial != nullptr) {
+    const float* qp = p.q_partial + static_cast<size_t>(row) * p.n_slabs;
+    for (int k = lane; k < p.n_slabs; k += 32) Q += qp[k];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) Q += __shfl_xor_sync(0xffffffffu, Q, o);
+  }
   const int t = p.tgt[row];
   const bool valid = t >= 0;
   if (lane == 0 && p.from_partials) {
@@ -323,6 +336,9 @@ __global__ void __launch_bounds__(256) row_finish_kernel(const RowFinishParams p
     encode_row_e5m2(p, row, at, t, S);
     return;
   }
+  if (p.cdot != nullptr && lane == 0)
+    p.cdot[at] = r != 0.f ? r * (Q - S * p.der_t[row] * p.z_t[row]) / static_cast<float>(p.d)
+                          : 0.f;
   if (lane == 0) {
     p.r[at] = r;
     if (valid) {
@@ -367,11 +383,13 @@ __global__ void __launch_bounds__(1024) loss_kernel(const float* __restrict__ ro
   }
 }
 
-// dX *= g, dW *= g for gradients formed with g = 1; returns at once when g == 1.  dW is fp32
+// dX *= g, dW *= g (and dg *= g, fp32) for gradients formed with g = 1; returns at once when
+// g == 1.  dW is fp32
 // (nW = elements / 4, float4 groups) or bf16 (dW_bf16 = 1, nW = elements / 8, groups of 8).
 __global__ void scale_grads_kernel(__nv_bfloat16* __restrict__ dX, long long nX8,
                                    void* __restrict__ dW, long long nW, int dW_bf16,
-                                   const float* __restrict__ grad_out) {
+                                   const float* __restrict__ grad_out,
+                                   float* __restrict__ dg = nullptr, long long n_dg = 0) {
   const float g = *grad_out;
   if (g == 1.f) return;
   const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
@@ -403,6 +421,9 @@ __global__ void scale_grads_kernel(__nv_bfloat16* __restrict__ dX, long long nX8
       }
     }
   }
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n_dg;
+       i += stride)
+    dg[i] *= g;
 }
 
 // ---------------------------------------------------------------- tensorwise e4m3 quantisation
@@ -580,6 +601,21 @@ __global__ void __launch_bounds__(256) rmsnorm_dgamma_partial_kernel(
   float* prow = partial + static_cast<long long>(blockIdx.y) * d;
   prow[k] = acc0;
   prow[k + 1] = acc1;
+}
+
+// dgamma (+)= the column sums of one chunk's dX . xh, from the dX epilogue's per-32-row-block
+// partials summed in block order over the blocks of the chunk's rows (its rows in the loss when
+// compacted: a device-side count).
+__global__ void rmsnorm_dgamma_chunk_kernel(const float* __restrict__ partial, int d, int rows,
+                                            const int* __restrict__ cnt, float* __restrict__ dgamma,
+                                            int accumulate) {
+  const int k = blockIdx.x * blockDim.x + threadIdx.x;
+  if (k >= d) return;
+  const int m = cnt != nullptr ? *cnt : rows;
+  const int blocks = (m + 31) / 32;
+  float acc = 0.f;
+  for (int b = 0; b < blocks; ++b) acc += partial[static_cast<long long>(b) * d + k];
+  dgamma[k] = accumulate ? dgamma[k] + acc : acc;
 }
 
 __global__ void rmsnorm_dgamma_final_kernel(const float* __restrict__ partial, int parts, int d,

@@ -202,6 +202,19 @@ def make_inputs(cfg: FlceConfig | str, seed: int | None = None, N: int | None = 
     return dict(X=X, W=W, targets=t, cfg=cfg)
 
 
+def make_rmsnorm_inputs(cfg: FlceConfig | str, seed: int | None = None, N: int | None = None,
+                        h_std: float = 2.0, gamma_std: float = 0.1):
+    """make_inputs plus the rows before the model's final RMSNorm and its gain:
+    H = uint16 [N,d] bf16 bits of N(0, h_std) (the residual stream has no fixed scale),
+    gamma = uint16 [d] bf16 bits of 1 + N(0, gamma_std)."""
+    inp = make_inputs(cfg, seed, N)
+    c = inp["cfg"]
+    inp["H"] = _normal_bf16(_rng(c.seed, "H"), (c.N, c.d), h_std)
+    g = 1.0 + gamma_std * _rng(c.seed, "gamma").standard_normal(c.d, dtype=np.float32)
+    inp["gamma"] = f32_to_bf16_bits(g.astype(np.float32))
+    return inp
+
+
 def custom_config(name: str, N: int, d: int, Vreal: int, Vpad: int, *, x_dist="normal",
                   w_std=0.02, target_dist="uniform", ignore_count=0, ignore_index=-1,
                   cap=15.0, seed=0) -> FlceConfig:

@@ -29,7 +29,8 @@ def test_exports_every_declared_symbol(L):
                           "flce_count_valid", "flce_forward_dp", "flce_forward_dp_bucketed",
                           "flce_rmsnorm_forward",
                           "flce_rmsnorm_workspace_bytes", "flce_rmsnorm_backward",
-                          "flce_check_pair_schedule"}
+                          "flce_workspace_bytes_rmsnorm", "flce_forward_rmsnorm",
+                          "flce_scale_grads_rmsnorm", "flce_check_pair_schedule"}
     for n in names:
         assert hasattr(L, n), n
     out = subprocess.run(["nm", "-D", "--defined-only", _abi.LIB_PATH], capture_output=True,
@@ -152,6 +153,31 @@ def test_rmsnorm_and_quantiser_reject_bad_arguments_before_launch(L):
     assert q(p, -1, p, p, None) == -1
     assert q(p, 16, None, p, None) == -1
     assert q(p, 16, p, p + 2, None) == -2
+
+
+def test_rmsnorm_head_rejects_bad_arguments_before_launch(L):
+    p = 0x10000000      # never dereferenced: argument checks come first
+    s = flce.make_shape(8, 64, 128, 100)
+    sp = ctypes.byref(s)
+    ws = L.flce_workspace_bytes_rmsnorm(sp, 1)
+    # beyond the head's workspace: the normalised rows and rstd, and the fold's partials
+    assert ws >= flce.workspace_bytes(s, True) + 8 * 64 * 2 + 8 * 4
+    f = L.flce_forward_rmsnorm
+    # H, gamma, eps, W, t, loss, lse, want_grads, g, dH, dgamma, dW, dW_dtype, acc, ws,
+    # ws_bytes, stream
+    assert f(sp, p, None, 1e-6, p, p, p, p, 1, None, p, p, p, 0, 0, p, ws, None) == -1  # gamma
+    assert f(sp, p, p, -1.0, p, p, p, p, 1, None, p, p, p, 0, 0, p, ws, None) == -1     # eps
+    assert f(sp, None, p, 1e-6, p, p, p, p, 1, None, p, p, p, 0, 0, p, ws, None) == -1  # H
+    assert f(sp, p + 8, p, 1e-6, p, p, p, p, 1, None, p, p, p, 0, 0, p, ws, None) == -2
+    assert f(sp, p, p, 1e-6, p, p, p, p, 1, None, p, p, p, 0, 0, p, ws - 1, None) == -3
+    assert f(sp, p, p, 1e-6, p, p, p, p, 1, None, p, None, p, 0, 0, p, ws, None) == -1  # dgamma
+    assert f(sp, p, p, 1e-6, p, p, p, p, 1, None, p, p + 2, p, 0, 0, p, ws, None) == -2
+    assert f(sp, p, p, 1e-6, p, p, p, p, 1, None, p, p, p, 5, 0, p, ws, None) == -1    # dtype
+    sg = L.flce_scale_grads_rmsnorm
+    assert sg(sp, p, p, None, p, 0, None) == -1
+    assert sg(sp, p, p, p, p, 2, None) == -1
+    assert sg(sp, p + 2, p, p, p, 0, None) == -2
+    assert sg(sp, p, p + 8, p, p, 0, None) == -2
 
 
 def test_fp8_dp_and_count_entry_points_reject_bad_arguments_before_launch(L):

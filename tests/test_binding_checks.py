@@ -118,6 +118,19 @@ def test_rmsnorm_checks_its_buffers():
                               dgamma=Buf((D,), torch.bfloat16))
 
 
+def test_rmsnorm_head_checks_its_buffers():
+    H, g, W = Buf((N, D), torch.bfloat16), Buf((D,), torch.bfloat16), Buf((V, D), torch.bfloat16)
+    t = Buf((N,), torch.int64)
+    with pytest.raises(ValueError):
+        _abi.forward_rmsnorm(H, Buf((D - 8,), torch.bfloat16), W, t, 1000)
+    with pytest.raises(TypeError):
+        _abi.forward_rmsnorm(H, g, W, t, 1000, want_grads=True, dgamma=Buf((D,), torch.bfloat16))
+    with pytest.raises(ValueError):
+        _abi.forward_rmsnorm(H, g, W, t, 1000, want_grads=True, dH=Buf((N, D + 8), torch.bfloat16))
+    with pytest.raises(TypeError):
+        _abi.forward_rmsnorm(H, g, W, t, 1000, want_grads=True, dW=Buf((V, D), torch.float16))
+
+
 def test_quantiser_checks_outputs():
     x = Buf((N, D), torch.bfloat16)
     with pytest.raises(TypeError):

@@ -233,6 +233,34 @@ def test_edge_cases(cuda_device):
     assert loss.item() == 0.0 and lse.numel() == 0 and float(dW.abs().max()) == 0.0
 
 
+def test_smallest_hidden_and_vocabulary(cuda_device):
+    """d = 8, the smallest hidden size the header allows (one 16-byte row: every tile is a K
+    tail and a ragged N block), and Vpad = 40, a multiple of 8 but not of 16 (gradient-operand
+    rows not 32-byte aligned), in one chunk and in chunks of 32 rows."""
+    inp = synth.make_inputs(synth.custom_config("d8", 70, 8, 33, 40, w_std=0.5, ignore_count=3))
+    ref = oracle_full(inp)
+    for chunk_rows in (0, 32):
+        got = run_gpu(inp, chunk_rows=chunk_rows)
+        assert got["status"] == 0
+        compare_full(got, ref)
+    compare_full(run_gpu(inp, recompute=True), ref)
+
+
+@pytest.mark.parametrize("ignore_index", [-100, 3])
+def test_other_ignore_index(cuda_device, ignore_index):
+    """ignore_index other than -1: PyTorch's default -100, and a vocabulary id (3), whose rows
+    leave the loss while column 3 stays in every row's softmax.  Neither is a bad target."""
+    cfg = synth.custom_config("ignore_other", N=300, d=200, Vreal=1500, Vpad=1544,
+                              w_std=0.05, ignore_count=11, ignore_index=ignore_index)
+    inp = synth.make_inputs(cfg)
+    assert int(np.count_nonzero(inp["targets"] == ignore_index)) >= 11
+    ref = oracle_full(inp)
+    for chunk_rows in (0, 128):
+        got = run_gpu(inp, chunk_rows=chunk_rows)
+        assert got["status"] == 0
+        compare_full(got, ref)
+
+
 def test_accumulate_and_upstream_gradient(cuda_device):
     import lm_head_linear_gemm_b200 as flce
     torch = _torch()
