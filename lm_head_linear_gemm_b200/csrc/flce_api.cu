@@ -645,7 +645,7 @@ int grad_chunk(const Ctx& c, int64_t row0, int rows, const __nv_bfloat16* X,
     }
   }
   if (fold) {
-    rmsnorm_dgamma_chunk_kernel<<<(d + 255) / 256, 256, 0, c.st>>>(
+    rmsnorm_dgamma_chunk_kernel<<<(d + 31) / 32, dim3(32, 8), 0, c.st>>>(
         xp.dg_part, d, rows, cnt, c.rms->dgamma, (row0 > 0 || c.rms->accumulate) ? 1 : 0);
     FLCE_TRY(launch_ok());
   }

@@ -946,22 +946,35 @@ struct DxEpi {
     const __nv_bfloat16* hrow = p.H + static_cast<size_t>(row_ok ? out_row : 0) * p.d;
     __nv_bfloat16* out = row_ok ? p.dX + static_cast<size_t>(out_row) * p.d : nullptr;
     float* dgp = p.dg_part + static_cast<size_t>(row >> 5) * p.d;   // the warp's 32-row block
+    // h is read one 32-column chunk ahead of its use, so that the load's latency overlaps the
+    // previous chunk's arithmetic (this epilogue is not overlapped with MMAs in wide tiles)
+    uint4 hn[4];
+    auto load_h = [&](int cbase) {
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        const int col = cbase + 8 * g;
+        hn[g] = (row_ok && col < p.d) ? __ldg(reinterpret_cast<const uint4*>(hrow + col))
+                                      : make_uint4(0, 0, 0, 0);
+      }
+    };
+    load_h(col0);
 #pragma unroll 1
     for (int cc = 0; cc < NCOLS / 32; ++cc) {
       float v[32];
       tmem_ld32_or_zero(taddr + cc * 32, v, zero);
       const int cbase = col0 + cc * 32;
       if (cbase >= p.d) continue;                      // the same for the whole warp
+      uint4 hc[4];
+#pragma unroll
+      for (int g = 0; g < 4; ++g) hc[g] = hn[g];
+      if (cc + 1 < NCOLS / 32) load_h(cbase + 32);
       float dg[32];
 #pragma unroll
       for (int g = 0; g < 4; ++g) {
         const int col = cbase + 8 * g;
-        uint4 hr = make_uint4(0, 0, 0, 0), gr = make_uint4(0, 0, 0, 0);
-        if (col < p.d) {
-          gr = __ldg(reinterpret_cast<const uint4*>(p.gamma + col));
-          if (row_ok) hr = __ldg(reinterpret_cast<const uint4*>(hrow + col));
-        }
-        const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&hr);
+        const uint4 gr = col < p.d ? __ldg(reinterpret_cast<const uint4*>(p.gamma + col))
+                                   : make_uint4(0, 0, 0, 0);
+        const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&hc[g]);
         const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&gr);
 #pragma unroll
         for (int q = 0; q < 4; ++q) {

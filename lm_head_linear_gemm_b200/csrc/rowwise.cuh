@@ -604,18 +604,27 @@ __global__ void __launch_bounds__(256) rmsnorm_dgamma_partial_kernel(
 }
 
 // dgamma (+)= the column sums of one chunk's dX . xh, from the dX epilogue's per-32-row-block
-// partials summed in block order over the blocks of the chunk's rows (its rows in the loss when
-// compacted: a device-side count).
-__global__ void rmsnorm_dgamma_chunk_kernel(const float* __restrict__ partial, int d, int rows,
-                                            const int* __restrict__ cnt, float* __restrict__ dgamma,
-                                            int accumulate) {
-  const int k = blockIdx.x * blockDim.x + threadIdx.x;
-  if (k >= d) return;
+// partials over the blocks of the chunk's rows (its rows in the loss when compacted: a device-side
+// count).  A block of 32 x 8 threads takes 32 columns: thread row y sums the blocks b = y mod 8
+// in order, then the eight sums are added in order (deterministic).
+__global__ void __launch_bounds__(256) rmsnorm_dgamma_chunk_kernel(
+    const float* __restrict__ partial, int d, int rows, const int* __restrict__ cnt,
+    float* __restrict__ dgamma, int accumulate) {
+  __shared__ float part[8][32];
+  const int k = blockIdx.x * 32 + threadIdx.x;
   const int m = cnt != nullptr ? *cnt : rows;
   const int blocks = (m + 31) / 32;
   float acc = 0.f;
-  for (int b = 0; b < blocks; ++b) acc += partial[static_cast<long long>(b) * d + k];
-  dgamma[k] = accumulate ? dgamma[k] + acc : acc;
+  if (k < d)
+    for (int b = threadIdx.y; b < blocks; b += 8) acc += partial[static_cast<long long>(b) * d + k];
+  part[threadIdx.y][threadIdx.x] = acc;
+  __syncthreads();
+  if (threadIdx.y == 0 && k < d) {
+    float sum = 0.f;
+#pragma unroll
+    for (int y = 0; y < 8; ++y) sum += part[y][threadIdx.x];
+    dgamma[k] = accumulate ? dgamma[k] + sum : sum;
+  }
 }
 
 __global__ void rmsnorm_dgamma_final_kernel(const float* __restrict__ partial, int parts, int d,
