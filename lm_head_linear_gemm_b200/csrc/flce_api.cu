@@ -106,6 +106,10 @@ using CfgL = PairCfg<FLCE_LOGITS_BN, FLCE_LOGITS_STAGES, FLCE_EPI_WARPS, 2, FLCE
 constexpr auto kLogitsKernel =
     gemm_pair_kernel<CfgL, LogitsEpi, LogitsEpi, Major::K, Major::K, Major::K, Major::K, false,
                      FLCE_LOGITS_ROUND>;
+// the same with the final RMSNorm's row sums in the epilogue (flce_forward_rmsnorm)
+constexpr auto kLogitsFoldKernel =
+    gemm_pair_kernel<CfgL, LogitsFoldEpi, LogitsFoldEpi, Major::K, Major::K, Major::K, Major::K,
+                     false, FLCE_LOGITS_ROUND>;
 // logits from e4m3 operands (kind::f8f6f4, tensorwise scales applied in the epilogue)
 using Cfg8 = PairCfg<FLCE_LOGITS_BN, FLCE_LOGITS_STAGES, FLCE_EPI_WARPS, 1, FLCE_LOGITS_KSUB>;
 constexpr auto kLogitsKernel8 =
@@ -246,6 +250,8 @@ int device_info(DeviceInfo** out) {
   if (!di.ok) return FLCE_ERR_DEVICE;
   if (!di.attrs_set) {
     if (cudaFuncSetAttribute(kLogitsKernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             CfgL::SMEM_BYTES) != cudaSuccess ||
+        cudaFuncSetAttribute(kLogitsFoldKernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              CfgL::SMEM_BYTES) != cudaSuccess ||
         cudaFuncSetAttribute(kGradKernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              Cfg::SMEM_BYTES) != cudaSuccess ||
@@ -442,6 +448,10 @@ int launch_logits_rows(const Ctx& c, int64_t row0, int rows, const __nv_bfloat16
   FLCE_TRY(make_map(&mX, X + row0 * s->d, d, rows, d, CfgL::BM_CTA));
   FLCE_TRY(make_map(&mW, W, d, Vpad, d, CfgL::BN_CTA));
   lp.scale_a = lp.scale_b = nullptr;
+  if (lp.q_partial != nullptr)
+    return launch_pair<LogitsFoldEpi, LogitsFoldEpi, CfgL>(kLogitsFoldKernel, c.di, mX, mW, mX,
+                                                          mW, logits, none, &c.hdr->status, lp,
+                                                          lp, c.st, 0);
   return launch_pair<LogitsEpi, LogitsEpi, CfgL>(kLogitsKernel, c.di, mX, mW, mX, mW, logits,
                                                   none, &c.hdr->status, lp, lp, c.st, 0);
 }

@@ -726,7 +726,10 @@ struct LogitsParams {
   float* z_t;                // [rows] (with q_partial)
 };
 
-struct LogitsEpi {
+// FOLD: also the per-slab sums of A_ij z_ij and the target's z (q_partial, z_t), for the final
+// RMSNorm's backward; a separate instantiation, so that the plain epilogue carries none of it.
+template <bool FOLD>
+struct LogitsEpiT {
   using Params = LogitsParams;
   static constexpr float LOG2E = 1.4426950408889634f;
 
@@ -748,8 +751,7 @@ struct LogitsEpi {
     float run_max = -INFINITY;
     float tv_s = 0.f, tv_der = 0.f, tv_e = 0.f, tv_z = 0.f;
     bool has_t = false;
-    const bool want_q = p.q_partial != nullptr;
-    float qsum = 0.f;                                  // sum of A_ij z_ij / zs
+    float qsum = 0.f;                                  // FOLD: sum of A_ij z_ij / zs
     __nv_bfloat16* arow = nullptr;
     if (write_a && row_ok) {
       const int at = p.pos != nullptr ? __ldg(p.pos + row) : row;
@@ -771,7 +773,7 @@ struct LogitsEpi {
           tv_s = sc.s;
           tv_der = sc.der;
           tv_e = sc.e;
-          tv_z = zt * zs;
+          if constexpr (FOLD) tv_z = zt * zs;
           has_t = true;
         }
         if (cbase + 32 <= p.Vreal) {
@@ -781,7 +783,7 @@ struct LogitsEpi {
             const Softcapped sc = softcap_fixed_ref(z, k_u, p.m2c_log2e, p.cap);
             sum += sc.e;
             v[k] = sc.e * sc.der;
-            if (want_q) qsum = fmaf(v[k], z, qsum);
+            if constexpr (FOLD) qsum = fmaf(v[k], z, qsum);
           }
         } else {                                            // last vocabulary tile: padded columns
 #pragma unroll
@@ -791,7 +793,7 @@ struct LogitsEpi {
             const float e = cbase + k < p.Vreal ? sc.e : 0.f;
             sum += e;
             v[k] = e * sc.der;
-            if (want_q) qsum = fmaf(v[k], z, qsum);
+            if constexpr (FOLD) qsum = fmaf(v[k], z, qsum);
           }
         }
       } else {
@@ -877,7 +879,8 @@ struct LogitsEpi {
     if (p.mode != LOGITS_RECOMPUTE) {
       if (!online) {
         p.partial[static_cast<size_t>(row) * p.n_slabs + slab_index] = sum;
-        if (want_q) p.q_partial[static_cast<size_t>(row) * p.n_slabs + slab_index] = qsum * zs;
+        if constexpr (FOLD)
+          p.q_partial[static_cast<size_t>(row) * p.n_slabs + slab_index] = qsum * zs;
       } else {
         float* pp = p.partial + (static_cast<size_t>(row) * p.n_slabs + slab_index) * 2;
         pp[0] = run_max;
@@ -888,10 +891,12 @@ struct LogitsEpi {
       p.s_t[row] = tv_s;
       p.der_t[row] = tv_der;
       p.e_t[row] = tv_e;
-      if (want_q) p.z_t[row] = tv_z;
+      if constexpr (FOLD) p.z_t[row] = tv_z;
     }
   }
 };
+using LogitsEpi = LogitsEpiT<false>;
+using LogitsFoldEpi = LogitsEpiT<true>;
 
 // ==============================================================================================
 // Epilogue 2: dX rows = r_i * (A' W)_i, stored as bf16.
