@@ -395,13 +395,21 @@ def main_gpu(args):
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
+    # one event pair per step as well (median / min / max of the same steps); recording an
+    # event adds no work to the stream
+    step_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                for _ in range(args.steps)]
     e0.record(stream)
-    for _ in range(args.steps):
+    for a, b in step_evs:
+        a.record(stream)
         loss = timed_step()
+        b.record(stream)
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
     elapsed_ms = e0.elapsed_time(e1)
+    per = [a.elapsed_time(b) for a, b in step_evs]
+    spread = {"median": statistics.median(per), "min": min(per), "max": max(per)}
     kstats = flce.instrument_read()
     flce.instrument(False)
     clk = clocks.stop()
@@ -522,6 +530,38 @@ def main_gpu(args):
                                    "4*(rows in the loss)*Vpad*d per launch (the gradient "
                                    "contractions skip rows outside the loss)"}
 
+    # After the timed region (the GPU already at its power cap): the recompute path -- a forward
+    # without gradients, then a backward that recomputes the logits with lse known (8 N d Vpad
+    # executed FLOPs against 6).
+    recompute = None
+    if world == 1:
+        if not fp8:
+            ws_fwd = flce.alloc_workspace(shape, False, dev)
+
+            def rec_step():
+                _, lse_r, _, _, _ = flce.forward(X, W, t, Vr, c.cap, c.ignore_index, False,
+                                                 workspace=ws_fwd, chunk_rows=args.chunk_rows)
+                flce.backward(X, W, t, lse_r, Vr, c.cap, c.ignore_index, grad_out=g_one, dX=dX,
+                              dW=dW, workspace=ws, chunk_rows=args.chunk_rows)
+
+            for _ in range(max(2, args.warmup)):
+                rec_step()
+            torch.cuda.synchronize()
+            r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            r0.record(stream)
+            for _ in range(args.steps):
+                rec_step()
+            r1.record(stream)
+            torch.cuda.synchronize()
+            rms = r0.elapsed_time(r1) / args.steps
+            recompute = {"ms_per_step": rms, "tokens_per_s": N / (rms / 1e3),
+                         "credited_tflops": credited / (rms / 1e3) / 1e12,
+                         "executed_tflops": (4.0 * N * d * Vp + grad_flop_step) / (rms / 1e3) / 1e12,
+                         "what": "flce_forward(want_grads=0), then flce_backward recomputing the "
+                                 "logits with lse known, timed after the fused steps; executed = "
+                                 "two logits passes + the gradient contractions over the rows in "
+                                 "the loss"}
+
     unfused = None
     cpu = None
     if rank == 0 and world == 1 and not args.no_unfused:
@@ -557,6 +597,7 @@ def main_gpu(args):
             "peak_mem_MiB": {"fused_step": peak_fused / 2**20,
                              "workspace": ws.numel() / 2**20,
                              "unfused_torch": unfused["peak_MiB"] if unfused else None},
+            "per_step_ms": spread, "recompute_path": recompute,
             "unfused_torch": unfused, "device_status": status, "n_valid": nv,
             "loss": float(loss.item()),
         }
