@@ -204,3 +204,53 @@ def test_headline_sampled(cuda_device):
                                       np.argsort(-counts)[:8], np.arange(c.Vreal, c.Vpad)]))
     ref_dW = oracle.dW_rows(x, W, t, f["lse"], vrows, c.Vreal, c.cap, c.ignore_index)
     _check("dW rows", got["dW"][vrows], ref_dW)
+
+
+def test_edge_cases(cuda_device):
+    """Loss only (lse against the oracle's forward); every row ignored (loss 0, zero gradients,
+    dgamma written as zeros); a bad target (flagged, treated as ignored); N = 0 (dgamma and dW
+    written as zeros, or left as they are when accumulating)."""
+    import torch
+    import lm_head_linear_gemm_b200 as flce
+    inp = synth.make_rmsnorm_inputs(RAGGED)
+    c = inp["cfg"]
+    H, gamma, W = _dev(inp["H"]), _dev(inp["gamma"]), _dev(inp["W"])
+    # loss and lse only
+    loss, lse, dH, dg, dW, _ = flce.forward_rmsnorm(H, gamma, W, _dev(inp["targets"]), c.Vreal,
+                                                    c.cap, c.ignore_index, EPS)
+    torch.cuda.synchronize()
+    assert dH is None and dg is None and dW is None
+    ref = _oracle(inp)
+    assert abs(float(loss.item()) - ref["loss"]) <= LOSS_TOL
+    assert np.abs(lse.double().cpu().numpy() - ref["lse"]).max() <= LSE_TOL
+    # every row ignored
+    got = _run(dict(inp, targets=np.full(c.N, -1, np.int64)))
+    assert got["loss"] == 0.0 and got["n_valid"] == 0 and got["status"] == 0
+    for k in ("dH", "dgamma", "dW"):
+        assert np.abs(got[k]).max() == 0.0, k
+    # a bad target: flagged and treated as ignored
+    t = inp["targets"].copy()
+    t[5] = c.Vreal + 3
+    bad = dict(inp, targets=t)
+    got = _run(bad)
+    assert got["status"] & flce.DEV_BAD_TARGET
+    t_ref = t.copy()
+    t_ref[5] = -1
+    _compare(dict(got, status=0), _oracle(dict(inp, targets=t_ref)))
+    # N = 0
+    H0 = torch.zeros((0, c.d), dtype=torch.bfloat16, device="cuda")
+    t0 = torch.zeros((0,), dtype=torch.int64, device="cuda")
+    dg0 = torch.full((c.d,), 7.0, device="cuda")
+    dW0 = torch.full((c.Vpad, c.d), 7.0, device="cuda")
+    loss, lse, _, dg0, dW0, _ = flce.forward_rmsnorm(H0, gamma, W, t0, c.Vreal, c.cap, -1, EPS,
+                                                     want_grads=True, dgamma=dg0, dW=dW0)
+    torch.cuda.synchronize()
+    assert float(loss.item()) == 0.0 and lse.numel() == 0
+    assert float(dg0.abs().max()) == 0.0 and float(dW0.abs().max()) == 0.0
+    dg1 = torch.full((c.d,), 7.0, device="cuda")
+    dW1 = torch.full((c.Vpad, c.d), 7.0, device="cuda")
+    flce.forward_rmsnorm(H0, gamma, W, t0, c.Vreal, c.cap, -1, EPS, want_grads=True, dgamma=dg1,
+                         dW=dW1, accumulate=True)
+    torch.cuda.synchronize()
+    assert float(dg1.min()) == 7.0 and float(dg1.max()) == 7.0
+    assert float(dW1.min()) == 7.0 and float(dW1.max()) == 7.0
