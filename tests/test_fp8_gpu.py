@@ -129,6 +129,56 @@ def test_fp8_gradients_against_quantisation_aware_oracle(cuda_device):
           f"dW {_rel(got['dW'], bw):.2e}")
 
 
+RAGGED8 = synth.custom_config("fp8_ragged", N=300, d=208, Vreal=1500, Vpad=1544, w_std=0.05,
+                              ignore_count=7)
+
+
+@pytest.mark.parametrize("chunk_rows", [0, 128])
+def test_fp8_ragged_shapes(cuda_device, chunk_rows):
+    """300 rows (ragged row tiles), d = 208 (a K tail inside the second 128-byte k-block of the
+    e4m3 operands, and ragged dX / dW column tiles), Vpad = 1544 (a ragged vocabulary tile and a
+    K tail of the gradient operand), 7 ignored rows; one chunk and 128-row chunks; the bf16 and
+    the FP8 gradient products, every element."""
+    inp = synth.make_fp8_inputs(RAGGED8)
+    c = inp["cfg"]
+    Xq, Wq = _dequantised(inp)
+    t = inp["targets"]
+    ref = oracle.forward_backward(Xq, Wq, t, c.Vreal, c.cap, c.ignore_index,
+                                  Xg=synth.bf16_to_f64(inp["X"]), Wg=synth.bf16_to_f64(inp["W"]))
+    got = _run_fp8(inp, chunk_rows=chunk_rows)
+    assert got["status"] == 0 and got["n_valid"] == ref["n_valid"]
+    assert abs(got["loss"] - ref["loss"]) <= LOSS_TOL
+    assert np.abs(got["lse"] - ref["lse"]).max() <= LSE_TOL
+    _check("dX", got["dX"], ref["dX"])
+    _check("dW", got["dW"], ref["dW"])
+    rX, rW = oracle.backward_fp8(Xq, Wq, t, c.Vreal, c.cap, c.ignore_index)
+    g8 = _run_fp8(inp, chunk_rows=chunk_rows, grad_fp8=True)
+    assert g8["status"] == 0 and g8["loss"] == got["loss"]
+    _check("dX (fp8 gradients)", g8["dX"], rX)
+    _check("dW (fp8 gradients)", g8["dW"], rW)
+    assert np.abs(g8["dW"][c.Vreal:]).max() == 0.0
+    assert np.abs(g8["dX"][t == c.ignore_index]).max() == 0.0
+
+
+@pytest.mark.parametrize("cap", [0.0, 50.0])
+def test_fp8_logits_without_fixed_reference(cuda_device, cap):
+    """No softcap, or a cap above 32: the e4m3 logits take the online-softmax statistics pass and
+    the recompute of the gradient operand with lse, the scales applied to z (not folded into the
+    exp2 argument as on the fixed-reference path); bf16 gradient products."""
+    inp = synth.make_fp8_inputs(RAGGED8)
+    c = inp["cfg"]
+    Xq, Wq = _dequantised(inp)
+    ref = oracle.forward_backward(Xq, Wq, inp["targets"], c.Vreal, cap, c.ignore_index,
+                                  Xg=synth.bf16_to_f64(inp["X"]), Wg=synth.bf16_to_f64(inp["W"]))
+    import dataclasses
+    got = _run_fp8(dict(inp, cfg=dataclasses.replace(c, cap=cap)), chunk_rows=128)
+    assert got["status"] == 0
+    assert abs(got["loss"] - ref["loss"]) <= LOSS_TOL
+    assert np.abs(got["lse"] - ref["lse"]).max() <= LSE_TOL
+    _check("dX", got["dX"], ref["dX"])
+    _check("dW", got["dW"], ref["dW"])
+
+
 def test_fp8_quantisation_error_against_bf16_oracle(cuda_device):
     """Reported figure: how far e4m3 logits move the loss and gradients from the bf16 result."""
     inp = synth.make_fp8_inputs("small", N=640)
