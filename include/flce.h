@@ -272,6 +272,17 @@ int flce_forward_rmsnorm(const flce_shape* shape, const void* H, const void* gam
                          size_t workspace_bytes, void* stream);
 int flce_scale_grads_rmsnorm(const flce_shape* shape, const float* grad_out, void* dH,
                              float* dgamma, void* dW, int dW_dtype, void* stream);
+/*
+ * flce_forward_rmsnorm for one data-parallel rank: the loss and gradients are normalised by
+ * *n_valid_total (device int64, 8-byte aligned: the rows in the loss over all ranks, e.g. the
+ * all-reduced flce_count_valid), as flce_forward_dp does for the head alone.  The loss is this
+ * rank's share of the global mean; dgamma and dW are its contributions, to be summed over ranks.
+ */
+int flce_forward_rmsnorm_dp(const flce_shape* shape, const void* H, const void* gamma, float eps,
+                            const void* W, const int64_t* targets, const int64_t* n_valid_total,
+                            float* loss, float* lse, int want_grads, const float* grad_scale,
+                            void* dH, float* dgamma, void* dW, int dW_dtype, int accumulate,
+                            void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * Self-test of failure detection (no counterpart on the pages): runs the library's bounded

@@ -14,7 +14,7 @@ from ._abi import (DEV_BAD_TARGET, DEV_TIMEOUT, FlceError, alloc_workspace, back
 from .autograd import (FusedLinearCrossEntropy, FusedRMSNormLinearCrossEntropy, RMSNorm,
                        fused_linear_cross_entropy, fused_rmsnorm_linear_cross_entropy, rmsnorm)
 from . import data_parallel
-from .data_parallel import dp_step
+from .data_parallel import dp_step, dp_step_rmsnorm
 
 __all__ = [
     "DEV_BAD_TARGET", "DEV_TIMEOUT", "FlceError", "alloc_workspace", "backward",
@@ -23,6 +23,7 @@ __all__ = [
     "raw_forward", "quantize_e4m3", "raw_forward_noalloc", "read_status", "rmsnorm_backward",
     "rmsnorm_forward", "scale_grads_rmsnorm", "selftest_wait_timeout", "status_string",
     "workspace_bytes", "FusedLinearCrossEntropy", "FusedRMSNormLinearCrossEntropy",
-    "fused_linear_cross_entropy", "fused_rmsnorm_linear_cross_entropy", "dp_step", "RMSNorm",
+    "fused_linear_cross_entropy", "fused_rmsnorm_linear_cross_entropy", "dp_step",
+    "dp_step_rmsnorm", "RMSNorm",
     "rmsnorm",
 ]

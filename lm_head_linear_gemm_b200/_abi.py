@@ -111,6 +111,9 @@ def lib() -> ctypes.CDLL:
     L.flce_forward_rmsnorm.argtypes = [shp, P, P, ctypes.c_float, P, P, P, P, I, P, P, P, P, I,
                                        I, P, ctypes.c_size_t, P]
     L.flce_forward_rmsnorm.restype = ctypes.c_int
+    L.flce_forward_rmsnorm_dp.argtypes = [shp, P, P, ctypes.c_float, P, P, P, P, P, I, P, P,
+                                          P, P, I, I, P, ctypes.c_size_t, P]
+    L.flce_forward_rmsnorm_dp.restype = ctypes.c_int
     L.flce_scale_grads_rmsnorm.argtypes = [shp, P, P, P, P, I, P]
     L.flce_scale_grads_rmsnorm.restype = ctypes.c_int
     L.flce_selftest_wait_timeout.argtypes = [P, ctypes.c_uint64, P]
@@ -462,11 +465,13 @@ def rmsnorm_forward(H, gamma, eps: float = 1e-6, X=None, rstd=None, stream=None)
 def forward_rmsnorm(H, gamma, W, targets, Vreal: int, cap: float = 15.0, ignore_index: int = -1,
                     eps: float = 1e-6, want_grads: bool = False, dH=None, dgamma=None, dW=None,
                     accumulate: bool = False, workspace=None, chunk_rows: int = 0, stream=None,
-                    grad_scale=None, dW_dtype=None):
+                    grad_scale=None, dW_dtype=None, n_valid_total=None):
     """The final RMSNorm and the head in one call (flce_forward_rmsnorm).  Returns
     ``(loss, lse, dH, dgamma, dW, workspace)``; the gradients (None unless ``want_grads``) are
     those of ``grad_scale * loss`` with respect to the rows before the norm, its gamma and the
-    head; ``accumulate`` adds into dgamma and dW."""
+    head; ``accumulate`` adds into dgamma and dW.  With ``n_valid_total`` (a one-element int64
+    device tensor: the rows in the loss over all data-parallel ranks) the call is one rank's
+    share (flce_forward_rmsnorm_dp)."""
     import torch
     _check(H, W, targets)
     N, d = H.shape
@@ -474,6 +479,7 @@ def forward_rmsnorm(H, gamma, W, targets, Vreal: int, cap: float = 15.0, ignore_
     _check_buffer(gamma, "gamma", torch.bfloat16, (d,), dev)
     if gamma is None:
         raise TypeError("gamma must be a bfloat16 CUDA tensor [d]")
+    _check_scalar(n_valid_total, "n_valid_total", torch.int64, dev)
     dw_t, dw_code = _dW_type(dW, dW_dtype)
     if want_grads:
         _check_buffer(dH, "dH", torch.bfloat16, H.shape, dev)
@@ -497,14 +503,17 @@ def forward_rmsnorm(H, gamma, W, targets, Vreal: int, cap: float = 15.0, ignore_
             raise FlceError(-1, "flce_workspace_bytes_rmsnorm")
         workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev)
     g = want_grads
-    rc = lib().flce_forward_rmsnorm(ctypes.byref(shape), _ptr(H), _ptr(gamma), float(eps),
-                                    _ptr(W), _ptr(targets), _ptr(loss), _ptr(lse), int(g),
-                                    _ptr(grad_scale) if g else None, _ptr(dH) if g else None,
-                                    _ptr(dgamma) if g else None, _ptr(dW) if g else None,
-                                    dw_code, int(accumulate), _ptr(workspace),
-                                    workspace.numel(), _stream(stream))
+    head = (ctypes.byref(shape), _ptr(H), _ptr(gamma), float(eps), _ptr(W), _ptr(targets))
+    tail = (_ptr(loss), _ptr(lse), int(g), _ptr(grad_scale) if g else None,
+            _ptr(dH) if g else None, _ptr(dgamma) if g else None, _ptr(dW) if g else None,
+            dw_code, int(accumulate), _ptr(workspace), workspace.numel(), _stream(stream))
+    if n_valid_total is None:
+        rc, name = lib().flce_forward_rmsnorm(*head, *tail), "flce_forward_rmsnorm"
+    else:
+        rc = lib().flce_forward_rmsnorm_dp(*head, _ptr(n_valid_total), *tail)
+        name = "flce_forward_rmsnorm_dp"
     if rc != FLCE_OK:
-        raise FlceError(rc, "flce_forward_rmsnorm")
+        raise FlceError(rc, name)
     if not g:
         return loss, lse, None, None, None, workspace
     return loss, lse, dH, dgamma, dW, workspace

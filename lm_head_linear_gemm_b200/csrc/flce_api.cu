@@ -1169,11 +1169,12 @@ size_t flce_workspace_bytes_rmsnorm(const flce_shape* shape, int want_grads) {
   return make_layout(shape, want_grads ? 1 : 0, 1).total;
 }
 
-int flce_forward_rmsnorm(const flce_shape* s, const void* H, const void* gamma, float eps,
-                         const void* W, const int64_t* targets, float* loss, float* lse,
-                         int want_grads, const float* grad_scale, void* dH, float* dgamma,
-                         void* dW, int dW_dtype, int accumulate, void* workspace,
-                         size_t workspace_bytes, void* stream) {
+static int forward_rmsnorm_impl(const flce_shape* s, const void* H, const void* gamma, float eps,
+                                const void* W, const int64_t* targets,
+                                const int64_t* n_valid_total, float* loss, float* lse,
+                                int want_grads, const float* grad_scale, void* dH, float* dgamma,
+                                void* dW, int dW_dtype, int accumulate, void* workspace,
+                                size_t workspace_bytes, void* stream) {
   want_grads = want_grads ? 1 : 0;
   if (!shape_ok(s)) return FLCE_ERR_ARG;
   FLCE_TRY(rms_args_ok(H, gamma, s->N, s->d));
@@ -1182,7 +1183,8 @@ int flce_forward_rmsnorm(const flce_shape* s, const void* H, const void* gamma, 
   if ((s->N > 0 && targets == nullptr) || W == nullptr || workspace == nullptr)
     return FLCE_ERR_ARG;
   if (!aligned16(W) || !aligned16(targets) ||
-      (reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0)
+      (reinterpret_cast<uintptr_t>(workspace) & (kAlign - 1)) != 0 ||
+      (reinterpret_cast<uintptr_t>(n_valid_total) & 7u) != 0)
     return FLCE_ERR_ALIGN;
   if (workspace_bytes < make_layout(s, want_grads, 1).total) return FLCE_ERR_WORKSPACE;
   if (want_grads) {
@@ -1193,8 +1195,29 @@ int flce_forward_rmsnorm(const flce_shape* s, const void* H, const void* gamma, 
                    eps, static_cast<__nv_bfloat16*>(dH), dgamma, accumulate ? 1 : 0};
   // the head's input is the normalised rows forward_impl writes; dH takes dX's place
   return forward_impl(s, nullptr, W, Fp8Logits{}, targets, loss, lse, want_grads, grad_scale, dH,
-                      dW, dW_dtype, accumulate, workspace, workspace_bytes, stream, nullptr,
+                      dW, dW_dtype, accumulate, workspace, workspace_bytes, stream, n_valid_total,
                       nullptr, 0, &rf);
+}
+
+int flce_forward_rmsnorm(const flce_shape* s, const void* H, const void* gamma, float eps,
+                         const void* W, const int64_t* targets, float* loss, float* lse,
+                         int want_grads, const float* grad_scale, void* dH, float* dgamma,
+                         void* dW, int dW_dtype, int accumulate, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+  return forward_rmsnorm_impl(s, H, gamma, eps, W, targets, nullptr, loss, lse, want_grads,
+                              grad_scale, dH, dgamma, dW, dW_dtype, accumulate, workspace,
+                              workspace_bytes, stream);
+}
+
+int flce_forward_rmsnorm_dp(const flce_shape* s, const void* H, const void* gamma, float eps,
+                            const void* W, const int64_t* targets, const int64_t* n_valid_total,
+                            float* loss, float* lse, int want_grads, const float* grad_scale,
+                            void* dH, float* dgamma, void* dW, int dW_dtype, int accumulate,
+                            void* workspace, size_t workspace_bytes, void* stream) {
+  if (n_valid_total == nullptr) return FLCE_ERR_ARG;
+  return forward_rmsnorm_impl(s, H, gamma, eps, W, targets, n_valid_total, loss, lse, want_grads,
+                              grad_scale, dH, dgamma, dW, dW_dtype, accumulate, workspace,
+                              workspace_bytes, stream);
 }
 
 int flce_scale_grads_rmsnorm(const flce_shape* s, const float* grad_out, void* dH, float* dgamma,

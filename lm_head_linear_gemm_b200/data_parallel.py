@@ -21,6 +21,9 @@ backward pass in the same way.
 With gradient accumulation over micro-batches (``accumulate_dW``, ``grad_scale`` = 1/m for m
 micro-batches) the dW all-reduce is needed only once per optimizer step; ``allreduce_dW=False``
 skips it for the intermediate micro-batches (as DDP's no_sync does).
+
+``dp_step_rmsnorm`` is the same step with the model's final RMSNorm in front of the head, in one
+library call per rank (``flce_forward_rmsnorm_dp``); its parameter gradients are dW and dgamma.
 """
 from __future__ import annotations
 
@@ -64,6 +67,16 @@ class LibraryOps:
         return loss, lse, dX, dW, [(slice(bounds[b], bounds[b + 1]), events[b])
                                    for b in range(n_buckets)]
 
+    def forward_rmsnorm(self, H, gamma, W, targets, n_valid_total, Vreal, cap, ignore_index, eps,
+                        dgamma, dW, accumulate, workspace, chunk_rows, grad_scale=None):
+        """The final RMSNorm and the head in one call, normalised by the global count.  Returns
+        (loss share, lse, dH, dgamma, dW)."""
+        loss, lse, dH, dgamma, dW, _ = _abi.forward_rmsnorm(
+            H, gamma, W, targets, Vreal, cap, ignore_index, eps, True, dgamma=dgamma, dW=dW,
+            accumulate=accumulate, workspace=workspace, chunk_rows=chunk_rows,
+            grad_scale=grad_scale, n_valid_total=n_valid_total)
+        return loss, lse, dH, dgamma, dW
+
     def allreduce_async(self, t, ready, group):
         """All-reduce ``t`` on this device's communication stream once ``ready`` has fired."""
         import torch
@@ -106,3 +119,30 @@ def dp_step(X, W, targets, Vreal: int, cap: float = 15.0, ignore_index: int = -1
         if allreduce_dW:
             dist.all_reduce(dW, group=group)
     return loss, lse, dX, dW, nv
+
+
+def dp_step_rmsnorm(H, gamma, W, targets, Vreal: int, cap: float = 15.0, ignore_index: int = -1,
+                    eps: float = 1e-6, *, group=None, dgamma=None, dW=None,
+                    accumulate: bool = False, allreduce_grads: bool = True, workspace=None,
+                    chunk_rows: int = 0, ops=None, grad_scale=None):
+    """One data-parallel step of the model's final RMSNorm and the head in one call (the norm's
+    backward folded into the dX contraction).  Steps 1-2 as in ``dp_step``; step 3 is
+    ``flce_forward_rmsnorm_dp``; step 4 all-reduces the loss shares, dW and dgamma (the
+    parameters' gradients; dH stays with the rank's rows).  Returns
+    ``(loss, lse, dH, dgamma, dW, n_valid_total)``, the same as one call on the union of all
+    ranks' rows."""
+    import torch.distributed as dist
+    ops = ops or LibraryOps()
+    distributed = dist.is_initialized()
+    nv = ops.count_valid(targets, Vreal, ignore_index)
+    if distributed:
+        dist.all_reduce(nv, group=group)
+    loss, lse, dH, dgamma, dW = ops.forward_rmsnorm(H, gamma, W, targets, nv, Vreal, cap,
+                                                    ignore_index, eps, dgamma, dW, accumulate,
+                                                    workspace, chunk_rows, grad_scale)
+    if distributed:
+        dist.all_reduce(loss, group=group)
+        if allreduce_grads:
+            dist.all_reduce(dW, group=group)
+            dist.all_reduce(dgamma, group=group)
+    return loss, lse, dH, dgamma, dW, nv

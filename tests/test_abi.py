@@ -30,7 +30,8 @@ def test_exports_every_declared_symbol(L):
                           "flce_rmsnorm_forward",
                           "flce_rmsnorm_workspace_bytes", "flce_rmsnorm_backward",
                           "flce_workspace_bytes_rmsnorm", "flce_forward_rmsnorm",
-                          "flce_scale_grads_rmsnorm", "flce_check_pair_schedule"}
+                          "flce_scale_grads_rmsnorm", "flce_forward_rmsnorm_dp",
+                          "flce_check_pair_schedule"}
     for n in names:
         assert hasattr(L, n), n
     out = subprocess.run(["nm", "-D", "--defined-only", _abi.LIB_PATH], capture_output=True,
@@ -173,6 +174,12 @@ def test_rmsnorm_head_rejects_bad_arguments_before_launch(L):
     assert f(sp, p, p, 1e-6, p, p, p, p, 1, None, p, None, p, 0, 0, p, ws, None) == -1  # dgamma
     assert f(sp, p, p, 1e-6, p, p, p, p, 1, None, p, p + 2, p, 0, 0, p, ws, None) == -2
     assert f(sp, p, p, 1e-6, p, p, p, p, 1, None, p, p, p, 5, 0, p, ws, None) == -1    # dtype
+    fd = L.flce_forward_rmsnorm_dp
+    # H, gamma, eps, W, t, n_valid_total, loss, lse, want_grads, g, dH, dgamma, dW, dtype, acc,
+    # ws, ws_bytes, stream
+    assert fd(sp, p, p, 1e-6, p, p, None, p, p, 1, None, p, p, p, 0, 0, p, ws, None) == -1
+    assert fd(sp, p, p, 1e-6, p, p, p + 4, p, p, 1, None, p, p, p, 0, 0, p, ws, None) == -2
+    assert fd(sp, p, p, 1e-6, p, p, p, p, p, 1, None, p, None, p, 0, 0, p, ws, None) == -1
     sg = L.flce_scale_grads_rmsnorm
     assert sg(sp, p, p, None, p, 0, None) == -1
     assert sg(sp, p, p, p, p, 2, None) == -1

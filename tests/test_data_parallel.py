@@ -53,6 +53,21 @@ class OracleOps:
         return loss, lse, dX, dWt, [(slice(edges[b], edges[b + 1]), None)
                                     for b in range(n_buckets)]
 
+    def forward_rmsnorm(self, H, gamma, W, targets, n_valid_total, Vreal, cap, ignore_index, eps,
+                        dgamma, dW, accumulate, workspace, chunk_rows, grad_scale=None):
+        t = targets.numpy()
+        nt = int(n_valid_total.item())
+        nl = int(oracle.valid_rows(t, Vreal, ignore_index)[0].sum())
+        share = nl / nt if nt else 0.0
+        gs = 1.0 if grad_scale is None else float(grad_scale)
+        f = oracle.rmsnorm_head(H.numpy(), gamma.numpy(), W.numpy(), t, Vreal, cap, ignore_index,
+                                eps, g=share * gs)
+        dg, dWt = torch.from_numpy(f["dgamma"]), torch.from_numpy(f["dW"])
+        if accumulate:
+            dg, dWt = dgamma + dg, dW + dWt
+        return (torch.tensor(f["loss"] * share, dtype=torch.float64), torch.from_numpy(f["lse"]),
+                torch.from_numpy(f["dH"]), dg, dWt)
+
     def allreduce_async(self, t, ready, group):
         return dist.all_reduce(t, group=group, async_op=True)
 
@@ -164,3 +179,57 @@ def test_two_rank_accumulation_over_micro_batches(buckets):
             assert abs(res[r][1][k] - f["loss"]) < 1e-12
     for r in (0, 1):
         np.testing.assert_allclose(res[r][3], ref_dW, atol=1e-14)
+
+
+def _rms_data(seed=3, N=30):
+    X, W, t = _data(seed, N)
+    rng = np.random.default_rng(seed + 100)
+    H = rng.standard_normal((N, D)) * 2.0
+    gamma = 1.0 + 0.2 * rng.standard_normal(D)
+    return H, gamma, W, t
+
+
+def _rms_worker(rank, world, store_path, split, q):
+    dist.init_process_group("gloo", init_method=f"file://{store_path}", rank=rank,
+                            world_size=world)
+    try:
+        from lm_head_linear_gemm_b200.data_parallel import dp_step_rmsnorm
+        H, gamma, W, t = _rms_data()
+        lo, hi = (0, split) if rank == 0 else (split, H.shape[0])
+        loss, lse, dH, dg, dW, nv = dp_step_rmsnorm(
+            torch.from_numpy(H[lo:hi].copy()), torch.from_numpy(gamma), torch.from_numpy(W),
+            torch.from_numpy(t[lo:hi].copy()), VR, CAP, -1, ops=OracleOps())
+        q.put((rank, float(loss), dH.numpy(), dg.numpy(), dW.numpy(), int(nv.item())))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("split", [13, 4])
+def test_two_rank_rmsnorm_step_equals_union_batch(split):
+    """dp_step_rmsnorm on two gloo ranks: the global loss, dgamma and dW on both ranks and the
+    ranks' dH rows equal one oracle step of the norm and the head on the union of their rows."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    store_dir = tempfile.mkdtemp(prefix="flce_gloo_")
+    procs = [ctx.Process(target=_rms_worker,
+                         args=(r, 2, os.path.join(store_dir, "rendezvous"), split, q))
+             for r in range(2)]
+    for p in procs:
+        p.start()
+    res = {}
+    for _ in range(2):
+        r = q.get(timeout=120)
+        res[r[0]] = r
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    shutil.rmtree(store_dir, ignore_errors=True)
+    H, gamma, W, t = _rms_data()
+    ref = oracle.rmsnorm_head(H, gamma, W, t, VR, CAP, -1)
+    for r in (0, 1):
+        assert abs(res[r][1] - ref["loss"]) < 1e-12
+        np.testing.assert_allclose(res[r][3], ref["dgamma"], rtol=1e-12, atol=1e-14)
+        np.testing.assert_allclose(res[r][4], ref["dW"], rtol=1e-12, atol=1e-14)
+        assert res[r][5] == ref["n_valid"]
+    np.testing.assert_allclose(np.concatenate([res[0][2], res[1][2]]), ref["dH"], rtol=1e-12,
+                               atol=1e-14)

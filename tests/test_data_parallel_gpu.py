@@ -158,3 +158,81 @@ def test_dp_step_bucketed_world_size_one_nccl(cuda_device):
         assert _rel(dW.double().cpu().numpy(), ref["dW"]) <= REL_L2
     finally:
         dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("parts,ignored_part", [([(0, 300), (300, 1000)], None),
+                                                ([(0, 300), (300, 1000)], 1)])
+def test_rmsnorm_rank_shares_match_the_oracle_on_the_union_batch(cuda_device, parts,
+                                                                  ignored_part):
+    """flce_forward_rmsnorm_dp: each emulated rank's loss share, its dH rows and its dgamma and
+    dW contributions add up to one oracle step of the final RMSNorm and the head on the union
+    of the ranks' rows (also when one rank has no row in the loss)."""
+    import torch
+    import lm_head_linear_gemm_b200 as flce
+    from lm_head_linear_gemm_b200.data_parallel import LibraryOps
+    inp = synth.make_rmsnorm_inputs("small", N=1000)
+    c = inp["cfg"]
+    t_np = inp["targets"].copy()
+    if ignored_part is not None:
+        a, b = parts[ignored_part]
+        t_np[a:b] = -1
+    ref = oracle.rmsnorm_head(synth.bf16_to_f64(inp["H"]), synth.bf16_to_f64(inp["gamma"]),
+                              synth.bf16_to_f64(inp["W"]), t_np, c.Vreal, c.cap, -1)
+    H, gamma, W, t = _dev(inp["H"]), _dev(inp["gamma"]), _dev(inp["W"]), _dev(t_np)
+    ops = LibraryOps()
+    nv = sum(ops.count_valid(t[a:b].contiguous(), c.Vreal, -1) for a, b in parts)
+    shares, dHs, lses = [], [], []
+    dgsum = torch.zeros(c.d, device="cuda")
+    dWsum = torch.zeros(W.shape, device="cuda")
+    for a, b in parts:
+        l, lse, dH, dg, dW, _ = flce.forward_rmsnorm(H[a:b].contiguous(), gamma, W,
+                                                     t[a:b].contiguous(), c.Vreal, c.cap, -1,
+                                                     1e-6, True, chunk_rows=256,
+                                                     n_valid_total=nv)
+        shares.append(float(l.item()))
+        dHs.append(dH.double().cpu().numpy())
+        lses.append(lse.double().cpu().numpy())
+        dgsum += dg
+        dWsum += dW
+    torch.cuda.synchronize()
+    assert int(nv.item()) == ref["n_valid"]
+    assert abs(sum(shares) - ref["loss"]) <= LOSS_TOL
+    if ignored_part is not None:
+        assert shares[ignored_part] == 0.0
+        assert np.abs(dHs[ignored_part]).max() == 0.0
+    assert np.abs(np.concatenate(lses) - ref["lse"]).max() <= LSE_TOL
+    assert _rel(np.concatenate(dHs), ref["dH"]) <= REL_L2
+    assert _rel(dgsum.double().cpu().numpy(), ref["dgamma"]) <= REL_L2
+    assert _rel(dWsum.double().cpu().numpy(), ref["dW"]) <= REL_L2
+
+
+def test_dp_step_rmsnorm_world_size_one_nccl(cuda_device):
+    import torch
+    import torch.distributed as dist
+    import lm_head_linear_gemm_b200 as flce
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("nccl", rank=0, world_size=1, device_id=torch.device("cuda", 0))
+    try:
+        inp = synth.make_rmsnorm_inputs(synth.custom_config("ragged", N=300, d=200, Vreal=1500,
+                                                            Vpad=1544, w_std=0.05,
+                                                            ignore_count=7))
+        c = inp["cfg"]
+        ref = oracle.rmsnorm_head(synth.bf16_to_f64(inp["H"]), synth.bf16_to_f64(inp["gamma"]),
+                                  synth.bf16_to_f64(inp["W"]), inp["targets"], c.Vreal, c.cap,
+                                  -1)
+        loss, lse, dH, dg, dW, nv = flce.dp_step_rmsnorm(_dev(inp["H"]), _dev(inp["gamma"]),
+                                                         _dev(inp["W"]), _dev(inp["targets"]),
+                                                         c.Vreal, c.cap, -1)
+        torch.cuda.synchronize()
+        assert int(nv.item()) == ref["n_valid"] == 293
+        assert abs(loss.item() - ref["loss"]) <= LOSS_TOL
+        assert np.abs(lse.double().cpu().numpy() - ref["lse"]).max() <= LSE_TOL
+        assert _rel(dH.double().cpu().numpy(), ref["dH"]) <= REL_L2
+        assert _rel(dg.double().cpu().numpy(), ref["dgamma"]) <= REL_L2
+        assert _rel(dW.double().cpu().numpy(), ref["dW"]) <= REL_L2
+    finally:
+        dist.destroy_process_group()
