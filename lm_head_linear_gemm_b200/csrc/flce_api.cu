@@ -111,7 +111,13 @@ constexpr auto kLogitsFoldKernel =
     gemm_pair_kernel<CfgL, LogitsFoldEpi, LogitsFoldEpi, Major::K, Major::K, Major::K, Major::K,
                      false, FLCE_LOGITS_ROUND>;
 // logits from e4m3 operands (kind::f8f6f4, tensorwise scales applied in the epilogue)
-using Cfg8 = PairCfg<FLCE_LOGITS_BN, FLCE_LOGITS_STAGES, FLCE_EPI_WARPS, 1, FLCE_LOGITS_KSUB>;
+#ifndef FLCE_LOGITS8_STAGES
+#define FLCE_LOGITS8_STAGES FLCE_LOGITS_STAGES
+#endif
+#ifndef FLCE_LOGITS8_KSUB
+#define FLCE_LOGITS8_KSUB FLCE_LOGITS_KSUB
+#endif
+using Cfg8 = PairCfg<FLCE_LOGITS_BN, FLCE_LOGITS8_STAGES, FLCE_EPI_WARPS, 1, FLCE_LOGITS8_KSUB>;
 constexpr auto kLogitsKernel8 =
     gemm_pair_kernel<Cfg8, LogitsEpi, LogitsEpi, Major::K, Major::K, Major::K, Major::K, false,
                      FLCE_LOGITS_ROUND>;
