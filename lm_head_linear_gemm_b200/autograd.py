@@ -150,7 +150,12 @@ def fused_rmsnorm_linear_cross_entropy(H, gamma, W, targets, Vreal: int, cap: fl
                                        chunk_rows: int = 0):
     """Mean softcapped cross entropy of ``rmsnorm(H, gamma) W^T`` over rows whose target is not
     ignore_index, with gradients into H, gamma and W (gamma's gradient is formed in float32 and
-    cast to gamma's dtype by autograd)."""
+    cast to gamma's dtype by autograd).
+
+    The gradients are formed in the forward for g = 1 and scaled by the upstream gradient in
+    backward, as in the plain mode of ``fused_linear_cross_entropy``; a ``main_grad`` on W is not
+    used here (accumulate into an fp32 buffer with ``_abi.forward_rmsnorm(..., accumulate=True,
+    grad_scale=g)`` instead)."""
     return FusedRMSNormLinearCrossEntropy.apply(H, gamma, W, targets, Vreal, cap, ignore_index,
                                                 eps, chunk_rows)
 

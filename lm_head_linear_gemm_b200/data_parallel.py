@@ -130,7 +130,8 @@ def dp_step_rmsnorm(H, gamma, W, targets, Vreal: int, cap: float = 15.0, ignore_
     ``flce_forward_rmsnorm_dp``; step 4 all-reduces the loss shares, dW and dgamma (the
     parameters' gradients; dH stays with the rank's rows).  Returns
     ``(loss, lse, dH, dgamma, dW, n_valid_total)``, the same as one call on the union of all
-    ranks' rows."""
+    ranks' rows.  The dW all-reduce follows the call (no vocabulary buckets on this path);
+    ``allreduce_grads=False`` skips the parameter all-reduces for intermediate micro-batches."""
     import torch.distributed as dist
     ops = ops or LibraryOps()
     distributed = dist.is_initialized()
