@@ -189,30 +189,44 @@ def _rms_data(seed=3, N=30):
     return H, gamma, W, t
 
 
-def _rms_worker(rank, world, store_path, split, q):
+def _rms_worker(rank, world, store_path, split, q, micro=1):
     dist.init_process_group("gloo", init_method=f"file://{store_path}", rank=rank,
                             world_size=world)
     try:
         from lm_head_linear_gemm_b200.data_parallel import dp_step_rmsnorm
         H, gamma, W, t = _rms_data()
         lo, hi = (0, split) if rank == 0 else (split, H.shape[0])
-        loss, lse, dH, dg, dW, nv = dp_step_rmsnorm(
-            torch.from_numpy(H[lo:hi].copy()), torch.from_numpy(gamma), torch.from_numpy(W),
-            torch.from_numpy(t[lo:hi].copy()), VR, CAP, -1, ops=OracleOps())
-        q.put((rank, float(loss), dH.numpy(), dg.numpy(), dW.numpy(), int(nv.item())))
+        Hr, tr = torch.from_numpy(H[lo:hi].copy()), torch.from_numpy(t[lo:hi].copy())
+        if micro == 1:
+            loss, lse, dH, dg, dW, nv = dp_step_rmsnorm(Hr, torch.from_numpy(gamma),
+                                                        torch.from_numpy(W), tr, VR, CAP, -1,
+                                                        ops=OracleOps())
+            q.put((rank, float(loss), dH.numpy(), dg.numpy(), dW.numpy(), int(nv.item())))
+            return
+        # this rank's rows as `micro` micro-batches, dgamma and dW accumulated with grad_scale
+        # 1/micro and all-reduced after the last one
+        cut = [(hi - lo) * k // micro for k in range(micro + 1)]
+        dg = dW = None
+        losses, dHs = [], []
+        for k in range(micro):
+            a, b = cut[k], cut[k + 1]
+            loss, _, dH, dg, dW, nv = dp_step_rmsnorm(
+                Hr[a:b], torch.from_numpy(gamma), torch.from_numpy(W), tr[a:b], VR, CAP, -1,
+                ops=OracleOps(), dgamma=dg, dW=dW, accumulate=k > 0,
+                allreduce_grads=k == micro - 1, grad_scale=1.0 / micro)
+            losses.append(float(loss))
+            dHs.append(dH.numpy())
+        q.put((rank, losses, np.concatenate(dHs), dg.numpy(), dW.numpy(), int(nv.item())))
     finally:
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("split", [13, 4])
-def test_two_rank_rmsnorm_step_equals_union_batch(split):
-    """dp_step_rmsnorm on two gloo ranks: the global loss, dgamma and dW on both ranks and the
-    ranks' dH rows equal one oracle step of the norm and the head on the union of their rows."""
+def _run_rms(split, micro=1):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     store_dir = tempfile.mkdtemp(prefix="flce_gloo_")
     procs = [ctx.Process(target=_rms_worker,
-                         args=(r, 2, os.path.join(store_dir, "rendezvous"), split, q))
+                         args=(r, 2, os.path.join(store_dir, "rendezvous"), split, q, micro))
              for r in range(2)]
     for p in procs:
         p.start()
@@ -224,6 +238,41 @@ def test_two_rank_rmsnorm_step_equals_union_batch(split):
         p.join(timeout=60)
         assert p.exitcode == 0
     shutil.rmtree(store_dir, ignore_errors=True)
+    return res
+
+
+def test_two_rank_rmsnorm_accumulation_over_micro_batches():
+    """Each rank's rows as two micro-batches with grad_scale 1/2, dgamma and dW accumulated and
+    all-reduced after the second: they equal half the sum of the oracle's gradients of the two
+    union micro-batches, whose losses both ranks hold."""
+    split = 14
+    res = _run_rms(split, micro=2)
+    H, gamma, W, t = _rms_data()
+    N = H.shape[0]
+    half0 = split // 2
+    half1 = split + (N - split) // 2
+    halves = [np.r_[0:half0, split:half1], np.r_[half0:split, half1:N]]
+    ref_dg, ref_dW = np.zeros_like(gamma), np.zeros_like(W)
+    ref_dH = np.zeros_like(H)
+    for k, rows in enumerate(halves):
+        f = oracle.rmsnorm_head(H[rows], gamma, W, t[rows], VR, CAP, -1, g=0.5)
+        ref_dg += f["dgamma"]
+        ref_dW += f["dW"]
+        ref_dH[rows] = f["dH"]
+        for r in (0, 1):
+            assert abs(res[r][1][k] - f["loss"]) < 1e-12
+    for r in (0, 1):
+        np.testing.assert_allclose(res[r][3], ref_dg, rtol=1e-12, atol=1e-14)
+        np.testing.assert_allclose(res[r][4], ref_dW, rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(np.concatenate([res[0][2], res[1][2]]), ref_dH, rtol=1e-12,
+                               atol=1e-14)
+
+
+@pytest.mark.parametrize("split", [13, 4])
+def test_two_rank_rmsnorm_step_equals_union_batch(split):
+    """dp_step_rmsnorm on two gloo ranks: the global loss, dgamma and dW on both ranks and the
+    ranks' dH rows equal one oracle step of the norm and the head on the union of their rows."""
+    res = _run_rms(split)
     H, gamma, W, t = _rms_data()
     ref = oracle.rmsnorm_head(H, gamma, W, t, VR, CAP, -1)
     for r in (0, 1):
