@@ -298,3 +298,37 @@ def test_one_call_captures_into_a_cuda_graph(cuda_device):
         torch.cuda.synchronize()
         assert torch.equal(out["loss"], ref[0])
         assert torch.equal(dH, ref[1]) and torch.equal(dg, ref[2]) and torch.equal(dW, ref[3])
+
+
+def test_one_call_beyond_32bit_element_offsets(cuda_device):
+    """N = 1400 x 512 = 716,800 rows at d = 3072: H, the normalised rows and dH hold 2.2e9
+    elements each, past 32-bit element offsets, in 88 chunks whose dgamma and dW contributions
+    accumulate.  The rows are 1400 copies of a 512-row base problem, so the oracle on the base
+    fixes every result: the loss and each row's lse equal the base's, each dH row is the base
+    row's divided by 1400 (1400 times as many rows in the loss), and dgamma and dW equal the
+    base's.  Copies of a row go through the same arithmetic and must agree bit for bit."""
+    import torch
+    import lm_head_linear_gemm_b200 as flce
+    k = 1400
+    inp = synth.make_rmsnorm_inputs("3.8b", N=512)
+    c = inp["cfg"]
+    ref = _oracle(inp)
+    H = _dev(inp["H"]).repeat(k, 1)
+    t = _dev(inp["targets"]).repeat(k)
+    assert H.numel() > 2**31
+    loss, lse, dH, dg, dW, ws = flce.forward_rmsnorm(H, _dev(inp["gamma"]), _dev(inp["W"]), t,
+                                                     c.Vreal, c.cap, c.ignore_index, EPS, True)
+    torch.cuda.synchronize()
+    status, nv = flce.read_status(ws)
+    assert status == 0 and nv == k * ref["n_valid"]
+    del H, ws
+    assert abs(float(loss.item()) - ref["loss"]) <= LOSS_TOL
+    lse_k = lse.view(k, 512)
+    assert torch.equal(lse_k, lse_k[:1].expand(k, 512))
+    assert np.abs(lse_k[0].double().cpu().numpy() - ref["lse"]).max() <= LSE_TOL
+    dH_k = dH.view(k, 512, c.d)
+    for i0 in range(0, k, 100):
+        assert torch.equal(dH_k[i0:i0 + 100], dH_k[:1].expand(min(100, k - i0), 512, c.d)), i0
+    _check("dH rows (x copies)", dH_k[0].double().cpu().numpy() * k, ref["dH"])
+    _check("dgamma", dg.double().cpu().numpy(), ref["dgamma"])
+    _check("dW", dW.double().cpu().numpy(), ref["dW"])
