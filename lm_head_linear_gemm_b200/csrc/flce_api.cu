@@ -101,7 +101,11 @@ namespace {
 #define FLCE_EPI_SECTOR32 1
 #endif
 using Cfg = PairCfg<256, FLCE_GRAD_STAGES, FLCE_EPI_WARPS>;
-using CfgL = PairCfg<FLCE_LOGITS_BN, FLCE_LOGITS_STAGES, FLCE_EPI_WARPS, 2, FLCE_LOGITS_KSUB>;
+// epilogue warps of the logits kernels (the gradient kernels keep FLCE_EPI_WARPS)
+#ifndef FLCE_LOGITS_EPI_WARPS
+#define FLCE_LOGITS_EPI_WARPS FLCE_EPI_WARPS
+#endif
+using CfgL = PairCfg<FLCE_LOGITS_BN, FLCE_LOGITS_STAGES, FLCE_LOGITS_EPI_WARPS, 2, FLCE_LOGITS_KSUB>;
 // logits: A = X (K-major), B = W (K-major)
 constexpr auto kLogitsKernel =
     gemm_pair_kernel<CfgL, LogitsEpi, LogitsEpi, Major::K, Major::K, Major::K, Major::K, false,
@@ -117,7 +121,8 @@ constexpr auto kLogitsFoldKernel =
 #ifndef FLCE_LOGITS8_KSUB
 #define FLCE_LOGITS8_KSUB FLCE_LOGITS_KSUB
 #endif
-using Cfg8 = PairCfg<FLCE_LOGITS_BN, FLCE_LOGITS8_STAGES, FLCE_EPI_WARPS, 1, FLCE_LOGITS8_KSUB>;
+using Cfg8 = PairCfg<FLCE_LOGITS_BN, FLCE_LOGITS8_STAGES, FLCE_LOGITS_EPI_WARPS, 1,
+                     FLCE_LOGITS8_KSUB>;
 constexpr auto kLogitsKernel8 =
     gemm_pair_kernel<Cfg8, LogitsEpi, LogitsEpi, Major::K, Major::K, Major::K, Major::K, false,
                      FLCE_LOGITS_ROUND>;
