@@ -132,6 +132,31 @@ def test_bucketed_forward_matches_oracle_and_unbucketed(cuda_device, n_buckets, 
     assert _rel(dW.double().cpu().numpy(), ref["dW"]) <= REL_L2
 
 
+def test_bucketed_forward_bf16_dW_accumulated(cuda_device):
+    """The bucketed launches writing a bf16 dW (the bucket offsets are in 2-byte elements) and
+    adding into it: equal bit for bit to the unbucketed call, and the sum of the two calls'
+    gradients (grad_scale 1/2 each) matches the oracle."""
+    import torch
+    import lm_head_linear_gemm_b200 as flce
+    from lm_head_linear_gemm_b200.data_parallel import LibraryOps
+    inp = synth.make_inputs("small", N=700)
+    c = inp["cfg"]
+    ref = _oracle(inp, inp["targets"])
+    X, W, t = _dev(inp["X"]), _dev(inp["W"]), _dev(inp["targets"])
+    nv = LibraryOps().count_valid(t, c.Vreal, -1)
+    events = [torch.cuda.Event() for _ in range(5)]
+    dWb = torch.zeros(W.shape, dtype=torch.bfloat16, device="cuda")
+    dWu = torch.zeros(W.shape, dtype=torch.bfloat16, device="cuda")
+    for k in range(2):
+        flce.forward_dp_bucketed(X, W, t, nv, c.Vreal, c.cap, -1, events, dW=dWb,
+                                 accumulate_dW=k > 0, chunk_rows=256, grad_scale=0.5)
+        flce.forward_dp(X, W, t, nv, c.Vreal, c.cap, -1, True, dW=dWu, accumulate_dW=k > 0,
+                        chunk_rows=256, grad_scale=0.5)
+    torch.cuda.synchronize()
+    assert torch.equal(dWb, dWu)
+    assert _rel(dWb.double().cpu().numpy(), ref["dW"]) <= REL_L2
+
+
 def test_dp_step_bucketed_world_size_one_nccl(cuda_device):
     """dp_step with the dW all-reduce in four buckets on a communication stream (NCCL, world
     size 1) against the oracle."""

@@ -129,6 +129,29 @@ def test_fp8_gradients_against_quantisation_aware_oracle(cuda_device):
           f"dW {_rel(got['dW'], bw):.2e}")
 
 
+def test_fp8_bf16_dW_written_and_accumulated(cuda_device):
+    """A bf16 dW from both gradient paths of the 8-bit workload (bf16 gradient products, and
+    e5m2 x e4m3 products whose epilogue applies the tensorwise factor before the bf16 add):
+    written by the first call with grad_scale 1/2, added to by the second, against the sum of
+    the oracle's gradients."""
+    import torch
+    inp = synth.make_fp8_inputs("small", N=640)
+    c = inp["cfg"]
+    Xq, Wq = _dequantised(inp)
+    t = inp["targets"]
+    ref = oracle.forward_backward(Xq, Wq, t, c.Vreal, c.cap, c.ignore_index,
+                                  Xg=synth.bf16_to_f64(inp["X"]), Wg=synth.bf16_to_f64(inp["W"]))
+    _, rW8 = oracle.backward_fp8(Xq, Wq, t, c.Vreal, c.cap, c.ignore_index)
+    for grad_fp8, rW in ((False, ref["dW"]), (True, rW8)):
+        dW = torch.empty((c.Vpad, c.d), dtype=torch.bfloat16, device="cuda")
+        for k in range(2):
+            got = _run_fp8(inp, chunk_rows=256, grad_fp8=grad_fp8, dW=dW, accumulate_dW=k > 0,
+                           grad_scale=0.5)
+            assert got["status"] == 0
+        _check(f"bf16 dW (grad_fp8={grad_fp8})", got["dW"], rW)
+        assert np.abs(got["dW"][c.Vreal:]).max() == 0.0
+
+
 RAGGED8 = synth.custom_config("fp8_ragged", N=300, d=208, Vreal=1500, Vpad=1544, w_std=0.05,
                               ignore_count=7)
 
